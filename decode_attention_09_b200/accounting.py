@@ -1,0 +1,31 @@
+"""Algorithmic byte accounting for decode attention (host logic, no kernels).
+
+The unit of work is one (sequence, attended position) pair of one layer.  The
+bytes that must cross HBM for it are the cached key row and value row of every KV
+head: ``n_kv_heads * head_dim * 2 bytes`` for K, the same again for V unless K
+serves as V, in which case the one tensor is read once.  Queries, outputs, LSE
+and split partials are overhead and are not counted.
+
+The per-token formula of the "Gemma 4 12B" record (KV GEOMETRY paragraph) counts
+K and V for every layer; ``count_shared_twice=True`` reproduces that figure.
+"""
+from __future__ import annotations
+
+BF16_BYTES = 2
+
+
+def kv_bytes_per_position(spec, count_shared_twice: bool = False) -> int:
+    """KV bytes read for one attended position of one sequence in one layer."""
+    tensors = 2 if (not spec.kv_shared or count_shared_twice) else 1
+    return spec.n_kv_heads * spec.head_dim * BF16_BYTES * tensors
+
+
+def attended_positions(spec, seqlen: int) -> int:
+    """Positions one decode step attends: min(L, w) for a sliding layer, L otherwise."""
+    return min(seqlen, spec.window) if spec.window > 0 else seqlen
+
+
+def layer_kv_bytes(spec, seqlens) -> int:
+    """Algorithmic KV bytes for one decode step of one layer over a batch."""
+    per = kv_bytes_per_position(spec)
+    return sum(attended_positions(spec, int(L)) * per for L in seqlens)

@@ -1,0 +1,54 @@
+"""The oracle pinned to facts outside itself (CPU only)."""
+import json
+import os
+
+import pytest
+
+import oracle
+import pins
+import workloads
+
+MUTATIONS = {
+    1: "window one position short",
+    2: "interleaved instead of contiguous GQA groups",
+    3: "soft-cap applied before the scale",
+    4: "LSE in log base 2",
+    5: "weights not normalised",
+    6: "values read from K when a separate V exists",
+    7: "ring slot off by one",
+    8: "scale dropped",
+}
+
+
+@pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda p: p.__name__)
+def test_oracle_pin(pin):
+    pin(oracle.get())
+
+
+@pytest.mark.parametrize("mutation", sorted(MUTATIONS), ids=lambda m: MUTATIONS[m])
+def test_pins_catch_planted_mistake(mutation, tmp_path):
+    """Each planted mistake in the oracle is caught by at least one pin."""
+    mutant = oracle.load(mutation, out_dir=str(tmp_path))
+    assert mutant.lib.oracle_version() == 1 + 1000 * mutation
+    failed = pins.failing_pins(mutant)
+    assert failed, f"no pin catches: {MUTATIONS[mutation]}"
+
+
+def test_golden_kv_bytes_per_token():
+    """The bench's per-token KV byte formula reproduces the figures printed for Gemma 4 12B."""
+    from decode_attention_09_b200 import accounting
+
+    with open(os.path.join(os.path.dirname(__file__), "golden", "gemma4_12b_kv_bytes.json")) as f:
+        g = json.load(f)
+    stack = workloads.gemma4_12b_stack(1024, 8192)
+    sl = [s for s in stack if s.kind == "sliding"]
+    gl = [s for s in stack if s.kind == "global"]
+    assert len(sl) == g["num_layers_sliding"] and len(gl) == g["num_layers_full"]
+    assert [i for i, s in enumerate(stack) if s.kind == "global"] == g["full_layer_indices"]
+    per_tok = lambda specs, twice: sum(accounting.kv_bytes_per_position(s, count_shared_twice=twice)
+                                       for s in specs)
+    assert per_tok(sl, True) == g["sliding_bytes_per_token"]
+    assert per_tok(gl, True) == g["full_bytes_per_token"]
+    assert per_tok(stack, True) == g["total_bytes_per_token"]
+    # K = V read once: the full layers' term halves.
+    assert per_tok(stack, False) == g["sliding_bytes_per_token"] + g["full_bytes_per_token"] // 2
