@@ -5,13 +5,6 @@ ABI declared in ``include/gdattn.h``).  ``binding`` marshals arguments to it;
 nothing here computes attention.  Importing the package does not load the
 library; the first call does, and raises if it has not been built.
 """
-from . import accounting  # noqa: F401
+from . import accounting, binding  # noqa: F401
 
 __all__ = ["accounting", "binding"]
-
-
-def __getattr__(name):
-    if name == "binding":
-        from . import binding
-        return binding
-    raise AttributeError(name)

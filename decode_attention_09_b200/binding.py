@@ -1,0 +1,192 @@
+"""ctypes binding of libgdattn's C ABI (include/gdattn.h).
+
+Argument marshalling only: every step of decode attention runs in the CUDA
+kernels of libgdattn.so.  Torch supplies device memory and streams.  There is no
+fallback: if the library has not been built, loading it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdattn.so")
+
+GDATTN_OK = 0
+GDATTN_ERR_INVALID_ARG = 1
+GDATTN_ERR_UNSUPPORTED = 2
+GDATTN_ERR_MISALIGNED = 3
+GDATTN_ERR_WORKSPACE = 4
+GDATTN_ERR_CUDA = 5
+GDATTN_ERR_DEVICE_TIMEOUT = 6
+GDATTN_ERR_DEVICE_SEQLEN = 7
+
+
+class LayerDesc(ctypes.Structure):
+    """Mirror of gdattn_layer_desc."""
+
+    _fields_ = [
+        ("n_q_heads", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("window", ctypes.c_int32),
+        ("softcap", ctypes.c_float),
+        ("scale", ctypes.c_float),
+        ("kv_shared", ctypes.c_int32),
+        ("cache_capacity", ctypes.c_int32),
+        ("cache_batch_stride", ctypes.c_int64),
+        ("split_ctas", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+
+class GdattnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libgdattn.so.  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libgdattn.so not found at {LIB_PATH}; build it with "
+                "`python decode_attention_09_b200/build.py` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
+        descp = ctypes.POINTER(LayerDesc)
+        L.gdattn_version.restype = i32
+        L.gdattn_status_string.argtypes = [ctypes.c_int]
+        L.gdattn_status_string.restype = ctypes.c_char_p
+        L.gdattn_workspace_size.argtypes = [i32, i32, descp]
+        L.gdattn_workspace_size.restype = sz
+        L.gdattn_plan_splits.argtypes = [i32, i32, descp]
+        L.gdattn_plan_splits.restype = i32
+        L.gdattn_workspace_init.argtypes = [vp, sz, vp]
+        L.gdattn_workspace_init.restype = ctypes.c_int
+        L.gdattn_decode.argtypes = [vp, vp, vp, vp, i32, i32, descp, vp, vp, vp, sz, vp]
+        L.gdattn_decode.restype = ctypes.c_int
+        L.gdattn_combine.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp]
+        L.gdattn_combine.restype = ctypes.c_int
+        L.gdattn_check_device_status.argtypes = [vp, vp]
+        L.gdattn_check_device_status.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().gdattn_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return int(lib().gdattn_version())
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def make_desc(n_q_heads: int, n_kv_heads: int, head_dim: int, window: int, softcap: float,
+              scale: float, kv_shared: bool, cache_capacity: int, cache_batch_stride: int = 0,
+              split_ctas: int = 0) -> LayerDesc:
+    return LayerDesc(int(n_q_heads), int(n_kv_heads), int(head_dim), int(window),
+                     float(softcap), float(scale), 1 if kv_shared else 0, int(cache_capacity),
+                     int(cache_batch_stride), int(split_ctas), 0)
+
+
+def desc_from_spec(spec, split_ctas: int = 0, capacity: Optional[int] = None) -> LayerDesc:
+    """Descriptor for a ``workloads.LayerSpec``."""
+    return make_desc(spec.n_q_heads, spec.n_kv_heads, spec.head_dim, spec.window, spec.softcap,
+                     spec.scale, spec.kv_shared,
+                     capacity if capacity is not None else spec.capacity, 0, split_ctas)
+
+
+def workspace_size(batch: int, max_seqlen: int, desc: LayerDesc) -> int:
+    return int(lib().gdattn_workspace_size(int(batch), int(max_seqlen), ctypes.byref(desc)))
+
+
+def plan_splits(batch: int, max_seqlen: int, desc: LayerDesc) -> int:
+    """CTAs the planner splits the KV range across (0 on invalid arguments)."""
+    return int(lib().gdattn_plan_splits(int(batch), int(max_seqlen), ctypes.byref(desc)))
+
+
+def launches_per_call(batch: int, max_seqlen: int, desc: LayerDesc) -> int:
+    """Kernel launches one gdattn_decode call makes: decode, plus combine when split."""
+    return 1 + (1 if plan_splits(batch, max_seqlen, desc) > 1 else 0)
+
+
+def workspace_init(workspace: torch.Tensor, stream=None) -> None:
+    st = lib().gdattn_workspace_init(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream_handle(stream))
+    if st != GDATTN_OK:
+        raise GdattnError(st, "gdattn_workspace_init")
+
+
+def alloc_workspace(batch: int, max_seqlen: int, desc: LayerDesc, device="cuda",
+                    stream=None) -> torch.Tensor:
+    n = workspace_size(batch, max_seqlen, desc)
+    if n == 0:
+        raise GdattnError(GDATTN_ERR_INVALID_ARG, "gdattn_workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    workspace_init(ws, stream)
+    return ws
+
+
+def decode_raw(q, k, v, seqlens, batch, max_seqlen, desc, out, lse, workspace, workspace_bytes,
+               stream) -> int:
+    """gdattn_decode on raw addresses (ints); returns the status code."""
+    return int(lib().gdattn_decode(q, k, v, seqlens, int(batch), int(max_seqlen),
+                                   ctypes.byref(desc), out, lse, workspace,
+                                   int(workspace_bytes), stream))
+
+
+def decode(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor], seqlens: torch.Tensor,
+           desc: LayerDesc, max_seqlen: int, out: Optional[torch.Tensor] = None,
+           lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+           stream=None, want_lse: bool = True):
+    """One decode-attention layer through gdattn_decode.  Returns (out, lse)."""
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, max_seqlen, desc, q.device, stream)
+    st = decode_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(seqlens), B, max_seqlen, desc, _ptr(out),
+                    _ptr(lse), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    if st != GDATTN_OK:
+        raise GdattnError(st, "gdattn_decode")
+    return out, lse
+
+
+def combine(o_partial: torch.Tensor, lse_partial: torch.Tensor, out: Optional[torch.Tensor] = None,
+            lse: Optional[torch.Tensor] = None, stream=None):
+    """gdattn_combine: o_partial fp32 [B,Hq,S,D], lse_partial fp32 [B,Hq,S]."""
+    B, Hq, S, D = o_partial.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=o_partial.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=o_partial.device)
+    st = lib().gdattn_combine(_ptr(o_partial), _ptr(lse_partial), B, Hq, S, D, _ptr(out), _ptr(lse),
+                              _stream_handle(stream))
+    if st != GDATTN_OK:
+        raise GdattnError(st, "gdattn_combine")
+    return out, lse
+
+
+def check_device_status(workspace: torch.Tensor, stream=None) -> int:
+    return int(lib().gdattn_check_device_status(_ptr(workspace), _stream_handle(stream)))

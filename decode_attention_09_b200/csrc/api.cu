@@ -1,0 +1,473 @@
+// C ABI of libgdattn (declared in include/gdattn.h): argument checks, the split
+// planner, tensor-map encoding and kernel launches.  All compute is in the
+// kernels included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "gdattn.h"
+
+#include "combine.cuh"
+#include "core_decode.cuh"
+#include "tc_decode.cuh"
+
+using namespace gdattn;
+
+namespace {
+
+enum class PathKind { kNone, kCore, kTc };
+
+struct LayerPlan {
+  PathKind kind = PathKind::kNone;
+  int32_t grid = 0;            // CTAs sharing the KV range (P)
+  int32_t units_per_seq = 1;   // query-head groups per sequence
+  int32_t heads_per_unit = 0;
+  int64_t slots = 0;           // partial slots: P + units
+  size_t off_lse = 0, off_o = 0, bytes = 0;
+};
+
+constexpr size_t kStatusBytes = 256;
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+// ----------------------------------------------------------------- kernels
+// Resolve the CUDA-core kernel instantiation for (D, G, Hkv, shared).
+struct CoreKernel {
+  void (*fn)(const CoreParams);
+  int threads;
+  int smem;
+  int tokens_per_stage;
+  int min_blocks;
+};
+
+template <int D, int G, int HKV, bool SH>
+CoreKernel core_kernel_entry() {
+  using Cfg = CoreConfig<D, G, HKV, SH>;
+  return CoreKernel{core_decode_kernel<D, G, HKV, SH>, Cfg::kThreads, Cfg::SMEM, Cfg::T,
+                    Cfg::MIN_BLOCKS};
+}
+
+template <int D, int G, int HKV>
+CoreKernel core_pick_shared(bool shared) {
+  return shared ? core_kernel_entry<D, G, HKV, true>() : core_kernel_entry<D, G, HKV, false>();
+}
+
+template <int D, int G>
+CoreKernel core_pick_hkv(int hkv, bool shared) {
+  switch (hkv) {
+    case 1: return core_pick_shared<D, G, 1>(shared);
+    case 2: return core_pick_shared<D, G, 2>(shared);
+    case 4: return core_pick_shared<D, G, 4>(shared);
+    case 8: return core_pick_shared<D, G, 8>(shared);
+    default: return CoreKernel{nullptr, 0, 0, 0, 0};
+  }
+}
+
+template <int D>
+CoreKernel core_pick_g(int g, int hkv, bool shared) {
+  switch (g) {
+    case 1: return core_pick_hkv<D, 1>(hkv, shared);
+    case 2: return core_pick_hkv<D, 2>(hkv, shared);
+    case 4: return core_pick_hkv<D, 4>(hkv, shared);
+    default: return CoreKernel{nullptr, 0, 0, 0, 0};
+  }
+}
+
+CoreKernel core_pick(int d, int g, int hkv, bool shared) {
+  switch (d) {
+    case 256: return core_pick_g<256>(g, hkv, shared);
+    case 512: return core_pick_g<512>(g, hkv, shared);
+    default: return CoreKernel{nullptr, 0, 0, 0, 0};
+  }
+}
+
+// Blocks of `fn` resident per SM with `smem` dynamic bytes (after opting in to
+// the shared-memory size).  Cached per kernel.
+template <class F>
+int blocks_per_sm(F fn, int threads, int smem) {
+  if (cudaFuncSetAttribute(reinterpret_cast<const void *>(fn),
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return 0;
+  int nb = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, smem) != cudaSuccess) return 0;
+  return nb;
+}
+
+struct KernelInfo {
+  const void *key;
+  int blocks;
+};
+
+// Resident blocks per SM for each kernel instantiation, measured once.
+int cached_blocks_per_sm(const void *key, int threads, int smem,
+                         int (*query)(const void *, int, int)) {
+  static std::mutex mu;
+  static KernelInfo cache[64];
+  static int used = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].key == key) return cache[i].blocks;
+  const int nb = query(key, threads, smem);
+  if (nb > 0 && used < 64) cache[used++] = KernelInfo{key, nb};
+  return nb;
+}
+
+int query_core(const void *fn, int threads, int smem) {
+  return blocks_per_sm(reinterpret_cast<void (*)(const CoreParams)>(const_cast<void *>(fn)),
+                       threads, smem);
+}
+int query_tc(const void *fn, int threads, int smem) {
+  using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const TcParams);
+  return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
+}
+
+// ---------------------------------------------------------------- planning
+gdattn_status check_desc(const gdattn_layer_desc *d) {
+  if (d == nullptr) return GDATTN_ERR_INVALID_ARG;
+  if (d->n_q_heads <= 0 || d->n_kv_heads <= 0 || d->head_dim <= 0 || d->cache_capacity <= 0)
+    return GDATTN_ERR_INVALID_ARG;
+  if (d->n_q_heads % d->n_kv_heads != 0) return GDATTN_ERR_INVALID_ARG;
+  if (d->window < 0 || d->split_ctas < 0 || d->reserved != 0) return GDATTN_ERR_INVALID_ARG;
+  if (!(d->softcap >= 0.f) || !std::isfinite(d->softcap) || !std::isfinite(d->scale))
+    return GDATTN_ERR_INVALID_ARG;
+  if (d->kv_shared != 0 && d->kv_shared != 1) return GDATTN_ERR_INVALID_ARG;
+  const int64_t dense = static_cast<int64_t>(d->cache_capacity) * d->n_kv_heads * d->head_dim;
+  if (d->cache_batch_stride != 0 && (d->cache_batch_stride < dense || d->cache_batch_stride % 8 != 0))
+    return GDATTN_ERR_INVALID_ARG;
+  return GDATTN_OK;
+}
+
+PathKind choose_path(const gdattn_layer_desc *d) {
+  const int g = d->n_q_heads / d->n_kv_heads;
+  if (g == 16 && d->head_dim == 512 && d->kv_shared == 1) return PathKind::kTc;
+  if ((d->head_dim == 256 || d->head_dim == 512) && (g == 1 || g == 2 || g == 4) &&
+      (d->n_kv_heads == 1 || d->n_kv_heads == 2 || d->n_kv_heads == 4 || d->n_kv_heads == 8))
+    return PathKind::kCore;
+  return PathKind::kNone;
+}
+
+gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *d,
+                        LayerPlan &pl) {
+  gdattn_status st = check_desc(d);
+  if (st != GDATTN_OK) return st;
+  if (batch <= 0 || max_seqlen <= 0) return GDATTN_ERR_INVALID_ARG;
+  pl.kind = choose_path(d);
+  if (pl.kind == PathKind::kNone) return GDATTN_ERR_UNSUPPORTED;
+  const int nsm = sm_count();
+  if (nsm <= 0) return GDATTN_ERR_CUDA;
+  int per_sm = 1, min_tokens = 64;
+  if (pl.kind == PathKind::kCore) {
+    const CoreKernel ck = core_pick(d->head_dim, d->n_q_heads / d->n_kv_heads, d->n_kv_heads,
+                                    d->kv_shared != 0);
+    if (ck.fn == nullptr) return GDATTN_ERR_UNSUPPORTED;
+    per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(ck.fn), ck.threads, ck.smem,
+                                  query_core);
+    min_tokens = 4 * ck.tokens_per_stage;
+    pl.units_per_seq = 1;
+    pl.heads_per_unit = d->n_q_heads;
+  } else {
+    per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_kernel),
+                                  TcConfig::kThreads, TcConfig::SMEM, query_tc);
+    min_tokens = 2 * TcConfig::TILE;
+    pl.units_per_seq = d->n_kv_heads;
+    pl.heads_per_unit = 16;
+  }
+  if (per_sm <= 0) return GDATTN_ERR_CUDA;
+  int64_t per_unit = max_seqlen;
+  if (d->window > 0 && d->window < per_unit) per_unit = d->window;
+  if (d->cache_capacity < per_unit) per_unit = d->cache_capacity;
+  const int64_t units = static_cast<int64_t>(batch) * pl.units_per_seq;
+  const int64_t total = units * per_unit;
+  int64_t grid = (total + min_tokens - 1) / min_tokens;
+  const int64_t cap = static_cast<int64_t>(nsm) * per_sm;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  if (d->split_ctas > 0) grid = d->split_ctas;
+  if (grid > 65535) return GDATTN_ERR_INVALID_ARG;
+  pl.grid = static_cast<int32_t>(grid);
+  pl.slots = grid + units;
+  pl.off_lse = kStatusBytes;
+  pl.off_o = align256(pl.off_lse + static_cast<size_t>(pl.slots) * pl.heads_per_unit * 4);
+  pl.bytes = align256(pl.off_o + static_cast<size_t>(pl.slots) * pl.heads_per_unit * d->head_dim * 4);
+  return GDATTN_OK;
+}
+
+// --------------------------------------------------------------- launching
+cudaLaunchConfig_t launch_config(dim3 grid, int threads, int smem, cudaStream_t stream,
+                                 cudaLaunchAttribute *attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  // Programmatic dependent launch: the kernel may start while its predecessor
+  // drains; every kernel here waits (griddepcontrol.wait) before touching memory.
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+gdattn_status launch_combine_internal(const LayerPlan &pl, const Geometry &geo, const float *ws_lse,
+                                      const float *ws_o, const gdattn_layer_desc *d, void *out,
+                                      float *lse, cudaStream_t stream) {
+  CombineParams cp = {};
+  cp.parts_o = ws_o;
+  cp.parts_lse = ws_lse;
+  cp.out = static_cast<uint16_t *>(out);
+  cp.lse = lse;
+  cp.n_q_heads = d->n_q_heads;
+  cp.head_dim = d->head_dim;
+  cp.geo = geo;
+  cp.heads_per_unit = pl.heads_per_unit;
+  cp.n_splits = 0;
+  const int smem = static_cast<int>(pl.grid) * 4 + 16;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg =
+      launch_config(dim3(static_cast<unsigned>(geo.batch * pl.units_per_seq),
+                         static_cast<unsigned>(pl.heads_per_unit)),
+                    kCombineThreads, smem, stream, attr);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(combine_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return GDATTN_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, combine_kernel<true>, cp) == cudaSuccess ? GDATTN_OK
+                                                                            : GDATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+// ===================================================================== ABI
+extern "C" {
+
+int32_t gdattn_version(void) { return GDATTN_VERSION; }
+
+const char *gdattn_status_string(gdattn_status s) {
+  switch (s) {
+    case GDATTN_OK: return "GDATTN_OK";
+    case GDATTN_ERR_INVALID_ARG: return "GDATTN_ERR_INVALID_ARG";
+    case GDATTN_ERR_UNSUPPORTED: return "GDATTN_ERR_UNSUPPORTED";
+    case GDATTN_ERR_MISALIGNED: return "GDATTN_ERR_MISALIGNED";
+    case GDATTN_ERR_WORKSPACE: return "GDATTN_ERR_WORKSPACE";
+    case GDATTN_ERR_CUDA: return "GDATTN_ERR_CUDA";
+    case GDATTN_ERR_DEVICE_TIMEOUT: return "GDATTN_ERR_DEVICE_TIMEOUT";
+    case GDATTN_ERR_DEVICE_SEQLEN: return "GDATTN_ERR_DEVICE_SEQLEN";
+  }
+  return "GDATTN_UNKNOWN_STATUS";
+}
+
+size_t gdattn_workspace_size(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc) {
+  LayerPlan pl;
+  if (make_plan(batch, max_seqlen, desc, pl) != GDATTN_OK) return 0;
+  return pl.bytes;
+}
+
+int32_t gdattn_plan_splits(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc) {
+  LayerPlan pl;
+  if (make_plan(batch, max_seqlen, desc, pl) != GDATTN_OK) return 0;
+  return pl.grid;
+}
+
+gdattn_status gdattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
+  if (workspace == nullptr || workspace_bytes < kStatusBytes) return GDATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GDATTN_ERR_MISALIGNED;
+  return cudaMemsetAsync(workspace, 0, kStatusBytes, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? GDATTN_OK
+             : GDATTN_ERR_CUDA;
+}
+
+gdattn_status gdattn_decode(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *seqlens, int32_t batch, int32_t max_seqlen,
+                            const gdattn_layer_desc *desc, void *out, float *lse,
+                            void *workspace, size_t workspace_bytes, void *stream_) {
+  // Host-only checks first: nothing below touches CUDA until they pass.
+  if (q == nullptr || k_cache == nullptr || seqlens == nullptr || out == nullptr || desc == nullptr)
+    return GDATTN_ERR_INVALID_ARG;
+  gdattn_status st = check_desc(desc);
+  if (st != GDATTN_OK) return st;
+  if ((desc->kv_shared == 1) != (v_cache == nullptr)) return GDATTN_ERR_INVALID_ARG;
+  if (batch <= 0 || max_seqlen <= 0) return GDATTN_ERR_INVALID_ARG;
+  if (choose_path(desc) == PathKind::kNone) return GDATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || (v_cache && !aligned16(v_cache)) ||
+      !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return GDATTN_ERR_MISALIGNED;
+  if (workspace == nullptr) return GDATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GDATTN_ERR_MISALIGNED;
+  LayerPlan pl;
+  st = make_plan(batch, max_seqlen, desc, pl);
+  if (st != GDATTN_OK) return st;
+  if (workspace_bytes < pl.bytes) return GDATTN_ERR_WORKSPACE;
+
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+  float *ws_lse = reinterpret_cast<float *>(ws + pl.off_lse);
+  float *ws_o = reinterpret_cast<float *>(ws + pl.off_o);
+  const int32_t D = desc->head_dim;
+  const int32_t Hkv = desc->n_kv_heads;
+  const int64_t bstride = desc->cache_batch_stride != 0
+                              ? desc->cache_batch_stride
+                              : static_cast<int64_t>(desc->cache_capacity) * Hkv * D;
+  const float log2e = 1.4426950408889634f;
+  const float qscale = desc->softcap > 0.f ? desc->scale / desc->softcap : desc->scale * log2e;
+  const float post = desc->softcap > 0.f ? desc->softcap * log2e : 0.f;
+
+  Geometry geo;
+  geo.seqlens = seqlens;
+  geo.batch = batch;
+  geo.units_per_seq = pl.units_per_seq;
+  geo.window = desc->window;
+  geo.capacity = desc->cache_capacity;
+  geo.nchunks = pl.grid;
+
+  cudaLaunchAttribute attr[1];
+  if (pl.kind == PathKind::kCore) {
+    const CoreKernel ck = core_pick(D, desc->n_q_heads / Hkv, Hkv, desc->kv_shared != 0);
+    CoreParams cp;
+    cp.q = static_cast<const uint16_t *>(q);
+    cp.k = static_cast<const uint16_t *>(k_cache);
+    cp.v = static_cast<const uint16_t *>(v_cache ? v_cache : k_cache);
+    cp.batch_stride = bstride;
+    cp.out = static_cast<uint16_t *>(out);
+    cp.lse = lse;
+    cp.ws_o = ws_o;
+    cp.ws_lse = ws_lse;
+    cp.status = status;
+    cp.geo = geo;
+    cp.n_q_heads = desc->n_q_heads;
+    cp.qscale = qscale;
+    cp.post = post;
+    cudaLaunchConfig_t cfg = launch_config(dim3(pl.grid), ck.threads, ck.smem, stream, attr);
+    if (cudaLaunchKernelEx(&cfg, ck.fn, cp) != cudaSuccess) return GDATTN_ERR_CUDA;
+  } else {
+    EncodeTiledFn enc = encode_tiled();
+    if (enc == nullptr) return GDATTN_ERR_CUDA;
+    CUtensorMap kmap, qmap;
+    {
+      const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv),
+                                  static_cast<cuuint64_t>(desc->cache_capacity),
+                                  static_cast<cuuint64_t>(batch)};
+      const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2,
+                                     static_cast<cuuint64_t>(Hkv) * D * 2,
+                                     static_cast<cuuint64_t>(bstride) * 2};
+      const cuuint32_t box[4] = {64, 1, TcConfig::TILE, 1};
+      const cuuint32_t estr[4] = {1, 1, 1, 1};
+      if (enc(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(k_cache), dims,
+              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return GDATTN_ERR_CUDA;
+    }
+    {
+      const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D),
+                                  static_cast<cuuint64_t>(batch) * desc->n_q_heads};
+      const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+      const cuuint32_t box[2] = {64, 16};
+      const cuuint32_t estr[2] = {1, 1};
+      if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(q), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return GDATTN_ERR_CUDA;
+    }
+    TcParams tp;
+    tp.q = static_cast<const uint16_t *>(q);
+    tp.out = static_cast<uint16_t *>(out);
+    tp.lse = lse;
+    tp.ws_o = ws_o;
+    tp.ws_lse = ws_lse;
+    tp.status = status;
+    tp.geo = geo;
+    tp.n_q_heads = desc->n_q_heads;
+    tp.qscale = qscale;
+    tp.post = post;
+    cudaLaunchConfig_t cfg =
+        launch_config(dim3(pl.grid), TcConfig::kThreads, TcConfig::SMEM, stream, attr);
+    if (cudaLaunchKernelEx(&cfg, tc_decode_kernel, kmap, qmap, tp) != cudaSuccess)
+      return GDATTN_ERR_CUDA;
+  }
+  if (pl.grid > 1)
+    return launch_combine_internal(pl, geo, ws_lse, ws_o, desc, out, lse, stream);
+  return GDATTN_OK;
+}
+
+gdattn_status gdattn_combine(const float *o_partial, const float *lse_partial, int32_t batch,
+                             int32_t n_q_heads, int32_t n_splits, int32_t head_dim, void *out,
+                             float *lse, void *stream) {
+  if (o_partial == nullptr || lse_partial == nullptr || out == nullptr)
+    return GDATTN_ERR_INVALID_ARG;
+  if (batch <= 0 || n_q_heads <= 0 || n_splits <= 0 || head_dim <= 0 || head_dim % 4 != 0 ||
+      head_dim > 1024 || n_splits > 8192 || batch > 65535 || n_q_heads > 65535)
+    return GDATTN_ERR_INVALID_ARG;
+  if (!aligned16(o_partial) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(lse_partial) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return GDATTN_ERR_MISALIGNED;
+  if ((head_dim % 8) != 0 && (reinterpret_cast<uintptr_t>(out) & 7u)) return GDATTN_ERR_MISALIGNED;
+  CombineParams cp = {};
+  cp.parts_o = o_partial;
+  cp.parts_lse = lse_partial;
+  cp.out = static_cast<uint16_t *>(out);
+  cp.lse = lse;
+  cp.n_q_heads = n_q_heads;
+  cp.head_dim = head_dim;
+  cp.heads_per_unit = 0;
+  cp.n_splits = n_splits;
+  const int smem = n_splits * 4 + 16;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(combine_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return GDATTN_ERR_CUDA;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = launch_config(dim3(batch, n_q_heads), kCombineThreads, smem,
+                                         static_cast<cudaStream_t>(stream), attr);
+  return cudaLaunchKernelEx(&cfg, combine_kernel<false>, cp) == cudaSuccess ? GDATTN_OK
+                                                                             : GDATTN_ERR_CUDA;
+}
+
+gdattn_status gdattn_check_device_status(void *workspace, void *stream_) {
+  if (workspace == nullptr) return GDATTN_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaMemsetAsync(workspace, 0, sizeof(word), stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return GDATTN_ERR_CUDA;
+  if (word & kStatusTimeout) return GDATTN_ERR_DEVICE_TIMEOUT;
+  if (word & kStatusSeqlen) return GDATTN_ERR_DEVICE_SEQLEN;
+  return GDATTN_OK;
+}
+
+}  // extern "C"

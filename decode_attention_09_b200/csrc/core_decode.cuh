@@ -1,0 +1,412 @@
+// Split-KV decode attention on CUDA cores, for small GQA groups (G = Hq/Hkv in
+// {1, 2, 4}) such as Gemma-4 sliding layers (16 q heads over 8 KV heads, G = 2).
+//
+// With G <= 4 a KV row feeds at most 4 query heads, about 1-2 flop per byte, so
+// the products are not a dense contraction and run as fp32 FMAs; the kernel is
+// bound by HBM bandwidth.
+//
+// CTA = 8 compute warps + 1 producer warp.  The producer streams whole token
+// rows (all Hkv heads, contiguous in the token-major cache) with 1-D bulk
+// copies into an NSTAGE-deep shared-memory ring, one mbarrier pair per stage.
+// Compute warp w owns KV head w % Hkv and, when Hkv < 8, every (8/Hkv)-th token
+// of a stage.  A lane holds D/32 consecutive-by-16-bytes elements of q, of the
+// output accumulator and of each K/V row it reads, so shared-memory reads are
+// 16-byte vectors with no bank conflicts.
+//
+// Per stage a warp handles TPW = 4 tokens: it forms TPW*G partial dot products
+// per lane, reduce-scatters them across the warp (each lane ends with one full
+// score), applies scale / soft-cap, updates the running max and sum of the
+// online softmax, broadcasts the TPW*G weights and accumulates P.V.
+#pragma once
+
+#include <cstdint>
+
+#include "partition.cuh"
+#include "ptx.cuh"
+
+namespace gdattn {
+
+struct CoreParams {
+  const uint16_t *q;      // [B, Hq, D]
+  const uint16_t *k;      // cache
+  const uint16_t *v;      // cache (== k when shared)
+  int64_t batch_stride;   // elements
+  uint16_t *out;          // [B, Hq, D]
+  float *lse;             // [B, Hq] or null
+  float *ws_o;            // partial outputs [slots][Hq][D]
+  float *ws_lse;          // partial lse [slots][Hq]
+  uint32_t *status;       // device status word
+  Geometry geo;           // units_per_seq == 1
+  int32_t n_q_heads;
+  float qscale;           // folded into q: scale*log2(e), or scale/softcap
+  float post;             // softcap*log2(e), or 0 when soft-cap is off
+};
+
+template <int D, int G, int HKV, bool SHARED>
+struct CoreConfig {
+  static constexpr int kComputeWarps = 8;
+  static constexpr int kThreads = (kComputeWarps + 1) * 32;
+  static constexpr int TS = kComputeWarps / HKV;      // warps sharing one KV head
+  static constexpr int TPW = 4;                       // tokens per warp per stage
+  static constexpr int T = TS * TPW;                  // tokens per stage
+  static constexpr int EPL = D / 32;                  // elements per lane
+  static constexpr int CH = EPL / 8;                  // 16-byte chunks per lane
+  static constexpr int ROWB = HKV * D * 2;            // bytes of one token row (one tensor)
+  static constexpr int NT = SHARED ? 1 : 2;
+  static constexpr int STAGEB = T * ROWB * NT;
+  static constexpr int NSTAGE = (98304 / STAGEB) < 2 ? 2 : (98304 / STAGEB);
+  static constexpr int NV = TPW * G;                  // scores per warp per stage
+  static constexpr int LOGNV = NV == 4 ? 2 : (NV == 8 ? 3 : 4);
+  static constexpr int LOGG = G == 1 ? 0 : (G == 2 ? 1 : 2);
+  static constexpr int MHDR = 8;                      // per-warp merge header (m[G], l[G])
+  static constexpr int MSTRIDE = MHDR + G * D;        // floats per warp, 16-byte multiple
+  static constexpr int MERGEB = TS > 1 ? kComputeWarps * MSTRIDE * 4 : 0;
+  static constexpr int SMEM = NSTAGE * STAGEB + 2 * NSTAGE * 8 + 128 + MERGEB + 1024;
+  static constexpr int MIN_BLOCKS = (EPL * G <= 32 && SMEM <= 110 * 1024) ? 2 : 1;
+  static_assert(HKV == 1 || HKV == 2 || HKV == 4 || HKV == 8, "HKV");
+  static_assert(G == 1 || G == 2 || G == 4, "G");
+  static_assert(D == 256 || D == 512, "D");
+};
+
+__device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
+
+template <int D, int G, int HKV, bool SHARED>
+__global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads,
+                                  CoreConfig<D, G, HKV, SHARED>::MIN_BLOCKS)
+    core_decode_kernel(const CoreParams p) {
+  using Cfg = CoreConfig<D, G, HKV, SHARED>;
+  constexpr int NSTAGE = Cfg::NSTAGE, T = Cfg::T, EPL = Cfg::EPL, CH = Cfg::CH;
+  constexpr int ROWB = Cfg::ROWB, NV = Cfg::NV, LOGNV = Cfg::LOGNV;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint8_t *stage_k = smem;
+  uint8_t *stage_v = smem + NSTAGE * T * ROWB;  // unused when SHARED
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + NSTAGE * Cfg::STAGEB);
+  uint64_t *empty = full + NSTAGE;
+  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(empty + NSTAGE);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(plan + 1);
+  float *merge = reinterpret_cast<float *>(smem + NSTAGE * Cfg::STAGEB + 2 * NSTAGE * 8 + 128);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], Cfg::kComputeWarps);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  grid_launch_dependents();
+  grid_dependency_wait();  // inputs / workspace may come from the previous kernel
+  if (warp == 0) plan_chunk(p.geo, c, plan);
+  __syncthreads();
+
+  if (c == 0 && warp == 0 && plan->bad) {
+    if (lane == 0) atomicOr(p.status, kStatusSeqlen);
+    // Sequences with nothing to attend get out = 0 and lse = -inf.
+    for (int32_t b = 0; b < p.geo.batch; ++b) {
+      bool dummy = false;
+      if (attended_count(__ldg(p.geo.seqlens + b), p.geo.window, p.geo.capacity, dummy) != 0)
+        continue;
+      for (int i = lane; i < p.n_q_heads * D; i += 32)
+        p.out[static_cast<int64_t>(b) * p.n_q_heads * D + i] = 0;
+      if (p.lse != nullptr)
+        for (int i = lane; i < p.n_q_heads; i += 32)
+          p.lse[static_cast<int64_t>(b) * p.n_q_heads + i] = -INFINITY;
+    }
+  }
+
+  const int32_t C = p.geo.capacity;
+
+  if (warp == Cfg::kComputeWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol = l2_evict_first_policy();
+      uint32_t fills = 0;
+      bool ok = true;
+      SegmentIter it;
+      it.init(p.geo, *plan);
+      Segment s;
+      while (ok && it.next(s)) {
+        const SlotRuns runs = segment_runs(s, C);
+        for (int r = 0; ok && r < runs.count; ++r) {
+          for (int32_t t0 = 0; t0 < runs.len(r); t0 += T) {
+            const int ntok = min(T, runs.len(r) - t0);
+            const int st = fills % NSTAGE;
+            if (fills >= NSTAGE &&
+                !mbar_wait(&empty[st], ((fills / NSTAGE) - 1) & 1, abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            const uint32_t bytes = static_cast<uint32_t>(ntok * ROWB);
+            const int64_t off = static_cast<int64_t>(s.b) * p.batch_stride +
+                                static_cast<int64_t>(runs.start(r) + t0) * (HKV * D);
+            mbar_arrive_expect_tx(&full[st], bytes * Cfg::NT);
+            bulk_g2s(stage_k + st * T * ROWB, p.k + off, bytes, &full[st], pol);
+            if (!SHARED) bulk_g2s(stage_v + st * T * ROWB, p.v + off, bytes, &full[st], pol);
+            ++fills;
+          }
+        }
+      }
+      // Never leave with copies in flight into this CTA's shared memory.
+      for (uint32_t f = fills > NSTAGE ? fills - NSTAGE : 0; f < fills; ++f) {
+        volatile int no_abort = 0;
+        mbar_wait(&full[f % NSTAGE], (f / NSTAGE) & 1, &no_abort, p.status);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- compute
+    const int kvh = warp % HKV;
+    const int tp = warp / HKV;
+    float q[G][EPL];
+    float o[G][EPL];
+    float m[G], l[G];
+    uint32_t fills = 0;
+    bool ok = true;
+    SegmentIter it;
+    it.init(p.geo, *plan);
+    Segment s;
+    while (it.next(s)) {
+      // Load this sequence's query rows for the warp's heads, pre-scaled.
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const uint16_t *qr = p.q + (static_cast<int64_t>(s.b) * p.n_q_heads + kvh * G + g) * D;
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+          const uint4 w = __ldg(reinterpret_cast<const uint4 *>(qr + 256 * j + 8 * lane));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            q[g][8 * j + 2 * e] = bf16lo(ww[e]) * p.qscale;
+            q[g][8 * j + 2 * e + 1] = bf16hi(ww[e]) * p.qscale;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) o[g][e] = 0.f;
+        m[g] = -INFINITY;
+        l[g] = 0.f;
+      }
+
+      const SlotRuns runs = segment_runs(s, C);
+      for (int r = 0; r < runs.count; ++r) {
+        for (int32_t t0 = 0; t0 < runs.len(r); t0 += T) {
+          const int ntok = min(T, runs.len(r) - t0);
+          const int st = fills % NSTAGE;
+          if (ok && !mbar_wait(&full[st], (fills / NSTAGE) & 1, abort_flag, p.status)) ok = false;
+          ok = __all_sync(0xffffffffu, ok);  // warp-uniform before warp-collective code
+          ++fills;
+          if (!ok) continue;
+          const uint8_t *kst = stage_k + st * T * ROWB + kvh * D * 2;
+          const uint8_t *vst = (SHARED ? stage_k : stage_v) + st * T * ROWB + kvh * D * 2;
+
+          // Partial dot products: part[i*G + g] over this lane's elements.
+          float part[NV];
+#pragma unroll
+          for (int i = 0; i < Cfg::TPW; ++i) {
+            const int t = tp + Cfg::TS * i;
+#pragma unroll
+            for (int g = 0; g < G; ++g) part[i * G + g] = 0.f;
+            if (t < ntok) {
+#pragma unroll
+              for (int j = 0; j < CH; ++j) {
+                const uint4 w =
+                    *reinterpret_cast<const uint4 *>(kst + t * ROWB + 512 * j + 16 * lane);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float k0 = bf16lo(ww[e]), k1 = bf16hi(ww[e]);
+#pragma unroll
+                  for (int g = 0; g < G; ++g) {
+                    part[i * G + g] = fmaf(q[g][8 * j + 2 * e], k0, part[i * G + g]);
+                    part[i * G + g] = fmaf(q[g][8 * j + 2 * e + 1], k1, part[i * G + g]);
+                  }
+                }
+              }
+            }
+          }
+          // Reduce-scatter: after log2(NV) halving steps lane holds one score,
+          // index bits k <-> lane bit (5 - LOGNV + k); the rest of the lanes
+          // that share an index sum up with the remaining xor steps.
+          {
+            int cnt = NV;
+#pragma unroll
+            for (int lev = 0; lev < LOGNV; ++lev) {
+              const int off = 16 >> lev;
+              const bool upper = (lane & off) != 0;
+              const int half = cnt >> 1;
+#pragma unroll
+              for (int i2 = 0; i2 < NV / 2; ++i2) {
+                if (i2 < half) {
+                  const float send = upper ? part[i2] : part[i2 + half];
+                  const float keep = upper ? part[i2 + half] : part[i2];
+                  part[i2] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                }
+              }
+              cnt = half;
+            }
+#pragma unroll
+            for (int off = 16 >> LOGNV; off > 0; off >>= 1)
+              part[0] += __shfl_xor_sync(0xffffffffu, part[0], off);
+          }
+          const int idx = (lane >> (5 - LOGNV)) & (NV - 1);
+          const int my_g = idx & (G - 1);
+          const int my_t = tp + Cfg::TS * (idx >> Cfg::LOGG);
+          float sc = part[0];
+          if (p.post != 0.f) sc = p.post * tanhf(sc);
+          if (my_t >= ntok) sc = -INFINITY;
+          // Max over this stage's tokens for the lane's head (token bits are
+          // the top lane bits: offsets 16, 8 for TPW = 4).
+          float tmax = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 16));
+          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+          float mnew[G], alpha[G];
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float mx = __shfl_sync(0xffffffffu, tmax, g << (5 - LOGNV));
+            mnew[g] = fmaxf(m[g], mx);
+            alpha[g] = (mnew[g] == -INFINITY) ? 1.f : fast_exp2(m[g] - mnew[g]);
+          }
+          float mine_m = mnew[0];
+#pragma unroll
+          for (int g = 1; g < G; ++g)
+            if (my_g == g) mine_m = mnew[g];
+          const float pe = (sc == -INFINITY) ? 0.f : fast_exp2(sc - mine_m);
+          float psum = pe + __shfl_xor_sync(0xffffffffu, pe, 16);
+          psum += __shfl_xor_sync(0xffffffffu, psum, 8);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float ps = __shfl_sync(0xffffffffu, psum, g << (5 - LOGNV));
+            l[g] = l[g] * alpha[g] + ps;
+            m[g] = mnew[g];
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) o[g][e] *= alpha[g];
+          }
+          // P.V for this warp's tokens.
+#pragma unroll
+          for (int i = 0; i < Cfg::TPW; ++i) {
+            const int t = tp + Cfg::TS * i;
+            float pw[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+              pw[g] = __shfl_sync(0xffffffffu, pe, (i * G + g) << (5 - LOGNV));
+            if (t < ntok) {
+#pragma unroll
+              for (int j = 0; j < CH; ++j) {
+                const uint4 w =
+                    *reinterpret_cast<const uint4 *>(vst + t * ROWB + 512 * j + 16 * lane);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float v0 = bf16lo(ww[e]), v1 = bf16hi(ww[e]);
+#pragma unroll
+                  for (int g = 0; g < G; ++g) {
+                    o[g][8 * j + 2 * e] = fmaf(pw[g], v0, o[g][8 * j + 2 * e]);
+                    o[g][8 * j + 2 * e + 1] = fmaf(pw[g], v1, o[g][8 * j + 2 * e + 1]);
+                  }
+                }
+              }
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[st]);
+        }
+      }
+
+      // ---------------------------------------------------- segment epilogue
+      if (Cfg::TS > 1) {
+        // Merge the TS warps that share a KV head through shared memory.
+        float *mine = merge + warp * Cfg::MSTRIDE;
+        if (lane == 0) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            mine[g] = m[g];
+            mine[4 + g] = l[g];
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int j = 0; j < CH; ++j) {
+            float4 *dst = reinterpret_cast<float4 *>(mine + Cfg::MHDR + g * D + 256 * j + 8 * lane);
+            dst[0] = make_float4(o[g][8 * j], o[g][8 * j + 1], o[g][8 * j + 2], o[g][8 * j + 3]);
+            dst[1] =
+                make_float4(o[g][8 * j + 4], o[g][8 * j + 5], o[g][8 * j + 6], o[g][8 * j + 7]);
+          }
+        named_bar_sync(1, Cfg::kComputeWarps * 32);
+        if (tp == 0) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            float M = -INFINITY;
+            for (int k = 0; k < Cfg::TS; ++k) M = fmaxf(M, merge[(kvh + HKV * k) * Cfg::MSTRIDE + g]);
+            float Ls = 0.f;
+            float wk[Cfg::TS];
+#pragma unroll
+            for (int k = 0; k < Cfg::TS; ++k) {
+              const float *src = merge + (kvh + HKV * k) * Cfg::MSTRIDE;
+              wk[k] = (src[g] == -INFINITY) ? 0.f : fast_exp2(src[g] - M);
+              Ls += src[4 + g] * wk[k];
+            }
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) o[g][e] = 0.f;
+#pragma unroll
+            for (int k = 0; k < Cfg::TS; ++k) {
+              const float *src = merge + (kvh + HKV * k) * Cfg::MSTRIDE + Cfg::MHDR + g * D;
+#pragma unroll
+              for (int j = 0; j < CH; ++j)
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  o[g][8 * j + e] = fmaf(wk[k], src[256 * j + 8 * lane + e], o[g][8 * j + e]);
+            }
+            m[g] = M;
+            l[g] = Ls;
+          }
+        }
+        named_bar_sync(1, Cfg::kComputeWarps * 32);
+      }
+      if (tp == 0 && ok) {
+        int32_t cf, cl;
+        unit_chunks(s.unit_start, s.n, plan->chunk, cf, cl);
+        const bool single = (cf == cl);
+        const int64_t slot = static_cast<int64_t>(c) + s.unit;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const int h = kvh * G + g;
+          const float inv = 1.f / l[g];
+          const float lse_v = (m[g] + log2f(l[g])) * 0.69314718055994530942f;
+          if (single) {
+            uint16_t *dst = p.out + (static_cast<int64_t>(s.b) * p.n_q_heads + h) * D;
+#pragma unroll
+            for (int j = 0; j < CH; ++j) {
+              uint4 w;
+              w.x = pack_bf16x2(o[g][8 * j] * inv, o[g][8 * j + 1] * inv);
+              w.y = pack_bf16x2(o[g][8 * j + 2] * inv, o[g][8 * j + 3] * inv);
+              w.z = pack_bf16x2(o[g][8 * j + 4] * inv, o[g][8 * j + 5] * inv);
+              w.w = pack_bf16x2(o[g][8 * j + 6] * inv, o[g][8 * j + 7] * inv);
+              *reinterpret_cast<uint4 *>(dst + 256 * j + 8 * lane) = w;
+            }
+            if (lane == 0 && p.lse != nullptr)
+              p.lse[static_cast<int64_t>(s.b) * p.n_q_heads + h] = lse_v;
+          } else {
+            float *dst = p.ws_o + (slot * p.n_q_heads + h) * D;
+#pragma unroll
+            for (int j = 0; j < CH; ++j) {
+              float4 *d4 = reinterpret_cast<float4 *>(dst + 256 * j + 8 * lane);
+              d4[0] = make_float4(o[g][8 * j] * inv, o[g][8 * j + 1] * inv, o[g][8 * j + 2] * inv,
+                                  o[g][8 * j + 3] * inv);
+              d4[1] = make_float4(o[g][8 * j + 4] * inv, o[g][8 * j + 5] * inv,
+                                  o[g][8 * j + 6] * inv, o[g][8 * j + 7] * inv);
+            }
+            if (lane == 0) p.ws_lse[slot * p.n_q_heads + h] = lse_v;
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
+}  // namespace gdattn

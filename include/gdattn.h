@@ -1,0 +1,165 @@
+/*
+ * libgdattn -- single-token (decode) attention over a per-layer KV cache for
+ * Gemma-4-style hybrid stacks, split along the KV sequence, on NVIDIA B200
+ * (sm_100a).
+ *
+ * What one call computes (one layer, one decode step, every sequence b of the
+ * batch and every query head h):
+ *
+ *   G    = n_q_heads / n_kv_heads; query head h reads KV head kv = h / G
+ *   L    = seqlens[b], the context length with the current token's K/V already
+ *          in the cache
+ *   positions attended: [max(0, L - window), L) when window > 0, else [0, L)
+ *   slot(j) = j mod cache_capacity          (ring buffer for sliding layers)
+ *   x_j  = scale * <q[b,h,:], K[b, slot(j), kv, :]>
+ *   s_j  = softcap * tanh(x_j / softcap)    when softcap > 0, else x_j
+ *   lse[b,h] = log sum_j exp(s_j)           (natural log)
+ *   out[b,h,:] = sum_j exp(s_j - lse[b,h]) * V'[b, slot(j), kv, :],
+ *                V' = K when kv_shared, else V
+ *
+ * Sources: sliding layers read exactly the last w positions from a rotating
+ * cache and full layers read the whole context ("Gemma 4 12B" record, KV
+ * GEOMETRY and serviceability join, item 6); sliding layers use head_dim 256
+ * with 8 KV heads, full layers a larger head_dim (512) with one KV head and key
+ * == value ("Gemma4-26B-A4B ... NO-GO", section 3 Break 4; "Gemma 4 12B" KV
+ * GEOMETRY, attention_k_eq_v); attention soft-capping and K = V global attention
+ * ("Gemma support" PR, summary); split decode attention for head sizes 256/512
+ * ("Gemma support" PR, Performance); the split count must match the GPU so
+ * that single-query global layers keep every SM busy ("Gemma 4 12B", item 4).
+ *
+ * Conventions for every entry point:
+ *  - All tensors are caller-owned.  The library allocates no device or host
+ *    memory and keeps no state between calls; calls are thread-safe.
+ *  - Device pointers must be 16-byte aligned and rows are contiguous along the
+ *    head dimension.  bf16 means IEEE bfloat16, stored as 16-bit words.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *    enqueued asynchronously; no call synchronises except
+ *    gdattn_check_device_status.  Decode and combine only enqueue kernels, so they
+ *    can be captured into a CUDA graph.
+ *  - Arguments are checked on the host before anything is enqueued; a failed
+ *    check returns its status and launches nothing.  A launch failure returns
+ *    GDATTN_ERR_CUDA.  Problems only the device can see (a context length that
+ *    needs more slots than the cache has, a pipeline wait that ran out) are
+ *    latched in the workspace status word and read by
+ *    gdattn_check_device_status.
+ */
+#ifndef GDATTN_H_
+#define GDATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDATTN_VERSION 100
+
+typedef enum gdattn_status {
+  GDATTN_OK = 0,
+  GDATTN_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, Hq % Hkv != 0, ... */
+  GDATTN_ERR_UNSUPPORTED = 2,   /* valid but not built: head_dim or GQA group size */
+  GDATTN_ERR_MISALIGNED = 3,    /* a device pointer or stride is not 16-byte aligned */
+  GDATTN_ERR_WORKSPACE = 4,     /* workspace missing or smaller than gdattn_workspace_size */
+  GDATTN_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
+  GDATTN_ERR_DEVICE_TIMEOUT = 6,/* device: a bounded pipeline wait expired (result invalid) */
+  GDATTN_ERR_DEVICE_SEQLEN = 7  /* device: seqlens[b] < 1, or the attended range needs more
+                                   slots than cache_capacity (range clamped, result invalid) */
+} gdattn_status;
+
+/* Geometry and numerics of one attention layer. */
+typedef struct gdattn_layer_desc {
+  int32_t n_q_heads;      /* Hq > 0 */
+  int32_t n_kv_heads;     /* Hkv > 0, Hq % Hkv == 0 */
+  int32_t head_dim;       /* D: 256 or 512 */
+  int32_t window;         /* 0: attend [0, L); w > 0: attend the last w positions [L-w, L) */
+  float softcap;          /* 0: off; > 0: s = softcap * tanh(s / softcap), after the scale */
+  float scale;            /* multiplies q.k (1/sqrt(D) for Gemma-4 geometries) */
+  int32_t kv_shared;      /* 1: K serves as V (attention_k_eq_v); v_cache must be NULL */
+  int32_t cache_capacity; /* C: slots per sequence; position j lives in slot j mod C */
+  int64_t cache_batch_stride; /* elements from sequence b to b+1 in K (and V); 0 = C*Hkv*D;
+                                 otherwise >= C*Hkv*D and a multiple of 8 */
+  int32_t split_ctas;     /* 0: the planner picks how many CTAs share the KV range; > 0
+                             forces that many (tests and tuning) */
+  int32_t reserved;       /* must be 0 */
+} gdattn_layer_desc;
+
+/*
+ * Bytes of device workspace gdattn_decode needs for this layer geometry and
+ * batch on the current CUDA device (partial results of split ranges plus a
+ * 256-byte status word).  max_seqlen is the host's upper bound on seqlens[];
+ * it only steers the split count.  Returns 0 on invalid arguments.
+ */
+size_t gdattn_workspace_size(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc);
+
+/*
+ * Number of CTAs the planner splits this layer's KV range across (the value
+ * gdattn_decode uses for the same arguments on the current device): one decode
+ * kernel launch, plus one LSE-combine launch when the result is above 1.
+ * Returns 0 on invalid arguments.
+ */
+int32_t gdattn_plan_splits(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc);
+
+/*
+ * Zero the workspace's status word.  Call once after allocating a workspace
+ * (or zero the whole buffer yourself); the library keeps it clear afterwards.
+ */
+gdattn_status gdattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Decode attention for one layer (the definition at the top of this file).
+ *
+ *  q        bf16 [batch, Hq, D], device, read only
+ *  k_cache  bf16, device, read only; sequence b at k_cache + b*cache_batch_stride
+ *           elements, laid out [C][Hkv][D] (token-major)
+ *  v_cache  bf16, same layout as k_cache, or NULL when desc->kv_shared == 1
+ *  seqlens  int32 [batch], device: L_b >= 1 and min(L_b, window or L_b) <= C
+ *  batch    > 0;  max_seqlen: host upper bound of seqlens[] (> 0)
+ *  out      bf16 [batch, Hq, D], device, written
+ *  lse      fp32 [batch, Hq], device, written (natural log), or NULL
+ *  workspace / workspace_bytes: device scratch of at least gdattn_workspace_size
+ *           bytes, status word zeroed once by gdattn_workspace_init.  Calls that
+ *           share a workspace must be ordered on one stream.
+ *
+ * Supported: D in {256, 512}; G = Hq / Hkv in {1, 2, 4} with Hkv in {1, 2, 4, 8, 16}
+ * (CUDA-core path), or G == 16 with D == 512 (tensor-core path).  Other
+ * geometries return GDATTN_ERR_UNSUPPORTED.
+ */
+gdattn_status gdattn_decode(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *seqlens, int32_t batch, int32_t max_seqlen,
+                            const gdattn_layer_desc *desc, void *out, float *lse,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Merge n_splits partial results per (sequence, head), each normalised over its
+ * own part of the position range:
+ *   lse = log sum_s exp(lse_s),  out = sum_s exp(lse_s - lse) * o_s.
+ * A part with lse_s = -INFINITY (empty) contributes nothing; if every part is
+ * empty the result is lse = -INFINITY and out = 0.
+ *
+ *  o_partial    fp32 [batch, Hq, n_splits, D], device
+ *  lse_partial  fp32 [batch, Hq, n_splits], device (natural log)
+ *  out          bf16 [batch, Hq, D], device;  lse: fp32 [batch, Hq] or NULL
+ *  head_dim     any multiple of 4 up to 1024; n_splits >= 1
+ */
+gdattn_status gdattn_combine(const float *o_partial, const float *lse_partial, int32_t batch,
+                             int32_t n_q_heads, int32_t n_splits, int32_t head_dim, void *out,
+                             float *lse, void *stream);
+
+/*
+ * Synchronise `stream`, read and clear the workspace status word, and return
+ * the first device-side error latched since the last check (GDATTN_OK if none).
+ */
+gdattn_status gdattn_check_device_status(void *workspace, void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *gdattn_status_string(gdattn_status status);
+
+/* GDATTN_VERSION of the built library. */
+int32_t gdattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDATTN_H_ */

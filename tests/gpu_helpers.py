@@ -1,0 +1,81 @@
+"""Shared helpers for the GPU tests: run one layer through the C ABI and compare
+with the float64 oracle on the very same bf16 inputs."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from decode_attention_09_b200 import binding
+
+OUT_TOL = 8e-3  # max |out_gpu - out_oracle|, bf16 output
+LSE_TOL = 1e-3  # max |lse_gpu - lse_oracle|, fp32
+
+
+def require_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 numbers at |x| (8 significant bits)."""
+    ax = np.maximum(np.abs(x), np.finfo(np.float32).tiny)
+    return np.exp2(np.floor(np.log2(ax)) - 7)
+
+
+class GpuLayer:
+    """Device copies of a layer's inputs plus a workspace."""
+
+    def __init__(self, inp, split_ctas=0, max_seqlen=None, device="cuda"):
+        self.inp = inp
+        self.q = inp.q.to(device)
+        self.k = inp.k.to(device)
+        self.v = inp.v.to(device) if inp.v is not None else None
+        self.seqlens = inp.seqlens.to(device=device, dtype=torch.int32)
+        self.B = inp.q.shape[0]
+        self.max_seqlen = int(max_seqlen or int(inp.seqlens.max()))
+        self.desc = binding.desc_from_spec(inp.spec, split_ctas, capacity=inp.k.shape[1])
+        self.ws = binding.alloc_workspace(self.B, self.max_seqlen, self.desc, device)
+
+    def run(self, check_status=True):
+        out, lse = binding.decode(self.q, self.k, self.v, self.seqlens, self.desc,
+                                  self.max_seqlen, workspace=self.ws)
+        if check_status:
+            st = binding.check_device_status(self.ws)
+            assert st == binding.GDATTN_OK, binding.status_string(st)
+        torch.cuda.synchronize()
+        return out, lse
+
+
+def compare(out_gpu, lse_gpu, out_ref, lse_ref, ulp_floor=False, what=""):
+    """Element-wise parity: |dout| <= 8e-3 (or 1 bf16 ulp of the reference when
+    ``ulp_floor``) and |dlse| <= 1e-3."""
+    og = out_gpu.float().cpu().numpy().astype(np.float64)
+    lg = lse_gpu.float().cpu().numpy().astype(np.float64)
+    assert og.shape == out_ref.shape and lg.shape == lse_ref.shape
+    assert np.all(np.isfinite(og)), f"{what}: non-finite output"
+    tol = OUT_TOL
+    if ulp_floor:
+        tol = np.maximum(OUT_TOL, bf16_ulp(out_ref))
+    err = np.abs(og - out_ref)
+    bad = err > tol
+    assert not bad.any(), (f"{what}: {bad.sum()} outputs off, max |d| = {err.max():.3e} at "
+                           f"{np.unravel_index(err.argmax(), err.shape)}")
+    lerr = np.abs(lg - lse_ref)
+    assert lerr.max() <= LSE_TOL, f"{what}: max |dlse| = {lerr.max():.3e}"
+    return float(err.max()), float(lerr.max())
+
+
+def oracle_for(inp, batch_index=None):
+    """Oracle result for all sequences, or for the listed ones."""
+    orc = oracle.get()
+    s = inp.spec
+    if batch_index is None:
+        return orc.decode(inp.q, inp.k, inp.v, inp.seqlens, s.window, s.softcap, s.scale)
+    idx = torch.as_tensor(batch_index, dtype=torch.long)
+    q = inp.q.index_select(0, idx.to(inp.q.device)).cpu()
+    k = inp.k.index_select(0, idx.to(inp.k.device)).cpu()
+    v = inp.v.index_select(0, idx.to(inp.v.device)).cpu() if inp.v is not None else None
+    sl = inp.seqlens.cpu().index_select(0, idx)
+    return orc.decode(q, k, v, sl, s.window, s.softcap, s.scale)

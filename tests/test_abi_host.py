@@ -1,0 +1,174 @@
+"""The C ABI without a GPU: exports, struct layout and host-side argument checks.
+
+Every call here is rejected by a host check before the library touches CUDA, so
+these run on a machine with no GPU.  Fake device addresses are never
+dereferenced.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from decode_attention_09_b200 import binding
+from decode_attention_09_b200 import build as libbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdattn.h")
+
+A = 0x100000  # a 16-byte-aligned fake device address (never dereferenced)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    libbuild.build()
+    return binding.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(gdattn_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_api():
+    names = declared_functions()
+    for n in ("gdattn_decode", "gdattn_combine", "gdattn_workspace_size", "gdattn_workspace_init",
+              "gdattn_plan_splits",
+              "gdattn_check_device_status", "gdattn_status_string", "gdattn_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], check=True,
+                         capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT\s+(gdattn_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    for n in declared_functions():
+        assert hasattr(lib, n)
+
+
+def test_desc_layout_matches_c(tmp_path):
+    """ctypes mirror of gdattn_layer_desc has the C compiler's size and offsets."""
+    src = tmp_path / "layout.c"
+    fields = [f for f, _ in binding.LayerDesc._fields_]
+    body = "\n".join(f'printf("%zu\\n", offsetof(gdattn_layer_desc, {f}));' for f in fields)
+    src.write_text("#include <stddef.h>\n#include <stdio.h>\n#include \"gdattn.h\"\n"
+                   "int main(void){" + body + 'printf("%zu\\n", sizeof(gdattn_layer_desc));'
+                   "return 0;}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                    str(exe)], check=True)
+    vals = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True,
+                                           text=True).stdout.split()]
+    expect = [getattr(binding.LayerDesc, f).offset for f in fields] + [
+        ctypes.sizeof(binding.LayerDesc)]
+    assert vals == expect
+
+
+def test_version_and_status_strings(lib):
+    assert binding.version() == 100
+    assert binding.status_string(0) == "GDATTN_OK"
+    assert binding.status_string(binding.GDATTN_ERR_DEVICE_SEQLEN) == "GDATTN_ERR_DEVICE_SEQLEN"
+    assert binding.status_string(999) == "GDATTN_UNKNOWN_STATUS"
+
+
+def good_desc(**kw):
+    d = dict(n_q_heads=16, n_kv_heads=8, head_dim=256, window=1024, softcap=0.0,
+             scale=1 / 16, kv_shared=False, cache_capacity=1024)
+    d.update(kw)
+    return binding.make_desc(**d)
+
+
+def call(desc, q=A, k=A, v=A, seqlens=A, batch=1, max_seqlen=8, out=A, lse=A, ws=A, ws_bytes=1 << 20):
+    return binding.decode_raw(q, k, v, seqlens, batch, max_seqlen, desc, out, lse, ws, ws_bytes,
+                              None)
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(q=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(k=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(seqlens=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(out=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(v=None), binding.GDATTN_ERR_INVALID_ARG),  # separate V expected
+    (dict(batch=0), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(max_seqlen=0), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(q=A + 8), binding.GDATTN_ERR_MISALIGNED),
+    (dict(k=A + 2), binding.GDATTN_ERR_MISALIGNED),
+    (dict(v=A + 4), binding.GDATTN_ERR_MISALIGNED),
+    (dict(out=A + 8), binding.GDATTN_ERR_MISALIGNED),
+    (dict(seqlens=A + 2), binding.GDATTN_ERR_MISALIGNED),
+    (dict(lse=A + 1), binding.GDATTN_ERR_MISALIGNED),
+    (dict(ws=None), binding.GDATTN_ERR_WORKSPACE),
+    (dict(ws=A + 8), binding.GDATTN_ERR_MISALIGNED),
+])
+def test_decode_rejects_bad_pointers(lib, case, expect):
+    assert call(good_desc(), **case) == expect
+
+
+@pytest.mark.parametrize("desc_kw,expect", [
+    (dict(n_q_heads=0), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(n_kv_heads=0), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(n_q_heads=12, n_kv_heads=8), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(head_dim=0), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(cache_capacity=0), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(window=-1), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(softcap=-1.0), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(softcap=float("nan")), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(split_ctas=-1), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(cache_batch_stride=100), binding.GDATTN_ERR_INVALID_ARG),  # < C*Hkv*D
+    (dict(cache_batch_stride=1024 * 8 * 256 + 4), binding.GDATTN_ERR_INVALID_ARG),  # not % 8
+    (dict(head_dim=128), binding.GDATTN_ERR_UNSUPPORTED),
+    (dict(n_q_heads=64, n_kv_heads=8), binding.GDATTN_ERR_UNSUPPORTED),  # G = 8
+    (dict(n_q_heads=32, n_kv_heads=16), binding.GDATTN_ERR_UNSUPPORTED),  # Hkv = 16
+])
+def test_decode_rejects_bad_desc(lib, desc_kw, expect):
+    assert call(good_desc(**desc_kw)) == expect
+
+
+def test_kv_shared_requires_null_v(lib):
+    d = good_desc(n_q_heads=16, n_kv_heads=1, head_dim=512, window=0, kv_shared=True)
+    assert call(d, v=A) == binding.GDATTN_ERR_INVALID_ARG
+    d.reserved = 1
+    assert call(d, v=None) == binding.GDATTN_ERR_INVALID_ARG
+
+
+def test_tensor_core_path_needs_shared_kv(lib):
+    d = good_desc(n_q_heads=16, n_kv_heads=1, head_dim=512, window=0, kv_shared=False)
+    assert call(d) == binding.GDATTN_ERR_UNSUPPORTED
+
+
+def test_workspace_size_rejects_bad_args(lib):
+    assert binding.workspace_size(0, 8, good_desc()) == 0
+    assert binding.workspace_size(1, 8, good_desc(head_dim=128)) == 0
+    assert lib.gdattn_workspace_size(1, 8, None) == 0
+    assert binding.plan_splits(0, 8, good_desc()) == 0
+    assert binding.plan_splits(1, 8, good_desc(n_q_heads=12)) == 0
+
+
+def test_workspace_init_and_status_reject_null(lib):
+    assert lib.gdattn_workspace_init(None, 1024, None) == binding.GDATTN_ERR_WORKSPACE
+    assert lib.gdattn_workspace_init(A, 16, None) == binding.GDATTN_ERR_WORKSPACE
+    assert lib.gdattn_workspace_init(A + 8, 1024, None) == binding.GDATTN_ERR_MISALIGNED
+    assert lib.gdattn_check_device_status(None, None) == binding.GDATTN_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((None, A, 1, 16, 2, 256, A, A), binding.GDATTN_ERR_INVALID_ARG),
+    ((A, None, 1, 16, 2, 256, A, A), binding.GDATTN_ERR_INVALID_ARG),
+    ((A, A, 1, 16, 2, 256, None, A), binding.GDATTN_ERR_INVALID_ARG),
+    ((A, A, 0, 16, 2, 256, A, A), binding.GDATTN_ERR_INVALID_ARG),
+    ((A, A, 1, 0, 2, 256, A, A), binding.GDATTN_ERR_INVALID_ARG),
+    ((A, A, 1, 16, 0, 256, A, A), binding.GDATTN_ERR_INVALID_ARG),
+    ((A, A, 1, 16, 2, 6, A, A), binding.GDATTN_ERR_INVALID_ARG),
+    ((A, A, 1, 16, 2, 2048, A, A), binding.GDATTN_ERR_INVALID_ARG),
+    ((A, A, 1, 16, 9000, 256, A, A), binding.GDATTN_ERR_INVALID_ARG),
+    ((A + 4, A, 1, 16, 2, 256, A, A), binding.GDATTN_ERR_MISALIGNED),
+    ((A, A + 2, 1, 16, 2, 256, A, A), binding.GDATTN_ERR_MISALIGNED),
+    ((A, A, 1, 16, 2, 256, A + 8, A), binding.GDATTN_ERR_MISALIGNED),
+])
+def test_combine_rejects_bad_args(lib, args, expect):
+    o, l, B, Hq, S, D, out, lse = args
+    assert lib.gdattn_combine(o, l, B, Hq, S, D, out, lse, None) == expect

@@ -1,0 +1,241 @@
+"""GPU parity: libgdattn through its C ABI versus the float64 oracle.
+
+Inputs are seeded bf16; both sides see the same bits.  Gates: max |dout| <= 8e-3
+on the bf16 output (with a one-bf16-ulp floor where heavy key rows push |out|
+above 1) and max |dlse| <= 1e-3 on the fp32 LSE.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from decode_attention_09_b200 import binding
+from gpu_helpers import GpuLayer, compare, oracle_for, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+SPLITS = [0, 1, 2, 3, 7, 33, 300]
+
+# (B, Hq, Hkv, D, C, seqlens, window, softcap, kv_shared)
+CASES = {
+    # CUDA-core path (G = 1, 2, 4)
+    "sliding_g2_nowrap_cap": (3, 16, 8, 256, 64, [64, 1, 37], 64, 50.0, False),
+    "sliding_g2_ring_wraps": (2, 16, 8, 256, 48, [100, 47], 48, 0.0, False),
+    "sliding_g2_window_lt_cap": (2, 16, 8, 256, 64, [130, 20], 40, 0.0, False),
+    "sliding_g2_edges": (5, 16, 8, 256, 32, [1, 2, 31, 32, 33], 32, 0.0, False),
+    "global_g1_shared_d512": (2, 8, 8, 512, 70, [70, 9], 0, 0.0, True),
+    "global_g4_hkv2": (2, 8, 2, 256, 90, [90, 33], 0, 0.0, False),
+    "global_g4_hkv1_d512": (1, 4, 1, 512, 200, [200], 0, 0.0, False),
+    "global_g1_hkv4_shared": (2, 4, 4, 256, 50, [50, 50], 0, 5.0, True),
+    # tensor-core path (G = 16, D = 512, K = V)
+    "tc_multi_tile_tail": (1, 16, 1, 512, 300, [300], 0, 0.0, True),
+    "tc_edges": (3, 16, 1, 512, 200, [1, 64, 200], 0, 0.0, True),
+    "tc_hkv2": (2, 32, 2, 512, 150, [150, 65], 0, 0.0, True),
+    "tc_window_ring": (2, 16, 1, 512, 96, [150, 96], 96, 0.0, True),
+    "tc_softcap": (2, 16, 1, 512, 129, [129, 128], 0, 30.0, True),
+}
+
+_ref_cache = {}
+
+
+def case_inputs(name):
+    B, Hq, Hkv, D, C, sl, w, cap, shared = CASES[name]
+    seed = 100 + sorted(CASES).index(name)
+    return workloads.random_case(seed, B, Hq, Hkv, D, C, sl, window=w, softcap=cap,
+                                 kv_shared=shared)
+
+
+def case_ref(name):
+    if name not in _ref_cache:
+        inp = case_inputs(name)
+        _ref_cache[name] = (inp, oracle_for(inp))
+    return _ref_cache[name]
+
+
+@pytest.mark.parametrize("split", SPLITS)
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_sweep(name, split):
+    require_gpu()
+    inp, (o_ref, l_ref) = case_ref(name)
+    out, lse = GpuLayer(inp, split_ctas=split).run()
+    compare(out, lse, o_ref, l_ref, what=f"{name} split={split}")
+
+
+# ---------------------------------------------------------------- workloads
+
+
+def test_single_sliding_layer():
+    """q [1,16,256], K/V [2048,8,256], w 512, cap 50, scale 1/16."""
+    require_gpu()
+    w = workloads.single_sliding()
+    inp = workloads.workload_layer_inputs(w, 0)
+    o_ref, l_ref = oracle_for(inp)
+    out, lse = GpuLayer(inp).run()
+    compare(out, lse, o_ref, l_ref, what=w.name)
+
+
+def test_single_global_layer():
+    """q [1,16,512], one K=V tensor [32768,1,512], split-KV + LSE combine."""
+    require_gpu()
+    w = workloads.single_global()
+    inp = workloads.workload_layer_inputs(w, 0)
+    o_ref, l_ref = oracle_for(inp)
+    out, lse = GpuLayer(inp).run()
+    compare(out, lse, o_ref, l_ref, what=w.name)
+
+
+@pytest.mark.parametrize("layer", [0, 5])
+def test_gemma4_12b_stack_layers(layer):
+    """Batch 8, context 8192: one sliding layer (ring of 1024) and one global K=V layer."""
+    require_gpu()
+    w = workloads.gemma4_12b_b8_l8192()
+    inp = workloads.workload_layer_inputs(w, layer)
+    o_ref, l_ref = oracle_for(inp)
+    out, lse = GpuLayer(inp).run()
+    compare(out, lse, o_ref, l_ref, what=f"{w.name} layer {layer}")
+
+
+@pytest.mark.parametrize("layer", [0, 1])
+def test_ragged_batch(layer):
+    """Batch 64, L ~ U[512, 32768]: all sequences on the GPU, 4 sampled by the oracle."""
+    require_gpu()
+    w = workloads.ragged_b64()
+    inp = workloads.workload_layer_inputs(w, layer, device="cuda")
+    sl = inp.seqlens.cpu()
+    g = torch.Generator().manual_seed(7)
+    pick = sorted(set([int(sl.argmin()), int(sl.argmax())] +
+                      torch.randint(0, w.batch, (2,), generator=g).tolist()))
+    o_ref, l_ref = oracle_for(inp, pick)
+    out, lse = GpuLayer(inp).run()
+    compare(out[pick], lse[pick], o_ref, l_ref, what=f"{w.name} layer {layer}")
+
+
+@pytest.mark.parametrize("layer", [0, 5])
+def test_long_context(layer):
+    """Batch 4, context 131072, 1 % of key rows x8: sampled sequences, ulp floor."""
+    require_gpu()
+    w = workloads.long_context_b4()
+    inp = workloads.workload_layer_inputs(w, layer, device="cuda")
+    pick = [1] if inp.spec.kind == "global" else [0, 1, 2, 3]
+    o_ref, l_ref = oracle_for(inp, pick)
+    out, lse = GpuLayer(inp).run()
+    compare(out[pick], lse[pick], o_ref, l_ref, ulp_floor=True, what=f"{w.name} layer {layer}")
+
+
+# --------------------------------------------------------------- invariants
+
+
+@pytest.mark.parametrize("name", ["sliding_g2_window_lt_cap", "sliding_g2_ring_wraps",
+                                  "tc_multi_tile_tail", "tc_window_ring", "tc_edges"])
+def test_unattended_slots_never_matter(name):
+    """NaN in every cache slot outside the attended range leaves the result unchanged."""
+    require_gpu()
+    inp, _ = case_ref(name)
+    clean_out, clean_lse = GpuLayer(inp, split_ctas=3).run()
+    k = inp.k.clone()
+    v = inp.v.clone() if inp.v is not None else None
+    C = k.shape[1]
+    w = inp.spec.window
+    for b, L in enumerate(inp.seqlens.tolist()):
+        n = min(L, w) if w > 0 else L
+        keep = torch.zeros(C, dtype=torch.bool)
+        for p in range(L - n, L):
+            keep[p % C] = True
+        k[b, ~keep] = float("nan")
+        if v is not None:
+            v[b, ~keep] = float("nan")
+    poisoned = workloads.LayerInputs(inp.q, k, v, inp.seqlens, inp.spec)
+    out, lse = GpuLayer(poisoned, split_ctas=3).run()
+    assert torch.equal(out, clean_out)
+    assert torch.equal(lse, clean_lse)
+
+
+@pytest.mark.parametrize("which", ["single_sliding", "single_global"])
+def test_split_count_invariance(which):
+    """One CTA or many: same result to fp32 rounding (one bf16 ulp on out)."""
+    require_gpu()
+    w = getattr(workloads, which)()
+    inp = workloads.workload_layer_inputs(w, 0)
+    o1, l1 = GpuLayer(inp, split_ctas=1).run()
+    for split in (2, 5, 148, 296):
+        o2, l2 = GpuLayer(inp, split_ctas=split).run()
+        d = (o1.float() - o2.float()).abs()
+        ulp = torch.from_numpy(np.exp2(np.floor(np.log2(np.maximum(
+            o1.float().abs().cpu().numpy(), 1e-30))) - 7)).to(d.device)
+        assert bool((d <= ulp + 1e-12).all()), f"split {split}: max {d.max().item()}"
+        assert (l1 - l2).abs().max().item() <= 2e-5
+
+
+def test_bitwise_reproducible():
+    require_gpu()
+    for name in ("sliding_g2_ring_wraps", "tc_multi_tile_tail"):
+        inp, _ = case_ref(name)
+        layer = GpuLayer(inp, split_ctas=7)
+        a = layer.run()
+        b = layer.run()
+        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_combine_matches_oracle_merge():
+    """gdattn_combine on oracle-made partials equals the oracle's own LSE merge."""
+    require_gpu()
+    orc = oracle.get()
+    inp = workloads.random_case(55, 2, 8, 2, 256, 120, [120, 77], window=0, softcap=0.0)
+    s = inp.spec
+    cuts = [[0, 10, 10, 64, 120], [0, 5, 40, 77, 77]]  # includes empty parts
+    parts_o, parts_l = [], []
+    for p in range(4):
+        lo = [c[p] for c in cuts]
+        hi = [c[p + 1] for c in cuts]
+        o, l = orc.attend(inp.q, inp.k, inp.v, lo, hi, s.softcap, s.scale)
+        parts_o.append(o)
+        parts_l.append(l)
+    po = np.stack(parts_o, axis=2)
+    pl = np.stack(parts_l, axis=2)
+    o_ref, l_ref = orc.combine(po, pl)
+    out, lse = binding.combine(torch.from_numpy(po).float().cuda().contiguous(),
+                               torch.from_numpy(pl).float().cuda().contiguous())
+    torch.cuda.synchronize()
+    compare(out, lse, o_ref, l_ref, what="combine")
+    # all-empty parts: out = 0, lse = -inf
+    out, lse = binding.combine(torch.zeros((1, 2, 3, 256), device="cuda"),
+                               torch.full((1, 2, 3), float("-inf"), device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_device_detects_impossible_seqlens():
+    """L = 0, or a global layer's L beyond the cache: status word says so, no fault."""
+    require_gpu()
+    inp = workloads.random_case(56, 3, 16, 8, 256, 32, [5, 0, 9], window=16)
+    layer = GpuLayer(inp, max_seqlen=16)
+    out, lse = binding.decode(layer.q, layer.k, layer.v, layer.seqlens, layer.desc, 16,
+                              workspace=layer.ws)
+    assert binding.check_device_status(layer.ws) == binding.GDATTN_ERR_DEVICE_SEQLEN
+    assert torch.all(out[1] == 0) and torch.all(torch.isneginf(lse[1]))
+    assert binding.check_device_status(layer.ws) == binding.GDATTN_OK  # cleared by the read
+    inp = workloads.random_case(57, 1, 16, 1, 512, 64, [100], window=0, kv_shared=True)
+    layer = GpuLayer(inp, max_seqlen=100)
+    binding.decode(layer.q, layer.k, layer.v, layer.seqlens, layer.desc, 100, workspace=layer.ws)
+    assert binding.check_device_status(layer.ws) == binding.GDATTN_ERR_DEVICE_SEQLEN
+
+
+def test_cuda_graph_replay_matches_eager():
+    """Decode calls captured in a CUDA graph give the eager results."""
+    require_gpu()
+    layers = [GpuLayer(case_ref(n)[0]) for n in ("sliding_g2_ring_wraps", "tc_multi_tile_tail")]
+    eager = [ly.run() for ly in layers]
+    outs = [(torch.empty_like(e[0]), torch.empty_like(e[1])) for e in eager]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for ly, (o, l) in zip(layers, outs):
+                binding.decode(ly.q, ly.k, ly.v, ly.seqlens, ly.desc, ly.max_seqlen, out=o, lse=l,
+                               workspace=ly.ws, stream=s)
+    g.replay()
+    torch.cuda.synchronize()
+    for (o, l), (eo, el) in zip(outs, eager):
+        assert torch.equal(o, eo) and torch.equal(l, el)
