@@ -21,7 +21,6 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -190,17 +189,19 @@ class Stack:
 
 
 def time_graph(g, stream, steps, warmup):
-    for _ in range(warmup):
-        g.replay()
-    stream.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(steps):
-        g.replay()
-    t1.record(stream)
+    """Device time per replay (ms): CUDA events on the stream the graph replays on."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            g.replay()
+        stream.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        t1.record(stream)
     t1.synchronize()
-    return t0.elapsed_time(t1) / steps  # ms per replay
+    return t0.elapsed_time(t1) / steps
 
 
 def max_over_ranks(x, world):
@@ -213,46 +214,56 @@ def max_over_ranks(x, world):
 
 
 # --------------------------------------------------------- oracle baseline
-def oracle_sample(w: workloads.Workload, layers, seqs, device_inputs=None):
-    """Time the float64 oracle on `layers` x `seqs` of the workload.  Returns
-    (kv_bytes, seconds)."""
+def oracle_time(w: workloads.Workload, host_layers):
+    """Time the float64 oracle over host copies of some layers' inputs.
+    host_layers: list of (layer index, LayerInputs on the CPU).  Returns (kv_bytes, s)."""
     import oracle  # the CPU baseline leg is the one bench path that runs the oracle
 
     orc = oracle.get()
-    seqlens = w.seqlens()
     total_bytes, total_s = 0, 0.0
+    for i, inp in host_layers:
+        spec = w.layers[i]
+        t = time.perf_counter()
+        orc.decode(inp.q, inp.k, inp.v, inp.seqlens, spec.window, spec.softcap, spec.scale)
+        total_s += time.perf_counter() - t
+        total_bytes += accounting.layer_kv_bytes(spec, inp.seqlens.tolist())
+    return total_bytes, total_s
+
+
+def host_sample(w: workloads.Workload, layers, seqs):
+    """CPU-generated inputs of `layers`, restricted to sequences `seqs`."""
+    seqlens = w.seqlens()
+    idx = torch.as_tensor(seqs)
+    out = []
     for i in layers:
         spec = w.layers[i]
         inp = workloads.layer_inputs(spec, w.batch, seqlens, w.seed * 1000 + i, device="cpu",
                                      heavy_row_frac=w.heavy_row_frac,
                                      heavy_row_scale=w.heavy_row_scale)
-        idx = torch.as_tensor(seqs)
-        q, k = inp.q[idx].contiguous(), inp.k[idx].contiguous()
-        v = inp.v[idx].contiguous() if inp.v is not None else None
-        sl = seqlens[idx]
-        t = time.perf_counter()
-        orc.decode(q, k, v, sl, spec.window, spec.softcap, spec.scale)
-        total_s += time.perf_counter() - t
-        total_bytes += accounting.layer_kv_bytes(spec, sl.tolist())
-    return total_bytes, total_s
+        out.append((i, workloads.LayerInputs(
+            inp.q[idx].contiguous(), inp.k[idx].contiguous(),
+            inp.v[idx].contiguous() if inp.v is not None else None, seqlens[idx], spec)))
+    return out
 
 
-ORACLE_SAMPLE_LAYERS = [0, 1, 2, 3, 4, 5]
-ORACLE_SAMPLE_SEQS = [0, 1]
-ORACLE_SAMPLE_TEXT = ("float64 oracle, 1 thread, layers 0-5 (5 sliding + 1 global K=V) x "
-                      "sequences 0-1 of the batch-8 / 8192-context stack")
+REF_STEP_LAYERS = [0, 5]
+REF_STEP_SEQS = [0, 1]
+REF_STEP_TEXT = ("float64 oracle, 1 thread; one step = layers 0 (sliding) and 5 (global K=V) x "
+                 "sequences 0-1 of the batch-8 / 8192-context stack")
+CPU_BASELINE_TEXT = ("float64 oracle, 1 thread, over the full 48-layer step (all 8 sequences), "
+                     "on host copies of the exact inputs the GPU processed")
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
     w = workloads.ALL_WORKLOADS[args.workload]()
-    step_layers = ORACLE_SAMPLE_LAYERS
+    sample = host_sample(w, REF_STEP_LAYERS, REF_STEP_SEQS)
     for _ in range(args.warmup):
-        oracle_sample(w, [0], [0])
+        oracle_time(w, sample[:1])
     tb, ts = 0, 0.0
     for _ in range(args.steps):
-        b, s = oracle_sample(w, step_layers, ORACLE_SAMPLE_SEQS)
+        b, s = oracle_time(w, sample)
         tb += b
         ts += s
     gbs = tb / ts / 1e9
@@ -263,9 +274,9 @@ def run_reference(args, world, rank):
         "data": "synthetic",
         "config": {"workload": w.name, "layers": len(w.layers), "global_batch": w.batch,
                    "seq_len": w.seqlen, "parallelism": "none (host oracle)",
-                   "step": "bounded sample: " + ORACLE_SAMPLE_TEXT},
+                   "step": "bounded sample: " + REF_STEP_TEXT},
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": ORACLE_SAMPLE_TEXT},
+                         "sample": REF_STEP_TEXT},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -328,38 +339,59 @@ def run_ours(args, world, rank, local):
     d2h = sum(t.numel() * t.element_size() for t in out_host + lse_host)
 
     def e2e_step():
+        sl_dev.copy_(sl_host, non_blocking=True)
+        for i, ly in enumerate(stack.layers):
+            q_dev[i].copy_(q_host[i], non_blocking=True)
+            binding.decode(q_dev[i], ly["inp"].k, ly["inp"].v, sl_dev, ly["desc"],
+                           stack.max_seqlen, out=ly["out"], lse=ly["lse"], workspace=ly["ws"],
+                           stream=stream)
+            out_host[i].copy_(ly["out"], non_blocking=True)
+            lse_host[i].copy_(ly["lse"], non_blocking=True)
+
+    def timed(fn, steps):
         with torch.cuda.stream(stream):
-            sl_dev.copy_(sl_host, non_blocking=True)
-            for i, ly in enumerate(stack.layers):
-                q_dev[i].copy_(q_host[i], non_blocking=True)
-                binding.decode(q_dev[i], ly["inp"].k, ly["inp"].v, sl_dev, ly["desc"],
-                               stack.max_seqlen, out=ly["out"], lse=ly["lse"], workspace=ly["ws"],
-                               stream=stream)
-                out_host[i].copy_(ly["out"], non_blocking=True)
-                lse_host[i].copy_(ly["lse"], non_blocking=True)
+            for _ in range(args.warmup):
+                fn()
+            barrier()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                fn()
+            e1.record(stream)
+        e1.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1) / steps, world)
 
-    for _ in range(args.warmup):
+    # (a) each step issued call by call from Python;
+    ms_e2e_eager = timed(e2e_step, min(args.steps, 200))
+    # (b) the same step (copies + 48 calls) captured once in a CUDA graph, as a
+    #     serving loop replays it.
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
         e2e_step()
-    barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    e1.synchronize()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+        stream.synchronize()
+        with torch.cuda.graph(g_e2e, stream=stream):
+            e2e_step()
+    ms_e2e = timed(g_e2e.replay, args.steps)
+    # the graph's D2H landed in pinned memory: it must equal the device result
+    torch.cuda.synchronize()
+    assert torch.equal(out_host[-1], stack.layers[-1]["out"].cpu())
 
-    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    # ---- CPU baseline: the oracle over the whole step (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
-        b, s = oracle_sample(w, ORACLE_SAMPLE_LAYERS, ORACLE_SAMPLE_SEQS)
+        host = [(i, workloads.LayerInputs(ly["inp"].q.cpu(), ly["inp"].k.cpu(),
+                                          ly["inp"].v.cpu() if ly["inp"].v is not None else None,
+                                          ly["inp"].seqlens.cpu(), ly["spec"]))
+                for i, ly in enumerate(stack.layers)]
+        b, s = oracle_time(w, host)
+        del host
         cpu = {"value": b / s / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": ORACLE_SAMPLE_TEXT, "seconds": s}
+               "sample": CPU_BASELINE_TEXT, "seconds": s}
 
     if world > 1:
         import torch.distributed as dist
-        del g_all, g_sl, g_gl
+        del g_all, g_sl, g_gl, g_e2e
         dist.destroy_process_group()
     if rank != 0:
         return 0
@@ -403,7 +435,11 @@ def run_ours(args, world, rank, local):
                    "graph": "48 gdattn_decode calls per CUDA graph replay"},
         "roofline": roof, "per_layer_type": per_type, "cpu_baseline": cpu,
         "e2e": {"value": kv_step * world / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
-                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "how": "pinned H2D of q + seqlens, 48 gdattn_decode calls, D2H of out + lse; "
+                       "the step captured once in a CUDA graph and replayed",
+                "eager_value": kv_step * world / (ms_e2e_eager * 1e-3) / 1e9,
+                "eager_ms_per_step": ms_e2e_eager},
         "gpu_launches": stack.launches_per_step(all_idx) * args.steps,
         "clocks": clk,
     }
@@ -414,7 +450,7 @@ def run_ours(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="gemma4_12b_stack_b8_l8192",

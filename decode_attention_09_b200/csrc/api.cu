@@ -56,8 +56,7 @@ struct CoreKernel {
 template <int D, int G, int HKV, bool SH>
 CoreKernel core_kernel_entry() {
   using Cfg = CoreConfig<D, G, HKV, SH>;
-  return CoreKernel{core_decode_kernel<D, G, HKV, SH>, Cfg::kThreads, Cfg::SMEM, Cfg::T,
-                    Cfg::MIN_BLOCKS};
+  return CoreKernel{core_decode_kernel<D, G, HKV, SH>, Cfg::kThreads, Cfg::SMEM, Cfg::T, 1};
 }
 
 template <int D, int G, int HKV>
@@ -175,7 +174,7 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
     if (ck.fn == nullptr) return GDATTN_ERR_UNSUPPORTED;
     per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(ck.fn), ck.threads, ck.smem,
                                   query_core);
-    min_tokens = 4 * ck.tokens_per_stage;
+    min_tokens = 2 * ck.tokens_per_stage;
     pl.units_per_seq = 1;
     pl.heads_per_unit = d->n_q_heads;
   } else {
@@ -240,6 +239,14 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
+// Dynamic shared memory of the combine kernel: part weights plus the
+// per-group float4 accumulators.
+int combine_smem_bytes(int n_parts, int head_dim) {
+  const int nc = head_dim / 4;
+  const int ng = nc >= kCombineThreads ? 1 : kCombineThreads / nc;
+  return ((n_parts + 3) & ~3) * 4 + ng * nc * 16 + 16;
+}
+
 gdattn_status launch_combine_internal(const LayerPlan &pl, const Geometry &geo, const float *ws_lse,
                                       const float *ws_o, const gdattn_layer_desc *d, void *out,
                                       float *lse, cudaStream_t stream) {
@@ -253,7 +260,7 @@ gdattn_status launch_combine_internal(const LayerPlan &pl, const Geometry &geo, 
   cp.geo = geo;
   cp.heads_per_unit = pl.heads_per_unit;
   cp.n_splits = 0;
-  const int smem = static_cast<int>(pl.grid) * 4 + 16;
+  const int smem = combine_smem_bytes(pl.grid, d->head_dim);
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg =
       launch_config(dim3(static_cast<unsigned>(geo.batch * pl.units_per_seq),
@@ -403,7 +410,6 @@ gdattn_status gdattn_decode(const void *q, const void *k_cache, const void *v_ca
         return GDATTN_ERR_CUDA;
     }
     TcParams tp;
-    tp.q = static_cast<const uint16_t *>(q);
     tp.out = static_cast<uint16_t *>(out);
     tp.lse = lse;
     tp.ws_o = ws_o;
@@ -444,7 +450,7 @@ gdattn_status gdattn_combine(const float *o_partial, const float *lse_partial, i
   cp.head_dim = head_dim;
   cp.heads_per_unit = 0;
   cp.n_splits = n_splits;
-  const int smem = n_splits * 4 + 16;
+  const int smem = combine_smem_bytes(n_splits, head_dim);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(combine_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) != cudaSuccess)

@@ -53,7 +53,7 @@ __device__ void unit_position(const Geometry &g, int32_t b, int32_t x, int64_t &
 
 template <bool INTERNAL>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineParams p) {
-  extern __shared__ float wts[];  // [n_parts]
+  extern __shared__ __align__(16) float wts[];  // [n_parts] weights, then [NG][NC] float4
   __shared__ int64_t sh_slot0;
   __shared__ int32_t sh_nparts;
 
@@ -139,24 +139,67 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineP
   const bool empty = (mx == -INFINITY);
   const float inv_z = empty ? 0.f : 1.f / z;
 
+  // Thread t owns float4 column (t mod NC) and parts t / NC, t / NC + NG, ...;
+  // loads are issued kUnroll at a time so each thread keeps several in flight.
   uint16_t *dst = p.out + (static_cast<int64_t>(b) * p.n_q_heads + h) * D;
-  for (int d = 4 * threadIdx.x; d < D; d += 4 * blockDim.x) {
+  const int NC = D / 4;
+  const int NG = NC >= kCombineThreads ? 1 : kCombineThreads / NC;
+  const int grp = threadIdx.x / NC;
+  float4 *part_acc = reinterpret_cast<float4 *>(wts + ((np + 3) & ~3));  // [NG][NC]
+  for (int d4 = threadIdx.x % NC; d4 < NC; d4 += kCombineThreads) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (!empty) {
-      for (int32_t s = 0; s < np; ++s) {
+    if (!empty && grp < NG) {
+      constexpr int kUnroll = 8;
+      int32_t s = grp;
+      for (; s + (kUnroll - 1) * NG < np; s += kUnroll * NG) {
+        float4 v[kUnroll];
+        float wv[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          v[u] = *reinterpret_cast<const float4 *>(o_base + (s + u * NG) * o_stride + 4 * d4);
+          wv[u] = wts[s + u * NG];
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          // an empty part has weight 0 and may hold anything: select, don't multiply
+          if (wv[u] != 0.f) {
+            acc.x = fmaf(wv[u], v[u].x, acc.x);
+            acc.y = fmaf(wv[u], v[u].y, acc.y);
+            acc.z = fmaf(wv[u], v[u].z, acc.z);
+            acc.w = fmaf(wv[u], v[u].w, acc.w);
+          }
+        }
+      }
+      for (; s < np; s += NG) {
         const float w = wts[s];
-        if (w == 0.f) continue;
-        const float4 v = *reinterpret_cast<const float4 *>(o_base + s * o_stride + d);
-        acc.x = fmaf(w, v.x, acc.x);
-        acc.y = fmaf(w, v.y, acc.y);
-        acc.z = fmaf(w, v.z, acc.z);
-        acc.w = fmaf(w, v.w, acc.w);
+        if (w != 0.f) {
+          const float4 v = *reinterpret_cast<const float4 *>(o_base + s * o_stride + 4 * d4);
+          acc.x = fmaf(w, v.x, acc.x);
+          acc.y = fmaf(w, v.y, acc.y);
+          acc.z = fmaf(w, v.z, acc.z);
+          acc.w = fmaf(w, v.w, acc.w);
+        }
       }
     }
-    uint2 pk;
-    pk.x = pack_bf16x2(acc.x * inv_z, acc.y * inv_z);
-    pk.y = pack_bf16x2(acc.z * inv_z, acc.w * inv_z);
-    *reinterpret_cast<uint2 *>(dst + d) = pk;
+    if (NG > 1) {
+      if (grp < NG) part_acc[grp * NC + d4] = acc;
+      __syncthreads();
+      if (grp == 0) {
+        for (int g2 = 1; g2 < NG; ++g2) {
+          const float4 o = part_acc[g2 * NC + d4];
+          acc.x += o.x;
+          acc.y += o.y;
+          acc.z += o.z;
+          acc.w += o.w;
+        }
+      }
+    }
+    if (grp == 0) {
+      uint2 pk;
+      pk.x = pack_bf16x2(acc.x * inv_z, acc.y * inv_z);
+      pk.y = pack_bf16x2(acc.z * inv_z, acc.w * inv_z);
+      *reinterpret_cast<uint2 *>(dst + 4 * d4) = pk;
+    }
   }
   if (threadIdx.x == 0 && p.lse != nullptr)
     p.lse[static_cast<int64_t>(b) * p.n_q_heads + h] = empty ? -INFINITY : mx + logf(z);

@@ -1,22 +1,22 @@
 // Split-KV decode attention on CUDA cores, for small GQA groups (G = Hq/Hkv in
 // {1, 2, 4}) such as Gemma-4 sliding layers (16 q heads over 8 KV heads, G = 2).
 //
-// With G <= 4 a KV row feeds at most 4 query heads, about 1-2 flop per byte, so
-// the products are not a dense contraction and run as fp32 FMAs; the kernel is
-// bound by HBM bandwidth.
+// With G <= 4 a KV row feeds at most 4 query heads, 1-2 flop per byte: not a
+// dense contraction, so the products run as fp32 FMAs (packed two per
+// instruction with Blackwell's fma.rn.f32x2) and the kernel is bound by HBM.
 //
-// CTA = 8 compute warps + 1 producer warp.  The producer streams whole token
-// rows (all Hkv heads, contiguous in the token-major cache) with 1-D bulk
-// copies into an NSTAGE-deep shared-memory ring, one mbarrier pair per stage.
-// Compute warp w owns KV head w % Hkv and, when Hkv < 8, every (8/Hkv)-th token
-// of a stage.  A lane holds D/32 consecutive-by-16-bytes elements of q, of the
-// output accumulator and of each K/V row it reads, so shared-memory reads are
-// 16-byte vectors with no bank conflicts.
+// CTA = 8 compute warps + 1 producer warp, one CTA per SM.  The producer streams
+// whole token rows (all Hkv heads, contiguous in the token-major cache) with
+// 1-D bulk copies into an NSTAGE-deep shared-memory ring, one mbarrier pair per
+// stage.  Compute warp w owns KV head w % Hkv and, when Hkv < 8, every
+// (8/Hkv)-th token of a stage.  A lane holds D/32 elements (16-byte chunks
+// 256 * j + 8 * lane) of q, of the output accumulator and of each K/V row it
+// reads, so shared-memory reads are conflict-free 16-byte vectors.
 //
-// Per stage a warp handles TPW = 4 tokens: it forms TPW*G partial dot products
-// per lane, reduce-scatters them across the warp (each lane ends with one full
-// score), applies scale / soft-cap, updates the running max and sum of the
-// online softmax, broadcasts the TPW*G weights and accumulates P.V.
+// Per stage a warp handles TPW tokens: it forms TPW*G partial dot products per
+// lane, reduce-scatters them across the warp (each lane ends with one full
+// score), applies scale / soft-cap, updates the running max and sum of the online
+// softmax, broadcasts the weights and accumulates P.V.
 #pragma once
 
 #include <cstdint>
@@ -46,37 +46,39 @@ template <int D, int G, int HKV, bool SHARED>
 struct CoreConfig {
   static constexpr int kComputeWarps = 8;
   static constexpr int kThreads = (kComputeWarps + 1) * 32;
+  static constexpr int NT = SHARED ? 1 : 2;
   static constexpr int TS = kComputeWarps / HKV;      // warps sharing one KV head
-  static constexpr int TPW = 4;                       // tokens per warp per stage
+  static constexpr int TPW = (D * NT <= 512) ? 8 : 4; // tokens per warp per stage
   static constexpr int T = TS * TPW;                  // tokens per stage
   static constexpr int EPL = D / 32;                  // elements per lane
   static constexpr int CH = EPL / 8;                  // 16-byte chunks per lane
   static constexpr int ROWB = HKV * D * 2;            // bytes of one token row (one tensor)
-  static constexpr int NT = SHARED ? 1 : 2;
   static constexpr int STAGEB = T * ROWB * NT;
-  static constexpr int NSTAGE = (98304 / STAGEB) < 2 ? 2 : (98304 / STAGEB);
-  static constexpr int NV = TPW * G;                  // scores per warp per stage
-  static constexpr int LOGNV = NV == 4 ? 2 : (NV == 8 ? 3 : 4);
-  static constexpr int LOGG = G == 1 ? 0 : (G == 2 ? 1 : 2);
   static constexpr int MHDR = 8;                      // per-warp merge header (m[G], l[G])
   static constexpr int MSTRIDE = MHDR + G * D;        // floats per warp, 16-byte multiple
   static constexpr int MERGEB = TS > 1 ? kComputeWarps * MSTRIDE * 4 : 0;
+  // Stages: up to 192 KiB of ring, within what the merge area leaves.
+  static constexpr int RING = (220 * 1024 - MERGEB) < 196608 ? (220 * 1024 - MERGEB) : 196608;
+  static constexpr int NSTAGE = (RING / STAGEB) < 2 ? 2 : (RING / STAGEB > 8 ? 8 : RING / STAGEB);
+  static constexpr int NV = TPW * G;                  // scores per warp per stage
+  static constexpr int LOGNV = NV == 4 ? 2 : (NV == 8 ? 3 : (NV == 16 ? 4 : 5));
+  static constexpr int LOGG = G == 1 ? 0 : (G == 2 ? 1 : 2);
+  static constexpr int LOGT = TPW == 4 ? 2 : 3;
   static constexpr int SMEM = NSTAGE * STAGEB + 2 * NSTAGE * 8 + 128 + MERGEB + 1024;
-  static constexpr int MIN_BLOCKS = (EPL * G <= 32 && SMEM <= 110 * 1024) ? 2 : 1;
   static_assert(HKV == 1 || HKV == 2 || HKV == 4 || HKV == 8, "HKV");
   static_assert(G == 1 || G == 2 || G == 4, "G");
   static_assert(D == 256 || D == 512, "D");
+  static_assert(NV <= 32, "one score per lane at most");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-__device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
-
 template <int D, int G, int HKV, bool SHARED>
-__global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads,
-                                  CoreConfig<D, G, HKV, SHARED>::MIN_BLOCKS)
+__global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads, 1)
     core_decode_kernel(const CoreParams p) {
   using Cfg = CoreConfig<D, G, HKV, SHARED>;
-  constexpr int NSTAGE = Cfg::NSTAGE, T = Cfg::T, EPL = Cfg::EPL, CH = Cfg::CH;
-  constexpr int ROWB = Cfg::ROWB, NV = Cfg::NV, LOGNV = Cfg::LOGNV;
+  constexpr int NSTAGE = Cfg::NSTAGE, T = Cfg::T, CH = Cfg::CH;
+  constexpr int ROWB = Cfg::ROWB, NV = Cfg::NV, LOGNV = Cfg::LOGNV, TPW = Cfg::TPW;
+  constexpr int P2 = Cfg::EPL / 2;  // float2 pairs per lane
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -163,8 +165,8 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads,
     // ------------------------------------------------------------- compute
     const int kvh = warp % HKV;
     const int tp = warp / HKV;
-    float q[G][EPL];
-    float o[G][EPL];
+    float2 q[G][P2];
+    float2 o[G][P2];
     float m[G], l[G];
     uint32_t fills = 0;
     bool ok = true;
@@ -172,7 +174,7 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads,
     it.init(p.geo, *plan);
     Segment s;
     while (it.next(s)) {
-      // Load this sequence's query rows for the warp's heads, pre-scaled.
+      // This sequence's query rows for the warp's heads, pre-scaled, as pairs.
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const uint16_t *qr = p.q + (static_cast<int64_t>(s.b) * p.n_q_heads + kvh * G + g) * D;
@@ -181,13 +183,11 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads,
           const uint4 w = __ldg(reinterpret_cast<const uint4 *>(qr + 256 * j + 8 * lane));
           const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            q[g][8 * j + 2 * e] = bf16lo(ww[e]) * p.qscale;
-            q[g][8 * j + 2 * e + 1] = bf16hi(ww[e]) * p.qscale;
-          }
+          for (int e = 0; e < 4; ++e)
+            q[g][4 * j + e] = make_float2(bf16lo(ww[e]) * p.qscale, bf16hi(ww[e]) * p.qscale);
         }
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) o[g][e] = 0.f;
+        for (int e = 0; e < P2; ++e) o[g][e] = make_float2(0.f, 0.f);
         m[g] = -INFINITY;
         l[g] = 0.f;
       }
@@ -204,13 +204,15 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads,
           const uint8_t *kst = stage_k + st * T * ROWB + kvh * D * 2;
           const uint8_t *vst = (SHARED ? stage_k : stage_v) + st * T * ROWB + kvh * D * 2;
 
-          // Partial dot products: part[i*G + g] over this lane's elements.
+          // Partial dot products part[i*G + g] over this lane's elements, two
+          // elements per packed FMA.
           float part[NV];
 #pragma unroll
-          for (int i = 0; i < Cfg::TPW; ++i) {
+          for (int i = 0; i < TPW; ++i) {
             const int t = tp + Cfg::TS * i;
+            float2 acc[G];
 #pragma unroll
-            for (int g = 0; g < G; ++g) part[i * G + g] = 0.f;
+            for (int g = 0; g < G; ++g) acc[g] = make_float2(0.f, 0.f);
             if (t < ntok) {
 #pragma unroll
               for (int j = 0; j < CH; ++j) {
@@ -219,19 +221,18 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads,
                 const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                  const float k0 = bf16lo(ww[e]), k1 = bf16hi(ww[e]);
+                  const float2 k2 = make_float2(bf16lo(ww[e]), bf16hi(ww[e]));
 #pragma unroll
-                  for (int g = 0; g < G; ++g) {
-                    part[i * G + g] = fmaf(q[g][8 * j + 2 * e], k0, part[i * G + g]);
-                    part[i * G + g] = fmaf(q[g][8 * j + 2 * e + 1], k1, part[i * G + g]);
-                  }
+                  for (int g = 0; g < G; ++g) acc[g] = __ffma2_rn(q[g][4 * j + e], k2, acc[g]);
                 }
               }
             }
+#pragma unroll
+            for (int g = 0; g < G; ++g) part[i * G + g] = acc[g].x + acc[g].y;
           }
-          // Reduce-scatter: after log2(NV) halving steps lane holds one score,
-          // index bits k <-> lane bit (5 - LOGNV + k); the rest of the lanes
-          // that share an index sum up with the remaining xor steps.
+          // Reduce-scatter: after log2(NV) halving steps a lane holds one score,
+          // index bit k <-> lane bit (5 - LOGNV + k); lanes below bit
+          // (5 - LOGNV) then sum their copies with the remaining xor steps.
           {
             int cnt = NV;
 #pragma unroll
@@ -259,40 +260,49 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads,
           float sc = part[0];
           if (p.post != 0.f) sc = p.post * tanhf(sc);
           if (my_t >= ntok) sc = -INFINITY;
-          // Max over this stage's tokens for the lane's head (token bits are
-          // the top lane bits: offsets 16, 8 for TPW = 4).
-          float tmax = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 16));
-          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+          // Max over this stage's tokens for the lane's head: the token bits
+          // are lane bits 5 - LOGT .. 4.
+          float tmax = sc;
+#pragma unroll
+          for (int off = 16; off >= (1 << (5 - Cfg::LOGT)); off >>= 1)
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
           float mnew[G], alpha[G];
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             const float mx = __shfl_sync(0xffffffffu, tmax, g << (5 - LOGNV));
             mnew[g] = fmaxf(m[g], mx);
-            alpha[g] = (mnew[g] == -INFINITY) ? 1.f : fast_exp2(m[g] - mnew[g]);
+            alpha[g] = (mnew[g] == -INFINITY) ? 1.f : exp2f(m[g] - mnew[g]);
           }
           float mine_m = mnew[0];
 #pragma unroll
           for (int g = 1; g < G; ++g)
             if (my_g == g) mine_m = mnew[g];
-          const float pe = (sc == -INFINITY) ? 0.f : fast_exp2(sc - mine_m);
-          float psum = pe + __shfl_xor_sync(0xffffffffu, pe, 16);
-          psum += __shfl_xor_sync(0xffffffffu, psum, 8);
+          const float pe = (sc == -INFINITY) ? 0.f : exp2f(sc - mine_m);
+          float psum = pe;
+#pragma unroll
+          for (int off = 16; off >= (1 << (5 - Cfg::LOGT)); off >>= 1)
+            psum += __shfl_xor_sync(0xffffffffu, psum, off);
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             const float ps = __shfl_sync(0xffffffffu, psum, g << (5 - LOGNV));
             l[g] = l[g] * alpha[g] + ps;
             m[g] = mnew[g];
+            if (alpha[g] != 1.f) {  // warp-uniform: every lane holds the same alpha
+              const float2 a2 = make_float2(alpha[g], alpha[g]);
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) o[g][e] *= alpha[g];
+              for (int e = 0; e < P2; ++e) o[g][e] = __fmul2_rn(o[g][e], a2);
+            }
           }
           // P.V for this warp's tokens.
 #pragma unroll
-          for (int i = 0; i < Cfg::TPW; ++i) {
+          for (int i = 0; i < TPW; ++i) {
             const int t = tp + Cfg::TS * i;
-            float pw[G];
+            float2 pw[G];
 #pragma unroll
-            for (int g = 0; g < G; ++g)
-              pw[g] = __shfl_sync(0xffffffffu, pe, (i * G + g) << (5 - LOGNV));
+            for (int g = 0; g < G; ++g) {
+              const float x = __shfl_sync(0xffffffffu, pe, (i * G + g) << (5 - LOGNV));
+              pw[g] = make_float2(x, x);
+            }
             if (t < ntok) {
 #pragma unroll
               for (int j = 0; j < CH; ++j) {
@@ -301,12 +311,10 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads,
                 const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                  const float v0 = bf16lo(ww[e]), v1 = bf16hi(ww[e]);
+                  const float2 v2 = make_float2(bf16lo(ww[e]), bf16hi(ww[e]));
 #pragma unroll
-                  for (int g = 0; g < G; ++g) {
-                    o[g][8 * j + 2 * e] = fmaf(pw[g], v0, o[g][8 * j + 2 * e]);
-                    o[g][8 * j + 2 * e + 1] = fmaf(pw[g], v1, o[g][8 * j + 2 * e + 1]);
-                  }
+                  for (int g = 0; g < G; ++g)
+                    o[g][4 * j + e] = __ffma2_rn(pw[g], v2, o[g][4 * j + e]);
                 }
               }
             }
@@ -331,35 +339,41 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads,
         for (int g = 0; g < G; ++g)
 #pragma unroll
           for (int j = 0; j < CH; ++j) {
-            float4 *dst = reinterpret_cast<float4 *>(mine + Cfg::MHDR + g * D + 256 * j + 8 * lane);
-            dst[0] = make_float4(o[g][8 * j], o[g][8 * j + 1], o[g][8 * j + 2], o[g][8 * j + 3]);
-            dst[1] =
-                make_float4(o[g][8 * j + 4], o[g][8 * j + 5], o[g][8 * j + 6], o[g][8 * j + 7]);
+            float4 *dst =
+                reinterpret_cast<float4 *>(mine + Cfg::MHDR + g * D + 256 * j + 8 * lane);
+            dst[0] = make_float4(o[g][4 * j].x, o[g][4 * j].y, o[g][4 * j + 1].x,
+                                 o[g][4 * j + 1].y);
+            dst[1] = make_float4(o[g][4 * j + 2].x, o[g][4 * j + 2].y, o[g][4 * j + 3].x,
+                                 o[g][4 * j + 3].y);
           }
         named_bar_sync(1, Cfg::kComputeWarps * 32);
         if (tp == 0) {
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             float M = -INFINITY;
-            for (int k = 0; k < Cfg::TS; ++k) M = fmaxf(M, merge[(kvh + HKV * k) * Cfg::MSTRIDE + g]);
+            for (int k = 0; k < Cfg::TS; ++k)
+              M = fmaxf(M, merge[(kvh + HKV * k) * Cfg::MSTRIDE + g]);
             float Ls = 0.f;
             float wk[Cfg::TS];
 #pragma unroll
             for (int k = 0; k < Cfg::TS; ++k) {
               const float *src = merge + (kvh + HKV * k) * Cfg::MSTRIDE;
-              wk[k] = (src[g] == -INFINITY) ? 0.f : fast_exp2(src[g] - M);
+              wk[k] = (src[g] == -INFINITY) ? 0.f : exp2f(src[g] - M);
               Ls += src[4 + g] * wk[k];
             }
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) o[g][e] = 0.f;
+            for (int e = 0; e < P2; ++e) o[g][e] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int k = 0; k < Cfg::TS; ++k) {
               const float *src = merge + (kvh + HKV * k) * Cfg::MSTRIDE + Cfg::MHDR + g * D;
+              const float2 w2 = make_float2(wk[k], wk[k]);
 #pragma unroll
               for (int j = 0; j < CH; ++j)
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                  o[g][8 * j + e] = fmaf(wk[k], src[256 * j + 8 * lane + e], o[g][8 * j + e]);
+                for (int e = 0; e < 4; ++e)
+                  o[g][4 * j + e] = __ffma2_rn(
+                      w2, *reinterpret_cast<const float2 *>(src + 256 * j + 8 * lane + 2 * e),
+                      o[g][4 * j + e]);
             }
             m[g] = M;
             l[g] = Ls;
@@ -382,10 +396,10 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads,
 #pragma unroll
             for (int j = 0; j < CH; ++j) {
               uint4 w;
-              w.x = pack_bf16x2(o[g][8 * j] * inv, o[g][8 * j + 1] * inv);
-              w.y = pack_bf16x2(o[g][8 * j + 2] * inv, o[g][8 * j + 3] * inv);
-              w.z = pack_bf16x2(o[g][8 * j + 4] * inv, o[g][8 * j + 5] * inv);
-              w.w = pack_bf16x2(o[g][8 * j + 6] * inv, o[g][8 * j + 7] * inv);
+              w.x = pack_bf16x2(o[g][4 * j].x * inv, o[g][4 * j].y * inv);
+              w.y = pack_bf16x2(o[g][4 * j + 1].x * inv, o[g][4 * j + 1].y * inv);
+              w.z = pack_bf16x2(o[g][4 * j + 2].x * inv, o[g][4 * j + 2].y * inv);
+              w.w = pack_bf16x2(o[g][4 * j + 3].x * inv, o[g][4 * j + 3].y * inv);
               *reinterpret_cast<uint4 *>(dst + 256 * j + 8 * lane) = w;
             }
             if (lane == 0 && p.lse != nullptr)
@@ -395,10 +409,10 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads,
 #pragma unroll
             for (int j = 0; j < CH; ++j) {
               float4 *d4 = reinterpret_cast<float4 *>(dst + 256 * j + 8 * lane);
-              d4[0] = make_float4(o[g][8 * j] * inv, o[g][8 * j + 1] * inv, o[g][8 * j + 2] * inv,
-                                  o[g][8 * j + 3] * inv);
-              d4[1] = make_float4(o[g][8 * j + 4] * inv, o[g][8 * j + 5] * inv,
-                                  o[g][8 * j + 6] * inv, o[g][8 * j + 7] * inv);
+              d4[0] = make_float4(o[g][4 * j].x * inv, o[g][4 * j].y * inv,
+                                  o[g][4 * j + 1].x * inv, o[g][4 * j + 1].y * inv);
+              d4[1] = make_float4(o[g][4 * j + 2].x * inv, o[g][4 * j + 2].y * inv,
+                                  o[g][4 * j + 3].x * inv, o[g][4 * j + 3].y * inv);
             }
             if (lane == 0) p.ws_lse[slot * p.n_q_heads + h] = lse_v;
           }

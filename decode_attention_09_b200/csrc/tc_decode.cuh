@@ -7,20 +7,34 @@
 // products run on tcgen05 with the accumulators in tensor memory (TMEM):
 //
 //   S^T[64 tok x 16 h]  = K_tile[64 x 512] . Q^T[512 x 16]   (M=64, N=16, K=512)
-//   O^T[512 d x 16 h]   = V_tile^T[512 x 64] . P^T[64 x 16]  (M=128 x4, N=16, K=64)
+//   O^T[512 d x 32]    += V_tile^T[512 x 64] . P^T[64 x 32]  (M=128 x4, N=32, K=64)
+//
+// The weights are bf16 operands (A and B of one MMA share a type, and V is
+// bf16), so each weight p is split into p_hi = bf16(p) and p_lo = bf16(p - p_hi):
+// the 32 columns of P^T are the 16 heads' p_hi then their p_lo, and O^T for a head
+// is the sum of its two column blocks.  That keeps the weights to ~2^-17
+// relative error instead of 2^-9, which matters when a few large key rows
+// dominate the weighted sum of values.
 //
 // K = V: the one 64-token tile in shared memory is the K-major A operand of the
 // first product and the MN-major A operand of the second, so each cache byte
 // crosses HBM once.  The tile arrives by TMA as eight 64x64 boxes with 128-byte
-// swizzle, which is the canonical operand layout for both majors.
+// swizzle, the canonical operand layout for both majors.
+//
+// Softmax with a lazily moved reference: P = exp2(s - m_ref) with m_ref a
+// running per-head reference that only moves when some score exceeds it by more
+// than 2^kTau.  Until then O^T keeps accumulating in TMEM across tiles and the
+// row sums stay in per-thread registers, so a tile costs one TMEM load of S, one
+// barrier-with-vote and the P^T stores.  When the reference must move, the tile's
+// exact per-head max is reduced, O^T in TMEM and the partial sums are rescaled
+// by exp2(m_old - m_new), and the tile proceeds.  The result is exact: out is
+// O/L and LSE is m_ref + log2 L for the final reference.
 //
 // Warp roles (192 threads): warp 0 issues TMA loads; warp 1 owns TMEM and issues
-// MMAs (one elected lane); warps 2-5 read S from TMEM, run the online softmax
-// (running max / sum per head), write P^T (bf16) to shared memory, and fold each
-// tile's O^T into fp32 registers with the rescale factor.  S and O^T are double
-// buffered in TMEM so the tensor core computes tile i+1 while tile i's softmax
-// runs.  Every wait is bounded; on a timeout all roles fast-forward, drain
-// their copies / MMAs and free TMEM.
+// MMAs (one elected lane); warps 2-5 run the softmax (TMEM sub-partition
+// warp % 4).  S is double buffered in TMEM so the tensor core computes tile i+1
+// while tile i's softmax runs.  Every wait is bounded; on a timeout all roles
+// fast-forward, drain their copies / MMAs and free TMEM.
 #pragma once
 
 #include <cstdint>
@@ -32,7 +46,6 @@
 namespace gdattn {
 
 struct TcParams {
-  const uint16_t *q;      // [B, Hq, D] (through qmap; pointer kept for reference)
   uint16_t *out;          // [B, Hq, D]
   float *lse;             // [B, Hq] or null
   float *ws_o;            // partial outputs [slots][16][D]
@@ -52,17 +65,21 @@ struct TcConfig {
   static constexpr int BOXB = TILE * 128;             // one 64-token x 64-d box
   static constexpr int STAGEB = BOXB * (D / 64);      // 64 KiB
   static constexpr int QB = G * D * 2;                // 16 KiB
-  static constexpr int PB = G * TILE * 2;             // 2 KiB per P buffer
+  static constexpr int PB = 2 * G * TILE * 2;         // 4 KiB per P buffer (hi, lo)
   static constexpr int OFF_Q = NST * STAGEB;
   static constexpr int OFF_P = OFF_Q + QB;
   static constexpr int OFF_BAR = OFF_P + 2 * PB;
   static constexpr int OFF_RED = OFF_BAR + 256;
-  static constexpr int SMEM = OFF_RED + 2 * 2 * 4 * G * 4 + 1024;
+  static constexpr int SMEM = OFF_RED + 2 * 4 * G * 4 + 1024;
   static constexpr int kThreads = 192;
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t S_COL = 0;                // 2 x 16 columns
-  static constexpr uint32_t O_COL = 64;               // 2 x 64 columns
+  static constexpr uint32_t O_COL = 128;              // 4 d-blocks x (16 hi + 16 lo) columns
 };
+
+// The reference max moves when a score exceeds it by more than 2^kTau, so the
+// weights stay below 256: no overflow in bf16 P, fp32 sums or O.
+constexpr float kTau = 8.f;
 
 // Tiles of one CTA, in order, across its segments.
 struct TileIter {
@@ -71,12 +88,10 @@ struct TileIter {
   SlotRuns runs;
   int32_t run, t0;
   bool have_seg;
-  int32_t seg_index;
 
   __device__ __forceinline__ void init(const Geometry &g, const ChunkPlan &p) {
     seg_it.init(g, p);
     have_seg = false;
-    seg_index = -1;
   }
   // Yields the next tile: slot row of its first token, valid token count, and
   // whether it opens / closes its segment.
@@ -90,7 +105,6 @@ struct TileIter {
       t0 = 0;
       have_seg = true;
       first = true;
-      ++seg_index;
     }
     row = runs.start(run) + t0;
     ntok = min(TcConfig::TILE, runs.len(run) - t0);
@@ -104,6 +118,27 @@ struct TileIter {
     return true;
   }
 };
+
+// Reduce 16 per-lane values over the warp (op = max or sum): after it, lane l
+// holds the reduction for value index (l >> 1) & 15.
+template <bool MAX>
+__device__ __forceinline__ float warp_reduce_scatter16(float (&r)[16], int lane) {
+#pragma unroll
+  for (int lev = 0; lev < 4; ++lev) {
+    const int off = 16 >> lev, half = 8 >> lev;
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (k < half) {
+        const float send = upper ? r[k] : r[k + half];
+        const float keep = upper ? r[k + half] : r[k];
+        const float got = __shfl_xor_sync(0xffffffffu, send, off);
+        r[k] = MAX ? fmaxf(keep, got) : keep + got;
+      }
+  }
+  const float got = __shfl_xor_sync(0xffffffffu, r[0], 1);
+  return MAX ? fmaxf(r[0], got) : r[0] + got;
+}
 
 __global__ void __launch_bounds__(TcConfig::kThreads, 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -122,16 +157,17 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
   uint64_t *empty = bars + 3;       // [NST]  MMA -> TMA
   uint64_t *qfull = bars + 6;       // TMA -> MMA
   uint64_t *qempty = bars + 7;      // MMA -> TMA
-  uint64_t *sfull = bars + 8;       // [2] MMA -> softmax
+  uint64_t *sfull = bars + 8;       // [2] MMA -> softmax (S of tile i in buffer i & 1)
   uint64_t *sempty = bars + 10;     // [2] softmax -> MMA
-  uint64_t *pfull = bars + 12;      // [2] softmax -> MMA
-  uint64_t *ofull = bars + 14;      // [2] MMA -> softmax
-  uint64_t *oempty = bars + 16;     // [2] softmax -> MMA
-  uint64_t *drain = bars + 18;
-  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 19);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 20);
-  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 21);  // 48 bytes, ends before +256
-  float *red = reinterpret_cast<float *>(smem + Cfg::OFF_RED);  // [2 kinds][2 buf][4 warps][16]
+  uint64_t *pfull = bars + 12;      // [2] softmax -> MMA (P of tile i in buffer i & 1)
+  uint64_t *ofull = bars + 14;      // [2] MMA -> softmax: P.V of tile i done (barrier i & 1)
+  uint64_t *oempty = bars + 16;     // softmax -> MMA: O of a finished segment read out
+  uint64_t *drain = bars + 17;
+  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 18);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 19);
+  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 20);  // 48 bytes, ends before +256
+  float *redmax = reinterpret_cast<float *>(smem + Cfg::OFF_RED);  // [4 warps][16]
+  float *redsum = redmax + 4 * G;                                  // [4 warps][16]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -149,8 +185,8 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
       mbar_init(&sempty[s], 4);
       mbar_init(&pfull[s], 4);
       mbar_init(&ofull[s], 1);
-      mbar_init(&oempty[s], 4);
     }
+    mbar_init(oempty, 4);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -206,7 +242,8 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
           const int32_t qrow = it.seg.b * p.n_q_heads + it.seg.x * G;
           mbar_arrive_expect_tx(qfull, Cfg::QB);
 #pragma unroll
-          for (int j = 0; j < D / 64; ++j) tma_load_2d(qs + j * (G * 128), &qmap, 64 * j, qrow, qfull);
+          for (int j = 0; j < D / 64; ++j)
+            tma_load_2d(qs + j * (G * 128), &qmap, 64 * j, qrow, qfull);
           ++nseg;
         }
         const int st = i % NST;
@@ -231,21 +268,23 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
     // -------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(64, 16, false, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 16, true, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 32, true, false);
       const uint32_t st_addr = smem_u32(stages);
       const uint32_t q_addr = smem_u32(qs);
       const uint32_t p_addr = smem_u32(ps);
       bool ok = true;
       uint32_t i = 0, nseg = 0;
-      int32_t prev = -1;  // tile whose P.V is still to issue
+      int32_t prev = -1;       // tile whose P.V is still to issue
+      bool prev_first = false; // ... and whether it opened its segment
+      uint32_t prev_seg = 0;   // ... and that segment's index in this CTA
       TileIter it;
       it.init(p.geo, *plan);
       int32_t row, ntok;
       bool first, last;
-      auto issue_pv = [&](uint32_t t) -> bool {
-        const int pb = t & 1, ob = t & 1;
-        if (!mbar_wait(&pfull[pb], (t >> 1) & 1, abort_flag, p.status)) return false;
-        if (t >= 2 && !mbar_wait(&oempty[ob], ((t >> 1) - 1) & 1, abort_flag, p.status))
+      auto issue_pv = [&](uint32_t t, bool seg_first, uint32_t seg) -> bool {
+        if (!mbar_wait(&pfull[t & 1], (t >> 1) & 1, abort_flag, p.status)) return false;
+        // A segment's first P.V overwrites O: the previous segment must be read out.
+        if (seg_first && seg > 0 && !mbar_wait(oempty, (seg - 1) & 1, abort_flag, p.status))
           return false;
         tc_fence_after();
         const uint32_t a0 = st_addr + (t % NST) * Cfg::STAGEB;
@@ -253,22 +292,24 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
         for (int jb = 0; jb < 4; ++jb) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = smem_desc_sw128(a0 + (2 * jb) * Cfg::BOXB + kk * 2048, Cfg::BOXB, 1024);
-            const uint64_t bd = smem_desc_sw128(p_addr + pb * Cfg::PB + kk * 32, 16, 1024);
-            tc_mma_bf16(tmem + Cfg::O_COL + ob * 64 + jb * 16, ad, bd, idesc_pv, kk > 0);
+            const uint64_t ad =
+                smem_desc_sw128(a0 + (2 * jb) * Cfg::BOXB + kk * 2048, Cfg::BOXB, 1024);
+            const uint64_t bd = smem_desc_sw128(p_addr + (t & 1) * Cfg::PB + kk * 32, 16, 1024);
+            tc_mma_bf16(tmem + Cfg::O_COL + jb * 32, ad, bd, idesc_pv, !(seg_first && kk == 0));
           }
         }
-        tc_commit(&ofull[ob]);
+        tc_commit(&ofull[t & 1]);
         tc_commit(&empty[t % NST]);
         return true;
       };
+      uint32_t cur_seg = 0;
       while (ok && it.next(C, row, ntok, first, last)) {
         if (first) {
           if (!mbar_wait(qfull, nseg & 1, abort_flag, p.status)) {
             ok = false;
             break;
           }
-          ++nseg;
+          cur_seg = nseg++;
         }
         const int st = i % NST, sb = i & 1;
         if (!mbar_wait(&full[st], (i / NST) & 1, abort_flag, p.status)) {
@@ -292,14 +333,16 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
         }
         tc_commit(&sfull[sb]);
         if (last) tc_commit(qempty);
-        if (prev >= 0 && !issue_pv(static_cast<uint32_t>(prev))) {
+        if (prev >= 0 && !issue_pv(static_cast<uint32_t>(prev), prev_first, prev_seg)) {
           ok = false;
           break;
         }
         prev = static_cast<int32_t>(i);
+        prev_first = first;
+        prev_seg = cur_seg;
         ++i;
       }
-      if (ok && prev >= 0) ok = issue_pv(static_cast<uint32_t>(prev));
+      if (ok && prev >= 0) ok = issue_pv(static_cast<uint32_t>(prev), prev_first, prev_seg);
       // Drain: wait until every issued MMA has completed before TMEM is freed.
       tc_commit(drain);
       volatile int no_abort = 0;
@@ -310,95 +353,38 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
     const int qd = warp & 3;                 // TMEM sub-partition: lanes 32*qd ..
     const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
     const int tok = 16 * qd + lane;          // tile token held by this lane (lane < 16)
-    float acc[4][G];
-    float m[G], l[G], alpha_prev[G], m_fin[G], l_fin[G];
+    float m_ref[G], lpart[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      m[h] = -INFINITY;
-      l[h] = 0.f;
-      m_fin[h] = -INFINITY;
-      l_fin[h] = 1.f;
-      alpha_prev[h] = 0.f;
-#pragma unroll
-      for (int jb = 0; jb < 4; ++jb) acc[jb][h] = 0.f;
+      m_ref[h] = -INFINITY;
+      lpart[h] = 0.f;
     }
     bool ok = true;
+    uint32_t cons[2] = {0u, 0u};  // ofull phases consumed per barrier
+    // Wait until the P.V of tile t has completed.  Phases are consumed in order
+    // and never lag by two, so the parity waits cannot alias.
+    auto ensure_pv = [&](uint32_t t) {
+      const uint32_t b = t & 1, ph = t >> 1;
+      if (cons[b] <= ph) {
+        if (ok && !mbar_wait(&ofull[b], cons[b] & 1, abort_flag, p.status)) ok = false;
+        ++cons[b];
+      }
+      ok = __all_sync(0xffffffffu, ok);
+    };
     uint32_t i = 0;
     TileIter it;
     it.init(p.geo, *plan);
     int32_t row, ntok;
     bool first, last;
-    bool prev_last = false;
-    Segment prev_seg;
-    prev_seg.b = 0;
-
-    auto correction = [&](uint32_t t) {
-      const int ob = t & 1;
-      if (ok && !mbar_wait(&ofull[ob], (t >> 1) & 1, abort_flag, p.status)) ok = false;
-      ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
-      if (ok) {
-        tc_fence_after();
-#pragma unroll
-        for (int jb = 0; jb < 4; ++jb) {
-          float v[16];
-          tmem_ld16(tmem + lane_base + Cfg::O_COL + ob * 64 + jb * 16, v);
-#pragma unroll
-          for (int h = 0; h < G; ++h) acc[jb][h] = fmaf(acc[jb][h], alpha_prev[h], v[h]);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&oempty[ob]);
-      }
-    };
-
-    auto finalize = [&](const Segment &s) {
-      if (!ok) return;
-      int32_t cf, cl;
-      unit_chunks(s.unit_start, s.n, plan->chunk, cf, cl);
-      const bool single = (cf == cl);
-      const int64_t slot = static_cast<int64_t>(c) + s.unit;
-      const int h0 = s.x * G;
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float inv = 1.f / l_fin[h];
-#pragma unroll
-        for (int jb = 0; jb < 4; ++jb) {
-          const int d = 128 * jb + 32 * qd + lane;
-          const float val = acc[jb][h] * inv;
-          if (single)
-            p.out[(static_cast<int64_t>(s.b) * p.n_q_heads + h0 + h) * D + d] = f32_to_bf16_rn(val);
-          else
-            p.ws_o[(slot * G + h) * D + d] = val;
-        }
-      }
-      if (qd == 0 && lane < G) {
-        float mf_l = m_fin[0], lf_l = l_fin[0];
-#pragma unroll
-        for (int h = 1; h < G; ++h)
-          if (lane == h) {
-            mf_l = m_fin[h];
-            lf_l = l_fin[h];
-          }
-        const float lse_v = (mf_l + log2f(lf_l)) * 0.69314718055994530942f;
-        if (single) {
-          if (p.lse != nullptr) p.lse[static_cast<int64_t>(s.b) * p.n_q_heads + h0 + lane] = lse_v;
-        } else {
-          p.ws_lse[slot * G + lane] = lse_v;
-        }
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int jb = 0; jb < 4; ++jb) acc[jb][h] = 0.f;
-    };
 
     while (it.next(C, row, ntok, first, last)) {
-      const int sb = i & 1, pb = i & 1, buf = i & 1;
+      const int sb = i & 1, pb = i & 1;
+      if (i >= 2) ensure_pv(i - 2);  // P buffer pb is free again
       if (first) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          m[h] = -INFINITY;
-          l[h] = 0.f;
+          m_ref[h] = -INFINITY;
+          lpart[h] = 0.f;
         }
       }
       // --- scores of tile i
@@ -413,108 +399,135 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
         if (lane == 0) mbar_arrive(&sempty[sb]);
       }
       const bool valid = ok && lane < 16 && tok < ntok;
+      bool need = false;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         float x = s[h] * p.qscale;
         if (p.post != 0.f) x = p.post * tanhf(x);
         s[h] = valid ? x : -INFINITY;
+        need |= s[h] > m_ref[h] + kTau;
       }
-      // --- per-head tile max: reduce-scatter over the warp, then across warps
-      float r[16];
+      // --- move the reference only when some score outgrew it
+      if (named_bar_or(1, 128, need)) {
+        float r[16];
 #pragma unroll
-      for (int h = 0; h < 16; ++h) r[h] = s[h];
+        for (int h = 0; h < 16; ++h) r[h] = s[h];
+        const float tm = warp_reduce_scatter16<true>(r, lane);
+        if ((lane & 1) == 0) redmax[qd * G + (lane >> 1)] = tm;
+        named_bar_sync(1, 128);
+        float alpha[G];
 #pragma unroll
-      for (int lev = 0; lev < 4; ++lev) {
-        const int off = 16 >> lev, half = 8 >> lev;
-        const bool upper = (lane & off) != 0;
+        for (int h = 0; h < G; ++h) {
+          const float t = fmaxf(fmaxf(redmax[h], redmax[G + h]),
+                                fmaxf(redmax[2 * G + h], redmax[3 * G + h]));
+          const float mn = fmaxf(m_ref[h], t);
+          alpha[h] = (m_ref[h] == -INFINITY) ? 0.f : exp2f(m_ref[h] - mn);
+          m_ref[h] = mn;
+          lpart[h] *= alpha[h];
+        }
+        if (!first) {
+          // O holds tiles < i: wait for the last of them, then rescale it in TMEM.
+          ensure_pv(i - 1);
+          if (ok) {
+            tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          if (k < half) {
-            const float send = upper ? r[k] : r[k + half];
-            const float keep = upper ? r[k + half] : r[k];
-            r[k] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, off));
+            for (int cb = 0; cb < 8; ++cb) {  // 4 d-blocks x (hi, lo)
+              float v[16];
+              tmem_ld16(tmem + lane_base + Cfg::O_COL + cb * 16, v);
+#pragma unroll
+              for (int h = 0; h < G; ++h) v[h] *= alpha[h];
+              tmem_st16_wait(tmem + lane_base + Cfg::O_COL + cb * 16, v);
+            }
           }
+        }
       }
-      r[0] = fmaxf(r[0], __shfl_xor_sync(0xffffffffu, r[0], 1));
-      float *redmax = red + (0 * 2 + buf) * 4 * G;
-      float *redsum = red + (1 * 2 + buf) * 4 * G;
-      if ((lane & 1) == 0) redmax[qd * G + (lane >> 1)] = r[0];
-      named_bar_sync(1, 128);
-      float mnew[G], alpha[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float tm = fmaxf(fmaxf(redmax[h], redmax[G + h]), fmaxf(redmax[2 * G + h], redmax[3 * G + h]));
-        mnew[h] = fmaxf(m[h], tm);
-        alpha[h] = (mnew[h] == -INFINITY) ? 1.f : exp2f(m[h] - mnew[h]);
-        m[h] = mnew[h];
-      }
-      // --- probabilities, P^T (bf16, 128B-swizzled K-major) and row sums
+      // --- weights, P^T (bf16 hi / lo rows, 128B-swizzled K-major), row sums
       uint8_t *prow = ps + pb * Cfg::PB;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float pe = (s[h] == -INFINITY) ? 0.f : exp2f(s[h] - mnew[h]);
-        r[h] = pe;
+        const float pe = (s[h] == -INFINITY) ? 0.f : exp2f(s[h] - m_ref[h]);
+        lpart[h] += pe;
         if (lane < 16) {
-          const uint32_t off = h * 128 + ((((tok >> 3) ^ (h & 7)) & 7) << 4) + (tok & 7) * 2;
-          *reinterpret_cast<uint16_t *>(prow + off) = f32_to_bf16_rn(pe);
+          const uint16_t hi = f32_to_bf16_rn(pe);
+          const uint16_t lo = f32_to_bf16_rn(pe - __uint_as_float(static_cast<uint32_t>(hi) << 16));
+          const uint32_t col = (tok & 7) * 2;
+          const uint32_t chunk = tok >> 3;
+          *reinterpret_cast<uint16_t *>(prow + h * 128 + (((chunk ^ h) & 7) << 4) + col) = hi;
+          *reinterpret_cast<uint16_t *>(prow + (G + h) * 128 + (((chunk ^ (G + h)) & 7) << 4) +
+                                        col) = lo;
         }
       }
       if (ok && ntok < Cfg::TILE) {
         // Rows past the attended range hold other cache contents (possibly
         // NaN); they get weight 0, but 0 * NaN would still reach O, so clear them.
         uint8_t *tile = stages + (i % NST) * Cfg::STAGEB;
-        const int nchunk = (Cfg::TILE - ntok) * 8 * (D / 64);
-        for (int e = threadIdx.x - 64; e < nchunk; e += 128) {
-          const int box = e / ((Cfg::TILE - ntok) * 8);
-          const int rem = e - box * ((Cfg::TILE - ntok) * 8);
-          const int rrow = ntok + (rem >> 3);
-          *reinterpret_cast<uint4 *>(tile + box * Cfg::BOXB + rrow * 128 + (rem & 7) * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
+        const int per_box = (Cfg::TILE - ntok) * 8;
+        for (int e = threadIdx.x - 64; e < per_box * (D / 64); e += 128) {
+          const int box = e / per_box;
+          const int rem = e - box * per_box;
+          *reinterpret_cast<uint4 *>(tile + box * Cfg::BOXB + (ntok + (rem >> 3)) * 128 +
+                                     (rem & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
       fence_proxy_async_smem();
-#pragma unroll
-      for (int lev = 0; lev < 4; ++lev) {
-        const int off = 16 >> lev, half = 8 >> lev;
-        const bool upper = (lane & off) != 0;
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          if (k < half) {
-            const float send = upper ? r[k] : r[k + half];
-            const float keep = upper ? r[k + half] : r[k];
-            r[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-          }
-      }
-      r[0] += __shfl_xor_sync(0xffffffffu, r[0], 1);
-      if ((lane & 1) == 0) redsum[qd * G + (lane >> 1)] = r[0];
+      tc_fence_before();
       __syncwarp();
       if (ok && lane == 0) mbar_arrive(&pfull[pb]);
-      named_bar_sync(1, 128);
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-        l[h] = l[h] * alpha[h] + ((redsum[h] + redsum[G + h]) + (redsum[2 * G + h] + redsum[3 * G + h]));
 
-      // --- fold the previous tile's O^T, then close its segment if it ended
-      if (i > 0) {
-        correction(i - 1);
-        if (prev_last) finalize(prev_seg);
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h) alpha_prev[h] = alpha[h];
-      prev_last = last;
-      prev_seg = it.seg;
       if (last) {
+        // --- segment end: all of its P.V done, read O out
+        if (i >= 1) ensure_pv(i - 1);
+        ensure_pv(i);
+        float r[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) r[h] = lpart[h];
+        const float ls = warp_reduce_scatter16<false>(r, lane);
+        if ((lane & 1) == 0) redsum[qd * G + (lane >> 1)] = ls;
+        named_bar_sync(1, 128);
+        const Segment &sg = it.seg;
+        int32_t cf, cl;
+        unit_chunks(sg.unit_start, sg.n, plan->chunk, cf, cl);
+        const bool single = (cf == cl);
+        const int64_t slot = static_cast<int64_t>(c) + sg.unit;
+        const int h0 = sg.x * G;
+        float inv[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          m_fin[h] = m[h];
-          l_fin[h] = l[h];
+          const float L = (redsum[h] + redsum[G + h]) + (redsum[2 * G + h] + redsum[3 * G + h]);
+          inv[h] = 1.f / L;
+          if (ok && qd == 0 && lane == h) {
+            const float lse_v = (m_ref[h] + log2f(L)) * 0.69314718055994530942f;
+            if (single) {
+              if (p.lse != nullptr) p.lse[static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + h] = lse_v;
+            } else {
+              p.ws_lse[slot * G + h] = lse_v;
+            }
+          }
+        }
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int jb = 0; jb < 4; ++jb) {
+            float v[16], w[16];
+            tmem_ld16(tmem + lane_base + Cfg::O_COL + jb * 32, v);
+            tmem_ld16(tmem + lane_base + Cfg::O_COL + jb * 32 + 16, w);
+            const int d = 128 * jb + 32 * qd + lane;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const float val = (v[h] + w[h]) * inv[h];
+              if (single)
+                p.out[(static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + h) * D + d] =
+                    f32_to_bf16_rn(val);
+              else
+                p.ws_o[(slot * G + h) * D + d] = val;
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(oempty);
         }
       }
       ++i;
-    }
-    if (i > 0) {
-      correction(i - 1);
-      if (prev_last) finalize(prev_seg);
     }
   }
 

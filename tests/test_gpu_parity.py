@@ -153,18 +153,30 @@ def test_unattended_slots_never_matter(name):
 
 @pytest.mark.parametrize("which", ["single_sliding", "single_global"])
 def test_split_count_invariance(which):
-    """One CTA or many: same result to fp32 rounding (one bf16 ulp on out)."""
+    """One CTA or many: the same result up to rounding.
+
+    The CUDA-core path keeps the softmax weights in fp32, so only the last bf16
+    rounding of out may differ (one ulp).  The tensor-core path rounds each
+    weight p = exp(s - m) to bf16 against the running max m, which depends on
+    where the range is cut; a weight's relative error is up to 2^-9, so two
+    splits may differ by ~2^-8 * max|v| in the worst case: gate at 4e-3, half
+    the oracle gate.
+    """
     require_gpu()
     w = getattr(workloads, which)()
     inp = workloads.workload_layer_inputs(w, 0)
     o1, l1 = GpuLayer(inp, split_ctas=1).run()
+    tensor_path = inp.spec.group == 16
     for split in (2, 5, 148, 296):
         o2, l2 = GpuLayer(inp, split_ctas=split).run()
         d = (o1.float() - o2.float()).abs()
-        ulp = torch.from_numpy(np.exp2(np.floor(np.log2(np.maximum(
-            o1.float().abs().cpu().numpy(), 1e-30))) - 7)).to(d.device)
-        assert bool((d <= ulp + 1e-12).all()), f"split {split}: max {d.max().item()}"
-        assert (l1 - l2).abs().max().item() <= 2e-5
+        if tensor_path:
+            tol = torch.full_like(d, 4e-3)
+        else:
+            tol = torch.from_numpy(np.exp2(np.floor(np.log2(np.maximum(
+                o1.float().abs().cpu().numpy(), 1e-30))) - 7)).to(d.device) + 1e-12
+        assert bool((d <= tol).all()), f"split {split}: max {d.max().item()}"
+        assert (l1 - l2).abs().max().item() <= (1e-4 if tensor_path else 2e-5)
 
 
 def test_bitwise_reproducible():
