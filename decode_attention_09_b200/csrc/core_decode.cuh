@@ -44,31 +44,35 @@ struct CoreParams {
 
 template <int D, int G, int HKV, bool SHARED>
 struct CoreConfig {
-  static constexpr int kComputeWarps = 8;
-  static constexpr int kThreads = (kComputeWarps + 1) * 32;
   static constexpr int NT = SHARED ? 1 : 2;
+  static constexpr int MHDR = 8;                      // per-warp merge header (m[G], l[G])
+  static constexpr int MSTRIDE = MHDR + G * D;        // floats per warp, 16-byte multiple
+  // 16 compute warps (two or more per KV head) hide latency better; 8 when the
+  // cross-warp merge area for 16 would not fit beside the ring.
+  static constexpr int kComputeWarps = (16 * MSTRIDE * 4 <= 40 * 1024) ? 16 : 8;
+  static constexpr int kThreads = (kComputeWarps + 1) * 32;
   static constexpr int TS = kComputeWarps / HKV;      // warps sharing one KV head
-  static constexpr int TPW = (D * NT <= 512) ? 8 : 4; // tokens per warp per stage
+  static constexpr int ROWB = HKV * D * 2;            // bytes of one token row (one tensor)
+  // Tokens per warp per stage: the largest of 8, 4, 2 that keeps a stage <= 64 KiB.
+  static constexpr int TPW = (TS * 8 * ROWB * NT <= 65536) ? 8
+                             : (TS * 4 * ROWB * NT <= 65536) ? 4 : 2;
   static constexpr int T = TS * TPW;                  // tokens per stage
   static constexpr int EPL = D / 32;                  // elements per lane
   static constexpr int CH = EPL / 8;                  // 16-byte chunks per lane
-  static constexpr int ROWB = HKV * D * 2;            // bytes of one token row (one tensor)
   static constexpr int STAGEB = T * ROWB * NT;
-  static constexpr int MHDR = 8;                      // per-warp merge header (m[G], l[G])
-  static constexpr int MSTRIDE = MHDR + G * D;        // floats per warp, 16-byte multiple
   static constexpr int MERGEB = TS > 1 ? kComputeWarps * MSTRIDE * 4 : 0;
   // Stages: up to 192 KiB of ring, within what the merge area leaves.
   static constexpr int RING = (220 * 1024 - MERGEB) < 196608 ? (220 * 1024 - MERGEB) : 196608;
   static constexpr int NSTAGE = (RING / STAGEB) < 2 ? 2 : (RING / STAGEB > 8 ? 8 : RING / STAGEB);
   static constexpr int NV = TPW * G;                  // scores per warp per stage
-  static constexpr int LOGNV = NV == 4 ? 2 : (NV == 8 ? 3 : (NV == 16 ? 4 : 5));
+  static constexpr int LOGNV = NV == 2 ? 1 : NV == 4 ? 2 : (NV == 8 ? 3 : (NV == 16 ? 4 : 5));
   static constexpr int LOGG = G == 1 ? 0 : (G == 2 ? 1 : 2);
-  static constexpr int LOGT = TPW == 4 ? 2 : 3;
+  static constexpr int LOGT = TPW == 2 ? 1 : (TPW == 4 ? 2 : 3);
   static constexpr int SMEM = NSTAGE * STAGEB + 2 * NSTAGE * 8 + 128 + MERGEB + 1024;
   static_assert(HKV == 1 || HKV == 2 || HKV == 4 || HKV == 8, "HKV");
   static_assert(G == 1 || G == 2 || G == 4, "G");
   static_assert(D == 256 || D == 512, "D");
-  static_assert(NV <= 32, "one score per lane at most");
+  static_assert(NV >= 2 && NV <= 32, "one score per lane at most");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -127,39 +131,43 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads, 1)
 
   if (warp == Cfg::kComputeWarps) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint64_t pol = l2_evict_first_policy();
-      uint32_t fills = 0;
-      bool ok = true;
-      SegmentIter it;
-      it.init(p.geo, *plan);
-      Segment s;
-      while (ok && it.next(s)) {
-        const SlotRuns runs = segment_runs(s, C);
-        for (int r = 0; ok && r < runs.count; ++r) {
-          for (int32_t t0 = 0; t0 < runs.len(r); t0 += T) {
-            const int ntok = min(T, runs.len(r) - t0);
-            const int st = fills % NSTAGE;
-            if (fills >= NSTAGE &&
-                !mbar_wait(&empty[st], ((fills / NSTAGE) - 1) & 1, abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            const uint32_t bytes = static_cast<uint32_t>(ntok * ROWB);
-            const int64_t off = static_cast<int64_t>(s.b) * p.batch_stride +
-                                static_cast<int64_t>(runs.start(r) + t0) * (HKV * D);
+    // The whole warp walks the schedule and waits; one elected lane copies.
+    const uint64_t pol = l2_evict_first_policy();
+    uint32_t fills = 0;
+    bool ok = true;
+    SegmentIter it;
+    it.init(p.geo, *plan);
+    Segment s;
+    while (ok && it.next(s)) {
+      const SlotRuns runs = segment_runs(s, C);
+      for (int r = 0; ok && r < runs.count; ++r) {
+        for (int32_t t0 = 0; t0 < runs.len(r); t0 += T) {
+          const int ntok = min(T, runs.len(r) - t0);
+          const int st = fills % NSTAGE;
+          if (fills >= NSTAGE &&
+              !mbar_wait(&empty[st], ((fills / NSTAGE) - 1) & 1, abort_flag, p.status))
+            ok = false;
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          const uint32_t bytes = static_cast<uint32_t>(ntok * ROWB);
+          const int64_t off = static_cast<int64_t>(s.b) * p.batch_stride +
+                              static_cast<int64_t>(runs.start(r) + t0) * (HKV * D);
+          if (elect_one()) {
             mbar_arrive_expect_tx(&full[st], bytes * Cfg::NT);
             bulk_g2s(stage_k + st * T * ROWB, p.k + off, bytes, &full[st], pol);
             if (!SHARED) bulk_g2s(stage_v + st * T * ROWB, p.v + off, bytes, &full[st], pol);
-            ++fills;
           }
+          __syncwarp();
+          ++fills;
         }
       }
-      // Never leave with copies in flight into this CTA's shared memory.
-      for (uint32_t f = fills > NSTAGE ? fills - NSTAGE : 0; f < fills; ++f) {
-        volatile int no_abort = 0;
-        mbar_wait(&full[f % NSTAGE], (f / NSTAGE) & 1, &no_abort, p.status);
-      }
+    }
+    // Never leave with copies in flight into this CTA's shared memory.
+    for (uint32_t f = fills > NSTAGE ? fills - NSTAGE : 0; f < fills; ++f) {
+      volatile int no_abort = 0;
+      mbar_wait(&full[f % NSTAGE], (f / NSTAGE) & 1, &no_abort, p.status);
     }
   } else {
     // ------------------------------------------------------------- compute

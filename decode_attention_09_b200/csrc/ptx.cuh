@@ -14,17 +14,12 @@ enum : uint32_t {
   kStatusSeqlen = 1u << 1,
 };
 
-// A pipeline wait gives up after this many nanoseconds of %globaltimer.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// A pipeline wait gives up after this many SM clock cycles (about 2 s at the
+// 1.965 GHz maximum, longer at lower clocks).
+constexpr long long kWaitLimitCycles = 4000000000ll;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t global_timer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
 }
 
 // ---------------------------------------------------------------- mbarrier
@@ -62,17 +57,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Gives up (returns
-// false) when *abort becomes non-zero or after kWaitLimitNs; on its own timeout
-// it raises *abort and latches kStatusTimeout in *status.
+// false) when *abort becomes non-zero or after kWaitLimitCycles of the SM clock
+// (the SM-local counter: reading the global nanosecond timer is far slower);
+// on its own timeout it raises *abort and latches kStatusTimeout in *status.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           uint32_t *status) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
+  const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
+    if ((it & 255u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (clock64() - t0 > kWaitLimitCycles) {
         *abort = 1;
         atomicOr(status, kStatusTimeout);
         return false;
@@ -135,6 +131,16 @@ __device__ __forceinline__ void grid_dependency_wait() {
 }
 __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// One lane of a converged warp (the same lane every time the full warp calls it).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .b32 rx;\n\t.reg .pred px;\n\telect.sync rx|px, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, px;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 // --------------------------------------------------------- named barriers
@@ -228,17 +234,22 @@ __device__ __forceinline__ void tmem_st16_wait(uint32_t taddr, const float (&v)[
       : "memory");
 }
 
-// Shared-memory matrix descriptor for a 128-byte-swizzled canonical layout
-// (atoms of 8 rows x 128 bytes, 1024-byte aligned).  lbo/sbo in bytes.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo,
-                                                    uint32_t sbo) {
+// Shared-memory matrix descriptor of a swizzled canonical operand layout.
+// layout: 2 = 128-byte swizzle (atoms of 8 rows x 128 B, 1024-byte aligned),
+// 4 = 64-byte swizzle (8 rows x 64 B, 512-byte aligned).  lbo/sbo in bytes.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
   d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
   d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
-  d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
+  d |= static_cast<uint64_t>(layout & 7u) << 61;
   return d;
+}
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo,
+                                                    uint32_t sbo) {
+  return smem_desc(saddr, lbo, sbo, 2);
 }
 
 // Instruction descriptor: kind::f16 with bf16 A/B, fp32 accumulator.

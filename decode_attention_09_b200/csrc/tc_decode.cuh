@@ -9,6 +9,11 @@
 //   S^T[64 tok x 16 h]  = K_tile[64 x 512] . Q^T[512 x 16]   (M=64, N=16, K=512)
 //   O^T[512 d x 32]    += V_tile^T[512 x 64] . P^T[64 x 32]  (M=128 x4, N=32, K=64)
 //
+// Consecutive MMAs never feed the same accumulator: S^T is split over four TMEM
+// accumulators (one per 16-wide k-step within each 64-wide d-chunk, summed when
+// S is read) and P.V is issued k-step by k-step across the four d-blocks, so the
+// tensor pipe overlaps them instead of waiting on each accumulation.
+//
 // The weights are bf16 operands (A and B of one MMA share a type, and V is
 // bf16), so each weight p is split into p_hi = bf16(p) and p_lo = bf16(p - p_hi):
 // the 32 columns of P^T are the 16 heads' p_hi then their p_lo, and O^T for a head
@@ -65,7 +70,7 @@ struct TcConfig {
   static constexpr int BOXB = TILE * 128;             // one 64-token x 64-d box
   static constexpr int STAGEB = BOXB * (D / 64);      // 64 KiB
   static constexpr int QB = G * D * 2;                // 16 KiB
-  static constexpr int PB = 2 * G * TILE * 2;         // 4 KiB per P buffer (hi, lo)
+  static constexpr int PB = TILE * 2 * G * 2;         // 4 KiB per P buffer: 64 tokens x 32 bf16
   static constexpr int OFF_Q = NST * STAGEB;
   static constexpr int OFF_P = OFF_Q + QB;
   static constexpr int OFF_BAR = OFF_P + 2 * PB;
@@ -73,7 +78,7 @@ struct TcConfig {
   static constexpr int SMEM = OFF_RED + 2 * 4 * G * 4 + 1024;
   static constexpr int kThreads = 192;
   static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr uint32_t S_COL = 0;                // 2 x 16 columns
+  static constexpr uint32_t S_COL = 0;                // 2 buffers x 4 partial sums x 16 columns
   static constexpr uint32_t O_COL = 128;              // 4 d-blocks x (16 hi + 16 lo) columns
 };
 
@@ -225,149 +230,161 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
 
   if (warp == 0) {
     // -------------------------------------------------------------- TMA
-    if (lane == 0) {
-      const uint64_t pol = l2_evict_first_policy();
-      bool ok = true;
-      uint32_t i = 0, nseg = 0;
-      TileIter it;
-      it.init(p.geo, *plan);
-      int32_t row, ntok;
-      bool first, last;
-      while (ok && it.next(C, row, ntok, first, last)) {
-        if (first) {
-          if (nseg > 0 && !mbar_wait(qempty, (nseg - 1) & 1, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          const int32_t qrow = it.seg.b * p.n_q_heads + it.seg.x * G;
+    // The whole warp walks the schedule and waits (values stay warp-uniform);
+    // one elected lane issues the copies.
+    const uint64_t pol = l2_evict_first_policy();
+    bool ok = true;
+    uint32_t i = 0, nseg = 0;
+    TileIter it;
+    it.init(p.geo, *plan);
+    int32_t row, ntok;
+    bool first, last;
+    while (ok && it.next(C, row, ntok, first, last)) {
+      if (first) {
+        if (nseg > 0 && !mbar_wait(qempty, (nseg - 1) & 1, abort_flag, p.status)) ok = false;
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const int32_t qrow = it.seg.b * p.n_q_heads + it.seg.x * G;
+        if (elect_one()) {
           mbar_arrive_expect_tx(qfull, Cfg::QB);
 #pragma unroll
           for (int j = 0; j < D / 64; ++j)
             tma_load_2d(qs + j * (G * 128), &qmap, 64 * j, qrow, qfull);
-          ++nseg;
         }
-        const int st = i % NST;
-        if (i >= NST && !mbar_wait(&empty[st], ((i / NST) - 1) & 1, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
+        __syncwarp();
+        ++nseg;
+      }
+      const int st = i % NST;
+      if (i >= NST && !mbar_wait(&empty[st], ((i / NST) - 1) & 1, abort_flag, p.status)) ok = false;
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (elect_one()) {
         mbar_arrive_expect_tx(&full[st], Cfg::STAGEB);
 #pragma unroll
         for (int j = 0; j < D / 64; ++j)
           tma_load_4d(stages + st * Cfg::STAGEB + j * Cfg::BOXB, &kmap, 64 * j, it.seg.x, row,
                       it.seg.b, &full[st], pol);
-        ++i;
       }
-      // Drain: never leave with copies in flight into shared memory.
-      volatile int no_abort = 0;
-      for (uint32_t f = i > NST ? i - NST : 0; f < i; ++f)
-        mbar_wait(&full[f % NST], (f / NST) & 1, &no_abort, p.status);
-      if (nseg > 0) mbar_wait(qfull, (nseg - 1) & 1, &no_abort, p.status);
+      __syncwarp();
+      ++i;
     }
+    // Drain: never leave with copies in flight into shared memory.
+    volatile int no_abort = 0;
+    for (uint32_t f = i > NST ? i - NST : 0; f < i; ++f)
+      mbar_wait(&full[f % NST], (f / NST) & 1, &no_abort, p.status);
+    if (nseg > 0) mbar_wait(qfull, (nseg - 1) & 1, &no_abort, p.status);
   } else if (warp == 1) {
     // -------------------------------------------------------------- MMA
-    if (lane == 0) {
-      const uint32_t idesc_qk = idesc_bf16_f32(64, 16, false, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 32, true, false);
-      const uint32_t st_addr = smem_u32(stages);
-      const uint32_t q_addr = smem_u32(qs);
-      const uint32_t p_addr = smem_u32(ps);
-      bool ok = true;
-      uint32_t i = 0, nseg = 0;
-      int32_t prev = -1;       // tile whose P.V is still to issue
-      bool prev_first = false; // ... and whether it opened its segment
-      uint32_t prev_seg = 0;   // ... and that segment's index in this CTA
-      TileIter it;
-      it.init(p.geo, *plan);
-      int32_t row, ntok;
-      bool first, last;
-      auto issue_pv = [&](uint32_t t, bool seg_first, uint32_t seg) -> bool {
-        if (!mbar_wait(&pfull[t & 1], (t >> 1) & 1, abort_flag, p.status)) return false;
-        // A segment's first P.V overwrites O: the previous segment must be read out.
-        if (seg_first && seg > 0 && !mbar_wait(oempty, (seg - 1) & 1, abort_flag, p.status))
-          return false;
-        tc_fence_after();
-        const uint32_t a0 = st_addr + (t % NST) * Cfg::STAGEB;
+    // Converged warp: descriptors are warp-uniform, one elected lane issues
+    // every MMA and commit (commits track that lane's MMAs).
+    const uint32_t idesc_qk = idesc_bf16_f32(64, 16, false, false);
+    const uint32_t idesc_pv = idesc_bf16_f32(128, 32, true, true);
+    // Base descriptors; an operand at byte offset o from a base is base + (o >> 4)
+    // (the 14-bit start field holds address >> 4 and never carries: smem < 256 KiB).
+    const uint64_t kdesc = smem_desc_sw128(smem_u32(stages), 16, 1024);       // K tile, K-major
+    const uint64_t qdesc = smem_desc_sw128(smem_u32(qs), 16, 1024);           // Q, K-major
+    const uint64_t vdesc = smem_desc_sw128(smem_u32(stages), Cfg::BOXB, 1024); // V^T, MN-major
+    const uint64_t pdesc = smem_desc(smem_u32(ps), 4096, 512, 4);              // P^T, MN-major SW64
+    bool ok = true;
+    uint32_t i = 0, nseg = 0;
+    int32_t prev = -1;       // tile whose P.V is still to issue
+    bool prev_first = false; // ... and whether it opened its segment
+    uint32_t prev_seg = 0;   // ... and that segment's index in this CTA
+    TileIter it;
+    it.init(p.geo, *plan);
+    int32_t row, ntok;
+    bool first, last;
+    auto issue_pv = [&](uint32_t t, bool seg_first, uint32_t seg) -> bool {
+      bool w = mbar_wait(&pfull[t & 1], (t >> 1) & 1, abort_flag, p.status);
+      // A segment's first P.V overwrites O: the previous segment must be read out.
+      if (w && seg_first && seg > 0) w = mbar_wait(oempty, (seg - 1) & 1, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      const uint64_t a0 = vdesc + (((t % NST) * Cfg::STAGEB) >> 4);
+      const uint64_t b0 = pdesc + (((t & 1) * Cfg::PB) >> 4);
+      if (elect_one()) {
 #pragma unroll
-        for (int jb = 0; jb < 4; ++jb) {
+        for (int kk = 0; kk < 4; ++kk) {
+          // P^T: MN-major, 64-byte swizzle, a token row of 32 bf16 = 64 B; 16 tokens
+          // per k-step = two 512-byte atoms.
+          const uint64_t bd = b0 + ((kk * 1024) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad =
-                smem_desc_sw128(a0 + (2 * jb) * Cfg::BOXB + kk * 2048, Cfg::BOXB, 1024);
-            const uint64_t bd = smem_desc_sw128(p_addr + (t & 1) * Cfg::PB + kk * 32, 16, 1024);
+          for (int jb = 0; jb < 4; ++jb) {
+            const uint64_t ad = a0 + ((2 * jb * Cfg::BOXB + kk * 2048) >> 4);
             tc_mma_bf16(tmem + Cfg::O_COL + jb * 32, ad, bd, idesc_pv, !(seg_first && kk == 0));
           }
         }
         tc_commit(&ofull[t & 1]);
         tc_commit(&empty[t % NST]);
-        return true;
-      };
-      uint32_t cur_seg = 0;
-      while (ok && it.next(C, row, ntok, first, last)) {
-        if (first) {
-          if (!mbar_wait(qfull, nseg & 1, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          cur_seg = nseg++;
-        }
-        const int st = i % NST, sb = i & 1;
-        if (!mbar_wait(&full[st], (i / NST) & 1, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        if (i >= 2 && !mbar_wait(&sempty[sb], ((i >> 1) - 1) & 1, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t a0 = st_addr + st * Cfg::STAGEB;
+      }
+      __syncwarp();
+      return true;
+    };
+    uint32_t cur_seg = 0;
+    while (ok && it.next(C, row, ntok, first, last)) {
+      if (first) {
+        if (!mbar_wait(qfull, nseg & 1, abort_flag, p.status)) ok = false;
+        if (!__all_sync(0xffffffffu, ok)) break;
+        cur_seg = nseg++;
+      }
+      const int st = i % NST, sb = i & 1;
+      if (!mbar_wait(&full[st], (i / NST) & 1, abort_flag, p.status)) ok = false;
+      if (ok && i >= 2 && !mbar_wait(&sempty[sb], ((i >> 1) - 1) & 1, abort_flag, p.status))
+        ok = false;
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const uint64_t a0 = kdesc + ((st * Cfg::STAGEB) >> 4);
+      if (elect_one()) {
 #pragma unroll
         for (int j = 0; j < D / 64; ++j) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = smem_desc_sw128(a0 + j * Cfg::BOXB + kk * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(q_addr + j * (G * 128) + kk * 32, 16, 1024);
-            tc_mma_bf16(tmem + Cfg::S_COL + sb * 16, ad, bd, idesc_qk, (j | kk) != 0);
+            const uint64_t ad = a0 + ((j * Cfg::BOXB + kk * 32) >> 4);
+            const uint64_t bd = qdesc + ((j * (G * 128) + kk * 32) >> 4);
+            tc_mma_bf16(tmem + Cfg::S_COL + sb * 64 + kk * 16, ad, bd, idesc_qk, j != 0);
           }
         }
         tc_commit(&sfull[sb]);
         if (last) tc_commit(qempty);
-        if (prev >= 0 && !issue_pv(static_cast<uint32_t>(prev), prev_first, prev_seg)) {
-          ok = false;
-          break;
-        }
-        prev = static_cast<int32_t>(i);
-        prev_first = first;
-        prev_seg = cur_seg;
-        ++i;
       }
-      if (ok && prev >= 0) ok = issue_pv(static_cast<uint32_t>(prev), prev_first, prev_seg);
-      // Drain: wait until every issued MMA has completed before TMEM is freed.
-      tc_commit(drain);
-      volatile int no_abort = 0;
-      mbar_wait(drain, 0, &no_abort, p.status);
+      __syncwarp();
+      if (prev >= 0 && !issue_pv(static_cast<uint32_t>(prev), prev_first, prev_seg)) {
+        ok = false;
+        break;
+      }
+      prev = static_cast<int32_t>(i);
+      prev_first = first;
+      prev_seg = cur_seg;
+      ++i;
     }
+    if (ok && prev >= 0) ok = issue_pv(static_cast<uint32_t>(prev), prev_first, prev_seg);
+    // Drain: wait until every issued MMA has completed before TMEM is freed.
+    if (elect_one()) tc_commit(drain);
+    __syncwarp();
+    volatile int no_abort = 0;
+    mbar_wait(drain, 0, &no_abort, p.status);
   } else {
     // ---------------------------------------------------------- softmax
+    // M=64 puts tile token r in TMEM lane (r % 16) + 32 * (r / 16): lanes 0-15 of
+    // each warp receive one token's 16 scores.  Lanes 16-31 take heads 8-15 of
+    // the token of lane - 16, so every lane handles one token and 8 heads.
     const int qd = warp & 3;                 // TMEM sub-partition: lanes 32*qd ..
     const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
-    const int tok = 16 * qd + lane;          // tile token held by this lane (lane < 16)
-    float m_ref[G], lpart[G];
+    const int tok = 16 * qd + (lane & 15);   // tile token of this lane
+    const int hb = (lane < 16) ? 0 : 8;      // first head of this lane (heads hb .. hb+7)
+    float m_ref[G], lpart[8];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      m_ref[h] = -INFINITY;
-      lpart[h] = 0.f;
-    }
+    for (int h = 0; h < G; ++h) m_ref[h] = -INFINITY;
+#pragma unroll
+    for (int h = 0; h < 8; ++h) lpart[h] = 0.f;
     bool ok = true;
-    uint32_t cons[2] = {0u, 0u};  // ofull phases consumed per barrier
+    uint32_t cons0 = 0, cons1 = 0;  // ofull phases consumed on barrier 0 / 1
     // Wait until the P.V of tile t has completed.  Phases are consumed in order
     // and never lag by two, so the parity waits cannot alias.
     auto ensure_pv = [&](uint32_t t) {
       const uint32_t b = t & 1, ph = t >> 1;
-      if (cons[b] <= ph) {
-        if (ok && !mbar_wait(&ofull[b], cons[b] & 1, abort_flag, p.status)) ok = false;
-        ++cons[b];
+      uint32_t &cons = b ? cons1 : cons0;
+      if (cons <= ph) {
+        if (ok && !mbar_wait(&ofull[b], cons & 1, abort_flag, p.status)) ok = false;
+        ++cons;
       }
       ok = __all_sync(0xffffffffu, ok);
     };
@@ -382,36 +399,51 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
       if (i >= 2) ensure_pv(i - 2);  // P buffer pb is free again
       if (first) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          m_ref[h] = -INFINITY;
-          lpart[h] = 0.f;
-        }
+        for (int h = 0; h < G; ++h) m_ref[h] = -INFINITY;
+#pragma unroll
+        for (int h = 0; h < 8; ++h) lpart[h] = 0.f;
       }
-      // --- scores of tile i
-      float s[16];
+      // --- scores of tile i: sum of the four partial accumulators
+      float s16[16];
       if (ok && !mbar_wait(&sfull[sb], (i >> 1) & 1, abort_flag, p.status)) ok = false;
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
-        tmem_ld16(tmem + lane_base + Cfg::S_COL + sb * 16, s);
+        float a[16], b[16], c2[16], d2[16];
+        tmem_ld16(tmem + lane_base + Cfg::S_COL + sb * 64, a);
+        tmem_ld16(tmem + lane_base + Cfg::S_COL + sb * 64 + 16, b);
+        tmem_ld16(tmem + lane_base + Cfg::S_COL + sb * 64 + 32, c2);
+        tmem_ld16(tmem + lane_base + Cfg::S_COL + sb * 64 + 48, d2);
+#pragma unroll
+        for (int h = 0; h < 16; ++h) s16[h] = (a[h] + b[h]) + (c2[h] + d2[h]);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sempty[sb]);
       }
-      const bool valid = ok && lane < 16 && tok < ntok;
+      float s[8];
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        const float mine = s16[h], theirs = s16[8 + h];
+        const float got = __shfl_xor_sync(0xffffffffu, (lane < 16) ? theirs : mine, 16);
+        s[h] = (lane < 16) ? mine : got;
+      }
+      const bool valid = ok && tok < ntok;
       bool need = false;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
+      for (int h = 0; h < 8; ++h) {
         float x = s[h] * p.qscale;
         if (p.post != 0.f) x = p.post * tanhf(x);
         s[h] = valid ? x : -INFINITY;
-        need |= s[h] > m_ref[h] + kTau;
+        need |= s[h] > ((lane < 16) ? m_ref[h] : m_ref[8 + h]) + kTau;
       }
       // --- move the reference only when some score outgrew it
       if (named_bar_or(1, 128, need)) {
-        float r[16];
+        float r[16];  // this lane's 8 heads in their slots, -inf elsewhere
 #pragma unroll
-        for (int h = 0; h < 16; ++h) r[h] = s[h];
+        for (int h = 0; h < 8; ++h) {
+          r[h] = (lane < 16) ? s[h] : -INFINITY;
+          r[8 + h] = (lane < 16) ? -INFINITY : s[h];
+        }
         const float tm = warp_reduce_scatter16<true>(r, lane);
         if ((lane & 1) == 0) redmax[qd * G + (lane >> 1)] = tm;
         named_bar_sync(1, 128);
@@ -423,8 +455,9 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
           const float mn = fmaxf(m_ref[h], t);
           alpha[h] = (m_ref[h] == -INFINITY) ? 0.f : exp2f(m_ref[h] - mn);
           m_ref[h] = mn;
-          lpart[h] *= alpha[h];
         }
+#pragma unroll
+        for (int h = 0; h < 8; ++h) lpart[h] *= (lane < 16) ? alpha[h] : alpha[8 + h];
         if (!first) {
           // O holds tiles < i: wait for the last of them, then rescale it in TMEM.
           ensure_pv(i - 1);
@@ -441,21 +474,29 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
           }
         }
       }
-      // --- weights, P^T (bf16 hi / lo rows, 128B-swizzled K-major), row sums
-      uint8_t *prow = ps + pb * Cfg::PB;
+      // --- weights: P^T row of this token, MN-major with 64-byte swizzle:
+      // 16-byte chunks (hi 0-7, hi 8-15, lo 0-7, lo 8-15), chunk c of row r at
+      // r * 64 + ((c ^ ((r >> 1) & 3)) * 16).
+      {
+        float pe[8];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float pe = (s[h] == -INFINITY) ? 0.f : exp2f(s[h] - m_ref[h]);
-        lpart[h] += pe;
-        if (lane < 16) {
-          const uint16_t hi = f32_to_bf16_rn(pe);
-          const uint16_t lo = f32_to_bf16_rn(pe - __uint_as_float(static_cast<uint32_t>(hi) << 16));
-          const uint32_t col = (tok & 7) * 2;
-          const uint32_t chunk = tok >> 3;
-          *reinterpret_cast<uint16_t *>(prow + h * 128 + (((chunk ^ h) & 7) << 4) + col) = hi;
-          *reinterpret_cast<uint16_t *>(prow + (G + h) * 128 + (((chunk ^ (G + h)) & 7) << 4) +
-                                        col) = lo;
+        for (int h = 0; h < 8; ++h) {
+          const float mr = (lane < 16) ? m_ref[h] : m_ref[8 + h];
+          pe[h] = (s[h] == -INFINITY) ? 0.f : exp2f(s[h] - mr);
+          lpart[h] += pe[h];
         }
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          hw[k] = pack_bf16x2(pe[2 * k], pe[2 * k + 1]);
+          lw[k] = pack_bf16x2(pe[2 * k] - bf16lo(hw[k]), pe[2 * k + 1] - bf16hi(hw[k]));
+        }
+        uint8_t *prow = ps + pb * Cfg::PB + tok * 64;
+        const int ch = hb >> 3;  // 0 or 1
+        const int sw = (tok >> 1) & 3;
+        *reinterpret_cast<uint4 *>(prow + ((ch ^ sw) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4 *>(prow + (((ch + 2) ^ sw) << 4)) =
+            make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
       if (ok && ntok < Cfg::TILE) {
         // Rows past the attended range hold other cache contents (possibly
@@ -478,9 +519,12 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
         // --- segment end: all of its P.V done, read O out
         if (i >= 1) ensure_pv(i - 1);
         ensure_pv(i);
-        float r[16];
+        float r[16];  // this lane's 8 partial sums in their slots, 0 elsewhere
 #pragma unroll
-        for (int h = 0; h < 16; ++h) r[h] = lpart[h];
+        for (int h = 0; h < 8; ++h) {
+          r[h] = (lane < 16) ? lpart[h] : 0.f;
+          r[8 + h] = (lane < 16) ? 0.f : lpart[h];
+        }
         const float ls = warp_reduce_scatter16<false>(r, lane);
         if ((lane & 1) == 0) redsum[qd * G + (lane >> 1)] = ls;
         named_bar_sync(1, 128);
