@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.gdattn_workspace_size.restype = sz
         L.gdattn_plan_splits.argtypes = [i32, i32, descp]
         L.gdattn_plan_splits.restype = i32
+        L.gdattn_plan_launches.argtypes = [i32, i32, descp]
+        L.gdattn_plan_launches.restype = i32
         L.gdattn_workspace_init.argtypes = [vp, sz, vp]
         L.gdattn_workspace_init.restype = ctypes.c_int
         L.gdattn_decode.argtypes = [vp, vp, vp, vp, i32, i32, descp, vp, vp, vp, sz, vp]
@@ -125,8 +127,8 @@ def plan_splits(batch: int, max_seqlen: int, desc: LayerDesc) -> int:
 
 
 def launches_per_call(batch: int, max_seqlen: int, desc: LayerDesc) -> int:
-    """Kernel launches one gdattn_decode call makes: decode, plus combine when split."""
-    return 1 + (1 if plan_splits(batch, max_seqlen, desc) > 1 else 0)
+    """Kernel launches one gdattn_decode call makes (1, or 2 with a separate combine)."""
+    return int(lib().gdattn_plan_launches(int(batch), int(max_seqlen), ctypes.byref(desc)))
 
 
 def workspace_init(workspace: torch.Tensor, stream=None) -> None:

@@ -27,6 +27,7 @@ struct LayerPlan {
   int32_t units_per_seq = 1;   // query-head groups per sequence
   int32_t heads_per_unit = 0;
   int64_t slots = 0;           // partial slots: P + units
+  int32_t align = 1;           // chunk granularity in tokens (one tile / stage)
   size_t off_lse = 0, off_o = 0, bytes = 0;
 };
 
@@ -175,12 +176,14 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
     per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(ck.fn), ck.threads, ck.smem,
                                   query_core);
     min_tokens = 2 * ck.tokens_per_stage;
+    pl.align = ck.tokens_per_stage;
     pl.units_per_seq = 1;
     pl.heads_per_unit = d->n_q_heads;
   } else {
     per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_kernel),
                                   TcConfig::kThreads, TcConfig::SMEM, query_tc);
     min_tokens = 2 * TcConfig::TILE;
+    pl.align = TcConfig::TILE;
     pl.units_per_seq = d->n_kv_heads;
     pl.heads_per_unit = 16;
   }
@@ -239,14 +242,6 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// Dynamic shared memory of the combine kernel: part weights plus the
-// per-group float4 accumulators.
-int combine_smem_bytes(int n_parts, int head_dim) {
-  const int nc = head_dim / 4;
-  const int ng = nc >= kCombineThreads ? 1 : kCombineThreads / nc;
-  return ((n_parts + 3) & ~3) * 4 + ng * nc * 16 + 16;
-}
-
 gdattn_status launch_combine_internal(const LayerPlan &pl, const Geometry &geo, const float *ws_lse,
                                       const float *ws_o, const gdattn_layer_desc *d, void *out,
                                       float *lse, cudaStream_t stream) {
@@ -260,16 +255,11 @@ gdattn_status launch_combine_internal(const LayerPlan &pl, const Geometry &geo, 
   cp.geo = geo;
   cp.heads_per_unit = pl.heads_per_unit;
   cp.n_splits = 0;
-  const int smem = combine_smem_bytes(pl.grid, d->head_dim);
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg =
       launch_config(dim3(static_cast<unsigned>(geo.batch * pl.units_per_seq),
                          static_cast<unsigned>(pl.heads_per_unit)),
-                    kCombineThreads, smem, stream, attr);
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(combine_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem) != cudaSuccess)
-    return GDATTN_ERR_CUDA;
+                    combine_threads(d->head_dim), 0, stream, attr);
   return cudaLaunchKernelEx(&cfg, combine_kernel<true>, cp) == cudaSuccess ? GDATTN_OK
                                                                             : GDATTN_ERR_CUDA;
 }
@@ -307,10 +297,16 @@ int32_t gdattn_plan_splits(int32_t batch, int32_t max_seqlen, const gdattn_layer
   return pl.grid;
 }
 
+int32_t gdattn_plan_launches(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc) {
+  LayerPlan pl;
+  if (make_plan(batch, max_seqlen, desc, pl) != GDATTN_OK) return 0;
+  return pl.grid > 1 ? 2 : 1;
+}
+
 gdattn_status gdattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
   if (workspace == nullptr || workspace_bytes < kStatusBytes) return GDATTN_ERR_WORKSPACE;
   if (!aligned16(workspace)) return GDATTN_ERR_MISALIGNED;
-  return cudaMemsetAsync(workspace, 0, kStatusBytes, static_cast<cudaStream_t>(stream)) ==
+  return cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
              ? GDATTN_OK
              : GDATTN_ERR_CUDA;
@@ -360,6 +356,7 @@ gdattn_status gdattn_decode(const void *q, const void *k_cache, const void *v_ca
   geo.window = desc->window;
   geo.capacity = desc->cache_capacity;
   geo.nchunks = pl.grid;
+  geo.align = pl.align;
 
   cudaLaunchAttribute attr[1];
   if (pl.kind == PathKind::kCore) {
@@ -450,13 +447,8 @@ gdattn_status gdattn_combine(const float *o_partial, const float *lse_partial, i
   cp.head_dim = head_dim;
   cp.heads_per_unit = 0;
   cp.n_splits = n_splits;
-  const int smem = combine_smem_bytes(n_splits, head_dim);
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(combine_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem) != cudaSuccess)
-    return GDATTN_ERR_CUDA;
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = launch_config(dim3(batch, n_q_heads), kCombineThreads, smem,
+  cudaLaunchConfig_t cfg = launch_config(dim3(batch, n_q_heads), combine_threads(head_dim), 0,
                                          static_cast<cudaStream_t>(stream), attr);
   return cudaLaunchKernelEx(&cfg, combine_kernel<false>, cp) == cudaSuccess ? GDATTN_OK
                                                                              : GDATTN_ERR_CUDA;

@@ -3,8 +3,14 @@
 // Each part s of a (sequence, head) holds o_s (normalised over its own
 // positions) and lse_s; the merged result is
 //   lse = log sum_s exp(lse_s),   out = sum_s exp(lse_s - lse) * o_s,
-// with empty parts (lse_s = -inf) contributing nothing.  One CTA per
-// (unit or sequence, head); a thread owns 4 consecutive elements of D.
+// with empty parts (lse_s = -inf) contributing nothing.
+//
+// One CTA per (unit or sequence, head); a thread owns one float4 column of D.
+// The merge is a single pass over the parts with a running maximum; the
+// parts' LSE and O loads do not depend on one another, so they are issued
+// kBatch parts at a time and the cost after the decode kernel completes is a
+// few L2 round trips.  Where the parts sit is worked out from seqlens before
+// waiting on the decode kernel (programmatic dependent launch).
 #pragma once
 
 #include <cstdint>
@@ -29,7 +35,10 @@ struct CombineParams {
   int32_t n_splits;
 };
 
-constexpr int kCombineThreads = 128;
+// Threads per combine CTA: one float4 column of D each, whole warps.
+__host__ __device__ constexpr int combine_threads(int head_dim) {
+  return (head_dim / 4 + 31) / 32 * 32;
+}
 
 // Flattened start of unit (b, x) and the split chunk size, from seqlens.
 __device__ void unit_position(const Geometry &g, int32_t b, int32_t x, int64_t &unit_start,
@@ -48,21 +57,20 @@ __device__ void unit_position(const Geometry &g, int32_t b, int32_t x, int64_t &
   before = warp_sum_i64(before);
   n = attended_count(__ldg(g.seqlens + b), g.window, g.capacity, bad);
   unit_start = before + static_cast<int64_t>(x) * n;
-  chunk = total > 0 ? ceil_div64(total, g.nchunks) : 1;
+  chunk = total > 0 ? ceil_div64(ceil_div64(total, g.nchunks), g.align) * g.align : 1;
 }
 
 template <bool INTERNAL>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineParams p) {
-  extern __shared__ __align__(16) float wts[];  // [n_parts] weights, then [NG][NC] float4
+__global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
+  constexpr int kBatch = 16;
   __shared__ int64_t sh_slot0;
   __shared__ int32_t sh_nparts;
 
   grid_launch_dependents();
-  grid_dependency_wait();
-
   int32_t b, h;
   const int32_t hh = blockIdx.y;
   if (INTERNAL) {
+    // seqlens do not change while the decode kernel runs: locate the parts first.
     const int32_t u = blockIdx.x;
     b = u / p.geo.units_per_seq;
     const int32_t x = u - b * p.geo.units_per_seq;
@@ -90,6 +98,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineP
   }
   const int32_t np = sh_nparts;
   if (np == 0) return;
+  grid_dependency_wait();  // the parts come from the preceding kernel
   const int32_t D = p.head_dim;
 
   // Part s of this (b, h): o at o_base + s * o_stride, lse at l_base + s * l_stride.
@@ -108,101 +117,54 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineP
     l_base = p.parts_lse + (static_cast<int64_t>(b) * p.n_q_heads + h) * np;
   }
 
-  // Max of the parts' lse, then weights exp(lse_s - max) and their sum.
-  float mx = -INFINITY;
-  for (int32_t s = threadIdx.x; s < np; s += blockDim.x) {
-    const float v = l_base[s * l_stride];
-    wts[s] = v;
-    mx = fmaxf(mx, v);
-  }
-  __shared__ float red[kCombineThreads / 32];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
-  __syncthreads();
-  mx = red[0];
-  for (int w = 1; w < kCombineThreads / 32; ++w) mx = fmaxf(mx, red[w]);
-  __syncthreads();
-  float z = 0.f;
-  for (int32_t s = threadIdx.x; s < np; s += blockDim.x) {
-    const float v = wts[s];
-    const float e = (v == -INFINITY) ? 0.f : __expf(v - mx);
-    wts[s] = e;
-    z += e;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = z;
-  __syncthreads();
-  z = 0.f;
-  for (int w = 0; w < kCombineThreads / 32; ++w) z += red[w];
-  const bool empty = (mx == -INFINITY);
-  const float inv_z = empty ? 0.f : 1.f / z;
-
-  // Thread t owns float4 column (t mod NC) and parts t / NC, t / NC + NG, ...;
-  // loads are issued kUnroll at a time so each thread keeps several in flight.
   uint16_t *dst = p.out + (static_cast<int64_t>(b) * p.n_q_heads + h) * D;
-  const int NC = D / 4;
-  const int NG = NC >= kCombineThreads ? 1 : kCombineThreads / NC;
-  const int grp = threadIdx.x / NC;
-  float4 *part_acc = reinterpret_cast<float4 *>(wts + ((np + 3) & ~3));  // [NG][NC]
-  for (int d4 = threadIdx.x % NC; d4 < NC; d4 += kCombineThreads) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (!empty && grp < NG) {
-      constexpr int kUnroll = 8;
-      int32_t s = grp;
-      for (; s + (kUnroll - 1) * NG < np; s += kUnroll * NG) {
-        float4 v[kUnroll];
-        float wv[kUnroll];
+  const int d = 4 * threadIdx.x;
+  const bool owner = d < D;
+  float m = -INFINITY, z = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int32_t s0 = 0; s0 < np; s0 += kBatch) {
+    float lv[kBatch];
+    float4 ov[kBatch];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          v[u] = *reinterpret_cast<const float4 *>(o_base + (s + u * NG) * o_stride + 4 * d4);
-          wv[u] = wts[s + u * NG];
-        }
+    for (int q = 0; q < kBatch; ++q) {
+      const bool in = s0 + q < np;
+      lv[q] = in ? __ldcg(l_base + (s0 + q) * l_stride) : -INFINITY;
+      ov[q] = (in && owner)
+                  ? __ldcg(reinterpret_cast<const float4 *>(o_base + (s0 + q) * o_stride + d))
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float bm = m;
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          // an empty part has weight 0 and may hold anything: select, don't multiply
-          if (wv[u] != 0.f) {
-            acc.x = fmaf(wv[u], v[u].x, acc.x);
-            acc.y = fmaf(wv[u], v[u].y, acc.y);
-            acc.z = fmaf(wv[u], v[u].z, acc.z);
-            acc.w = fmaf(wv[u], v[u].w, acc.w);
-          }
-        }
-      }
-      for (; s < np; s += NG) {
-        const float w = wts[s];
-        if (w != 0.f) {
-          const float4 v = *reinterpret_cast<const float4 *>(o_base + s * o_stride + 4 * d4);
-          acc.x = fmaf(w, v.x, acc.x);
-          acc.y = fmaf(w, v.y, acc.y);
-          acc.z = fmaf(w, v.z, acc.z);
-          acc.w = fmaf(w, v.w, acc.w);
-        }
-      }
+    for (int q = 0; q < kBatch; ++q) bm = fmaxf(bm, lv[q]);
+    if (bm == -INFINITY) continue;  // only empty parts so far
+    const float r = (m == -INFINITY) ? 0.f : __expf(m - bm);
+    z *= r;
+    acc.x *= r;
+    acc.y *= r;
+    acc.z *= r;
+    acc.w *= r;
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      // an empty part has weight 0 and may hold anything: select, don't multiply
+      if (lv[q] == -INFINITY) continue;
+      const float w = __expf(lv[q] - bm);
+      z += w;
+      acc.x = fmaf(w, ov[q].x, acc.x);
+      acc.y = fmaf(w, ov[q].y, acc.y);
+      acc.z = fmaf(w, ov[q].z, acc.z);
+      acc.w = fmaf(w, ov[q].w, acc.w);
     }
-    if (NG > 1) {
-      if (grp < NG) part_acc[grp * NC + d4] = acc;
-      __syncthreads();
-      if (grp == 0) {
-        for (int g2 = 1; g2 < NG; ++g2) {
-          const float4 o = part_acc[g2 * NC + d4];
-          acc.x += o.x;
-          acc.y += o.y;
-          acc.z += o.z;
-          acc.w += o.w;
-        }
-      }
-    }
-    if (grp == 0) {
-      uint2 pk;
-      pk.x = pack_bf16x2(acc.x * inv_z, acc.y * inv_z);
-      pk.y = pack_bf16x2(acc.z * inv_z, acc.w * inv_z);
-      *reinterpret_cast<uint2 *>(dst + 4 * d4) = pk;
-    }
+    m = bm;
+  }
+  const float inv_z = (m == -INFINITY) ? 0.f : __fdividef(1.f, z);
+  if (owner) {
+    uint2 pk;
+    pk.x = pack_bf16x2(acc.x * inv_z, acc.y * inv_z);
+    pk.y = pack_bf16x2(acc.z * inv_z, acc.w * inv_z);
+    *reinterpret_cast<uint2 *>(dst + d) = pk;
   }
   if (threadIdx.x == 0 && p.lse != nullptr)
-    p.lse[static_cast<int64_t>(b) * p.n_q_heads + h] = empty ? -INFINITY : mx + logf(z);
+    p.lse[static_cast<int64_t>(b) * p.n_q_heads + h] = (m == -INFINITY) ? -INFINITY : m + logf(z);
 }
 
 }  // namespace gdattn

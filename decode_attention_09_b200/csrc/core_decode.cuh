@@ -49,7 +49,7 @@ struct CoreConfig {
   static constexpr int MSTRIDE = MHDR + G * D;        // floats per warp, 16-byte multiple
   // 16 compute warps (two or more per KV head) hide latency better; 8 when the
   // cross-warp merge area for 16 would not fit beside the ring.
-  static constexpr int kComputeWarps = (16 * MSTRIDE * 4 <= 40 * 1024) ? 16 : 8;
+  static constexpr int kComputeWarps = ((16 - HKV) * MSTRIDE * 4 <= 40 * 1024) ? 16 : 8;
   static constexpr int kThreads = (kComputeWarps + 1) * 32;
   static constexpr int TS = kComputeWarps / HKV;      // warps sharing one KV head
   static constexpr int ROWB = HKV * D * 2;            // bytes of one token row (one tensor)
@@ -60,9 +60,10 @@ struct CoreConfig {
   static constexpr int EPL = D / 32;                  // elements per lane
   static constexpr int CH = EPL / 8;                  // 16-byte chunks per lane
   static constexpr int STAGEB = T * ROWB * NT;
-  static constexpr int MERGEB = TS > 1 ? kComputeWarps * MSTRIDE * 4 : 0;
-  // Stages: up to 192 KiB of ring, within what the merge area leaves.
-  static constexpr int RING = (220 * 1024 - MERGEB) < 196608 ? (220 * 1024 - MERGEB) : 196608;
+  static constexpr int MERGEB = TS > 1 ? (kComputeWarps - HKV) * MSTRIDE * 4 : 0;
+  // Stages: up to 192 KiB of ring, within what the merge area leaves of the
+  // 227 KiB a CTA may use (3 KiB kept for barriers, alignment and statics).
+  static constexpr int RING = (224 * 1024 - MERGEB) < 196608 ? (224 * 1024 - MERGEB) : 196608;
   static constexpr int NSTAGE = (RING / STAGEB) < 2 ? 2 : (RING / STAGEB > 8 ? 8 : RING / STAGEB);
   static constexpr int NV = TPW * G;                  // scores per warp per stage
   static constexpr int LOGNV = NV == 2 ? 1 : NV == 4 ? 2 : (NV == 8 ? 3 : (NV == 16 ? 4 : 5));
@@ -73,7 +74,7 @@ struct CoreConfig {
   static_assert(G == 1 || G == 2 || G == 4, "G");
   static_assert(D == 256 || D == 512, "D");
   static_assert(NV >= 2 && NV <= 32, "one score per lane at most");
-  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(SMEM <= 226 * 1024, "shared memory");
 };
 
 template <int D, int G, int HKV, bool SHARED>
@@ -108,11 +109,14 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads, 1)
     fence_barrier_init();
   }
   grid_launch_dependents();
-  grid_dependency_wait();  // inputs / workspace may come from the previous kernel
+  // The split plan reads only seqlens, so it (and the producer's first KV
+  // loads below) may run before the preceding kernel has completed; every other
+  // global access waits for it (griddepcontrol.wait) in the role that makes it.
   if (warp == 0) plan_chunk(p.geo, c, plan);
   __syncthreads();
 
   if (c == 0 && warp == 0 && plan->bad) {
+    grid_dependency_wait();
     if (lane == 0) atomicOr(p.status, kStatusSeqlen);
     // Sequences with nothing to attend get out = 0 and lse = -inf.
     for (int32_t b = 0; b < p.geo.batch; ++b) {
@@ -135,6 +139,9 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads, 1)
     const uint64_t pol = l2_evict_first_policy();
     uint32_t fills = 0;
     bool ok = true;
+    // Until the preceding kernel completes, only cache rows of positions before
+    // each sequence's newest one are read (earlier decode steps wrote them).
+    bool waited = false;
     SegmentIter it;
     it.init(p.geo, *plan);
     Segment s;
@@ -144,6 +151,11 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads, 1)
         for (int32_t t0 = 0; t0 < runs.len(r); t0 += T) {
           const int ntok = min(T, runs.len(r) - t0);
           const int st = fills % NSTAGE;
+          const bool newest = s.lo + (r == 1 ? runs.len0 : 0) + t0 + ntok == s.n;
+          if (!waited && (fills >= NSTAGE || newest)) {
+            grid_dependency_wait();
+            waited = true;
+          }
           if (fills >= NSTAGE &&
               !mbar_wait(&empty[st], ((fills / NSTAGE) - 1) & 1, abort_flag, p.status))
             ok = false;
@@ -171,6 +183,7 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------- compute
+    grid_dependency_wait();  // q, outputs and workspace
     const int kvh = warp % HKV;
     const int tp = warp / HKV;
     float2 q[G][P2];
@@ -334,47 +347,48 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads, 1)
 
       // ---------------------------------------------------- segment epilogue
       if (Cfg::TS > 1) {
-        // Merge the TS warps that share a KV head through shared memory.
-        float *mine = merge + warp * Cfg::MSTRIDE;
-        if (lane == 0) {
+        // Merge the TS warps that share a KV head: warps tp > 0 hand their state
+        // to the tp == 0 warp through shared memory.
+        if (tp > 0) {
+          float *mine = merge + ((tp - 1) * HKV + kvh) * Cfg::MSTRIDE;
+          if (lane == 0) {
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            mine[g] = m[g];
-            mine[4 + g] = l[g];
+            for (int g = 0; g < G; ++g) {
+              mine[g] = m[g];
+              mine[4 + g] = l[g];
+            }
           }
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int j = 0; j < CH; ++j) {
+              float4 *dst =
+                  reinterpret_cast<float4 *>(mine + Cfg::MHDR + g * D + 256 * j + 8 * lane);
+              dst[0] = make_float4(o[g][4 * j].x, o[g][4 * j].y, o[g][4 * j + 1].x,
+                                   o[g][4 * j + 1].y);
+              dst[1] = make_float4(o[g][4 * j + 2].x, o[g][4 * j + 2].y, o[g][4 * j + 3].x,
+                                   o[g][4 * j + 3].y);
+            }
         }
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-          for (int j = 0; j < CH; ++j) {
-            float4 *dst =
-                reinterpret_cast<float4 *>(mine + Cfg::MHDR + g * D + 256 * j + 8 * lane);
-            dst[0] = make_float4(o[g][4 * j].x, o[g][4 * j].y, o[g][4 * j + 1].x,
-                                 o[g][4 * j + 1].y);
-            dst[1] = make_float4(o[g][4 * j + 2].x, o[g][4 * j + 2].y, o[g][4 * j + 3].x,
-                                 o[g][4 * j + 3].y);
-          }
         named_bar_sync(1, Cfg::kComputeWarps * 32);
         if (tp == 0) {
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            float M = -INFINITY;
-            for (int k = 0; k < Cfg::TS; ++k)
-              M = fmaxf(M, merge[(kvh + HKV * k) * Cfg::MSTRIDE + g]);
-            float Ls = 0.f;
-            float wk[Cfg::TS];
+            float M = m[g];
+            for (int k = 1; k < Cfg::TS; ++k)
+              M = fmaxf(M, merge[((k - 1) * HKV + kvh) * Cfg::MSTRIDE + g]);
+            const float w0 = (m[g] == -INFINITY) ? 0.f : exp2f(m[g] - M);
+            float Ls = l[g] * w0;
+            const float2 w02 = make_float2(w0, w0);
 #pragma unroll
-            for (int k = 0; k < Cfg::TS; ++k) {
-              const float *src = merge + (kvh + HKV * k) * Cfg::MSTRIDE;
-              wk[k] = (src[g] == -INFINITY) ? 0.f : exp2f(src[g] - M);
-              Ls += src[4 + g] * wk[k];
-            }
+            for (int e = 0; e < P2; ++e) o[g][e] = __fmul2_rn(o[g][e], w02);
 #pragma unroll
-            for (int e = 0; e < P2; ++e) o[g][e] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int k = 0; k < Cfg::TS; ++k) {
-              const float *src = merge + (kvh + HKV * k) * Cfg::MSTRIDE + Cfg::MHDR + g * D;
-              const float2 w2 = make_float2(wk[k], wk[k]);
+            for (int k = 1; k < Cfg::TS; ++k) {
+              const float *src = merge + ((k - 1) * HKV + kvh) * Cfg::MSTRIDE;
+              const float wk = (src[g] == -INFINITY) ? 0.f : exp2f(src[g] - M);
+              Ls += src[4 + g] * wk;
+              const float2 w2 = make_float2(wk, wk);
+              src += Cfg::MHDR + g * D;
 #pragma unroll
               for (int j = 0; j < CH; ++j)
 #pragma unroll
@@ -390,14 +404,12 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads, 1)
         named_bar_sync(1, Cfg::kComputeWarps * 32);
       }
       if (tp == 0 && ok) {
-        int32_t cf, cl;
-        unit_chunks(s.unit_start, s.n, plan->chunk, cf, cl);
-        const bool single = (cf == cl);
+        const bool single = s.whole();
         const int64_t slot = static_cast<int64_t>(c) + s.unit;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const int h = kvh * G + g;
-          const float inv = 1.f / l[g];
+          const float inv = __fdividef(1.f, l[g]);
           const float lse_v = (m[g] + log2f(l[g])) * 0.69314718055994530942f;
           if (single) {
             uint16_t *dst = p.out + (static_cast<int64_t>(s.b) * p.n_q_heads + h) * D;

@@ -31,6 +31,7 @@ struct Geometry {
   int32_t window;
   int32_t capacity;
   int32_t nchunks;  // P = gridDim.x of the decode kernel
+  int32_t align;    // chunk sizes are rounded up to a multiple of this (tokens)
 };
 
 // Positions one decode step attends for context length L (clamped to the cache;
@@ -86,7 +87,7 @@ __device__ void plan_chunk(const Geometry &g, int32_t c, ChunkPlan *plan) {
     acc += attended_count(__ldg(g.seqlens + b), g.window, g.capacity, bad);
   const int64_t total = warp_sum_i64(acc) * g.units_per_seq;
   const int anybad = __any_sync(0xffffffffu, bad);
-  const int64_t chunk = total > 0 ? ceil_div64(total, g.nchunks) : 1;
+  const int64_t chunk = total > 0 ? ceil_div64(ceil_div64(total, g.nchunks), g.align) * g.align : 1;
   const int64_t cs = imin64(static_cast<int64_t>(c) * chunk, total);
   const int64_t ce = imin64(cs + chunk, total);
   // First sequence whose flattened range ends after cs.
@@ -131,6 +132,8 @@ struct Segment {
   int32_t lo, hi;     // local offsets [lo, hi) within the unit's attended range
   int32_t first_pos;  // logical position of local offset 0 (= L_b - n)
   int64_t unit_start; // flattened offset of the unit
+  // The segment covers its whole unit: the result is final, no partial.
+  __device__ __forceinline__ bool whole() const { return lo == 0 && hi == n; }
 };
 
 // Walks the segments of one chunk in order.  Every thread of a CTA may run its

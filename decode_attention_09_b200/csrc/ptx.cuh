@@ -56,23 +56,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended (not issuing) for up to
+// `hint_ns` while the phase is incomplete; it resumes when the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t parity,
+                                                      uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Suspend limit of one wait attempt: waiting warps sleep instead of spinning
+// (so they take no issue slots from the warps doing the work) and notice an
+// abort within this time.
+constexpr uint32_t kSuspendHintNs = 1000000;
+
 // Wait for the phase with the given parity to complete.  Gives up (returns
-// false) when *abort becomes non-zero or after kWaitLimitCycles of the SM clock
-// (the SM-local counter: reading the global nanosecond timer is far slower);
+// false) when *abort becomes non-zero or after kWaitLimitCycles of the SM clock;
 // on its own timeout it raises *abort and latches kStatusTimeout in *status.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           uint32_t *status) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (*abort) return false;
-      if (clock64() - t0 > kWaitLimitCycles) {
-        *abort = 1;
-        atomicOr(status, kStatusTimeout);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      *abort = 1;
+      atomicOr(status, kStatusTimeout);
+      return false;
     }
   }
 }

@@ -35,11 +35,13 @@
 // by exp2(m_old - m_new), and the tile proceeds.  The result is exact: out is
 // O/L and LSE is m_ref + log2 L for the final reference.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads; warp 1 owns TMEM and issues
-// MMAs (one elected lane); warps 2-5 run the softmax (TMEM sub-partition
-// warp % 4).  S is double buffered in TMEM so the tensor core computes tile i+1
-// while tile i's softmax runs.  Every wait is bounded; on a timeout all roles
-// fast-forward, drain their copies / MMAs and free TMEM.
+// Warp roles (224 threads): warp 0 issues TMA loads; warp 1 owns TMEM and issues
+// the QK MMAs; warp 6 issues the P.V MMAs and releases KV stages (one elected
+// lane each, so a P.V never waits behind the next tile's data); warps 2-5 run
+// the softmax (TMEM sub-partition warp % 4).  S is double buffered in TMEM so
+// the tensor core computes tile i+1 while tile i's softmax runs.  Every wait is
+// bounded; on a timeout all roles fast-forward, drain their copies / MMAs and
+// free TMEM.
 #pragma once
 
 #include <cstdint>
@@ -76,7 +78,7 @@ struct TcConfig {
   static constexpr int OFF_BAR = OFF_P + 2 * PB;
   static constexpr int OFF_RED = OFF_BAR + 256;
   static constexpr int SMEM = OFF_RED + 2 * 4 * G * 4 + 1024;
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 224;
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t S_COL = 0;                // 2 buffers x 4 partial sums x 16 columns
   static constexpr uint32_t O_COL = 128;              // 4 d-blocks x (16 hi + 16 lo) columns
@@ -93,6 +95,7 @@ struct TileIter {
   SlotRuns runs;
   int32_t run, t0;
   bool have_seg;
+  bool newest;  // the last tile yielded holds the unit's newest position (L - 1)
 
   __device__ __forceinline__ void init(const Geometry &g, const ChunkPlan &p) {
     seg_it.init(g, p);
@@ -113,6 +116,7 @@ struct TileIter {
     }
     row = runs.start(run) + t0;
     ntok = min(TcConfig::TILE, runs.len(run) - t0);
+    newest = seg.lo + (run == 1 ? runs.len0 : 0) + t0 + ntok == seg.n;
     t0 += TcConfig::TILE;
     if (t0 >= runs.len(run)) {
       ++run;
@@ -167,10 +171,10 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
   uint64_t *pfull = bars + 12;      // [2] softmax -> MMA (P of tile i in buffer i & 1)
   uint64_t *ofull = bars + 14;      // [2] MMA -> softmax: P.V of tile i done (barrier i & 1)
   uint64_t *oempty = bars + 16;     // softmax -> MMA: O of a finished segment read out
-  uint64_t *drain = bars + 17;
-  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 18);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 19);
-  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 20);  // 48 bytes, ends before +256
+  uint64_t *drain = bars + 17;      // [2] QK warp, P.V warp: all their MMAs done
+  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 19);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 20);
+  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 21);  // 48 bytes, ends before +256
   float *redmax = reinterpret_cast<float *>(smem + Cfg::OFF_RED);  // [4 warps][16]
   float *redsum = redmax + 4 * G;                                  // [4 warps][16]
 
@@ -192,7 +196,8 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
       mbar_init(&ofull[s], 1);
     }
     mbar_init(oempty, 4);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -205,7 +210,9 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
     tmem_relinquish();
   }
   grid_launch_dependents();
-  grid_dependency_wait();
+  // The split plan reads only seqlens, so it (and the producer's first KV
+  // loads below) may run before the preceding kernel has completed; every other
+  // global access waits for it (griddepcontrol.wait) in the role that makes it.
   if (warp == 2) plan_chunk(p.geo, c, plan);
   tc_fence_before();
   __syncthreads();
@@ -213,6 +220,7 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
   const uint32_t tmem = *tmem_base_smem;
 
   if (c == 0 && warp == 2 && plan->bad) {
+    grid_dependency_wait();
     if (lane == 0) atomicOr(p.status, kStatusSeqlen);
     for (int32_t b = 0; b < p.geo.batch; ++b) {
       bool dummy = false;
@@ -231,31 +239,66 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
   if (warp == 0) {
     // -------------------------------------------------------------- TMA
     // The whole warp walks the schedule and waits (values stay warp-uniform);
-    // one elected lane issues the copies.
+    // one elected lane issues the copies.  A new segment's Q may only replace
+    // the previous one once that segment's last QK is done; instead of stalling
+    // the KV stream on it, the Q load is issued as soon as that has happened,
+    // and at the latest before waiting on a stage whose release needs it.
     const uint64_t pol = l2_evict_first_policy();
     bool ok = true;
-    uint32_t i = 0, nseg = 0;
+    uint32_t i = 0, seg_count = 0, q_issued = 0;
+    int32_t qrows[8];            // Q rows of segments whose Q is not issued yet
+    uint32_t stage_seg[NST];     // segment of the tile last loaded into each stage
+    auto issue_q = [&](bool block) -> bool {  // warp-uniform result
+      if (q_issued > 0) {
+        bool got = block ? mbar_wait(qempty, (q_issued - 1) & 1, abort_flag, p.status)
+                         : mbar_try_wait(qempty, (q_issued - 1) & 1);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (block) ok = false;
+          return false;
+        }
+      }
+      const int32_t qrow = qrows[q_issued & 7];
+      if (elect_one()) {
+        mbar_arrive_expect_tx(qfull, Cfg::QB);
+#pragma unroll
+        for (int j = 0; j < D / 64; ++j)
+          tma_load_2d(qs + j * (G * 128), &qmap, 64 * j, qrow, qfull);
+      }
+      __syncwarp();
+      ++q_issued;
+      return true;
+    };
     TileIter it;
     it.init(p.geo, *plan);
     int32_t row, ntok;
     bool first, last;
+    // Until the preceding kernel completes, only cache rows of positions before
+    // each sequence's newest one are read (earlier decode steps wrote them);
+    // q and the newest row are loaded after griddepcontrol.wait.
+    bool waited = false;
+    auto ensure_waited = [&]() {
+      if (!waited) {
+        grid_dependency_wait();
+        waited = true;
+      }
+    };
     while (ok && it.next(C, row, ntok, first, last)) {
       if (first) {
-        if (nseg > 0 && !mbar_wait(qempty, (nseg - 1) & 1, abort_flag, p.status)) ok = false;
-        if (!__all_sync(0xffffffffu, ok)) break;
-        const int32_t qrow = it.seg.b * p.n_q_heads + it.seg.x * G;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(qfull, Cfg::QB);
-#pragma unroll
-          for (int j = 0; j < D / 64; ++j)
-            tma_load_2d(qs + j * (G * 128), &qmap, 64 * j, qrow, qfull);
-        }
-        __syncwarp();
-        ++nseg;
+        // At most NST + 1 segments can be pending (see the wait below), so 8 slots do.
+        qrows[seg_count & 7] = it.seg.b * p.n_q_heads + it.seg.x * G;
+        ++seg_count;
+      }
+      if (i >= NST || it.newest) ensure_waited();
+      while (ok && waited && q_issued < seg_count && issue_q(false)) {
       }
       const int st = i % NST;
-      if (i >= NST && !mbar_wait(&empty[st], ((i / NST) - 1) & 1, abort_flag, p.status)) ok = false;
+      if (i >= NST) {
+        // The tile in this stage is released after its P.V, which needs its Q.
+        while (ok && q_issued <= stage_seg[st]) issue_q(true);
+        if (ok && !mbar_wait(&empty[st], ((i / NST) - 1) & 1, abort_flag, p.status)) ok = false;
+      }
       if (!__all_sync(0xffffffffu, ok)) break;
+      stage_seg[st] = seg_count - 1;
       if (elect_one()) {
         mbar_arrive_expect_tx(&full[st], Cfg::STAGEB);
 #pragma unroll
@@ -266,64 +309,33 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
       __syncwarp();
       ++i;
     }
+    ensure_waited();
+    while (ok && q_issued < seg_count) issue_q(true);
     // Drain: never leave with copies in flight into shared memory.
     volatile int no_abort = 0;
     for (uint32_t f = i > NST ? i - NST : 0; f < i; ++f)
       mbar_wait(&full[f % NST], (f / NST) & 1, &no_abort, p.status);
-    if (nseg > 0) mbar_wait(qfull, (nseg - 1) & 1, &no_abort, p.status);
+    if (q_issued > 0) mbar_wait(qfull, (q_issued - 1) & 1, &no_abort, p.status);
   } else if (warp == 1) {
-    // -------------------------------------------------------------- MMA
+    // ----------------------------------------------------------- QK MMA
     // Converged warp: descriptors are warp-uniform, one elected lane issues
     // every MMA and commit (commits track that lane's MMAs).
     const uint32_t idesc_qk = idesc_bf16_f32(64, 16, false, false);
-    const uint32_t idesc_pv = idesc_bf16_f32(128, 32, true, true);
     // Base descriptors; an operand at byte offset o from a base is base + (o >> 4)
     // (the 14-bit start field holds address >> 4 and never carries: smem < 256 KiB).
-    const uint64_t kdesc = smem_desc_sw128(smem_u32(stages), 16, 1024);       // K tile, K-major
-    const uint64_t qdesc = smem_desc_sw128(smem_u32(qs), 16, 1024);           // Q, K-major
-    const uint64_t vdesc = smem_desc_sw128(smem_u32(stages), Cfg::BOXB, 1024); // V^T, MN-major
-    const uint64_t pdesc = smem_desc(smem_u32(ps), 4096, 512, 4);              // P^T, MN-major SW64
+    const uint64_t kdesc = smem_desc_sw128(smem_u32(stages), 16, 1024);  // K tile, K-major
+    const uint64_t qdesc = smem_desc_sw128(smem_u32(qs), 16, 1024);      // Q, K-major
     bool ok = true;
     uint32_t i = 0, nseg = 0;
-    int32_t prev = -1;       // tile whose P.V is still to issue
-    bool prev_first = false; // ... and whether it opened its segment
-    uint32_t prev_seg = 0;   // ... and that segment's index in this CTA
     TileIter it;
     it.init(p.geo, *plan);
     int32_t row, ntok;
     bool first, last;
-    auto issue_pv = [&](uint32_t t, bool seg_first, uint32_t seg) -> bool {
-      bool w = mbar_wait(&pfull[t & 1], (t >> 1) & 1, abort_flag, p.status);
-      // A segment's first P.V overwrites O: the previous segment must be read out.
-      if (w && seg_first && seg > 0) w = mbar_wait(oempty, (seg - 1) & 1, abort_flag, p.status);
-      if (!__all_sync(0xffffffffu, w)) return false;
-      tc_fence_after();
-      const uint64_t a0 = vdesc + (((t % NST) * Cfg::STAGEB) >> 4);
-      const uint64_t b0 = pdesc + (((t & 1) * Cfg::PB) >> 4);
-      if (elect_one()) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          // P^T: MN-major, 64-byte swizzle, a token row of 32 bf16 = 64 B; 16 tokens
-          // per k-step = two 512-byte atoms.
-          const uint64_t bd = b0 + ((kk * 1024) >> 4);
-#pragma unroll
-          for (int jb = 0; jb < 4; ++jb) {
-            const uint64_t ad = a0 + ((2 * jb * Cfg::BOXB + kk * 2048) >> 4);
-            tc_mma_bf16(tmem + Cfg::O_COL + jb * 32, ad, bd, idesc_pv, !(seg_first && kk == 0));
-          }
-        }
-        tc_commit(&ofull[t & 1]);
-        tc_commit(&empty[t % NST]);
-      }
-      __syncwarp();
-      return true;
-    };
-    uint32_t cur_seg = 0;
     while (ok && it.next(C, row, ntok, first, last)) {
       if (first) {
         if (!mbar_wait(qfull, nseg & 1, abort_flag, p.status)) ok = false;
         if (!__all_sync(0xffffffffu, ok)) break;
-        cur_seg = nseg++;
+        ++nseg;
       }
       const int st = i % NST, sb = i & 1;
       if (!mbar_wait(&full[st], (i / NST) & 1, abort_flag, p.status)) ok = false;
@@ -346,23 +358,61 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
         if (last) tc_commit(qempty);
       }
       __syncwarp();
-      if (prev >= 0 && !issue_pv(static_cast<uint32_t>(prev), prev_first, prev_seg)) {
+      ++i;
+    }
+    // Drain: wait until every issued MMA has completed before TMEM is freed.
+    if (elect_one()) tc_commit(&drain[0]);
+    __syncwarp();
+    volatile int no_abort = 0;
+    mbar_wait(&drain[0], 0, &no_abort, p.status);
+  } else if (warp == 6) {
+    // ---------------------------------------------------------- P.V MMA
+    const uint32_t idesc_pv = idesc_bf16_f32(128, 32, true, true);
+    const uint64_t vdesc = smem_desc_sw128(smem_u32(stages), Cfg::BOXB, 1024);  // V^T, MN-major
+    const uint64_t pdesc = smem_desc(smem_u32(ps), 4096, 512, 4);               // P^T, MN-major SW64
+    bool ok = true;
+    uint32_t t = 0, nseg = 0;
+    TileIter it;
+    it.init(p.geo, *plan);
+    int32_t row, ntok;
+    bool first, last;
+    while (ok && it.next(C, row, ntok, first, last)) {
+      bool w = mbar_wait(&pfull[t & 1], (t >> 1) & 1, abort_flag, p.status);
+      // A segment's first P.V overwrites O: the previous segment must be read out.
+      if (w && first && nseg > 0) w = mbar_wait(oempty, (nseg - 1) & 1, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         break;
       }
-      prev = static_cast<int32_t>(i);
-      prev_first = first;
-      prev_seg = cur_seg;
-      ++i;
+      if (first) ++nseg;
+      tc_fence_after();
+      const uint64_t a0 = vdesc + (((t % NST) * Cfg::STAGEB) >> 4);
+      const uint64_t b0 = pdesc + (((t & 1) * Cfg::PB) >> 4);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          // P^T: MN-major, 64-byte swizzle, a token row of 32 bf16 = 64 B; 16 tokens
+          // per k-step = two 512-byte atoms.
+          const uint64_t bd = b0 + ((kk * 1024) >> 4);
+#pragma unroll
+          for (int jb = 0; jb < 4; ++jb) {
+            const uint64_t ad = a0 + ((2 * jb * Cfg::BOXB + kk * 2048) >> 4);
+            tc_mma_bf16(tmem + Cfg::O_COL + jb * 32, ad, bd, idesc_pv, !(first && kk == 0));
+          }
+        }
+        tc_commit(&ofull[t & 1]);
+        tc_commit(&empty[t % NST]);
+      }
+      __syncwarp();
+      ++t;
     }
-    if (ok && prev >= 0) ok = issue_pv(static_cast<uint32_t>(prev), prev_first, prev_seg);
-    // Drain: wait until every issued MMA has completed before TMEM is freed.
-    if (elect_one()) tc_commit(drain);
+    if (elect_one()) tc_commit(&drain[1]);
     __syncwarp();
     volatile int no_abort = 0;
-    mbar_wait(drain, 0, &no_abort, p.status);
+    mbar_wait(&drain[1], 0, &no_abort, p.status);
   } else {
     // ---------------------------------------------------------- softmax
+    grid_dependency_wait();  // outputs and workspace are written below
     // M=64 puts tile token r in TMEM lane (r % 16) + 32 * (r / 16): lanes 0-15 of
     // each warp receive one token's 16 scores.  Lanes 16-31 take heads 8-15 of
     // the token of lane - 16, so every lane handles one token and 8 heads.
@@ -502,13 +552,12 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
         // Rows past the attended range hold other cache contents (possibly
         // NaN); they get weight 0, but 0 * NaN would still reach O, so clear them.
         uint8_t *tile = stages + (i % NST) * Cfg::STAGEB;
-        const int per_box = (Cfg::TILE - ntok) * 8;
-        for (int e = threadIdx.x - 64; e < per_box * (D / 64); e += 128) {
-          const int box = e / per_box;
-          const int rem = e - box * per_box;
-          *reinterpret_cast<uint4 *>(tile + box * Cfg::BOXB + (ntok + (rem >> 3)) * 128 +
-                                     (rem & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
-        }
+        const int per_box = (Cfg::TILE - ntok) * 8;  // 16-byte chunks past row ntok
+#pragma unroll 1
+        for (int box = 0; box < D / 64; ++box)
+          for (int e = threadIdx.x - 64; e < per_box; e += 128)
+            *reinterpret_cast<uint4 *>(tile + box * Cfg::BOXB + (ntok + (e >> 3)) * 128 +
+                                       (e & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -529,25 +578,13 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
         if ((lane & 1) == 0) redsum[qd * G + (lane >> 1)] = ls;
         named_bar_sync(1, 128);
         const Segment &sg = it.seg;
-        int32_t cf, cl;
-        unit_chunks(sg.unit_start, sg.n, plan->chunk, cf, cl);
-        const bool single = (cf == cl);
+        const bool single = sg.whole();
         const int64_t slot = static_cast<int64_t>(c) + sg.unit;
         const int h0 = sg.x * G;
         float inv[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float L = (redsum[h] + redsum[G + h]) + (redsum[2 * G + h] + redsum[3 * G + h]);
-          inv[h] = 1.f / L;
-          if (ok && qd == 0 && lane == h) {
-            const float lse_v = (m_ref[h] + log2f(L)) * 0.69314718055994530942f;
-            if (single) {
-              if (p.lse != nullptr) p.lse[static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + h] = lse_v;
-            } else {
-              p.ws_lse[slot * G + h] = lse_v;
-            }
-          }
-        }
+        for (int h = 0; h < G; ++h)
+          inv[h] = __fdividef(1.f, (redsum[h] + redsum[G + h]) + (redsum[2 * G + h] + redsum[3 * G + h]));
         if (ok) {
           tc_fence_after();
 #pragma unroll
@@ -569,6 +606,19 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(oempty);
+          if (qd == 0 && lane < G) {  // LSE of head `lane`: one store per lane
+            float mr = m_ref[0];
+#pragma unroll
+            for (int h = 1; h < G; ++h) mr = (lane == h) ? m_ref[h] : mr;
+            const float L = (redsum[lane] + redsum[G + lane]) +
+                            (redsum[2 * G + lane] + redsum[3 * G + lane]);
+            const float lse_v = (mr + log2f(L)) * 0.69314718055994530942f;
+            if (single) {
+              if (p.lse != nullptr) p.lse[static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + lane] = lse_v;
+            } else {
+              p.ws_lse[slot * G + lane] = lse_v;
+            }
+          }
         }
       }
       ++i;

@@ -36,6 +36,15 @@
  *    enqueued asynchronously; no call synchronises except
  *    gdattn_check_device_status.  Decode and combine only enqueue kernels, so they
  *    can be captured into a CUDA graph.
+ *  - Kernels are launched with programmatic dependent launch: gdattn_decode may
+ *    start while the preceding kernel on the stream is still draining (once that
+ *    kernel has signalled griddepcontrol.launch_dependents, or exited).  In that
+ *    window it reads only seqlens and the cache rows of positions below each
+ *    sequence's newest one (L_b - 1), i.e. rows written by earlier decode steps.
+ *    q, the newest cache row, out, lse and the workspace are accessed only after
+ *    the preceding kernel has completed.  A preceding kernel that triggers its
+ *    dependents early must therefore not write seqlens or older cache rows after
+ *    its trigger; kernels that never trigger early (the default) are unaffected.
  *  - Arguments are checked on the host before anything is enqueued; a failed
  *    check returns its status and launches nothing.  A launch failure returns
  *    GDATTN_ERR_CUDA.  Problems only the device can see (a context length that
@@ -94,15 +103,22 @@ size_t gdattn_workspace_size(int32_t batch, int32_t max_seqlen, const gdattn_lay
 
 /*
  * Number of CTAs the planner splits this layer's KV range across (the value
- * gdattn_decode uses for the same arguments on the current device): one decode
- * kernel launch, plus one LSE-combine launch when the result is above 1.
- * Returns 0 on invalid arguments.
+ * gdattn_decode uses for the same arguments on the current device).  Returns 0
+ * on invalid arguments.
  */
 int32_t gdattn_plan_splits(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc);
 
 /*
- * Zero the workspace's status word.  Call once after allocating a workspace
- * (or zero the whole buffer yourself); the library keeps it clear afterwards.
+ * Kernel launches gdattn_decode makes for these arguments: the decode kernel,
+ * plus the LSE-combine kernel when the KV range is split over more than one
+ * CTA.  Returns 0 on invalid arguments.
+ */
+int32_t gdattn_plan_launches(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc);
+
+/*
+ * Zero the workspace (its status word and partials).  Call once after
+ * allocating a workspace, or zero it yourself; the library keeps the status
+ * word clear afterwards.
  */
 gdattn_status gdattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 

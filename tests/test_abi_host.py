@@ -34,7 +34,7 @@ def declared_functions():
 def test_header_declares_the_api():
     names = declared_functions()
     for n in ("gdattn_decode", "gdattn_combine", "gdattn_workspace_size", "gdattn_workspace_init",
-              "gdattn_plan_splits",
+              "gdattn_plan_splits", "gdattn_plan_launches",
               "gdattn_check_device_status", "gdattn_status_string", "gdattn_version"):
         assert n in names
 
