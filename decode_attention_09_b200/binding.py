@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.gdattn_workspace_init.restype = ctypes.c_int
         L.gdattn_decode.argtypes = [vp, vp, vp, vp, i32, i32, descp, vp, vp, vp, sz, vp]
         L.gdattn_decode.restype = ctypes.c_int
+        L.gdattn_decode_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, descp, vp, vp, vp]
+        L.gdattn_decode_noalloc.restype = ctypes.c_int
         L.gdattn_combine.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp]
         L.gdattn_combine.restype = ctypes.c_int
         L.gdattn_check_device_status.argtypes = [vp, vp]
@@ -175,6 +177,31 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor], seqlens:
     return out, lse
 
 
+NOALLOC_SCRATCH_BYTES = 8 << 20  # GDATTN_NOALLOC_SCRATCH_BYTES
+
+
+def decode_noalloc_raw(q, k, v, seqlens, batch, max_seqlen, desc, out, lse, stream) -> int:
+    """gdattn_decode_noalloc on raw addresses (ints); returns the status code."""
+    return int(lib().gdattn_decode_noalloc(q, k, v, seqlens, int(batch), int(max_seqlen),
+                                           ctypes.byref(desc), out, lse, stream))
+
+
+def decode_noalloc(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor],
+                   seqlens: torch.Tensor, desc: LayerDesc, max_seqlen: int,
+                   out: torch.Tensor, lse: Optional[torch.Tensor] = None, stream=None):
+    """One layer through gdattn_decode_noalloc (scratch inside the library).
+
+    `out` (and `lse`, if wanted) are caller-owned; nothing is allocated here.
+    Calls that can overlap in time on one device race on the shared scratch.
+    """
+    B = q.shape[0]
+    st = decode_noalloc_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(seqlens), B, max_seqlen, desc,
+                            _ptr(out), _ptr(lse), _stream_handle(stream))
+    if st != GDATTN_OK:
+        raise GdattnError(st, "gdattn_decode_noalloc")
+    return out, lse
+
+
 def combine(o_partial: torch.Tensor, lse_partial: torch.Tensor, out: Optional[torch.Tensor] = None,
             lse: Optional[torch.Tensor] = None, stream=None):
     """gdattn_combine: o_partial fp32 [B,Hq,S,D], lse_partial fp32 [B,Hq,S]."""
@@ -190,5 +217,6 @@ def combine(o_partial: torch.Tensor, lse_partial: torch.Tensor, out: Optional[to
     return out, lse
 
 
-def check_device_status(workspace: torch.Tensor, stream=None) -> int:
+def check_device_status(workspace: Optional[torch.Tensor], stream=None) -> int:
+    """Read and clear a workspace's status word (None: the no-alloc scratch)."""
     return int(lib().gdattn_check_device_status(_ptr(workspace), _stream_handle(stream)))

@@ -17,6 +17,12 @@
 
 using namespace gdattn;
 
+// Split-KV scratch of gdattn_decode_noalloc: one array per device context,
+// laid out like a caller workspace (status word, partial LSE, partial O).
+// A __device__ array without initialiser occupies no space in the binary.
+constexpr size_t kNoallocScratchBytes = GDATTN_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
+
 namespace {
 
 enum class PathKind { kNone, kCore, kTc };
@@ -264,59 +270,10 @@ gdattn_status launch_combine_internal(const LayerPlan &pl, const Geometry &geo, 
                                                                             : GDATTN_ERR_CUDA;
 }
 
-}  // namespace
-
-// ===================================================================== ABI
-extern "C" {
-
-int32_t gdattn_version(void) { return GDATTN_VERSION; }
-
-const char *gdattn_status_string(gdattn_status s) {
-  switch (s) {
-    case GDATTN_OK: return "GDATTN_OK";
-    case GDATTN_ERR_INVALID_ARG: return "GDATTN_ERR_INVALID_ARG";
-    case GDATTN_ERR_UNSUPPORTED: return "GDATTN_ERR_UNSUPPORTED";
-    case GDATTN_ERR_MISALIGNED: return "GDATTN_ERR_MISALIGNED";
-    case GDATTN_ERR_WORKSPACE: return "GDATTN_ERR_WORKSPACE";
-    case GDATTN_ERR_CUDA: return "GDATTN_ERR_CUDA";
-    case GDATTN_ERR_DEVICE_TIMEOUT: return "GDATTN_ERR_DEVICE_TIMEOUT";
-    case GDATTN_ERR_DEVICE_SEQLEN: return "GDATTN_ERR_DEVICE_SEQLEN";
-  }
-  return "GDATTN_UNKNOWN_STATUS";
-}
-
-size_t gdattn_workspace_size(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc) {
-  LayerPlan pl;
-  if (make_plan(batch, max_seqlen, desc, pl) != GDATTN_OK) return 0;
-  return pl.bytes;
-}
-
-int32_t gdattn_plan_splits(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc) {
-  LayerPlan pl;
-  if (make_plan(batch, max_seqlen, desc, pl) != GDATTN_OK) return 0;
-  return pl.grid;
-}
-
-int32_t gdattn_plan_launches(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc) {
-  LayerPlan pl;
-  if (make_plan(batch, max_seqlen, desc, pl) != GDATTN_OK) return 0;
-  return pl.grid > 1 ? 2 : 1;
-}
-
-gdattn_status gdattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
-  if (workspace == nullptr || workspace_bytes < kStatusBytes) return GDATTN_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return GDATTN_ERR_MISALIGNED;
-  return cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) ==
-                 cudaSuccess
-             ? GDATTN_OK
-             : GDATTN_ERR_CUDA;
-}
-
-gdattn_status gdattn_decode(const void *q, const void *k_cache, const void *v_cache,
-                            const int32_t *seqlens, int32_t batch, int32_t max_seqlen,
-                            const gdattn_layer_desc *desc, void *out, float *lse,
-                            void *workspace, size_t workspace_bytes, void *stream_) {
-  // Host-only checks first: nothing below touches CUDA until they pass.
+// Host checks shared by both decode entry points (the workspace aside).
+gdattn_status check_decode_args(const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *seqlens, int32_t batch, int32_t max_seqlen,
+                                const gdattn_layer_desc *desc, const void *out, const float *lse) {
   if (q == nullptr || k_cache == nullptr || seqlens == nullptr || out == nullptr || desc == nullptr)
     return GDATTN_ERR_INVALID_ARG;
   gdattn_status st = check_desc(desc);
@@ -328,15 +285,15 @@ gdattn_status gdattn_decode(const void *q, const void *k_cache, const void *v_ca
       !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return GDATTN_ERR_MISALIGNED;
-  if (workspace == nullptr) return GDATTN_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return GDATTN_ERR_MISALIGNED;
-  LayerPlan pl;
-  st = make_plan(batch, max_seqlen, desc, pl);
-  if (st != GDATTN_OK) return st;
-  if (workspace_bytes < pl.bytes) return GDATTN_ERR_WORKSPACE;
+  return GDATTN_OK;
+}
 
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  uint8_t *ws = static_cast<uint8_t *>(workspace);
+// Enqueues the decode kernel (and the combine when the plan splits) with the
+// split-KV scratch at `ws`: status word, then partial LSE, then partial O.
+gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_cache,
+                             const void *v_cache, const int32_t *seqlens, int32_t batch,
+                             const gdattn_layer_desc *desc, void *out, float *lse, uint8_t *ws,
+                             cudaStream_t stream) {
   uint32_t *status = reinterpret_cast<uint32_t *>(ws);
   float *ws_lse = reinterpret_cast<float *>(ws + pl.off_lse);
   float *ws_o = reinterpret_cast<float *>(ws + pl.off_o);
@@ -426,6 +383,114 @@ gdattn_status gdattn_decode(const void *q, const void *k_cache, const void *v_ca
   return GDATTN_OK;
 }
 
+// -------------------------------------------------- fixed scratch (no alloc)
+constexpr int kMaxDevices = 64;
+
+// Address of g_noalloc_scratch on the current device.  The first call on a
+// device looks it up and enqueues a clear of the status word on `stream`
+// (the only part that must start at zero: every partial slot the combine
+// reads is written first by the decode kernel of the same call).
+gdattn_status noalloc_scratch(cudaStream_t stream, uint8_t **addr) {
+  static std::mutex mu;
+  static void *by_device[kMaxDevices] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (by_device[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return GDATTN_ERR_CUDA;
+    if (cudaMemsetAsync(p, 0, kStatusBytes, stream) != cudaSuccess) return GDATTN_ERR_CUDA;
+    by_device[dev] = p;
+  }
+  *addr = static_cast<uint8_t *>(by_device[dev]);
+  return GDATTN_OK;
+}
+
+}  // namespace
+
+// ===================================================================== ABI
+extern "C" {
+
+int32_t gdattn_version(void) { return GDATTN_VERSION; }
+
+const char *gdattn_status_string(gdattn_status s) {
+  switch (s) {
+    case GDATTN_OK: return "GDATTN_OK";
+    case GDATTN_ERR_INVALID_ARG: return "GDATTN_ERR_INVALID_ARG";
+    case GDATTN_ERR_UNSUPPORTED: return "GDATTN_ERR_UNSUPPORTED";
+    case GDATTN_ERR_MISALIGNED: return "GDATTN_ERR_MISALIGNED";
+    case GDATTN_ERR_WORKSPACE: return "GDATTN_ERR_WORKSPACE";
+    case GDATTN_ERR_CUDA: return "GDATTN_ERR_CUDA";
+    case GDATTN_ERR_DEVICE_TIMEOUT: return "GDATTN_ERR_DEVICE_TIMEOUT";
+    case GDATTN_ERR_DEVICE_SEQLEN: return "GDATTN_ERR_DEVICE_SEQLEN";
+  }
+  return "GDATTN_UNKNOWN_STATUS";
+}
+
+size_t gdattn_workspace_size(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc) {
+  LayerPlan pl;
+  if (make_plan(batch, max_seqlen, desc, pl) != GDATTN_OK) return 0;
+  return pl.bytes;
+}
+
+int32_t gdattn_plan_splits(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc) {
+  LayerPlan pl;
+  if (make_plan(batch, max_seqlen, desc, pl) != GDATTN_OK) return 0;
+  return pl.grid;
+}
+
+int32_t gdattn_plan_launches(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc) {
+  LayerPlan pl;
+  if (make_plan(batch, max_seqlen, desc, pl) != GDATTN_OK) return 0;
+  return pl.grid > 1 ? 2 : 1;
+}
+
+gdattn_status gdattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
+  if (workspace == nullptr || workspace_bytes < kStatusBytes) return GDATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GDATTN_ERR_MISALIGNED;
+  return cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? GDATTN_OK
+             : GDATTN_ERR_CUDA;
+}
+
+gdattn_status gdattn_decode(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *seqlens, int32_t batch, int32_t max_seqlen,
+                            const gdattn_layer_desc *desc, void *out, float *lse,
+                            void *workspace, size_t workspace_bytes, void *stream) {
+  // Host-only checks first: nothing below touches CUDA until they pass.
+  gdattn_status st = check_decode_args(q, k_cache, v_cache, seqlens, batch, max_seqlen, desc,
+                                       out, lse);
+  if (st != GDATTN_OK) return st;
+  if (workspace == nullptr) return GDATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GDATTN_ERR_MISALIGNED;
+  LayerPlan pl;
+  st = make_plan(batch, max_seqlen, desc, pl);
+  if (st != GDATTN_OK) return st;
+  if (workspace_bytes < pl.bytes) return GDATTN_ERR_WORKSPACE;
+  return enqueue_decode(pl, q, k_cache, v_cache, seqlens, batch, desc, out, lse,
+                        static_cast<uint8_t *>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+gdattn_status gdattn_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                    const int32_t *seqlens, int32_t batch, int32_t max_seqlen,
+                                    const gdattn_layer_desc *desc, void *out, float *lse,
+                                    void *stream_) {
+  gdattn_status st = check_decode_args(q, k_cache, v_cache, seqlens, batch, max_seqlen, desc,
+                                       out, lse);
+  if (st != GDATTN_OK) return st;
+  LayerPlan pl;
+  st = make_plan(batch, max_seqlen, desc, pl);
+  if (st != GDATTN_OK) return st;
+  if (pl.bytes > kNoallocScratchBytes) return GDATTN_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint8_t *scratch = nullptr;
+  st = noalloc_scratch(stream, &scratch);
+  if (st != GDATTN_OK) return st;
+  return enqueue_decode(pl, q, k_cache, v_cache, seqlens, batch, desc, out, lse, scratch, stream);
+}
+
 gdattn_status gdattn_combine(const float *o_partial, const float *lse_partial, int32_t batch,
                              int32_t n_q_heads, int32_t n_splits, int32_t head_dim, void *out,
                              float *lse, void *stream) {
@@ -455,8 +520,13 @@ gdattn_status gdattn_combine(const float *o_partial, const float *lse_partial, i
 }
 
 gdattn_status gdattn_check_device_status(void *workspace, void *stream_) {
-  if (workspace == nullptr) return GDATTN_ERR_WORKSPACE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (workspace == nullptr) {  // the fixed scratch of gdattn_decode_noalloc
+    uint8_t *scratch = nullptr;
+    const gdattn_status st = noalloc_scratch(stream, &scratch);
+    if (st != GDATTN_OK) return st;
+    workspace = scratch;
+  }
   uint32_t word = 0;
   if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, stream) !=
           cudaSuccess ||

@@ -163,8 +163,40 @@ gdattn_status gdattn_combine(const float *o_partial, const float *lse_partial, i
                              float *lse, void *stream);
 
 /*
- * Synchronise `stream`, read and clear the workspace status word, and return
- * the first device-side error latched since the last check (GDATTN_OK if none).
+ * gdattn_decode without a caller workspace.  A library addition: the paper
+ * has no counterpart; it computes exactly what gdattn_decode computes.
+ *
+ * Same arguments (workspace and workspace_bytes dropped), host checks, kernels
+ * and results as gdattn_decode: for the same inputs on the same device both
+ * produce bit-identical out and lse.  The split-KV scratch (status word,
+ * partial LSE, partial O) is one fixed array inside the library,
+ * GDATTN_NOALLOC_SCRATCH_BYTES per device context, reserved when the library's
+ * device code is loaded, so no call allocates device or host memory.
+ *  - The first call on each device looks the array up (cudaGetSymbolAddress)
+ *    and enqueues a clear of its status word on `stream`; make that first call
+ *    outside stream capture.  Later calls only enqueue kernels.
+ *  - A layer whose gdattn_workspace_size exceeds GDATTN_NOALLOC_SCRATCH_BYTES
+ *    returns GDATTN_ERR_WORKSPACE and enqueues nothing; use gdattn_decode.
+ *  - One array per device: calls that can overlap in time on one device (on
+ *    streams with no ordering between them, from host threads racing on one
+ *    stream, or in graph replays that can run concurrently) race on it, and
+ *    their results are undefined.  Calls ordered on one stream are safe,
+ *    including the early start of programmatic dependent launch.
+ *  - Device-side errors latch in the array's status word; read and clear them
+ *    with gdattn_check_device_status(NULL, stream).
+ */
+#define GDATTN_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+gdattn_status gdattn_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                    const int32_t *seqlens, int32_t batch, int32_t max_seqlen,
+                                    const gdattn_layer_desc *desc, void *out, float *lse,
+                                    void *stream);
+
+/*
+ * Synchronise `stream`, read and clear the status word of `workspace` (NULL:
+ * the fixed scratch of gdattn_decode_noalloc on the current device), and
+ * return the first device-side error latched since the last check (GDATTN_OK
+ * if none).
  */
 gdattn_status gdattn_check_device_status(void *workspace, void *stream);
 

@@ -1,0 +1,214 @@
+"""gdattn_decode_noalloc: gdattn_decode with its split-KV scratch in a fixed
+device array inside the library (a library addition with no counterpart in the
+papers).  Its results must be bit-identical to gdattn_decode's, whatever the
+previous call left in the shared scratch.
+
+This file sorts last so that its GPU tests also run after everything else in
+one process; they pass on their own too.
+"""
+from __future__ import annotations
+
+import pytest
+import torch
+
+import workloads
+from decode_attention_09_b200 import binding
+from gpu_helpers import require_gpu
+
+A = 1 << 20  # a 16-byte aligned non-null address; host checks never dereference it
+
+
+def sliding_desc(**kw):
+    d = dict(n_q_heads=16, n_kv_heads=8, head_dim=256, window=1024, softcap=0.0,
+             scale=1 / 16, kv_shared=False, cache_capacity=1024)
+    d.update(kw)
+    return binding.make_desc(**d)
+
+
+def call(desc, q=A, k=A, v=A, seqlens=A, batch=1, max_seqlen=8, out=A, lse=A):
+    return binding.decode_noalloc_raw(q, k, v, seqlens, batch, max_seqlen, desc, out, lse, None)
+
+
+# ---------------------------------------------------------------- host checks
+@pytest.mark.parametrize("case,expect", [
+    (dict(q=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(k=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(seqlens=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(out=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(v=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(batch=0), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(max_seqlen=-3), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(q=A + 8), binding.GDATTN_ERR_MISALIGNED),
+    (dict(v=A + 4), binding.GDATTN_ERR_MISALIGNED),
+    (dict(lse=A + 2), binding.GDATTN_ERR_MISALIGNED),
+])
+def test_noalloc_host_checks(case, expect):
+    """The same argument checks as gdattn_decode, made before any CUDA call."""
+    binding.lib()
+    assert call(sliding_desc(), **case) == expect
+
+
+@pytest.mark.parametrize("desc_kw,expect", [
+    (dict(n_q_heads=12), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(softcap=float("nan")), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(head_dim=128), binding.GDATTN_ERR_UNSUPPORTED),
+])
+def test_noalloc_rejects_bad_desc(desc_kw, expect):
+    binding.lib()
+    assert call(sliding_desc(**desc_kw)) == expect
+
+
+def test_scratch_size_constant_matches_header():
+    import os
+    import re
+    hdr = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                            "include", "gdattn.h")).read()
+    m = re.search(r"#define GDATTN_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", hdr)
+    assert m and int(m.group(1)) << int(m.group(2)) == binding.NOALLOC_SCRATCH_BYTES
+
+
+# ------------------------------------------------------------------ GPU tests
+def _layers():
+    """Two sliding (CUDA-core path) and two global (tcgen05 path) inputs; each
+    pair differs in seed and lengths, so stale scratch would change results."""
+    core = [
+        (workloads.random_case(901, 4, 16, 8, 256, 1024, [1500, 700, 1, 4096], window=1024), 0),
+        (workloads.random_case(902, 4, 16, 8, 256, 1024, [333, 4000, 1024, 90], window=1024), 37),
+    ]
+    tc = [
+        (workloads.random_case(903, 3, 16, 1, 512, 4096, [4096, 1234, 65], window=0,
+                               kv_shared=True), 0),
+        (workloads.random_case(904, 3, 16, 1, 512, 4096, [17, 3000, 4000], window=0,
+                               kv_shared=True, softcap=30.0), 11),
+    ]
+    return [core[0], tc[0], core[1], tc[1]]
+
+
+class Dev:
+    def __init__(self, inp, split):
+        self.q = inp.q.cuda()
+        self.k = inp.k.cuda()
+        self.v = inp.v.cuda() if inp.v is not None else None
+        self.seqlens = inp.seqlens.to(device="cuda", dtype=torch.int32)
+        self.B = inp.q.shape[0]
+        self.max_seqlen = int(inp.seqlens.max())
+        self.desc = binding.desc_from_spec(inp.spec, split, capacity=inp.k.shape[1])
+        assert binding.workspace_size(self.B, self.max_seqlen, self.desc) <= \
+            binding.NOALLOC_SCRATCH_BYTES
+
+    def outputs(self):
+        return (torch.full_like(self.q, float("nan")),
+                torch.full((self.B, self.q.shape[1]), float("nan"), device="cuda"))
+
+    def with_workspace(self):
+        out, lse = self.outputs()
+        ws = binding.alloc_workspace(self.B, self.max_seqlen, self.desc)
+        binding.decode(self.q, self.k, self.v, self.seqlens, self.desc, self.max_seqlen, out=out,
+                       lse=lse, workspace=ws)
+        assert binding.check_device_status(ws) == binding.GDATTN_OK
+        return out, lse
+
+    def noalloc(self, out, lse, stream=None):
+        binding.decode_noalloc(self.q, self.k, self.v, self.seqlens, self.desc, self.max_seqlen,
+                               out, lse, stream=stream)
+
+
+def assert_same(a, b, what):
+    ao, al = a
+    bo, bl = b
+    assert torch.equal(ao.view(torch.int16), bo.view(torch.int16)), f"{what}: out differs"
+    assert torch.equal(al.view(torch.int32), bl.view(torch.int32)), f"{what}: lse differs"
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_workspace_decode_on_consecutive_calls():
+    """Back-to-back calls on one stream, alternating the two kernels' scratch
+    layouts, equal gdattn_decode bit for bit; then the same sequence again."""
+    require_gpu()
+    layers = [Dev(inp, split) for inp, split in _layers()]
+    ref = [ly.with_workspace() for ly in layers]
+    for rep in range(2):
+        got = [ly.outputs() for ly in layers]
+        for ly, (o, l) in zip(layers, got):
+            ly.noalloc(o, l)  # no synchronisation between the calls
+        torch.cuda.synchronize()
+        assert binding.check_device_status(None) == binding.GDATTN_OK
+        for i, (g, r) in enumerate(zip(got, ref)):
+            assert_same(g, r, f"pass {rep} layer {i}")
+
+
+@pytest.mark.gpu
+def test_noalloc_rejects_oversize_and_enqueues_nothing():
+    require_gpu()
+    inp, _ = _layers()[1]
+    ly = Dev(inp, 0)
+    big = binding.desc_from_spec(inp.spec, 4000, capacity=inp.k.shape[1])
+    assert binding.workspace_size(ly.B, ly.max_seqlen, big) > binding.NOALLOC_SCRATCH_BYTES
+    out, lse = ly.outputs()
+    st = binding.decode_noalloc_raw(binding._ptr(ly.q), binding._ptr(ly.k), None,
+                                    binding._ptr(ly.seqlens), ly.B, ly.max_seqlen, big,
+                                    binding._ptr(out), binding._ptr(lse), None)
+    assert st == binding.GDATTN_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert torch.isnan(out.float()).all() and torch.isnan(lse).all()
+
+
+@pytest.mark.gpu
+def test_noalloc_calls_take_no_device_memory():
+    """After a first call, further calls leave the device's free memory as it was."""
+    require_gpu()
+    layers = [Dev(inp, split) for inp, split in _layers()]
+    bufs = [ly.outputs() for ly in layers]
+    for ly, (o, l) in zip(layers, bufs):
+        ly.noalloc(o, l)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(5):
+        for ly, (o, l) in zip(layers, bufs):
+            ly.noalloc(o, l)
+    torch.cuda.synchronize()
+    assert binding.check_device_status(None) == binding.GDATTN_OK
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+
+
+@pytest.mark.gpu
+def test_noalloc_status_word_latches_and_clears():
+    """A device-side error lands in the fixed scratch's status word."""
+    require_gpu()
+    inp = workloads.random_case(905, 3, 16, 8, 256, 32, [5, 0, 9], window=16)
+    ly = Dev(inp, 0)
+    ly.max_seqlen = 16
+    out, lse = ly.outputs()
+    assert binding.check_device_status(None) == binding.GDATTN_OK
+    ly.noalloc(out, lse)
+    assert binding.check_device_status(None) == binding.GDATTN_ERR_DEVICE_SEQLEN
+    assert torch.all(out[1] == 0) and torch.all(torch.isneginf(lse[1]))
+    assert binding.check_device_status(None) == binding.GDATTN_OK
+
+
+@pytest.mark.gpu
+def test_noalloc_graph_replay_matches_workspace_decode():
+    require_gpu()
+    layers = [Dev(inp, split) for inp, split in _layers()]
+    ref = [ly.with_workspace() for ly in layers]
+    bufs = [ly.outputs() for ly in layers]
+    layers[0].noalloc(*bufs[0])  # first call on the device outside capture
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for ly, (o, l) in zip(layers, bufs):
+                ly.noalloc(o, l, stream=s)
+    for _ in range(2):
+        for o, l in bufs:
+            o.fill_(float("nan"))
+            l.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        for i, (b, r) in enumerate(zip(bufs, ref)):
+            assert_same(b, r, f"graph layer {i}")
+    assert binding.check_device_status(None) == binding.GDATTN_OK
+    del g
