@@ -409,7 +409,7 @@ def run_ours(args, world, rank, local):
         ach = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                 "frac": ach / peak, "peak_kind": peak_kind,
-                "kernel": "sliding layer: core_decode_kernel<256,2,8,false> + LSE combine",
+                "kernel": "sliding layer: tc_pair_decode_kernel (tcgen05) + LSE combine",
                 "bytes_per_launch": per_launch_bytes, "us_per_launch": per_launch_ms * 1e3,
                 "traffic": traffic_for("sliding")}
     per_type = {}

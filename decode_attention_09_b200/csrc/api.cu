@@ -14,6 +14,7 @@
 #include "combine.cuh"
 #include "core_decode.cuh"
 #include "tc_decode.cuh"
+#include "tc_pair_decode.cuh"
 
 using namespace gdattn;
 
@@ -25,7 +26,7 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes]
 
 namespace {
 
-enum class PathKind { kNone, kCore, kTc };
+enum class PathKind { kNone, kCore, kTc, kTcPair };
 
 struct LayerPlan {
   PathKind kind = PathKind::kNone;
@@ -139,6 +140,10 @@ int query_tc(const void *fn, int threads, int smem) {
   using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const TcParams);
   return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
 }
+int query_tc_pair(const void *fn, int threads, int smem) {
+  using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const TcParams);
+  return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
+}
 
 // ---------------------------------------------------------------- planning
 gdattn_status check_desc(const gdattn_layer_desc *d) {
@@ -159,6 +164,7 @@ gdattn_status check_desc(const gdattn_layer_desc *d) {
 PathKind choose_path(const gdattn_layer_desc *d) {
   const int g = d->n_q_heads / d->n_kv_heads;
   if (g == 16 && d->head_dim == 512 && d->kv_shared == 1) return PathKind::kTc;
+  if (g == 2 && d->head_dim == 256 && d->kv_shared == 0) return PathKind::kTcPair;
   if ((d->head_dim == 256 || d->head_dim == 512) && (g == 1 || g == 2 || g == 4) &&
       (d->n_kv_heads == 1 || d->n_kv_heads == 2 || d->n_kv_heads == 4 || d->n_kv_heads == 8))
     return PathKind::kCore;
@@ -185,13 +191,20 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
     pl.align = ck.tokens_per_stage;
     pl.units_per_seq = 1;
     pl.heads_per_unit = d->n_q_heads;
-  } else {
+  } else if (pl.kind == PathKind::kTc) {
     per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_kernel),
                                   TcConfig::kThreads, TcConfig::SMEM, query_tc);
     min_tokens = 2 * TcConfig::TILE;
     pl.align = TcConfig::TILE;
     pl.units_per_seq = d->n_kv_heads;
-    pl.heads_per_unit = 16;
+    pl.heads_per_unit = TcConfig::G;
+  } else {
+    per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_decode_kernel),
+                                  TcPairConfig::kThreads, TcPairConfig::SMEM, query_tc_pair);
+    min_tokens = 2 * TcPairConfig::TILE;
+    pl.align = TcPairConfig::TILE;
+    pl.units_per_seq = d->n_kv_heads;
+    pl.heads_per_unit = TcPairConfig::G;
   }
   if (per_sm <= 0) return GDATTN_ERR_CUDA;
   int64_t per_unit = max_seqlen;
@@ -246,6 +259,33 @@ EncodeTiledFn encode_tiled() {
     return reinterpret_cast<EncodeTiledFn>(p);
   }();
   return fn;
+}
+
+// K or V cache [B][C][Hkv][D] bf16 as a 4-D tensor map {D, Hkv, C, B} read in
+// 64-d x 1-head x 64-token boxes with 128-byte swizzle.
+bool encode_cache_map(EncodeTiledFn enc, CUtensorMap *map, const void *base, int32_t D,
+                      int32_t Hkv, int32_t C, int32_t batch, int64_t bstride, uint32_t tile) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv),
+                              static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(batch)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2,
+                                 static_cast<cuuint64_t>(Hkv) * D * 2,
+                                 static_cast<cuuint64_t>(bstride) * 2};
+  const cuuint32_t box[4] = {64, 1, tile, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// q [B * Hq][D] bf16 as a 2-D tensor map read in 64-d x 16-row boxes.
+bool encode_q_map(EncodeTiledFn enc, CUtensorMap *map, const void *q, int32_t D, int64_t rows) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  const cuuint32_t box[2] = {64, 16};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(q), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 gdattn_status launch_combine_internal(const LayerPlan &pl, const Geometry &geo, const float *ws_lse,
@@ -337,32 +377,11 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
   } else {
     EncodeTiledFn enc = encode_tiled();
     if (enc == nullptr) return GDATTN_ERR_CUDA;
-    CUtensorMap kmap, qmap;
-    {
-      const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv),
-                                  static_cast<cuuint64_t>(desc->cache_capacity),
-                                  static_cast<cuuint64_t>(batch)};
-      const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2,
-                                     static_cast<cuuint64_t>(Hkv) * D * 2,
-                                     static_cast<cuuint64_t>(bstride) * 2};
-      const cuuint32_t box[4] = {64, 1, TcConfig::TILE, 1};
-      const cuuint32_t estr[4] = {1, 1, 1, 1};
-      if (enc(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(k_cache), dims,
-              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return GDATTN_ERR_CUDA;
-    }
-    {
-      const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D),
-                                  static_cast<cuuint64_t>(batch) * desc->n_q_heads};
-      const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-      const cuuint32_t box[2] = {64, 16};
-      const cuuint32_t estr[2] = {1, 1};
-      if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(q), dims, strides,
-              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return GDATTN_ERR_CUDA;
-    }
+    CUtensorMap kmap, vmap, qmap;
+    if (!encode_cache_map(enc, &kmap, k_cache, D, Hkv, desc->cache_capacity, batch, bstride,
+                          TcConfig::TILE) ||
+        !encode_q_map(enc, &qmap, q, D, static_cast<int64_t>(batch) * desc->n_q_heads))
+      return GDATTN_ERR_CUDA;
     TcParams tp;
     tp.out = static_cast<uint16_t *>(out);
     tp.lse = lse;
@@ -373,10 +392,20 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     tp.n_q_heads = desc->n_q_heads;
     tp.qscale = qscale;
     tp.post = post;
-    cudaLaunchConfig_t cfg =
-        launch_config(dim3(pl.grid), TcConfig::kThreads, TcConfig::SMEM, stream, attr);
-    if (cudaLaunchKernelEx(&cfg, tc_decode_kernel, kmap, qmap, tp) != cudaSuccess)
-      return GDATTN_ERR_CUDA;
+    if (pl.kind == PathKind::kTc) {
+      cudaLaunchConfig_t cfg =
+          launch_config(dim3(pl.grid), TcConfig::kThreads, TcConfig::SMEM, stream, attr);
+      if (cudaLaunchKernelEx(&cfg, tc_decode_kernel, kmap, qmap, tp) != cudaSuccess)
+        return GDATTN_ERR_CUDA;
+    } else {
+      if (!encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, batch, bstride,
+                            TcPairConfig::TILE))
+        return GDATTN_ERR_CUDA;
+      cudaLaunchConfig_t cfg =
+          launch_config(dim3(pl.grid), TcPairConfig::kThreads, TcPairConfig::SMEM, stream, attr);
+      if (cudaLaunchKernelEx(&cfg, tc_pair_decode_kernel, kmap, vmap, qmap, tp) != cudaSuccess)
+        return GDATTN_ERR_CUDA;
+    }
   }
   if (pl.grid > 1)
     return launch_combine_internal(pl, geo, ws_lse, ws_o, desc, out, lse, stream);

@@ -55,8 +55,8 @@ namespace gdattn {
 struct TcParams {
   uint16_t *out;          // [B, Hq, D]
   float *lse;             // [B, Hq] or null
-  float *ws_o;            // partial outputs [slots][16][D]
-  float *ws_lse;          // partial lse [slots][16]
+  float *ws_o;            // partial outputs [slots][G][D]
+  float *ws_lse;          // partial lse [slots][G]
   uint32_t *status;
   Geometry geo;           // units_per_seq == n_kv_heads
   int32_t n_q_heads;
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
     const uint64_t pol = l2_evict_first_policy();
     bool ok = true;
     uint32_t i = 0, seg_count = 0, q_issued = 0;
-    int32_t qrows[8];            // Q rows of segments whose Q is not issued yet
+    int32_t qrows[8] = {};       // Q rows of segments whose Q is not issued yet
     uint32_t stage_seg[NST];     // segment of the tile last loaded into each stage
     auto issue_q = [&](bool block) -> bool {  // warp-uniform result
       if (q_issued > 0) {

@@ -1,0 +1,529 @@
+// Split-KV decode attention on the 5th-generation tensor cores (tcgen05) for
+// GQA pairs: two query heads per KV head, separate K and V caches, head_dim
+// 256 (Gemma-4 sliding-window layers).
+//
+// A pair of query rows is a thin contraction (2 flop per KV byte), yet on CUDA
+// cores the dot products, their cross-lane reductions and the bf16 unpacking
+// cost about three instructions per KV element, which caps an SM near 50 GB/s,
+// below its share of HBM bandwidth.  The tensor core does the same work in 24
+// MMA instructions per 64-token tile, so the SM only streams.  The MMAs are
+// padded to N = 16 (the smallest width valid for both shapes below); the unused
+// columns cost no extra instructions.
+//
+// One work unit is one (sequence, KV head); per 64-token tile of it:
+//
+//   S^T[64 tok x 16]  = K_tile[64 x 256] . Q^T[256 x 16]    (M=64,  N=16, K=256)
+//   O^T[256 d x 16]  += V_tile^T[256 x 64] . P[64 x 16]      (M=128 x2, N=16, K=64)
+//
+// Q rows 0-1 are the pair's query heads (rows 2-15 are whatever follows them, or
+// TMA zero fill; their score columns are never read).  P's columns are p_hi of
+// heads 0, 1, then p_lo of heads 0, 1 (rows 4-15 stay zero), so O^T column h
+// plus column 2 + h is head h's output: the same bf16 hi/lo split of the
+// weights as the 16-head kernel, for fp32-grade weights on a bf16 MMA.
+//
+// K and V tiles arrive by TMA as 64-token x 64-d boxes with 128-byte swizzle:
+// the K-major A operand of the first product and the MN-major A operand of the
+// second.  P is stored K-major (a row of 64 token weights per column), the same
+// canonical layout as Q.  S^T is split over four TMEM accumulators (one per
+// 16-wide k-step within each 64-wide d-chunk) so consecutive MMAs never feed
+// the same accumulator.  Softmax keeps a lazily moved reference max per head
+// (see tc_decode.cuh), so a tile normally costs one TMEM load, one vote and two
+// P stores per thread.
+//
+// Warp roles (224 threads) as in the 16-head kernel: warp 0 TMA, warp 1 QK MMA
+// and TMEM owner, warp 6 P.V MMA, warps 2-5 softmax (TMEM sub-partition warp %
+// 4).  Every wait is bounded.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+
+#include "partition.cuh"
+#include "ptx.cuh"
+#include "tc_decode.cuh"
+
+namespace gdattn {
+
+struct TcPairConfig {
+  static constexpr int D = 256;
+  static constexpr int G = 2;
+  static constexpr int N = 16;                        // MMA width (QK and P.V)
+  static constexpr int TILE = 64;                     // tokens per tile
+  static constexpr int NST = 3;                       // KV stages
+  static constexpr int BOXB = TILE * 128;             // one 64-token x 64-d box, 8 KiB
+  static constexpr int KB = BOXB * (D / 64);          // K tile, 32 KiB
+  static constexpr int STAGEB = 2 * KB;               // K tile then V tile, 64 KiB
+  static constexpr int QBOXB = N * 128;               // 16 Q rows x 64 d, 2 KiB
+  static constexpr int QB = QBOXB * (D / 64);         // 8 KiB
+  static constexpr int PB = N * 128;                  // P: 16 rows x 64 tokens bf16, 2 KiB
+  static constexpr int OFF_Q = NST * STAGEB;
+  static constexpr int OFF_P = OFF_Q + QB;
+  static constexpr int OFF_BAR = OFF_P + 2 * PB;
+  static constexpr int OFF_RED = OFF_BAR + 256;
+  static constexpr int SMEM = OFF_RED + 2 * 4 * G * 4 + 1024;
+  static constexpr int kThreads = 224;
+  static constexpr uint32_t TMEM_COLS = 256;
+  static constexpr uint32_t S_COL = 0;                // 2 buffers x 4 partial sums x 16 columns
+  static constexpr uint32_t O_COL = 128;              // 2 d-blocks x 16 columns
+};
+static_assert(TcPairConfig::TILE == TcConfig::TILE, "TileIter walks 64-token tiles");
+static_assert(TcPairConfig::SMEM <= 227 * 1024, "shared memory budget");
+
+// Byte offset of element (row n, token t) in a K-major 128-byte-swizzled
+// 64-column bf16 tile: 16-byte chunk t / 8 of row n sits at chunk (t / 8) ^ (n % 8).
+__device__ __forceinline__ uint32_t sw128_offset(int n, int t) {
+  return static_cast<uint32_t>(n * 128 + ((((t >> 3) ^ (n & 7)) << 4) | ((t & 7) << 1)));
+}
+
+__global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
+    tc_pair_decode_kernel(const __grid_constant__ CUtensorMap kmap,
+                          const __grid_constant__ CUtensorMap vmap,
+                          const __grid_constant__ CUtensorMap qmap, const TcParams p) {
+  using Cfg = TcPairConfig;
+  constexpr int G = Cfg::G, D = Cfg::D, NST = Cfg::NST;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint8_t *stages = smem;
+  uint8_t *qs = smem + Cfg::OFF_Q;
+  uint8_t *ps = smem + Cfg::OFF_P;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
+  uint64_t *full = bars;            // [NST]  TMA -> MMA
+  uint64_t *empty = bars + 3;       // [NST]  P.V -> TMA
+  uint64_t *qfull = bars + 6;       // TMA -> MMA
+  uint64_t *qempty = bars + 7;      // MMA -> TMA
+  uint64_t *sfull = bars + 8;       // [2] MMA -> softmax (S of tile i in buffer i & 1)
+  uint64_t *sempty = bars + 10;     // [2] softmax -> MMA
+  uint64_t *pfull = bars + 12;      // [2] softmax -> MMA (P of tile i in buffer i & 1)
+  uint64_t *ofull = bars + 14;      // [2] MMA -> softmax: P.V of tile i done (barrier i & 1)
+  uint64_t *oempty = bars + 16;     // softmax -> MMA: O of a finished segment read out
+  uint64_t *drain = bars + 17;      // [2] QK warp, P.V warp: all their MMAs done
+  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 19);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 20);
+  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 21);  // 48 bytes, ends before +256
+  float *redmax = reinterpret_cast<float *>(smem + Cfg::OFF_RED);  // [4 warps][G]
+  float *redsum = redmax + 4 * G;                                  // [4 warps][G]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(qfull, 1);
+    mbar_init(qempty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], 4);
+      mbar_init(&pfull[s], 4);
+      mbar_init(&ofull[s], 1);
+    }
+    mbar_init(oempty, 4);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+    prefetch_tensormap(&qmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_smem, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  grid_launch_dependents();
+  // The split plan reads only seqlens, so it (and the producer's first KV
+  // loads below) may run before the preceding kernel has completed; every other
+  // global access waits for it (griddepcontrol.wait) in the role that makes it.
+  if (warp == 2) plan_chunk(p.geo, c, plan);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_smem;
+
+  if (c == 0 && warp == 2 && plan->bad) {
+    grid_dependency_wait();
+    if (lane == 0) atomicOr(p.status, kStatusSeqlen);
+    for (int32_t b = 0; b < p.geo.batch; ++b) {
+      bool dummy = false;
+      if (attended_count(__ldg(p.geo.seqlens + b), p.geo.window, p.geo.capacity, dummy) != 0)
+        continue;
+      for (int i = lane; i < p.n_q_heads * D; i += 32)
+        p.out[static_cast<int64_t>(b) * p.n_q_heads * D + i] = 0;
+      if (p.lse != nullptr)
+        for (int i = lane; i < p.n_q_heads; i += 32)
+          p.lse[static_cast<int64_t>(b) * p.n_q_heads + i] = -INFINITY;
+    }
+  }
+
+  const int32_t C = p.geo.capacity;
+
+  if (warp == 0) {
+    // -------------------------------------------------------------- TMA
+    // As in the 16-head kernel: the warp walks the schedule, one elected lane
+    // copies, and a segment's Q is loaded as soon as the previous segment's
+    // last QK has released the buffer.
+    const uint64_t pol = l2_evict_first_policy();
+    bool ok = true;
+    uint32_t i = 0, seg_count = 0, q_issued = 0;
+    int32_t qrows[8] = {};       // Q rows of segments whose Q is not issued yet
+    uint32_t stage_seg[NST];     // segment of the tile last loaded into each stage
+    auto issue_q = [&](bool block) -> bool {  // warp-uniform result
+      if (q_issued > 0) {
+        bool got = block ? mbar_wait(qempty, (q_issued - 1) & 1, abort_flag, p.status)
+                         : mbar_try_wait(qempty, (q_issued - 1) & 1);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (block) ok = false;
+          return false;
+        }
+      }
+      const int32_t qrow = qrows[q_issued & 7];
+      if (elect_one()) {
+        mbar_arrive_expect_tx(qfull, Cfg::QB);
+#pragma unroll
+        for (int j = 0; j < D / 64; ++j)
+          tma_load_2d(qs + j * Cfg::QBOXB, &qmap, 64 * j, qrow, qfull);
+      }
+      __syncwarp();
+      ++q_issued;
+      return true;
+    };
+    TileIter it;
+    it.init(p.geo, *plan);
+    int32_t row, ntok;
+    bool first, last;
+    // Until the preceding kernel completes, only cache rows of positions before
+    // each sequence's newest one are read; q and the newest row come after.
+    bool waited = false;
+    auto ensure_waited = [&]() {
+      if (!waited) {
+        grid_dependency_wait();
+        waited = true;
+      }
+    };
+    while (ok && it.next(C, row, ntok, first, last)) {
+      if (first) {
+        // At most NST + 1 segments can be pending (see the wait below), so 8 slots do.
+        qrows[seg_count & 7] = it.seg.b * p.n_q_heads + it.seg.x * G;
+        ++seg_count;
+      }
+      if (i >= NST || it.newest) ensure_waited();
+      while (ok && waited && q_issued < seg_count && issue_q(false)) {
+      }
+      const int st = i % NST;
+      if (i >= NST) {
+        // The tile in this stage is released after its P.V, which needs its Q.
+        while (ok && q_issued <= stage_seg[st]) issue_q(true);
+        if (ok && !mbar_wait(&empty[st], ((i / NST) - 1) & 1, abort_flag, p.status)) ok = false;
+      }
+      if (!__all_sync(0xffffffffu, ok)) break;
+      stage_seg[st] = seg_count - 1;
+      if (elect_one()) {
+        uint8_t *kdst = stages + st * Cfg::STAGEB;
+        mbar_arrive_expect_tx(&full[st], Cfg::STAGEB);
+#pragma unroll
+        for (int j = 0; j < D / 64; ++j) {
+          tma_load_4d(kdst + j * Cfg::BOXB, &kmap, 64 * j, it.seg.x, row, it.seg.b, &full[st], pol);
+          tma_load_4d(kdst + Cfg::KB + j * Cfg::BOXB, &vmap, 64 * j, it.seg.x, row, it.seg.b,
+                      &full[st], pol);
+        }
+      }
+      __syncwarp();
+      ++i;
+    }
+    ensure_waited();
+    while (ok && q_issued < seg_count) issue_q(true);
+    // Drain: never leave with copies in flight into shared memory.
+    volatile int no_abort = 0;
+    for (uint32_t f = i > NST ? i - NST : 0; f < i; ++f)
+      mbar_wait(&full[f % NST], (f / NST) & 1, &no_abort, p.status);
+    if (q_issued > 0) mbar_wait(qfull, (q_issued - 1) & 1, &no_abort, p.status);
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- QK MMA
+    const uint32_t idesc_qk = idesc_bf16_f32(64, Cfg::N, false, false);
+    // An operand at byte offset o from a base descriptor is base + (o >> 4).
+    const uint64_t kdesc = smem_desc_sw128(smem_u32(stages), 16, 1024);  // K tile, K-major
+    const uint64_t qdesc = smem_desc_sw128(smem_u32(qs), 16, 1024);      // Q, K-major
+    bool ok = true;
+    uint32_t i = 0, nseg = 0;
+    TileIter it;
+    it.init(p.geo, *plan);
+    int32_t row, ntok;
+    bool first, last;
+    while (ok && it.next(C, row, ntok, first, last)) {
+      if (first) {
+        if (!mbar_wait(qfull, nseg & 1, abort_flag, p.status)) ok = false;
+        if (!__all_sync(0xffffffffu, ok)) break;
+        ++nseg;
+      }
+      const int st = i % NST, sb = i & 1;
+      if (!mbar_wait(&full[st], (i / NST) & 1, abort_flag, p.status)) ok = false;
+      if (ok && i >= 2 && !mbar_wait(&sempty[sb], ((i >> 1) - 1) & 1, abort_flag, p.status))
+        ok = false;
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const uint64_t a0 = kdesc + ((st * Cfg::STAGEB) >> 4);
+      if (elect_one()) {
+#pragma unroll
+        for (int j = 0; j < D / 64; ++j) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = a0 + ((j * Cfg::BOXB + kk * 32) >> 4);
+            const uint64_t bd = qdesc + ((j * Cfg::QBOXB + kk * 32) >> 4);
+            tc_mma_bf16(tmem + Cfg::S_COL + sb * 64 + kk * 16, ad, bd, idesc_qk, j != 0);
+          }
+        }
+        tc_commit(&sfull[sb]);
+        if (last) tc_commit(qempty);
+      }
+      __syncwarp();
+      ++i;
+    }
+    // Drain: wait until every issued MMA has completed before TMEM is freed.
+    if (elect_one()) tc_commit(&drain[0]);
+    __syncwarp();
+    volatile int no_abort = 0;
+    mbar_wait(&drain[0], 0, &no_abort, p.status);
+  } else if (warp == 6) {
+    // ---------------------------------------------------------- P.V MMA
+    const uint32_t idesc_pv = idesc_bf16_f32(128, Cfg::N, true, false);
+    const uint64_t vdesc =
+        smem_desc_sw128(smem_u32(stages + Cfg::KB), Cfg::BOXB, 1024);  // V^T, MN-major
+    const uint64_t pdesc = smem_desc_sw128(smem_u32(ps), 16, 1024);    // P, K-major
+    bool ok = true;
+    uint32_t t = 0, nseg = 0;
+    TileIter it;
+    it.init(p.geo, *plan);
+    int32_t row, ntok;
+    bool first, last;
+    while (ok && it.next(C, row, ntok, first, last)) {
+      bool w = mbar_wait(&pfull[t & 1], (t >> 1) & 1, abort_flag, p.status);
+      // A segment's first P.V overwrites O: the previous segment must be read out.
+      if (w && first && nseg > 0) w = mbar_wait(oempty, (nseg - 1) & 1, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      if (first) ++nseg;
+      tc_fence_after();
+      const uint64_t a0 = vdesc + (((t % NST) * Cfg::STAGEB) >> 4);
+      const uint64_t b0 = pdesc + (((t & 1) * Cfg::PB) >> 4);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bd = b0 + ((kk * 32) >> 4);  // 16 tokens = 32 bytes of each P row
+#pragma unroll
+          for (int jb = 0; jb < 2; ++jb) {
+            const uint64_t ad = a0 + ((2 * jb * Cfg::BOXB + kk * 2048) >> 4);
+            tc_mma_bf16(tmem + Cfg::O_COL + jb * 16, ad, bd, idesc_pv, !(first && kk == 0));
+          }
+        }
+        tc_commit(&ofull[t & 1]);
+        tc_commit(&empty[t % NST]);
+      }
+      __syncwarp();
+      ++t;
+    }
+    if (elect_one()) tc_commit(&drain[1]);
+    __syncwarp();
+    volatile int no_abort = 0;
+    mbar_wait(&drain[1], 0, &no_abort, p.status);
+  } else {
+    // ---------------------------------------------------------- softmax
+    grid_dependency_wait();  // outputs and workspace are written below
+    // M=64 puts tile token r in TMEM lane (r % 16) + 32 * (r / 16): lanes 0-15 of
+    // each warp receive one token's scores.  Lanes 0-15 take head 0 of their
+    // token, lanes 16-31 head 1 of the token of lane - 16.
+    const int qd = warp & 3;                 // TMEM sub-partition: lanes 32*qd ..
+    const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
+    const int tok = 16 * qd + (lane & 15);   // tile token of this lane
+    const int hd = lane >> 4;                // head of this lane's score
+    // P rows 2G .. N-1 multiply O columns nobody reads; keep them finite (zero).
+    for (int e = threadIdx.x - 64; e < 2 * (Cfg::N - 2 * G) * 8; e += 128) {
+      const int buf = e / ((Cfg::N - 2 * G) * 8), r = e % ((Cfg::N - 2 * G) * 8);
+      *reinterpret_cast<uint4 *>(ps + buf * Cfg::PB + (2 * G + (r >> 3)) * 128 + (r & 7) * 16) =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    float m_ref[G], lpart = 0.f;
+#pragma unroll
+    for (int h = 0; h < G; ++h) m_ref[h] = -INFINITY;
+    bool ok = true;
+    uint32_t cons0 = 0, cons1 = 0;  // ofull phases consumed on barrier 0 / 1
+    // Wait until the P.V of tile t has completed.  Phases are consumed in order
+    // and never lag by two, so the parity waits cannot alias.
+    auto ensure_pv = [&](uint32_t t) {
+      const uint32_t b = t & 1, ph = t >> 1;
+      uint32_t &cons = b ? cons1 : cons0;
+      if (cons <= ph) {
+        if (ok && !mbar_wait(&ofull[b], cons & 1, abort_flag, p.status)) ok = false;
+        ++cons;
+      }
+      ok = __all_sync(0xffffffffu, ok);
+    };
+    uint32_t i = 0;
+    TileIter it;
+    it.init(p.geo, *plan);
+    int32_t row, ntok;
+    bool first, last;
+
+    while (it.next(C, row, ntok, first, last)) {
+      const int sb = i & 1, pb = i & 1;
+      if (i >= 2) ensure_pv(i - 2);  // P buffer pb is free again
+      if (first) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) m_ref[h] = -INFINITY;
+        lpart = 0.f;
+      }
+      // --- scores of tile i: sum of the four partial accumulators
+      float s0 = 0.f, s1 = 0.f;
+      if (ok && !mbar_wait(&sfull[sb], (i >> 1) & 1, abort_flag, p.status)) ok = false;
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+        float v[8];
+        tmem_ld2x4(tmem + lane_base + Cfg::S_COL + sb * 64, v);
+        s0 = (v[0] + v[2]) + (v[4] + v[6]);
+        s1 = (v[1] + v[3]) + (v[5] + v[7]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty[sb]);
+      }
+      const float other = __shfl_xor_sync(0xffffffffu, s1, 16);
+      const bool valid = ok && tok < ntok;
+      float x = ((lane < 16) ? s0 : other) * p.qscale;
+      if (p.post != 0.f) x = p.post * tanhf(x);
+      x = valid ? x : -INFINITY;
+      const float mine_ref = hd ? m_ref[1] : m_ref[0];
+      // --- move the reference only when some score outgrew it
+      if (named_bar_or(1, 128, x > mine_ref + kTau)) {
+        float tm = x;
+#pragma unroll
+        for (int off = 1; off < 16; off <<= 1) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, off));
+        if ((lane & 15) == 0) redmax[qd * G + hd] = tm;
+        named_bar_sync(1, 128);
+        float alpha[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float t = fmaxf(fmaxf(redmax[h], redmax[G + h]),
+                                fmaxf(redmax[2 * G + h], redmax[3 * G + h]));
+          const float mn = fmaxf(m_ref[h], t);
+          alpha[h] = (m_ref[h] == -INFINITY) ? 0.f : exp2f(m_ref[h] - mn);
+          m_ref[h] = mn;
+        }
+        lpart *= hd ? alpha[1] : alpha[0];
+        if (!first) {
+          // O holds tiles < i: wait for the last of them, then rescale it in TMEM.
+          ensure_pv(i - 1);
+          if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int jb = 0; jb < 2; ++jb) {
+              float o[4];  // columns: hi of heads 0, 1, lo of heads 0, 1
+              tmem_ld4(tmem + lane_base + Cfg::O_COL + jb * 16, o);
+              o[0] *= alpha[0];
+              o[1] *= alpha[1];
+              o[2] *= alpha[0];
+              o[3] *= alpha[1];
+              tmem_st4_wait(tmem + lane_base + Cfg::O_COL + jb * 16, o);
+            }
+          }
+        }
+      }
+      // --- weight of this (token, head): hi part in P row hd, lo part in row G + hd
+      {
+        const float mr = hd ? m_ref[1] : m_ref[0];
+        const float pe = (x == -INFINITY) ? 0.f : exp2f(x - mr);
+        lpart += pe;
+        const uint16_t hi = f32_to_bf16_rn(pe);
+        const uint16_t lo = f32_to_bf16_rn(pe - __uint_as_float(static_cast<uint32_t>(hi) << 16));
+        uint8_t *pbuf = ps + pb * Cfg::PB;
+        *reinterpret_cast<uint16_t *>(pbuf + sw128_offset(hd, tok)) = hi;
+        *reinterpret_cast<uint16_t *>(pbuf + sw128_offset(G + hd, tok)) = lo;
+      }
+      if (ok && ntok < Cfg::TILE) {
+        // V rows past the attended range hold other cache contents (possibly
+        // NaN); they get weight 0, but 0 * NaN would still reach O, so clear them.
+        uint8_t *vt = stages + (i % NST) * Cfg::STAGEB + Cfg::KB;
+        const int per_box = (Cfg::TILE - ntok) * 8;  // 16-byte chunks past row ntok
+#pragma unroll 1
+        for (int box = 0; box < D / 64; ++box)
+          for (int e = threadIdx.x - 64; e < per_box; e += 128)
+            *reinterpret_cast<uint4 *>(vt + box * Cfg::BOXB + (ntok + (e >> 3)) * 128 +
+                                       (e & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (ok && lane == 0) mbar_arrive(&pfull[pb]);
+
+      if (last) {
+        // --- segment end: all of its P.V done, read O out
+        if (i >= 1) ensure_pv(i - 1);
+        ensure_pv(i);
+        float ls = lpart;
+#pragma unroll
+        for (int off = 1; off < 16; off <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
+        if ((lane & 15) == 0) redsum[qd * G + hd] = ls;
+        named_bar_sync(1, 128);
+        const Segment &sg = it.seg;
+        const bool single = sg.whole();
+        const int64_t slot = static_cast<int64_t>(c) + sg.unit;
+        const int h0 = sg.x * G;
+        float L[G], inv[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          L[h] = (redsum[h] + redsum[G + h]) + (redsum[2 * G + h] + redsum[3 * G + h]);
+          inv[h] = __fdividef(1.f, L[h]);
+        }
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int jb = 0; jb < 2; ++jb) {
+            float o[4];
+            tmem_ld4(tmem + lane_base + Cfg::O_COL + jb * 16, o);
+            const int d = 128 * jb + 32 * qd + lane;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const float val = (o[h] + o[G + h]) * inv[h];
+              if (single)
+                p.out[(static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + h) * D + d] =
+                    f32_to_bf16_rn(val);
+              else
+                p.ws_o[(slot * G + h) * D + d] = val;
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(oempty);
+          if (qd == 0 && lane < G) {  // LSE of head `lane`
+            const float mr = lane ? m_ref[1] : m_ref[0];
+            const float Lh = lane ? L[1] : L[0];
+            const float lse_v = (mr + log2f(Lh)) * 0.69314718055994530942f;
+            if (single) {
+              if (p.lse != nullptr)
+                p.lse[static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + lane] = lse_v;
+            } else {
+              p.ws_lse[slot * G + lane] = lse_v;
+            }
+          }
+        }
+      }
+      ++i;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace gdattn

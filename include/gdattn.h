@@ -137,9 +137,11 @@ gdattn_status gdattn_workspace_init(void *workspace, size_t workspace_bytes, voi
  *           bytes, status word zeroed once by gdattn_workspace_init.  Calls that
  *           share a workspace must be ordered on one stream.
  *
- * Supported: D in {256, 512}; G = Hq / Hkv in {1, 2, 4} with Hkv in {1, 2, 4, 8, 16}
- * (CUDA-core path), or G == 16 with D == 512 (tensor-core path).  Other
- * geometries return GDATTN_ERR_UNSUPPORTED.
+ * Supported geometries (G = Hq / Hkv), by the kernel that runs them:
+ *  - G == 2, D == 256, separate V, any Hkv: tcgen05 pair kernel;
+ *  - G == 16, D == 512, kv_shared, any Hkv: tcgen05 16-head kernel;
+ *  - otherwise D in {256, 512}, G in {1, 2, 4}, Hkv in {1, 2, 4, 8}: CUDA-core kernel.
+ * Other geometries return GDATTN_ERR_UNSUPPORTED.
  */
 gdattn_status gdattn_decode(const void *q, const void *k_cache, const void *v_cache,
                             const int32_t *seqlens, int32_t batch, int32_t max_seqlen,

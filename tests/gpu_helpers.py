@@ -18,6 +18,15 @@ def require_gpu():
         pytest.skip("no CUDA device")
 
 
+def uses_tensor_cores(spec) -> bool:
+    """Whether the library runs this geometry on its tcgen05 kernels: 16 query
+    heads per KV head with head_dim 512 and K = V, or pairs of query heads with
+    head_dim 256 and separate V.  Other geometries take the CUDA-core kernel."""
+    g = spec.n_q_heads // spec.n_kv_heads
+    return ((g == 16 and spec.head_dim == 512 and spec.kv_shared)
+            or (g == 2 and spec.head_dim == 256 and not spec.kv_shared))
+
+
 def bf16_ulp(x: np.ndarray) -> np.ndarray:
     """Spacing of bf16 numbers at |x| (8 significant bits)."""
     ax = np.maximum(np.abs(x), np.finfo(np.float32).tiny)

@@ -122,7 +122,7 @@ def test_decode_rejects_bad_pointers(lib, case, expect):
     (dict(cache_batch_stride=1024 * 8 * 256 + 4), binding.GDATTN_ERR_INVALID_ARG),  # not % 8
     (dict(head_dim=128), binding.GDATTN_ERR_UNSUPPORTED),
     (dict(n_q_heads=64, n_kv_heads=8), binding.GDATTN_ERR_UNSUPPORTED),  # G = 8
-    (dict(n_q_heads=32, n_kv_heads=16), binding.GDATTN_ERR_UNSUPPORTED),  # Hkv = 16
+    (dict(n_q_heads=64, n_kv_heads=16), binding.GDATTN_ERR_UNSUPPORTED),  # G = 4, Hkv = 16
 ])
 def test_decode_rejects_bad_desc(lib, desc_kw, expect):
     assert call(good_desc(**desc_kw)) == expect

@@ -11,7 +11,7 @@ import torch
 import oracle
 import workloads
 from decode_attention_09_b200 import binding
-from gpu_helpers import GpuLayer, compare, oracle_for, require_gpu
+from gpu_helpers import GpuLayer, compare, oracle_for, require_gpu, uses_tensor_cores
 
 pytestmark = pytest.mark.gpu
 
@@ -19,11 +19,16 @@ SPLITS = [0, 1, 2, 3, 7, 33, 300]
 
 # (B, Hq, Hkv, D, C, seqlens, window, softcap, kv_shared)
 CASES = {
-    # CUDA-core path (G = 1, 2, 4)
+    # tensor-core pair path (G = 2, D = 256, separate V)
     "sliding_g2_nowrap_cap": (3, 16, 8, 256, 64, [64, 1, 37], 64, 50.0, False),
     "sliding_g2_ring_wraps": (2, 16, 8, 256, 48, [100, 47], 48, 0.0, False),
     "sliding_g2_window_lt_cap": (2, 16, 8, 256, 64, [130, 20], 40, 0.0, False),
     "sliding_g2_edges": (5, 16, 8, 256, 32, [1, 2, 31, 32, 33], 32, 0.0, False),
+    "pair_multi_tile_ring": (2, 16, 8, 256, 200, [450, 130], 200, 0.0, False),
+    "pair_hkv1_long": (1, 2, 1, 256, 700, [700], 0, 0.0, False),
+    "pair_softcap_hkv4": (3, 8, 4, 256, 130, [130, 64, 65], 0, 30.0, False),
+    # CUDA-core path (G = 1, 2, 4 otherwise)
+    "core_g2_shared_d256": (2, 16, 8, 256, 90, [90, 17], 0, 0.0, True),
     "global_g1_shared_d512": (2, 8, 8, 512, 70, [70, 9], 0, 0.0, True),
     "global_g4_hkv2": (2, 8, 2, 256, 90, [90, 33], 0, 0.0, False),
     "global_g4_hkv1_d512": (1, 4, 1, 512, 200, [200], 0, 0.0, False),
@@ -127,7 +132,7 @@ def test_long_context(layer):
 
 
 @pytest.mark.parametrize("name", ["sliding_g2_window_lt_cap", "sliding_g2_ring_wraps",
-                                  "tc_multi_tile_tail", "tc_window_ring", "tc_edges"])
+                                  "pair_multi_tile_ring", "tc_multi_tile_tail", "tc_window_ring", "tc_edges"])
 def test_unattended_slots_never_matter(name):
     """NaN in every cache slot outside the attended range leaves the result unchanged."""
     require_gpu()
@@ -166,7 +171,7 @@ def test_split_count_invariance(which):
     w = getattr(workloads, which)()
     inp = workloads.workload_layer_inputs(w, 0)
     o1, l1 = GpuLayer(inp, split_ctas=1).run()
-    tensor_path = inp.spec.group == 16
+    tensor_path = uses_tensor_cores(inp.spec)
     for split in (2, 5, 148, 296):
         o2, l2 = GpuLayer(inp, split_ctas=split).run()
         d = (o1.float() - o2.float()).abs()
