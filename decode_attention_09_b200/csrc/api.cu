@@ -35,7 +35,9 @@ struct LayerPlan {
   int32_t heads_per_unit = 0;
   int64_t slots = 0;           // partial slots: P + units
   int32_t align = 1;           // chunk granularity in tokens (one tile / stage)
-  size_t off_lse = 0, off_o = 0, bytes = 0;
+  bool merge_in_kernel = false;  // the decode kernel merges split units itself
+  // Workspace: status word | per-unit part counters | partial LSE | partial O.
+  size_t off_cnt = 0, off_lse = 0, off_o = 0, bytes = 0;
 };
 
 constexpr size_t kStatusBytes = 256;
@@ -220,7 +222,9 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
   if (grid > 65535) return GDATTN_ERR_INVALID_ARG;
   pl.grid = static_cast<int32_t>(grid);
   pl.slots = grid + units;
-  pl.off_lse = kStatusBytes;
+  pl.merge_in_kernel = pl.kind == PathKind::kTcPair;
+  pl.off_cnt = kStatusBytes;
+  pl.off_lse = align256(pl.off_cnt + static_cast<size_t>(units) * 4);
   pl.off_o = align256(pl.off_lse + static_cast<size_t>(pl.slots) * pl.heads_per_unit * 4);
   pl.bytes = align256(pl.off_o + static_cast<size_t>(pl.slots) * pl.heads_per_unit * d->head_dim * 4);
   return GDATTN_OK;
@@ -335,6 +339,7 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
                              const gdattn_layer_desc *desc, void *out, float *lse, uint8_t *ws,
                              cudaStream_t stream) {
   uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+  uint32_t *counters = reinterpret_cast<uint32_t *>(ws + pl.off_cnt);
   float *ws_lse = reinterpret_cast<float *>(ws + pl.off_lse);
   float *ws_o = reinterpret_cast<float *>(ws + pl.off_o);
   const int32_t D = desc->head_dim;
@@ -388,6 +393,8 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     tp.ws_o = ws_o;
     tp.ws_lse = ws_lse;
     tp.status = status;
+    tp.counters = counters;
+    tp.merge_in_kernel = pl.merge_in_kernel ? 1 : 0;
     tp.geo = geo;
     tp.n_q_heads = desc->n_q_heads;
     tp.qscale = qscale;
@@ -407,7 +414,7 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
         return GDATTN_ERR_CUDA;
     }
   }
-  if (pl.grid > 1)
+  if (pl.grid > 1 && !pl.merge_in_kernel)
     return launch_combine_internal(pl, geo, ws_lse, ws_o, desc, out, lse, stream);
   return GDATTN_OK;
 }
@@ -416,9 +423,9 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
 constexpr int kMaxDevices = 64;
 
 // Address of g_noalloc_scratch on the current device.  The first call on a
-// device looks it up and enqueues a clear of the status word on `stream`
-// (the only part that must start at zero: every partial slot the combine
-// reads is written first by the decode kernel of the same call).
+// device looks it up and enqueues a clear of the array on `stream`: the status
+// word and the per-unit part counters must start at zero (every call leaves
+// the counters at zero again); partial slots are written before they are read.
 gdattn_status noalloc_scratch(cudaStream_t stream, uint8_t **addr) {
   static std::mutex mu;
   static void *by_device[kMaxDevices] = {};
@@ -429,7 +436,7 @@ gdattn_status noalloc_scratch(cudaStream_t stream, uint8_t **addr) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return GDATTN_ERR_CUDA;
-    if (cudaMemsetAsync(p, 0, kStatusBytes, stream) != cudaSuccess) return GDATTN_ERR_CUDA;
+    if (cudaMemsetAsync(p, 0, kNoallocScratchBytes, stream) != cudaSuccess) return GDATTN_ERR_CUDA;
     by_device[dev] = p;
   }
   *addr = static_cast<uint8_t *>(by_device[dev]);
@@ -472,7 +479,7 @@ int32_t gdattn_plan_splits(int32_t batch, int32_t max_seqlen, const gdattn_layer
 int32_t gdattn_plan_launches(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc) {
   LayerPlan pl;
   if (make_plan(batch, max_seqlen, desc, pl) != GDATTN_OK) return 0;
-  return pl.grid > 1 ? 2 : 1;
+  return (pl.grid > 1 && !pl.merge_in_kernel) ? 2 : 1;
 }
 
 gdattn_status gdattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {

@@ -60,6 +60,62 @@ __device__ void unit_position(const Geometry &g, int32_t b, int32_t x, int64_t &
   chunk = total > 0 ? ceil_div64(ceil_div64(total, g.nchunks), g.align) * g.align : 1;
 }
 
+// Merges np parts for one float4 column: part s holds o at o_base + s * o_stride
+// (4 floats) and lse at l_base[s * l_stride].  The loads of kBatch parts are
+// issued together; one running maximum rescales the sums between batches.
+// Returns the normalised column; m and z end as the max and the sum of
+// exp(lse_s - m), so lse = m + log z (m = -inf when every part is empty).
+template <int kBatch>
+__device__ __forceinline__ float4 merge_column(const float *o_base, int64_t o_stride,
+                                               const float *l_base, int64_t l_stride, int32_t np,
+                                               bool load_o, float &m, float &z) {
+  m = -INFINITY;
+  z = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int32_t s0 = 0; s0 < np; s0 += kBatch) {
+    float lv[kBatch];
+    float4 ov[kBatch];
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const bool in = s0 + q < np;
+      lv[q] = in ? __ldcg(l_base + (s0 + q) * l_stride) : -INFINITY;
+      ov[q] = (in && load_o) ? __ldcg(reinterpret_cast<const float4 *>(o_base + (s0 + q) * o_stride))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float bm = m;
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) bm = fmaxf(bm, lv[q]);
+    if (bm == -INFINITY) continue;  // only empty parts so far
+    const float r = (m == -INFINITY) ? 0.f : __expf(m - bm);
+    z *= r;
+    acc.x *= r;
+    acc.y *= r;
+    acc.z *= r;
+    acc.w *= r;
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      // an empty part has weight 0 and may hold anything: select, don't multiply
+      if (lv[q] == -INFINITY) continue;
+      const float w = __expf(lv[q] - bm);
+      z += w;
+      acc.x = fmaf(w, ov[q].x, acc.x);
+      acc.y = fmaf(w, ov[q].y, acc.y);
+      acc.z = fmaf(w, ov[q].z, acc.z);
+      acc.w = fmaf(w, ov[q].w, acc.w);
+    }
+    m = bm;
+  }
+  const float inv_z = (m == -INFINITY) ? 0.f : __fdividef(1.f, z);
+  return make_float4(acc.x * inv_z, acc.y * inv_z, acc.z * inv_z, acc.w * inv_z);
+}
+
+__device__ __forceinline__ void store_bf16x4(uint16_t *dst, float4 v) {
+  uint2 pk;
+  pk.x = pack_bf16x2(v.x, v.y);
+  pk.y = pack_bf16x2(v.z, v.w);
+  *reinterpret_cast<uint2 *>(dst) = pk;
+}
+
 template <bool INTERNAL>
 __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
   constexpr int kBatch = 16;
@@ -120,49 +176,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
   uint16_t *dst = p.out + (static_cast<int64_t>(b) * p.n_q_heads + h) * D;
   const int d = 4 * threadIdx.x;
   const bool owner = d < D;
-  float m = -INFINITY, z = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int32_t s0 = 0; s0 < np; s0 += kBatch) {
-    float lv[kBatch];
-    float4 ov[kBatch];
-#pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-      const bool in = s0 + q < np;
-      lv[q] = in ? __ldcg(l_base + (s0 + q) * l_stride) : -INFINITY;
-      ov[q] = (in && owner)
-                  ? __ldcg(reinterpret_cast<const float4 *>(o_base + (s0 + q) * o_stride + d))
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    float bm = m;
-#pragma unroll
-    for (int q = 0; q < kBatch; ++q) bm = fmaxf(bm, lv[q]);
-    if (bm == -INFINITY) continue;  // only empty parts so far
-    const float r = (m == -INFINITY) ? 0.f : __expf(m - bm);
-    z *= r;
-    acc.x *= r;
-    acc.y *= r;
-    acc.z *= r;
-    acc.w *= r;
-#pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-      // an empty part has weight 0 and may hold anything: select, don't multiply
-      if (lv[q] == -INFINITY) continue;
-      const float w = __expf(lv[q] - bm);
-      z += w;
-      acc.x = fmaf(w, ov[q].x, acc.x);
-      acc.y = fmaf(w, ov[q].y, acc.y);
-      acc.z = fmaf(w, ov[q].z, acc.z);
-      acc.w = fmaf(w, ov[q].w, acc.w);
-    }
-    m = bm;
-  }
-  const float inv_z = (m == -INFINITY) ? 0.f : __fdividef(1.f, z);
-  if (owner) {
-    uint2 pk;
-    pk.x = pack_bf16x2(acc.x * inv_z, acc.y * inv_z);
-    pk.y = pack_bf16x2(acc.z * inv_z, acc.w * inv_z);
-    *reinterpret_cast<uint2 *>(dst + d) = pk;
-  }
+  float m, z;
+  const float4 v = merge_column<kBatch>(o_base + (owner ? d : 0), o_stride, l_base, l_stride, np,
+                                        owner, m, z);
+  if (owner) store_bf16x4(dst + d, v);
   if (threadIdx.x == 0 && p.lse != nullptr)
     p.lse[static_cast<int64_t>(b) * p.n_q_heads + h] = (m == -INFINITY) ? -INFINITY : m + logf(z);
 }

@@ -131,6 +131,17 @@ __device__ __forceinline__ void tma_load_4d(void *dst_smem, const CUtensorMap *m
       : "memory");
 }
 
+// Atomic add at GPU scope with acquire-release semantics; returns the old value.
+// After a CTA barrier, one thread's release publishes the whole CTA's prior
+// stores; its acquire makes other CTAs' released stores visible to the CTA
+// after the next barrier.
+__device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t *addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v)
+               : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }

@@ -58,6 +58,8 @@ struct TcParams {
   float *ws_o;            // partial outputs [slots][G][D]
   float *ws_lse;          // partial lse [slots][G]
   uint32_t *status;
+  uint32_t *counters;     // per unit: parts finished in this call (zero between calls)
+  int32_t merge_in_kernel;  // 1: the CTA finishing a unit's last part merges it
   Geometry geo;           // units_per_seq == n_kv_heads
   int32_t n_q_heads;
   float qscale;           // multiplies raw scores: scale*log2(e), or scale/softcap

@@ -30,6 +30,12 @@
 // (see tc_decode.cuh), so a tile normally costs one TMEM load, one vote and two
 // P stores per thread.
 //
+// A unit split over several CTAs is merged where its last part finishes: each
+// CTA stores its part (normalised O and LSE) to the workspace and counts it in
+// the unit's counter; the CTA that brings the count to the number of parts
+// merges them (the LSE combine) and resets the counter for the next call.
+// Nobody waits for another CTA and no combine kernel is launched.
+//
 // Warp roles (224 threads) as in the 16-head kernel: warp 0 TMA, warp 1 QK MMA
 // and TMEM owner, warp 6 P.V MMA, warps 2-5 softmax (TMEM sub-partition warp %
 // 4).  Every wait is bounded.
@@ -38,6 +44,7 @@
 #include <cstdint>
 #include <cuda.h>
 
+#include "combine.cuh"
 #include "partition.cuh"
 #include "ptx.cuh"
 #include "tc_decode.cuh"
@@ -101,7 +108,8 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
   uint64_t *drain = bars + 17;      // [2] QK warp, P.V warp: all their MMAs done
   uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 19);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 20);
-  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 21);  // 48 bytes, ends before +256
+  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 21);  // 48 bytes, ends before +28
+  int32_t *merge = reinterpret_cast<int32_t *>(bars + 28);     // parts to merge, first chunk
   float *redmax = reinterpret_cast<float *>(smem + Cfg::OFF_RED);  // [4 warps][G]
   float *redsum = redmax + 4 * G;                                  // [4 warps][G]
 
@@ -200,6 +208,8 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
     bool first, last;
     // Until the preceding kernel completes, only cache rows of positions before
     // each sequence's newest one are read; q and the newest row come after.
+    // (Sending the rest of the chunk to L2 before the wait was measured to
+    // lose: the flood delays the latency-bound loads after the wait.)
     bool waited = false;
     auto ensure_waited = [&]() {
       if (!waited) {
@@ -511,6 +521,35 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
             } else {
               p.ws_lse[slot * G + lane] = lse_v;
             }
+          }
+        }
+        if (!single && p.merge_in_kernel) {
+          // Count this part (also after a failed wait, so the counter returns
+          // to zero); the CTA that completes the count merges the unit.  The
+          // barrier orders every softmax thread's part stores before the one
+          // release, whose acquire side orders the other parts before the reads.
+          named_bar_sync(1, 128);
+          if (threadIdx.x == 64) {
+            int32_t cf, cl;
+            unit_chunks(sg.unit_start, sg.n, plan->chunk, cf, cl);
+            const uint32_t done = atomic_add_acq_rel_gpu(p.counters + sg.unit, 1u);
+            const bool mine = done == static_cast<uint32_t>(cl - cf);
+            if (mine) p.counters[sg.unit] = 0u;
+            merge[0] = mine ? cl - cf + 1 : 0;
+            merge[1] = cf;
+          }
+          named_bar_sync(1, 128);
+          const int32_t np = merge[0];
+          if (np > 0) {
+            // G * D / 4 float4 columns, one per softmax thread.
+            const int e = threadIdx.x - 64, h = e / (D / 4), d = (e % (D / 4)) * 4;
+            const int64_t slot0 = static_cast<int64_t>(merge[1]) + sg.unit;
+            float m, z;
+            const float4 v = merge_column<4>(p.ws_o + (slot0 * G + h) * D + d, G * D,
+                                             p.ws_lse + slot0 * G + h, G, np, true, m, z);
+            const int64_t orow = static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + h;
+            store_bf16x4(p.out + orow * D + d, v);
+            if (d == 0 && p.lse != nullptr) p.lse[orow] = (m == -INFINITY) ? -INFINITY : m + logf(z);
           }
         }
       }

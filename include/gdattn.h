@@ -111,14 +111,16 @@ int32_t gdattn_plan_splits(int32_t batch, int32_t max_seqlen, const gdattn_layer
 /*
  * Kernel launches gdattn_decode makes for these arguments: the decode kernel,
  * plus the LSE-combine kernel when the KV range is split over more than one
- * CTA.  Returns 0 on invalid arguments.
+ * CTA and the decode kernel does not merge split units itself (the tcgen05
+ * pair kernel does).  Returns 0 on invalid arguments.
  */
 int32_t gdattn_plan_launches(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc);
 
 /*
- * Zero the workspace (its status word and partials).  Call once after
- * allocating a workspace, or zero it yourself; the library keeps the status
- * word clear afterwards.
+ * Zero the workspace.  Its status word and per-unit part counters must start
+ * at zero: call this once after allocating a workspace (or zero it yourself).
+ * Every decode call leaves the counters at zero again; the status word latches
+ * device-side errors until gdattn_check_device_status reads and clears it.
  */
 gdattn_status gdattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
@@ -171,11 +173,11 @@ gdattn_status gdattn_combine(const float *o_partial, const float *lse_partial, i
  * Same arguments (workspace and workspace_bytes dropped), host checks, kernels
  * and results as gdattn_decode: for the same inputs on the same device both
  * produce bit-identical out and lse.  The split-KV scratch (status word,
- * partial LSE, partial O) is one fixed array inside the library,
+ * part counters, partial LSE, partial O) is one fixed array inside the library,
  * GDATTN_NOALLOC_SCRATCH_BYTES per device context, reserved when the library's
  * device code is loaded, so no call allocates device or host memory.
  *  - The first call on each device looks the array up (cudaGetSymbolAddress)
- *    and enqueues a clear of its status word on `stream`; make that first call
+ *    and enqueues a clear of the whole array on `stream`; make that first call
  *    outside stream capture.  Later calls only enqueue kernels.
  *  - A layer whose gdattn_workspace_size exceeds GDATTN_NOALLOC_SCRATCH_BYTES
  *    returns GDATTN_ERR_WORKSPACE and enqueues nothing; use gdattn_decode.

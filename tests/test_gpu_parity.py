@@ -256,3 +256,18 @@ def test_cuda_graph_replay_matches_eager():
     torch.cuda.synchronize()
     for (o, l), (eo, el) in zip(outs, eager):
         assert torch.equal(o, eo) and torch.equal(l, el)
+
+
+@pytest.mark.parametrize("split", [2, 7, 33])
+def test_part_counters_return_to_zero(split):
+    """Units merged inside the decode kernel leave their arrival counters at
+    zero (the workspace holds the status word, then one counter per unit)."""
+    require_gpu()
+    inp, (o_ref, l_ref) = case_ref("pair_multi_tile_ring")
+    layer = GpuLayer(inp, split_ctas=split)
+    for _ in range(3):
+        out, lse = layer.run()
+        units = inp.q.shape[0] * inp.spec.n_kv_heads
+        cnt = layer.ws[256:256 + 4 * units].view(torch.int32)
+        assert int(cnt.abs().sum()) == 0
+    compare(out, lse, o_ref, l_ref, ulp_floor=True, what=f"split {split}")
