@@ -39,7 +39,7 @@ class LayerDesc(ctypes.Structure):
         ("cache_capacity", ctypes.c_int32),
         ("cache_batch_stride", ctypes.c_int64),
         ("split_ctas", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("flags", ctypes.c_int32),
     ]
 
 
@@ -104,19 +104,23 @@ def _stream_handle(stream) -> Optional[int]:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
+GDATTN_FLAG_EVEN_UNITS = 1
+
+
 def make_desc(n_q_heads: int, n_kv_heads: int, head_dim: int, window: int, softcap: float,
               scale: float, kv_shared: bool, cache_capacity: int, cache_batch_stride: int = 0,
-              split_ctas: int = 0) -> LayerDesc:
+              split_ctas: int = 0, flags: int = 0) -> LayerDesc:
     return LayerDesc(int(n_q_heads), int(n_kv_heads), int(head_dim), int(window),
                      float(softcap), float(scale), 1 if kv_shared else 0, int(cache_capacity),
-                     int(cache_batch_stride), int(split_ctas), 0)
+                     int(cache_batch_stride), int(split_ctas), int(flags))
 
 
-def desc_from_spec(spec, split_ctas: int = 0, capacity: Optional[int] = None) -> LayerDesc:
+def desc_from_spec(spec, split_ctas: int = 0, capacity: Optional[int] = None,
+                   flags: int = 0) -> LayerDesc:
     """Descriptor for a ``workloads.LayerSpec``."""
     return make_desc(spec.n_q_heads, spec.n_kv_heads, spec.head_dim, spec.window, spec.softcap,
                      spec.scale, spec.kv_shared,
-                     capacity if capacity is not None else spec.capacity, 0, split_ctas)
+                     capacity if capacity is not None else spec.capacity, 0, split_ctas, flags)
 
 
 def workspace_size(batch: int, max_seqlen: int, desc: LayerDesc) -> int:

@@ -36,6 +36,9 @@ struct LayerPlan {
   int64_t slots = 0;           // partial slots: P + units
   int32_t align = 1;           // chunk granularity in tokens (one tile / stage)
   bool merge_in_kernel = false;  // the decode kernel merges split units itself
+  int32_t cluster = 1;           // > 1: each unit split over a cluster of this many CTAs
+  // A separate LSE-combine launch follows the decode kernel.
+  bool needs_combine() const { return grid > 1 && cluster == 1 && !merge_in_kernel; }
   // Workspace: status word | per-unit part counters | partial LSE | partial O.
   size_t off_cnt = 0, off_lse = 0, off_o = 0, bytes = 0;
 };
@@ -147,13 +150,52 @@ int query_tc_pair(const void *fn, int threads, int smem) {
   return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
 }
 
+// Clusters of k CTAs of a kernel that can be resident at once (0 on error),
+// measured once per (kernel, k).
+int cached_clusters(const void *fn, int threads, int smem, int k) {
+  struct Entry {
+    const void *fn;
+    int k, n;
+  };
+  static std::mutex mu;
+  static Entry cache[32];
+  static int used = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].fn == fn && cache[i].k == k) return cache[i].n;
+  int n = 0;
+  if (k > 8 && cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                   cudaSuccess) {
+    cudaGetLastError();
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(k);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = k;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+  }
+  if (used < 32) cache[used++] = Entry{fn, k, n};
+  return n;
+}
+
 // ---------------------------------------------------------------- planning
 gdattn_status check_desc(const gdattn_layer_desc *d) {
   if (d == nullptr) return GDATTN_ERR_INVALID_ARG;
   if (d->n_q_heads <= 0 || d->n_kv_heads <= 0 || d->head_dim <= 0 || d->cache_capacity <= 0)
     return GDATTN_ERR_INVALID_ARG;
   if (d->n_q_heads % d->n_kv_heads != 0) return GDATTN_ERR_INVALID_ARG;
-  if (d->window < 0 || d->split_ctas < 0 || d->reserved != 0) return GDATTN_ERR_INVALID_ARG;
+  if (d->window < 0 || d->split_ctas < 0 || (d->flags & ~GDATTN_FLAG_EVEN_UNITS) != 0)
+    return GDATTN_ERR_INVALID_ARG;
   if (!(d->softcap >= 0.f) || !std::isfinite(d->softcap) || !std::isfinite(d->scale))
     return GDATTN_ERR_INVALID_ARG;
   if (d->kv_shared != 0 && d->kv_shared != 1) return GDATTN_ERR_INVALID_ARG;
@@ -219,9 +261,25 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   if (d->split_ctas > 0) grid = d->split_ctas;
+  // Even units on the pair kernel: one cluster of k CTAs per unit, k the largest
+  // power of two with all units * k CTAs resident at once and a tile per rank.
+  pl.cluster = 1;
+  if ((d->flags & GDATTN_FLAG_EVEN_UNITS) && d->split_ctas == 0 &&
+      pl.kind == PathKind::kTcPair) {
+    const int64_t tiles = (per_unit + TcPairConfig::TILE - 1) / TcPairConfig::TILE;
+    for (int k = 16; k >= 2; k /= 2) {
+      if (units * k > cap || k > tiles) continue;
+      if (cached_clusters(reinterpret_cast<const void *>(tc_pair_decode_kernel),
+                          TcPairConfig::kThreads, TcPairConfig::SMEM, k) < units)
+        continue;
+      pl.cluster = k;
+      grid = units * k;
+      break;
+    }
+  }
   if (grid > 65535) return GDATTN_ERR_INVALID_ARG;
   pl.grid = static_cast<int32_t>(grid);
-  pl.slots = grid + units;
+  pl.slots = pl.cluster > 1 ? 0 : grid + units;  // cluster mode merges in shared memory
   pl.merge_in_kernel = pl.kind == PathKind::kTcPair;
   pl.off_cnt = kStatusBytes;
   pl.off_lse = align256(pl.off_cnt + static_cast<size_t>(units) * 4);
@@ -231,8 +289,9 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
 }
 
 // --------------------------------------------------------------- launching
+// attr must hold two entries.  cluster > 1 groups CTAs into 1-D clusters.
 cudaLaunchConfig_t launch_config(dim3 grid, int threads, int smem, cudaStream_t stream,
-                                 cudaLaunchAttribute *attr) {
+                                 cudaLaunchAttribute *attr, int cluster = 1) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(threads);
@@ -244,6 +303,13 @@ cudaLaunchConfig_t launch_config(dim3 grid, int threads, int smem, cudaStream_t 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (cluster > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
   return cfg;
 }
 
@@ -305,7 +371,7 @@ gdattn_status launch_combine_internal(const LayerPlan &pl, const Geometry &geo, 
   cp.geo = geo;
   cp.heads_per_unit = pl.heads_per_unit;
   cp.n_splits = 0;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg =
       launch_config(dim3(static_cast<unsigned>(geo.batch * pl.units_per_seq),
                          static_cast<unsigned>(pl.heads_per_unit)),
@@ -360,7 +426,7 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
   geo.nchunks = pl.grid;
   geo.align = pl.align;
 
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   if (pl.kind == PathKind::kCore) {
     const CoreKernel ck = core_pick(D, desc->n_q_heads / Hkv, Hkv, desc->kv_shared != 0);
     CoreParams cp;
@@ -394,7 +460,8 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     tp.ws_lse = ws_lse;
     tp.status = status;
     tp.counters = counters;
-    tp.merge_in_kernel = pl.merge_in_kernel ? 1 : 0;
+    tp.merge_in_kernel = (pl.merge_in_kernel && pl.cluster == 1) ? 1 : 0;
+    tp.cluster = pl.cluster;
     tp.geo = geo;
     tp.n_q_heads = desc->n_q_heads;
     tp.qscale = qscale;
@@ -408,13 +475,13 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
       if (!encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, batch, bstride,
                             TcPairConfig::TILE))
         return GDATTN_ERR_CUDA;
-      cudaLaunchConfig_t cfg =
-          launch_config(dim3(pl.grid), TcPairConfig::kThreads, TcPairConfig::SMEM, stream, attr);
+      cudaLaunchConfig_t cfg = launch_config(dim3(pl.grid), TcPairConfig::kThreads,
+                                             TcPairConfig::SMEM, stream, attr, pl.cluster);
       if (cudaLaunchKernelEx(&cfg, tc_pair_decode_kernel, kmap, vmap, qmap, tp) != cudaSuccess)
         return GDATTN_ERR_CUDA;
     }
   }
-  if (pl.grid > 1 && !pl.merge_in_kernel)
+  if (pl.needs_combine())
     return launch_combine_internal(pl, geo, ws_lse, ws_o, desc, out, lse, stream);
   return GDATTN_OK;
 }
@@ -479,7 +546,7 @@ int32_t gdattn_plan_splits(int32_t batch, int32_t max_seqlen, const gdattn_layer
 int32_t gdattn_plan_launches(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc) {
   LayerPlan pl;
   if (make_plan(batch, max_seqlen, desc, pl) != GDATTN_OK) return 0;
-  return (pl.grid > 1 && !pl.merge_in_kernel) ? 2 : 1;
+  return pl.needs_combine() ? 2 : 1;
 }
 
 gdattn_status gdattn_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
@@ -548,7 +615,7 @@ gdattn_status gdattn_combine(const float *o_partial, const float *lse_partial, i
   cp.head_dim = head_dim;
   cp.heads_per_unit = 0;
   cp.n_splits = n_splits;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = launch_config(dim3(batch, n_q_heads), combine_threads(head_dim), 0,
                                          static_cast<cudaStream_t>(stream), attr);
   return cudaLaunchKernelEx(&cfg, combine_kernel<false>, cp) == cudaSuccess ? GDATTN_OK

@@ -60,53 +60,84 @@ __device__ void unit_position(const Geometry &g, int32_t b, int32_t x, int64_t &
   chunk = total > 0 ? ceil_div64(ceil_div64(total, g.nchunks), g.align) * g.align : 1;
 }
 
-// Merges np parts for one float4 column: part s holds o at o_base + s * o_stride
-// (4 floats) and lse at l_base[s * l_stride].  The loads of kBatch parts are
-// issued together; one running maximum rescales the sums between batches.
-// Returns the normalised column; m and z end as the max and the sum of
-// exp(lse_s - m), so lse = m + log z (m = -inf when every part is empty).
+// Merges np parts for NC float4 columns at once: for column c, part s holds
+// o at o_col[c] + s * o_stride (4 floats) and lse at l_col[c][s * l_stride].
+// The loads of kBatch parts for all NC columns are issued together; a running
+// maximum rescales the sums between batches.  res[c] is the normalised column;
+// m[c] and z[c] end as the max and the sum of exp(lse_s - m), so lse = m + log z
+// (m = -inf when every part is empty).  load_o = false skips the O loads.
+template <int NC, int kBatch>
+__device__ __forceinline__ void merge_columns(const float *const (&o_col)[NC],
+                                              const float *const (&l_col)[NC], int64_t o_stride,
+                                              int64_t l_stride, int32_t np, bool load_o,
+                                              float4 (&res)[NC], float (&m)[NC], float (&z)[NC]) {
+  float4 acc[NC];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    m[c] = -INFINITY;
+    z[c] = 0.f;
+    acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int32_t s0 = 0; s0 < np; s0 += kBatch) {
+    float lv[NC][kBatch];
+    float4 ov[NC][kBatch];
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const bool in = s0 + q < np;
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        lv[c][q] = in ? __ldcg(l_col[c] + (s0 + q) * l_stride) : -INFINITY;
+        ov[c][q] = (in && load_o)
+                       ? __ldcg(reinterpret_cast<const float4 *>(o_col[c] + (s0 + q) * o_stride))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      float bm = m[c];
+#pragma unroll
+      for (int q = 0; q < kBatch; ++q) bm = fmaxf(bm, lv[c][q]);
+      if (bm == -INFINITY) continue;  // only empty parts so far
+      const float r = (m[c] == -INFINITY) ? 0.f : __expf(m[c] - bm);
+      z[c] *= r;
+      acc[c].x *= r;
+      acc[c].y *= r;
+      acc[c].z *= r;
+      acc[c].w *= r;
+#pragma unroll
+      for (int q = 0; q < kBatch; ++q) {
+        // an empty part has weight 0 and may hold anything: select, don't multiply
+        if (lv[c][q] == -INFINITY) continue;
+        const float w = __expf(lv[c][q] - bm);
+        z[c] += w;
+        acc[c].x = fmaf(w, ov[c][q].x, acc[c].x);
+        acc[c].y = fmaf(w, ov[c][q].y, acc[c].y);
+        acc[c].z = fmaf(w, ov[c][q].z, acc[c].z);
+        acc[c].w = fmaf(w, ov[c][q].w, acc[c].w);
+      }
+      m[c] = bm;
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    const float inv_z = (m[c] == -INFINITY) ? 0.f : __fdividef(1.f, z[c]);
+    res[c] = make_float4(acc[c].x * inv_z, acc[c].y * inv_z, acc[c].z * inv_z, acc[c].w * inv_z);
+  }
+}
+
+// One column (see merge_columns).
 template <int kBatch>
 __device__ __forceinline__ float4 merge_column(const float *o_base, int64_t o_stride,
                                                const float *l_base, int64_t l_stride, int32_t np,
                                                bool load_o, float &m, float &z) {
-  m = -INFINITY;
-  z = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int32_t s0 = 0; s0 < np; s0 += kBatch) {
-    float lv[kBatch];
-    float4 ov[kBatch];
-#pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-      const bool in = s0 + q < np;
-      lv[q] = in ? __ldcg(l_base + (s0 + q) * l_stride) : -INFINITY;
-      ov[q] = (in && load_o) ? __ldcg(reinterpret_cast<const float4 *>(o_base + (s0 + q) * o_stride))
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    float bm = m;
-#pragma unroll
-    for (int q = 0; q < kBatch; ++q) bm = fmaxf(bm, lv[q]);
-    if (bm == -INFINITY) continue;  // only empty parts so far
-    const float r = (m == -INFINITY) ? 0.f : __expf(m - bm);
-    z *= r;
-    acc.x *= r;
-    acc.y *= r;
-    acc.z *= r;
-    acc.w *= r;
-#pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-      // an empty part has weight 0 and may hold anything: select, don't multiply
-      if (lv[q] == -INFINITY) continue;
-      const float w = __expf(lv[q] - bm);
-      z += w;
-      acc.x = fmaf(w, ov[q].x, acc.x);
-      acc.y = fmaf(w, ov[q].y, acc.y);
-      acc.z = fmaf(w, ov[q].z, acc.z);
-      acc.w = fmaf(w, ov[q].w, acc.w);
-    }
-    m = bm;
-  }
-  const float inv_z = (m == -INFINITY) ? 0.f : __fdividef(1.f, z);
-  return make_float4(acc.x * inv_z, acc.y * inv_z, acc.z * inv_z, acc.w * inv_z);
+  const float *const o_col[1] = {o_base};
+  const float *const l_col[1] = {l_base};
+  float4 res[1];
+  float mm[1], zz[1];
+  merge_columns<1, kBatch>(o_col, l_col, o_stride, l_stride, np, load_o, res, mm, zz);
+  m = mm[0];
+  z = zz[0];
+  return res[0];
 }
 
 __device__ __forceinline__ void store_bf16x4(uint16_t *dst, float4 v) {

@@ -179,6 +179,44 @@ struct SegmentIter {
   }
 };
 
+// Cluster split: unit u (sequence u / units_per_seq, group u % units_per_seq)
+// is shared by the k CTAs of one thread-block cluster; rank r takes whole
+// tiles [r * T / k, (r + 1) * T / k) of the unit's T = ceil(n / tile) tiles.
+// The range is expressed as a chunk so the segment and tile iterators apply
+// unchanged (it holds one segment, or none when the unit is too short).  Run
+// by one whole warp.
+__device__ void plan_unit_split(const Geometry &g, int32_t u, int32_t r, int32_t k, int32_t tile,
+                                ChunkPlan *plan) {
+  const int lane = threadIdx.x & 31;
+  const int32_t b = u / g.units_per_seq;
+  const int32_t x = u - b * g.units_per_seq;
+  bool bad = false;
+  int64_t all = 0, before = 0;
+  for (int32_t bb = lane; bb < g.batch; bb += 32) {
+    const int64_t n_bb = attended_count(__ldg(g.seqlens + bb), g.window, g.capacity, bad);
+    all += n_bb;
+    if (bb < b) before += n_bb;
+  }
+  const int64_t total = warp_sum_i64(all) * g.units_per_seq;
+  const int64_t pre = warp_sum_i64(before) * g.units_per_seq;
+  const int anybad = __any_sync(0xffffffffu, bad);
+  bool dummy = false;
+  const int32_t n = attended_count(__ldg(g.seqlens + b), g.window, g.capacity, dummy);
+  const int64_t tiles = ceil_div64(n, tile);
+  const int64_t lo = imin64(r * tiles / k * tile, n);
+  const int64_t hi = imin64((r + 1) * tiles / k * tile, n);
+  const int64_t ustart = pre + static_cast<int64_t>(x) * n;
+  if (lane == 0) {
+    plan->total = total;
+    plan->chunk = hi - lo;
+    plan->cs = ustart + lo;
+    plan->ce = ustart + hi;
+    plan->pre0 = pre;
+    plan->b0 = b;
+    plan->bad = anybad;
+  }
+}
+
 // Chunks covering [unit_start, unit_start + n).
 __device__ __forceinline__ void unit_chunks(int64_t unit_start, int32_t n, int64_t chunk,
                                             int32_t &c_first, int32_t &c_last) {

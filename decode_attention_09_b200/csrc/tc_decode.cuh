@@ -60,6 +60,7 @@ struct TcParams {
   uint32_t *status;
   uint32_t *counters;     // per unit: parts finished in this call (zero between calls)
   int32_t merge_in_kernel;  // 1: the CTA finishing a unit's last part merges it
+  int32_t cluster;        // > 1: each unit split over one cluster of this many CTAs
   Geometry geo;           // units_per_seq == n_kv_heads
   int32_t n_q_heads;
   float qscale;           // multiplies raw scores: scale*log2(e), or scale/softcap

@@ -34,11 +34,22 @@
 // CTA stores its part (normalised O and LSE) to the workspace and counts it in
 // the unit's counter; the CTA that brings the count to the number of parts
 // merges them (the LSE combine) and resets the counter for the next call.
-// Nobody waits for another CTA and no combine kernel is launched.
+// Nobody waits for another CTA and no combine kernel is launched.  Counting and
+// merging run in a warp of their own, so the softmax warps hand a part over at
+// a barrier and go straight on with the next segment.
 //
-// Warp roles (224 threads) as in the 16-head kernel: warp 0 TMA, warp 1 QK MMA
-// and TMEM owner, warp 6 P.V MMA, warps 2-5 softmax (TMEM sub-partition warp %
-// 4).  Every wait is bounded.
+// Cluster mode (p.cluster = k > 1, for units of even length): unit u is split
+// over the k CTAs of one thread-block cluster instead of the flattened chunks.
+// Each CTA leaves its part (normalised O, LSE) in its own shared memory; after
+// a cluster barrier every CTA merges a 1/k slice of the unit's outputs, reading
+// the k parts over distributed shared memory, and a second barrier keeps each
+// CTA's shared memory alive until its peers have read it.  No workspace
+// traffic, no counters, no segment straddles a CTA boundary.
+//
+// Warp roles (256 threads): warp 0 TMA, warp 1 QK MMA and TMEM owner, warp 6
+// P.V MMA, warps 2-5 softmax (TMEM sub-partition warp % 4), warp 7 part count
+// and merge.  Q is double buffered, so the next segment's Q is loaded while the
+// current one is still in use.  Every wait is bounded.
 #pragma once
 
 #include <cstdint>
@@ -61,14 +72,15 @@ struct TcPairConfig {
   static constexpr int KB = BOXB * (D / 64);          // K tile, 32 KiB
   static constexpr int STAGEB = 2 * KB;               // K tile then V tile, 64 KiB
   static constexpr int QBOXB = N * 128;               // 16 Q rows x 64 d, 2 KiB
-  static constexpr int QB = QBOXB * (D / 64);         // 8 KiB
+  static constexpr int QB = QBOXB * (D / 64);         // 8 KiB per Q buffer
   static constexpr int PB = N * 128;                  // P: 16 rows x 64 tokens bf16, 2 KiB
-  static constexpr int OFF_Q = NST * STAGEB;
-  static constexpr int OFF_P = OFF_Q + QB;
+  static constexpr int OFF_Q = NST * STAGEB;          // 2 Q buffers
+  static constexpr int OFF_P = OFF_Q + 2 * QB;
   static constexpr int OFF_BAR = OFF_P + 2 * PB;
   static constexpr int OFF_RED = OFF_BAR + 256;
-  static constexpr int SMEM = OFF_RED + 2 * 4 * G * 4 + 1024;
-  static constexpr int kThreads = 224;
+  static constexpr int OFF_PLSE = OFF_RED + 2 * 4 * G * 4;  // cluster mode: this CTA's part LSE
+  static constexpr int SMEM = OFF_PLSE + G * 4 + 1024;
+  static constexpr int kThreads = 256;
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t S_COL = 0;                // 2 buffers x 4 partial sums x 16 columns
   static constexpr uint32_t O_COL = 128;              // 2 d-blocks x 16 columns
@@ -98,20 +110,22 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
   uint64_t *full = bars;            // [NST]  TMA -> MMA
   uint64_t *empty = bars + 3;       // [NST]  P.V -> TMA
-  uint64_t *qfull = bars + 6;       // TMA -> MMA
-  uint64_t *qempty = bars + 7;      // MMA -> TMA
-  uint64_t *sfull = bars + 8;       // [2] MMA -> softmax (S of tile i in buffer i & 1)
-  uint64_t *sempty = bars + 10;     // [2] softmax -> MMA
-  uint64_t *pfull = bars + 12;      // [2] softmax -> MMA (P of tile i in buffer i & 1)
-  uint64_t *ofull = bars + 14;      // [2] MMA -> softmax: P.V of tile i done (barrier i & 1)
-  uint64_t *oempty = bars + 16;     // softmax -> MMA: O of a finished segment read out
-  uint64_t *drain = bars + 17;      // [2] QK warp, P.V warp: all their MMAs done
-  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 19);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 20);
-  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 21);  // 48 bytes, ends before +28
-  int32_t *merge = reinterpret_cast<int32_t *>(bars + 28);     // parts to merge, first chunk
+  uint64_t *qfull = bars + 6;       // [2] TMA -> MMA (Q of segment k in buffer k & 1)
+  uint64_t *qempty = bars + 8;      // [2] MMA -> TMA
+  uint64_t *sfull = bars + 10;      // [2] MMA -> softmax (S of tile i in buffer i & 1)
+  uint64_t *sempty = bars + 12;     // [2] softmax -> MMA
+  uint64_t *pfull = bars + 14;      // [2] softmax -> MMA (P of tile i in buffer i & 1)
+  uint64_t *ofull = bars + 16;      // [2] MMA -> softmax: P.V of tile i done (barrier i & 1)
+  uint64_t *oempty = bars + 18;     // softmax -> MMA: O of a finished segment read out
+  uint64_t *drain = bars + 19;      // [2] QK warp, P.V warp: all their MMAs done
+  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 21);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 22);
+  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 23);  // 48 bytes, ends before +29
   float *redmax = reinterpret_cast<float *>(smem + Cfg::OFF_RED);  // [4 warps][G]
   float *redsum = redmax + 4 * G;                                  // [4 warps][G]
+  // Cluster mode: this CTA's part, O in the (by then idle) first KV stage.
+  float *part_lse = reinterpret_cast<float *>(smem + Cfg::OFF_PLSE);  // [G]
+  float *part_o = reinterpret_cast<float *>(stages);                   // [G][D]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -122,9 +136,9 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(qfull, 1);
-    mbar_init(qempty, 1);
     for (int s = 0; s < 2; ++s) {
+      mbar_init(&qfull[s], 1);
+      mbar_init(&qempty[s], 1);
       mbar_init(&sfull[s], 1);
       mbar_init(&sempty[s], 4);
       mbar_init(&pfull[s], 4);
@@ -134,6 +148,7 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
     *abort_flag = 0;
+    for (int h = 0; h < G; ++h) part_lse[h] = -INFINITY;  // an empty rank's part
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -149,7 +164,13 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
   // The split plan reads only seqlens, so it (and the producer's first KV
   // loads below) may run before the preceding kernel has completed; every other
   // global access waits for it (griddepcontrol.wait) in the role that makes it.
-  if (warp == 2) plan_chunk(p.geo, c, plan);
+  const int32_t crank = p.cluster > 1 ? static_cast<int32_t>(cluster_ctarank()) : 0;
+  if (warp == 2) {
+    if (p.cluster > 1)
+      plan_unit_split(p.geo, c / p.cluster, crank, p.cluster, Cfg::TILE, plan);
+    else
+      plan_chunk(p.geo, c, plan);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -183,9 +204,11 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
     int32_t qrows[8] = {};       // Q rows of segments whose Q is not issued yet
     uint32_t stage_seg[NST];     // segment of the tile last loaded into each stage
     auto issue_q = [&](bool block) -> bool {  // warp-uniform result
-      if (q_issued > 0) {
-        bool got = block ? mbar_wait(qempty, (q_issued - 1) & 1, abort_flag, p.status)
-                         : mbar_try_wait(qempty, (q_issued - 1) & 1);
+      const uint32_t qb = q_issued & 1;
+      if (q_issued >= 2) {  // buffer qb is free once segment q_issued - 2's last QK is done
+        const uint32_t ph = ((q_issued >> 1) - 1) & 1;
+        bool got = block ? mbar_wait(&qempty[qb], ph, abort_flag, p.status)
+                         : mbar_try_wait(&qempty[qb], ph);
         if (!__all_sync(0xffffffffu, got)) {
           if (block) ok = false;
           return false;
@@ -193,10 +216,10 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
       }
       const int32_t qrow = qrows[q_issued & 7];
       if (elect_one()) {
-        mbar_arrive_expect_tx(qfull, Cfg::QB);
+        mbar_arrive_expect_tx(&qfull[qb], Cfg::QB);
 #pragma unroll
         for (int j = 0; j < D / 64; ++j)
-          tma_load_2d(qs + j * Cfg::QBOXB, &qmap, 64 * j, qrow, qfull);
+          tma_load_2d(qs + qb * Cfg::QB + j * Cfg::QBOXB, &qmap, 64 * j, qrow, &qfull[qb]);
       }
       __syncwarp();
       ++q_issued;
@@ -253,7 +276,8 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
     volatile int no_abort = 0;
     for (uint32_t f = i > NST ? i - NST : 0; f < i; ++f)
       mbar_wait(&full[f % NST], (f / NST) & 1, &no_abort, p.status);
-    if (q_issued > 0) mbar_wait(qfull, (q_issued - 1) & 1, &no_abort, p.status);
+    for (uint32_t k = q_issued > 2 ? q_issued - 2 : 0; k < q_issued; ++k)
+      mbar_wait(&qfull[k & 1], (k >> 1) & 1, &no_abort, p.status);
   } else if (warp == 1) {
     // ----------------------------------------------------------- QK MMA
     const uint32_t idesc_qk = idesc_bf16_f32(64, Cfg::N, false, false);
@@ -268,10 +292,11 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
     bool first, last;
     while (ok && it.next(C, row, ntok, first, last)) {
       if (first) {
-        if (!mbar_wait(qfull, nseg & 1, abort_flag, p.status)) ok = false;
+        if (!mbar_wait(&qfull[nseg & 1], (nseg >> 1) & 1, abort_flag, p.status)) ok = false;
         if (!__all_sync(0xffffffffu, ok)) break;
         ++nseg;
       }
+      const uint32_t qb = (nseg - 1) & 1;
       const int st = i % NST, sb = i & 1;
       if (!mbar_wait(&full[st], (i / NST) & 1, abort_flag, p.status)) ok = false;
       if (ok && i >= 2 && !mbar_wait(&sempty[sb], ((i >> 1) - 1) & 1, abort_flag, p.status))
@@ -285,12 +310,12 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = a0 + ((j * Cfg::BOXB + kk * 32) >> 4);
-            const uint64_t bd = qdesc + ((j * Cfg::QBOXB + kk * 32) >> 4);
+            const uint64_t bd = qdesc + ((qb * Cfg::QB + j * Cfg::QBOXB + kk * 32) >> 4);
             tc_mma_bf16(tmem + Cfg::S_COL + sb * 64 + kk * 16, ad, bd, idesc_qk, j != 0);
           }
         }
         tc_commit(&sfull[sb]);
-        if (last) tc_commit(qempty);
+        if (last) tc_commit(&qempty[qb]);
       }
       __syncwarp();
       ++i;
@@ -344,6 +369,52 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
     __syncwarp();
     volatile int no_abort = 0;
     mbar_wait(&drain[1], 0, &no_abort, p.status);
+  } else if (warp == 7) {
+    // -------------------------------------------------- part count, merge
+    // Segment by segment in the softmax warps' order: after a partial is
+    // stored (barrier 2), count it with one acq_rel atomic; the CTA whose count
+    // completes the unit merges all of its parts (lane c takes float4 columns
+    // c, c + 32, c + 64, c + 96) and resets the counter.  Parts are counted
+    // after a failed wait too, so the counters always return to zero.
+    if (p.merge_in_kernel) {
+      grid_dependency_wait();  // counters, workspace and outputs
+      SegmentIter sit;
+      sit.init(p.geo, *plan);
+      Segment sg;
+      while (sit.next(sg)) {
+        if (sg.whole()) continue;
+        named_bar_sync(2, 160);
+        int32_t cf, cl;
+        unit_chunks(sg.unit_start, sg.n, plan->chunk, cf, cl);
+        uint32_t done = 0;
+        if (lane == 0) done = atomic_add_acq_rel_gpu(p.counters + sg.unit, 1u);
+        done = __shfl_sync(0xffffffffu, done, 0);
+        __syncwarp();  // lane 0's acquire before every lane's reads
+        if (done != static_cast<uint32_t>(cl - cf)) continue;
+        if (lane == 0) p.counters[sg.unit] = 0u;
+        constexpr int NC = G * D / 4 / 32;  // float4 columns per lane
+        const int64_t slot0 = static_cast<int64_t>(cf) + sg.unit;
+        const float *o_col[NC];
+        const float *l_col[NC];
+#pragma unroll
+        for (int k = 0; k < NC; ++k) {
+          const int e = lane + 32 * k, h = e / (D / 4), d = (e % (D / 4)) * 4;
+          o_col[k] = p.ws_o + (slot0 * G + h) * D + d;
+          l_col[k] = p.ws_lse + slot0 * G + h;
+        }
+        float4 res[NC];
+        float m[NC], z[NC];
+        merge_columns<NC, 4>(o_col, l_col, G * D, G, cl - cf + 1, true, res, m, z);
+#pragma unroll
+        for (int k = 0; k < NC; ++k) {
+          const int e = lane + 32 * k, h = e / (D / 4), d = (e % (D / 4)) * 4;
+          const int64_t orow = static_cast<int64_t>(sg.b) * p.n_q_heads + sg.x * G + h;
+          store_bf16x4(p.out + orow * D + d, res[k]);
+          if (d == 0 && p.lse != nullptr)
+            p.lse[orow] = (m[k] == -INFINITY) ? -INFINITY : m[k] + logf(z[k]);
+        }
+      }
+    }
   } else {
     // ---------------------------------------------------------- softmax
     grid_dependency_wait();  // outputs and workspace are written below
@@ -482,7 +553,8 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
         if ((lane & 15) == 0) redsum[qd * G + hd] = ls;
         named_bar_sync(1, 128);
         const Segment &sg = it.seg;
-        const bool single = sg.whole();
+        const bool part_local = p.cluster > 1;  // the part stays in shared memory
+        const bool single = sg.whole() && !part_local;
         const int64_t slot = static_cast<int64_t>(c) + sg.unit;
         const int h0 = sg.x * G;
         float L[G], inv[G];
@@ -501,7 +573,9 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
 #pragma unroll
             for (int h = 0; h < G; ++h) {
               const float val = (o[h] + o[G + h]) * inv[h];
-              if (single)
+              if (part_local)
+                part_o[h * D + d] = val;
+              else if (single)
                 p.out[(static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + h) * D + d] =
                     f32_to_bf16_rn(val);
               else
@@ -515,7 +589,9 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
             const float mr = lane ? m_ref[1] : m_ref[0];
             const float Lh = lane ? L[1] : L[0];
             const float lse_v = (mr + log2f(Lh)) * 0.69314718055994530942f;
-            if (single) {
+            if (part_local) {
+              part_lse[lane] = lse_v;
+            } else if (single) {
               if (p.lse != nullptr)
                 p.lse[static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + lane] = lse_v;
             } else {
@@ -523,35 +599,8 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
             }
           }
         }
-        if (!single && p.merge_in_kernel) {
-          // Count this part (also after a failed wait, so the counter returns
-          // to zero); the CTA that completes the count merges the unit.  The
-          // barrier orders every softmax thread's part stores before the one
-          // release, whose acquire side orders the other parts before the reads.
-          named_bar_sync(1, 128);
-          if (threadIdx.x == 64) {
-            int32_t cf, cl;
-            unit_chunks(sg.unit_start, sg.n, plan->chunk, cf, cl);
-            const uint32_t done = atomic_add_acq_rel_gpu(p.counters + sg.unit, 1u);
-            const bool mine = done == static_cast<uint32_t>(cl - cf);
-            if (mine) p.counters[sg.unit] = 0u;
-            merge[0] = mine ? cl - cf + 1 : 0;
-            merge[1] = cf;
-          }
-          named_bar_sync(1, 128);
-          const int32_t np = merge[0];
-          if (np > 0) {
-            // G * D / 4 float4 columns, one per softmax thread.
-            const int e = threadIdx.x - 64, h = e / (D / 4), d = (e % (D / 4)) * 4;
-            const int64_t slot0 = static_cast<int64_t>(merge[1]) + sg.unit;
-            float m, z;
-            const float4 v = merge_column<4>(p.ws_o + (slot0 * G + h) * D + d, G * D,
-                                             p.ws_lse + slot0 * G + h, G, np, true, m, z);
-            const int64_t orow = static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + h;
-            store_bf16x4(p.out + orow * D + d, v);
-            if (d == 0 && p.lse != nullptr) p.lse[orow] = (m == -INFINITY) ? -INFINITY : m + logf(z);
-          }
-        }
+        // Hand a partial over to the merge warp (it counts it after the barrier).
+        if (!single && !part_local && p.merge_in_kernel) named_bar_sync(2, 160);
       }
       ++i;
     }
@@ -559,6 +608,52 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (p.cluster > 1) {
+    // --- cluster merge: CTA `crank` finalises float4 columns
+    // [crank * per, (crank + 1) * per) of the unit's G x D outputs.
+    cluster_sync();  // every CTA's part is in its shared memory
+    grid_dependency_wait();
+    const int32_t k = p.cluster;
+    const int per = G * D / 4 / k;
+    const int32_t u = c / k;
+    const int32_t b = u / p.geo.units_per_seq, x = u - b * p.geo.units_per_seq;
+    for (int t = threadIdx.x; t < per; t += Cfg::kThreads) {
+      const int e = crank * per + t, h = e / (D / 4), d = (e % (D / 4)) * 4;
+      float lv[16];
+      float4 ov[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        if (q < k) {
+          lv[q] = ld_cluster_f32(map_cluster(part_lse + h, q));
+          ov[q] = ld_cluster_f32x4(map_cluster(part_o + h * D + d, q));
+        }
+      }
+      float m = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (q < k) m = fmaxf(m, lv[q]);
+      float z = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        // an empty part has weight 0 and may hold anything: select, don't multiply
+        if (q < k && lv[q] != -INFINITY) {
+          const float w = __expf(lv[q] - m);
+          z += w;
+          acc.x = fmaf(w, ov[q].x, acc.x);
+          acc.y = fmaf(w, ov[q].y, acc.y);
+          acc.z = fmaf(w, ov[q].z, acc.z);
+          acc.w = fmaf(w, ov[q].w, acc.w);
+        }
+      }
+      const float inv_z = (m == -INFINITY) ? 0.f : __fdividef(1.f, z);
+      const int64_t orow = static_cast<int64_t>(b) * p.n_q_heads + x * G + h;
+      store_bf16x4(p.out + orow * D + d,
+                   make_float4(acc.x * inv_z, acc.y * inv_z, acc.z * inv_z, acc.w * inv_z));
+      if (d == 0 && p.lse != nullptr) p.lse[orow] = (m == -INFINITY) ? -INFINITY : m + logf(z);
+    }
+    cluster_sync();  // the peers are done reading this CTA's shared memory
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TMEM_COLS);

@@ -90,8 +90,19 @@ typedef struct gdattn_layer_desc {
                                  otherwise >= C*Hkv*D and a multiple of 8 */
   int32_t split_ctas;     /* 0: the planner picks how many CTAs share the KV range; > 0
                              forces that many (tests and tuning) */
-  int32_t reserved;       /* must be 0 */
+  int32_t flags;          /* GDATTN_FLAG_* bits; other bits must be 0 */
 } gdattn_layer_desc;
+
+/*
+ * The caller expects every sequence of a call to attend about the same number
+ * of positions (uniform context lengths, or all of them past the window).  The
+ * tcgen05 kernels may then split each (sequence, KV head) unit evenly over the
+ * CTAs of one thread-block cluster and merge the parts in distributed shared
+ * memory; with uneven lengths that split stays correct but loses balance.
+ * Without the flag (or with split_ctas > 0) the KV ranges of all units are laid
+ * end to end and cut into equal chunks.
+ */
+#define GDATTN_FLAG_EVEN_UNITS 1
 
 /*
  * Bytes of device workspace gdattn_decode needs for this layer geometry and

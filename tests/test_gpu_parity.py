@@ -271,3 +271,35 @@ def test_part_counters_return_to_zero(split):
         cnt = layer.ws[256:256 + 4 * units].view(torch.int32)
         assert int(cnt.abs().sum()) == 0
     compare(out, lse, o_ref, l_ref, ulp_floor=True, what=f"split {split}")
+
+
+# (B, Hq, Hkv, D, C, seqlens, window, softcap): pair-kernel geometries run with
+# GDATTN_FLAG_EVEN_UNITS, i.e. one thread-block cluster per (sequence, KV head)
+CLUSTER_CASES = {
+    "k4_empty_rank": (2, 16, 8, 256, 200, [450, 130], 200, 0.0),
+    "k8_one_unit": (1, 2, 1, 256, 700, [700], 0, 0.0),
+    "k16_long": (1, 4, 2, 256, 2048, [2048], 0, 0.0),
+    "ragged_mostly_empty": (3, 8, 4, 256, 1000, [1000, 64, 1], 0, 0.0),
+    "softcap_ring": (2, 16, 8, 256, 512, [1300, 700], 512, 30.0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CLUSTER_CASES))
+def test_cluster_split_matches_oracle(name):
+    """Units split over thread-block clusters and merged in distributed shared
+    memory give the oracle's result, ragged lengths and empty ranks included."""
+    require_gpu()
+    B, Hq, Hkv, D, C, sl, w, cap = CLUSTER_CASES[name]
+    inp = workloads.random_case(300 + sorted(CLUSTER_CASES).index(name), B, Hq, Hkv, D, C, sl,
+                                window=w, softcap=cap)
+    o_ref, l_ref = oracle_for(inp)
+    layer = GpuLayer(inp)
+    layer.desc = binding.desc_from_spec(inp.spec, capacity=C, flags=binding.GDATTN_FLAG_EVEN_UNITS)
+    layer.ws = binding.alloc_workspace(B, layer.max_seqlen, layer.desc)
+    units = B * Hkv
+    splits = binding.plan_splits(B, layer.max_seqlen, layer.desc)
+    assert splits % units == 0 and splits // units >= 2, splits  # cluster mode was taken
+    assert binding.launches_per_call(B, layer.max_seqlen, layer.desc) == 1
+    for _ in range(2):
+        out, lse = layer.run()
+        compare(out, lse, o_ref, l_ref, ulp_floor=True, what=f"{name} k={splits // units}")
