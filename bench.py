@@ -154,7 +154,10 @@ class Stack:
             inp = workloads.layer_inputs(spec, w.batch, seqlens, w.seed * 1000 + i + seed_offset,
                                          device=device, heavy_row_frac=w.heavy_row_frac,
                                          heavy_row_scale=w.heavy_row_scale)
-            desc = binding.desc_from_spec(spec)
+            # all sequences of an even workload attend the same number of positions:
+            # tell the planner, so it splits each unit into equal whole-tile parts
+            desc = binding.desc_from_spec(
+                spec, flags=binding.GDATTN_FLAG_EVEN_UNITS if w.ragged is None else 0)
             ws = binding.alloc_workspace(w.batch, self.max_seqlen, desc, device)
             out = torch.empty_like(inp.q)
             lse = torch.empty(inp.q.shape[:2], dtype=torch.float32, device=device)

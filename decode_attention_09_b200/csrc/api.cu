@@ -36,9 +36,9 @@ struct LayerPlan {
   int64_t slots = 0;           // partial slots: P + units
   int32_t align = 1;           // chunk granularity in tokens (one tile / stage)
   bool merge_in_kernel = false;  // the decode kernel merges split units itself
-  int32_t cluster = 1;           // > 1: each unit split over a cluster of this many CTAs
+  int32_t split_k = 1;           // > 1: each unit cut into split_k whole-tile parts
   // A separate LSE-combine launch follows the decode kernel.
-  bool needs_combine() const { return grid > 1 && cluster == 1 && !merge_in_kernel; }
+  bool needs_combine() const { return grid > 1 && !merge_in_kernel; }
   // Workspace: status word | per-unit part counters | partial LSE | partial O.
   size_t off_cnt = 0, off_lse = 0, off_o = 0, bytes = 0;
 };
@@ -150,44 +150,6 @@ int query_tc_pair(const void *fn, int threads, int smem) {
   return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
 }
 
-// Clusters of k CTAs of a kernel that can be resident at once (0 on error),
-// measured once per (kernel, k).
-int cached_clusters(const void *fn, int threads, int smem, int k) {
-  struct Entry {
-    const void *fn;
-    int k, n;
-  };
-  static std::mutex mu;
-  static Entry cache[32];
-  static int used = 0;
-  std::lock_guard<std::mutex> lock(mu);
-  for (int i = 0; i < used; ++i)
-    if (cache[i].fn == fn && cache[i].k == k) return cache[i].n;
-  int n = 0;
-  if (k > 8 && cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-                   cudaSuccess) {
-    cudaGetLastError();
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(k);
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = k;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
-      cudaGetLastError();
-      n = 0;
-    }
-  }
-  if (used < 32) cache[used++] = Entry{fn, k, n};
-  return n;
-}
-
 // ---------------------------------------------------------------- planning
 gdattn_status check_desc(const gdattn_layer_desc *d) {
   if (d == nullptr) return GDATTN_ERR_INVALID_ARG;
@@ -261,25 +223,25 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   if (d->split_ctas > 0) grid = d->split_ctas;
-  // Even units on the pair kernel: one cluster of k CTAs per unit, k the largest
-  // power of two with all units * k CTAs resident at once and a tile per rank.
-  pl.cluster = 1;
-  if ((d->flags & GDATTN_FLAG_EVEN_UNITS) && d->split_ctas == 0 &&
-      pl.kind == PathKind::kTcPair) {
-    const int64_t tiles = (per_unit + TcPairConfig::TILE - 1) / TcPairConfig::TILE;
-    for (int k = 16; k >= 2; k /= 2) {
-      if (units * k > cap || k > tiles) continue;
-      if (cached_clusters(reinterpret_cast<const void *>(tc_pair_decode_kernel),
-                          TcPairConfig::kThreads, TcPairConfig::SMEM, k) < units)
-        continue;
-      pl.cluster = k;
-      grid = units * k;
-      break;
+  // Even units on the tcgen05 kernels: cut every unit into k whole-tile parts,
+  // k minimising the largest part (the smallest such k, for cheaper merges)
+  // with all units * k CTAs resident at once.  No CTA then straddles two units.
+  pl.split_k = 1;
+  if ((d->flags & GDATTN_FLAG_EVEN_UNITS) && d->split_ctas == 0 && pl.kind != PathKind::kCore) {
+    const int64_t tiles = (per_unit + 63) / 64;
+    int64_t best = tiles;
+    for (int64_t k = 2; k <= tiles && units * k <= cap && k <= 64; ++k) {
+      const int64_t most = (tiles + k - 1) / k;
+      if (most < best) {
+        best = most;
+        pl.split_k = static_cast<int32_t>(k);
+      }
     }
+    if (pl.split_k > 1) grid = units * pl.split_k;
   }
   if (grid > 65535) return GDATTN_ERR_INVALID_ARG;
   pl.grid = static_cast<int32_t>(grid);
-  pl.slots = pl.cluster > 1 ? 0 : grid + units;  // cluster mode merges in shared memory
+  pl.slots = grid + units;
   pl.merge_in_kernel = pl.kind == PathKind::kTcPair;
   pl.off_cnt = kStatusBytes;
   pl.off_lse = align256(pl.off_cnt + static_cast<size_t>(units) * 4);
@@ -289,9 +251,8 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
 }
 
 // --------------------------------------------------------------- launching
-// attr must hold two entries.  cluster > 1 groups CTAs into 1-D clusters.
 cudaLaunchConfig_t launch_config(dim3 grid, int threads, int smem, cudaStream_t stream,
-                                 cudaLaunchAttribute *attr, int cluster = 1) {
+                                 cudaLaunchAttribute *attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(threads);
@@ -303,13 +264,6 @@ cudaLaunchConfig_t launch_config(dim3 grid, int threads, int smem, cudaStream_t 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cluster > 1) {
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = cluster;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.numAttrs = 2;
-  }
   return cfg;
 }
 
@@ -371,7 +325,8 @@ gdattn_status launch_combine_internal(const LayerPlan &pl, const Geometry &geo, 
   cp.geo = geo;
   cp.heads_per_unit = pl.heads_per_unit;
   cp.n_splits = 0;
-  cudaLaunchAttribute attr[2];
+  cp.split_k = pl.split_k;
+  cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg =
       launch_config(dim3(static_cast<unsigned>(geo.batch * pl.units_per_seq),
                          static_cast<unsigned>(pl.heads_per_unit)),
@@ -426,7 +381,7 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
   geo.nchunks = pl.grid;
   geo.align = pl.align;
 
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   if (pl.kind == PathKind::kCore) {
     const CoreKernel ck = core_pick(D, desc->n_q_heads / Hkv, Hkv, desc->kv_shared != 0);
     CoreParams cp;
@@ -460,8 +415,8 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     tp.ws_lse = ws_lse;
     tp.status = status;
     tp.counters = counters;
-    tp.merge_in_kernel = (pl.merge_in_kernel && pl.cluster == 1) ? 1 : 0;
-    tp.cluster = pl.cluster;
+    tp.merge_in_kernel = pl.merge_in_kernel ? 1 : 0;
+    tp.split_k = pl.split_k;
     tp.geo = geo;
     tp.n_q_heads = desc->n_q_heads;
     tp.qscale = qscale;
@@ -475,8 +430,8 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
       if (!encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, batch, bstride,
                             TcPairConfig::TILE))
         return GDATTN_ERR_CUDA;
-      cudaLaunchConfig_t cfg = launch_config(dim3(pl.grid), TcPairConfig::kThreads,
-                                             TcPairConfig::SMEM, stream, attr, pl.cluster);
+      cudaLaunchConfig_t cfg =
+          launch_config(dim3(pl.grid), TcPairConfig::kThreads, TcPairConfig::SMEM, stream, attr);
       if (cudaLaunchKernelEx(&cfg, tc_pair_decode_kernel, kmap, vmap, qmap, tp) != cudaSuccess)
         return GDATTN_ERR_CUDA;
     }
@@ -615,7 +570,8 @@ gdattn_status gdattn_combine(const float *o_partial, const float *lse_partial, i
   cp.head_dim = head_dim;
   cp.heads_per_unit = 0;
   cp.n_splits = n_splits;
-  cudaLaunchAttribute attr[2];
+  cp.split_k = 0;
+  cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = launch_config(dim3(batch, n_q_heads), combine_threads(head_dim), 0,
                                          static_cast<cudaStream_t>(stream), attr);
   return cudaLaunchKernelEx(&cfg, combine_kernel<false>, cp) == cudaSuccess ? GDATTN_OK

@@ -33,6 +33,9 @@ struct CombineParams {
   int32_t heads_per_unit;
   // Caller layout: o [B, Hq, n_splits, D], lse [B, Hq, n_splits].
   int32_t n_splits;
+  // Internal layout with units cut into split_k parts (> 1): unit u's parts are
+  // in slots u * split_k + u .. + split_k - 1, empty ones with LSE -inf.
+  int32_t split_k;
 };
 
 // Threads per combine CTA: one float4 column of D each, whole warps.
@@ -162,7 +165,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
     b = u / p.geo.units_per_seq;
     const int32_t x = u - b * p.geo.units_per_seq;
     h = x * p.heads_per_unit + hh;
-    if (threadIdx.x < 32) {
+    if (p.split_k > 1) {
+      if (threadIdx.x == 0) {
+        sh_nparts = p.split_k;
+        sh_slot0 = static_cast<int64_t>(u) * p.split_k + u;
+      }
+    } else if (threadIdx.x < 32) {
       int64_t ustart, chunk;
       int32_t n;
       unit_position(p.geo, b, x, ustart, n, chunk);

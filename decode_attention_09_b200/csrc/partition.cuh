@@ -179,9 +179,9 @@ struct SegmentIter {
   }
 };
 
-// Cluster split: unit u (sequence u / units_per_seq, group u % units_per_seq)
-// is shared by the k CTAs of one thread-block cluster; rank r takes whole
-// tiles [r * T / k, (r + 1) * T / k) of the unit's T = ceil(n / tile) tiles.
+// Unit split: unit u (sequence u / units_per_seq, group u % units_per_seq) is
+// cut into k parts; part r takes whole tiles [r * T / k, (r + 1) * T / k) of
+// the unit's T = ceil(n / tile) tiles.
 // The range is expressed as a chunk so the segment and tile iterators apply
 // unchanged (it holds one segment, or none when the unit is too short).  Run
 // by one whole warp.

@@ -60,7 +60,8 @@ struct TcParams {
   uint32_t *status;
   uint32_t *counters;     // per unit: parts finished in this call (zero between calls)
   int32_t merge_in_kernel;  // 1: the CTA finishing a unit's last part merges it
-  int32_t cluster;        // > 1: each unit split over one cluster of this many CTAs
+  int32_t split_k;        // > 1: unit u is cut into split_k whole-tile parts, part r on
+                          // CTA u * split_k + r (units of even length); else flattened chunks
   Geometry geo;           // units_per_seq == n_kv_heads
   int32_t n_q_heads;
   float qscale;           // multiplies raw scores: scale*log2(e), or scale/softcap
@@ -216,7 +217,14 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
   // The split plan reads only seqlens, so it (and the producer's first KV
   // loads below) may run before the preceding kernel has completed; every other
   // global access waits for it (griddepcontrol.wait) in the role that makes it.
-  if (warp == 2) plan_chunk(p.geo, c, plan);
+  const int32_t split_k = p.split_k > 1 ? p.split_k : 1;
+  const bool usplit = split_k > 1;  // unit c / split_k, part c % split_k (see TcParams)
+  if (warp == 2) {
+    if (usplit)
+      plan_unit_split(p.geo, c / split_k, c % split_k, split_k, Cfg::TILE, plan);
+    else
+      plan_chunk(p.geo, c, plan);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -581,7 +589,7 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
         if ((lane & 1) == 0) redsum[qd * G + (lane >> 1)] = ls;
         named_bar_sync(1, 128);
         const Segment &sg = it.seg;
-        const bool single = sg.whole();
+        const bool single = sg.whole() && !usplit;  // a split unit always has parts
         const int64_t slot = static_cast<int64_t>(c) + sg.unit;
         const int h0 = sg.x * G;
         float inv[G];
@@ -625,6 +633,11 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
         }
       }
       ++i;
+    }
+    if (usplit && i == 0 && qd == 0 && lane < G) {
+      // An empty part (the unit is shorter than split_k tiles): LSE -inf.
+      const int64_t slot = static_cast<int64_t>(c) + c / split_k;
+      p.ws_lse[slot * G + lane] = -INFINITY;
     }
   }
 

@@ -38,13 +38,10 @@
 // merging run in a warp of their own, so the softmax warps hand a part over at
 // a barrier and go straight on with the next segment.
 //
-// Cluster mode (p.cluster = k > 1, for units of even length): unit u is split
-// over the k CTAs of one thread-block cluster instead of the flattened chunks.
-// Each CTA leaves its part (normalised O, LSE) in its own shared memory; after
-// a cluster barrier every CTA merges a 1/k slice of the unit's outputs, reading
-// the k parts over distributed shared memory, and a second barrier keeps each
-// CTA's shared memory alive until its peers have read it.  No workspace
-// traffic, no counters, no segment straddles a CTA boundary.
+// Unit split (p.split_k = k > 1, for units of even length): instead of the
+// flattened chunks, unit u is cut into k whole-tile parts, part r on CTA
+// u * k + r, so no CTA straddles two units.  Every part goes through the merge
+// (an empty part has LSE -inf).
 //
 // Warp roles (256 threads): warp 0 TMA, warp 1 QK MMA and TMEM owner, warp 6
 // P.V MMA, warps 2-5 softmax (TMEM sub-partition warp % 4), warp 7 part count
@@ -78,8 +75,7 @@ struct TcPairConfig {
   static constexpr int OFF_P = OFF_Q + 2 * QB;
   static constexpr int OFF_BAR = OFF_P + 2 * PB;
   static constexpr int OFF_RED = OFF_BAR + 256;
-  static constexpr int OFF_PLSE = OFF_RED + 2 * 4 * G * 4;  // cluster mode: this CTA's part LSE
-  static constexpr int SMEM = OFF_PLSE + G * 4 + 1024;
+  static constexpr int SMEM = OFF_RED + 2 * 4 * G * 4 + 1024;
   static constexpr int kThreads = 256;
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t S_COL = 0;                // 2 buffers x 4 partial sums x 16 columns
@@ -123,9 +119,6 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
   ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 23);  // 48 bytes, ends before +29
   float *redmax = reinterpret_cast<float *>(smem + Cfg::OFF_RED);  // [4 warps][G]
   float *redsum = redmax + 4 * G;                                  // [4 warps][G]
-  // Cluster mode: this CTA's part, O in the (by then idle) first KV stage.
-  float *part_lse = reinterpret_cast<float *>(smem + Cfg::OFF_PLSE);  // [G]
-  float *part_o = reinterpret_cast<float *>(stages);                   // [G][D]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -148,7 +141,6 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
     *abort_flag = 0;
-    for (int h = 0; h < G; ++h) part_lse[h] = -INFINITY;  // an empty rank's part
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -164,10 +156,12 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
   // The split plan reads only seqlens, so it (and the producer's first KV
   // loads below) may run before the preceding kernel has completed; every other
   // global access waits for it (griddepcontrol.wait) in the role that makes it.
-  const int32_t crank = p.cluster > 1 ? static_cast<int32_t>(cluster_ctarank()) : 0;
+  const int32_t split_k = p.split_k > 1 ? p.split_k : 1;
+  const bool usplit = split_k > 1;
+  const int32_t crank = c % split_k;
   if (warp == 2) {
-    if (p.cluster > 1)
-      plan_unit_split(p.geo, c / p.cluster, crank, p.cluster, Cfg::TILE, plan);
+    if (usplit)
+      plan_unit_split(p.geo, c / split_k, crank, split_k, Cfg::TILE, plan);
     else
       plan_chunk(p.geo, c, plan);
   }
@@ -378,22 +372,16 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
     // after a failed wait too, so the counters always return to zero.
     if (p.merge_in_kernel) {
       grid_dependency_wait();  // counters, workspace and outputs
-      SegmentIter sit;
-      sit.init(p.geo, *plan);
-      Segment sg;
-      while (sit.next(sg)) {
-        if (sg.whole()) continue;
-        named_bar_sync(2, 160);
-        int32_t cf, cl;
-        unit_chunks(sg.unit_start, sg.n, plan->chunk, cf, cl);
+      // Count one part of unit `unit` (parts in slots slot0 .. slot0 + np - 1);
+      // the last one merges.
+      auto count_and_merge = [&](int32_t unit, int32_t b, int32_t x, int64_t slot0, int32_t np) {
         uint32_t done = 0;
-        if (lane == 0) done = atomic_add_acq_rel_gpu(p.counters + sg.unit, 1u);
+        if (lane == 0) done = atomic_add_acq_rel_gpu(p.counters + unit, 1u);
         done = __shfl_sync(0xffffffffu, done, 0);
         __syncwarp();  // lane 0's acquire before every lane's reads
-        if (done != static_cast<uint32_t>(cl - cf)) continue;
-        if (lane == 0) p.counters[sg.unit] = 0u;
+        if (done != static_cast<uint32_t>(np - 1)) return;
+        if (lane == 0) p.counters[unit] = 0u;
         constexpr int NC = G * D / 4 / 32;  // float4 columns per lane
-        const int64_t slot0 = static_cast<int64_t>(cf) + sg.unit;
         const float *o_col[NC];
         const float *l_col[NC];
 #pragma unroll
@@ -404,14 +392,38 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
         }
         float4 res[NC];
         float m[NC], z[NC];
-        merge_columns<NC, 4>(o_col, l_col, G * D, G, cl - cf + 1, true, res, m, z);
+        merge_columns<NC, 4>(o_col, l_col, G * D, G, np, true, res, m, z);
 #pragma unroll
         for (int k = 0; k < NC; ++k) {
           const int e = lane + 32 * k, h = e / (D / 4), d = (e % (D / 4)) * 4;
-          const int64_t orow = static_cast<int64_t>(sg.b) * p.n_q_heads + sg.x * G + h;
+          const int64_t orow = static_cast<int64_t>(b) * p.n_q_heads + x * G + h;
           store_bf16x4(p.out + orow * D + d, res[k]);
           if (d == 0 && p.lse != nullptr)
             p.lse[orow] = (m[k] == -INFINITY) ? -INFINITY : m[k] + logf(z[k]);
+        }
+      };
+      if (usplit) {
+        // One part per CTA, part r of unit c / k in slot c + unit.
+        const int32_t unit = c / split_k;
+        const int32_t b = unit / p.geo.units_per_seq, x = unit - b * p.geo.units_per_seq;
+        const int64_t slot = static_cast<int64_t>(c) + unit;
+        if (plan->cs < plan->ce) {
+          named_bar_sync(2, 160);  // the softmax warps stored the part
+        } else {
+          if (lane < G) p.ws_lse[slot * G + lane] = -INFINITY;  // an empty part
+          __syncwarp();
+        }
+        count_and_merge(unit, b, x, slot - crank, split_k);
+      } else {
+        SegmentIter sit;
+        sit.init(p.geo, *plan);
+        Segment sg;
+        while (sit.next(sg)) {
+          if (sg.whole()) continue;
+          named_bar_sync(2, 160);
+          int32_t cf, cl;
+          unit_chunks(sg.unit_start, sg.n, plan->chunk, cf, cl);
+          count_and_merge(sg.unit, sg.b, sg.x, static_cast<int64_t>(cf) + sg.unit, cl - cf + 1);
         }
       }
     }
@@ -553,8 +565,7 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
         if ((lane & 15) == 0) redsum[qd * G + hd] = ls;
         named_bar_sync(1, 128);
         const Segment &sg = it.seg;
-        const bool part_local = p.cluster > 1;  // the part stays in shared memory
-        const bool single = sg.whole() && !part_local;
+        const bool single = sg.whole() && !usplit;  // a split unit always has parts
         const int64_t slot = static_cast<int64_t>(c) + sg.unit;
         const int h0 = sg.x * G;
         float L[G], inv[G];
@@ -573,9 +584,7 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
 #pragma unroll
             for (int h = 0; h < G; ++h) {
               const float val = (o[h] + o[G + h]) * inv[h];
-              if (part_local)
-                part_o[h * D + d] = val;
-              else if (single)
+              if (single)
                 p.out[(static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + h) * D + d] =
                     f32_to_bf16_rn(val);
               else
@@ -589,9 +598,7 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
             const float mr = lane ? m_ref[1] : m_ref[0];
             const float Lh = lane ? L[1] : L[0];
             const float lse_v = (mr + log2f(Lh)) * 0.69314718055994530942f;
-            if (part_local) {
-              part_lse[lane] = lse_v;
-            } else if (single) {
+            if (single) {
               if (p.lse != nullptr)
                 p.lse[static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + lane] = lse_v;
             } else {
@@ -600,7 +607,7 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
           }
         }
         // Hand a partial over to the merge warp (it counts it after the barrier).
-        if (!single && !part_local && p.merge_in_kernel) named_bar_sync(2, 160);
+        if (!single && p.merge_in_kernel) named_bar_sync(2, 160);
       }
       ++i;
     }
@@ -608,52 +615,6 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (p.cluster > 1) {
-    // --- cluster merge: CTA `crank` finalises float4 columns
-    // [crank * per, (crank + 1) * per) of the unit's G x D outputs.
-    cluster_sync();  // every CTA's part is in its shared memory
-    grid_dependency_wait();
-    const int32_t k = p.cluster;
-    const int per = G * D / 4 / k;
-    const int32_t u = c / k;
-    const int32_t b = u / p.geo.units_per_seq, x = u - b * p.geo.units_per_seq;
-    for (int t = threadIdx.x; t < per; t += Cfg::kThreads) {
-      const int e = crank * per + t, h = e / (D / 4), d = (e % (D / 4)) * 4;
-      float lv[16];
-      float4 ov[16];
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        if (q < k) {
-          lv[q] = ld_cluster_f32(map_cluster(part_lse + h, q));
-          ov[q] = ld_cluster_f32x4(map_cluster(part_o + h * D + d, q));
-        }
-      }
-      float m = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < 16; ++q)
-        if (q < k) m = fmaxf(m, lv[q]);
-      float z = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        // an empty part has weight 0 and may hold anything: select, don't multiply
-        if (q < k && lv[q] != -INFINITY) {
-          const float w = __expf(lv[q] - m);
-          z += w;
-          acc.x = fmaf(w, ov[q].x, acc.x);
-          acc.y = fmaf(w, ov[q].y, acc.y);
-          acc.z = fmaf(w, ov[q].z, acc.z);
-          acc.w = fmaf(w, ov[q].w, acc.w);
-        }
-      }
-      const float inv_z = (m == -INFINITY) ? 0.f : __fdividef(1.f, z);
-      const int64_t orow = static_cast<int64_t>(b) * p.n_q_heads + x * G + h;
-      store_bf16x4(p.out + orow * D + d,
-                   make_float4(acc.x * inv_z, acc.y * inv_z, acc.z * inv_z, acc.w * inv_z));
-      if (d == 0 && p.lse != nullptr) p.lse[orow] = (m == -INFINITY) ? -INFINITY : m + logf(z);
-    }
-    cluster_sync();  // the peers are done reading this CTA's shared memory
-  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TMEM_COLS);

@@ -96,11 +96,12 @@ typedef struct gdattn_layer_desc {
 /*
  * The caller expects every sequence of a call to attend about the same number
  * of positions (uniform context lengths, or all of them past the window).  The
- * tcgen05 kernels may then split each (sequence, KV head) unit evenly over the
- * CTAs of one thread-block cluster and merge the parts in distributed shared
- * memory; with uneven lengths that split stays correct but loses balance.
- * Without the flag (or with split_ctas > 0) the KV ranges of all units are laid
- * end to end and cut into equal chunks.
+ * tcgen05 kernels then cut each (sequence, KV head) unit into the same number k
+ * of whole-tile parts, one CTA each (k chosen so all parts run at once), so no
+ * CTA straddles two units; the parts are merged as split-KV partials.  With
+ * uneven lengths that split stays correct but loses balance.  Without the flag
+ * (or with split_ctas > 0) the KV ranges of all units are laid end to end and
+ * cut into equal chunks.
  */
 #define GDATTN_FLAG_EVEN_UNITS 1
 

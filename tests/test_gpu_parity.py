@@ -273,33 +273,37 @@ def test_part_counters_return_to_zero(split):
     compare(out, lse, o_ref, l_ref, ulp_floor=True, what=f"split {split}")
 
 
-# (B, Hq, Hkv, D, C, seqlens, window, softcap): pair-kernel geometries run with
-# GDATTN_FLAG_EVEN_UNITS, i.e. one thread-block cluster per (sequence, KV head)
-CLUSTER_CASES = {
-    "k4_empty_rank": (2, 16, 8, 256, 200, [450, 130], 200, 0.0),
-    "k8_one_unit": (1, 2, 1, 256, 700, [700], 0, 0.0),
-    "k16_long": (1, 4, 2, 256, 2048, [2048], 0, 0.0),
-    "ragged_mostly_empty": (3, 8, 4, 256, 1000, [1000, 64, 1], 0, 0.0),
-    "softcap_ring": (2, 16, 8, 256, 512, [1300, 700], 512, 30.0),
+# (B, Hq, Hkv, D, C, seqlens, window, softcap, kv_shared) run with
+# GDATTN_FLAG_EVEN_UNITS: every (sequence, KV head) unit cut into k whole-tile parts
+EVEN_CASES = {
+    "pair_k2_empty_rank": (2, 16, 8, 256, 200, [450, 130], 200, 0.0, False),
+    "pair_one_unit": (1, 2, 1, 256, 700, [700], 0, 0.0, False),
+    "pair_long": (1, 4, 2, 256, 2048, [2048], 0, 0.0, False),
+    "pair_ragged_mostly_empty": (3, 8, 4, 256, 1000, [1000, 64, 1], 0, 0.0, False),
+    "pair_softcap_ring": (2, 16, 8, 256, 512, [1300, 700], 512, 30.0, False),
+    "tc16_one_unit": (1, 16, 1, 512, 3000, [3000], 0, 0.0, True),
+    "tc16_ragged": (3, 16, 1, 512, 2000, [2000, 100, 1], 0, 0.0, True),
+    "tc16_hkv2_softcap": (2, 32, 2, 512, 700, [700, 650], 0, 20.0, True),
 }
 
 
-@pytest.mark.parametrize("name", sorted(CLUSTER_CASES))
-def test_cluster_split_matches_oracle(name):
-    """Units split over thread-block clusters and merged in distributed shared
-    memory give the oracle's result, ragged lengths and empty ranks included."""
+@pytest.mark.parametrize("name", sorted(EVEN_CASES))
+def test_even_unit_split_matches_oracle(name):
+    """Units cut into k whole-tile parts (ragged lengths and empty parts
+    included: the flag only promises balance) give the oracle's result."""
     require_gpu()
-    B, Hq, Hkv, D, C, sl, w, cap = CLUSTER_CASES[name]
-    inp = workloads.random_case(300 + sorted(CLUSTER_CASES).index(name), B, Hq, Hkv, D, C, sl,
-                                window=w, softcap=cap)
+    B, Hq, Hkv, D, C, sl, w, cap, shared = EVEN_CASES[name]
+    inp = workloads.random_case(300 + sorted(EVEN_CASES).index(name), B, Hq, Hkv, D, C, sl,
+                                window=w, softcap=cap, kv_shared=shared)
     o_ref, l_ref = oracle_for(inp)
     layer = GpuLayer(inp)
     layer.desc = binding.desc_from_spec(inp.spec, capacity=C, flags=binding.GDATTN_FLAG_EVEN_UNITS)
     layer.ws = binding.alloc_workspace(B, layer.max_seqlen, layer.desc)
     units = B * Hkv
     splits = binding.plan_splits(B, layer.max_seqlen, layer.desc)
-    assert splits % units == 0 and splits // units >= 2, splits  # cluster mode was taken
-    assert binding.launches_per_call(B, layer.max_seqlen, layer.desc) == 1
+    assert splits % units == 0 and splits // units >= 2, splits  # the unit split was taken
+    expect_launches = 2 if shared else 1  # the 16-head kernel merges in the combine kernel
+    assert binding.launches_per_call(B, layer.max_seqlen, layer.desc) == expect_launches
     for _ in range(2):
         out, lse = layer.run()
         compare(out, lse, o_ref, l_ref, ulp_floor=True, what=f"{name} k={splits // units}")
