@@ -37,10 +37,12 @@ struct LayerPlan {
   int32_t align = 1;           // chunk granularity in tokens (one tile / stage)
   bool merge_in_kernel = false;  // the decode kernel merges split units itself
   int32_t split_k = 1;           // > 1: each unit cut into split_k whole-tile parts
+  bool tagged = false;           // parts stored as 64-bit (value, tag) words
   // A separate LSE-combine launch follows the decode kernel.
   bool needs_combine() const { return grid > 1 && !merge_in_kernel; }
-  // Workspace: status word | per-unit part counters | partial LSE | partial O.
-  size_t off_cnt = 0, off_lse = 0, off_o = 0, bytes = 0;
+  // Workspace: status word | per-unit part counters | per-unit epochs |
+  // partial LSE | partial O.
+  size_t off_cnt = 0, off_epoch = 0, off_lse = 0, off_o = 0, bytes = 0;
 };
 
 constexpr size_t kStatusBytes = 256;
@@ -243,10 +245,14 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
   pl.grid = static_cast<int32_t>(grid);
   pl.slots = grid + units;
   pl.merge_in_kernel = pl.kind == PathKind::kTcPair;
+  pl.tagged = pl.merge_in_kernel && pl.split_k > 1;
+  const size_t elem = pl.tagged ? 8 : 4;
   pl.off_cnt = kStatusBytes;
-  pl.off_lse = align256(pl.off_cnt + static_cast<size_t>(units) * 4);
-  pl.off_o = align256(pl.off_lse + static_cast<size_t>(pl.slots) * pl.heads_per_unit * 4);
-  pl.bytes = align256(pl.off_o + static_cast<size_t>(pl.slots) * pl.heads_per_unit * d->head_dim * 4);
+  pl.off_epoch = align256(pl.off_cnt + static_cast<size_t>(units) * 4);
+  pl.off_lse = align256(pl.off_epoch + static_cast<size_t>(units) * 4);
+  pl.off_o = align256(pl.off_lse + static_cast<size_t>(pl.slots) * pl.heads_per_unit * elem);
+  pl.bytes =
+      align256(pl.off_o + static_cast<size_t>(pl.slots) * pl.heads_per_unit * d->head_dim * elem);
   return GDATTN_OK;
 }
 
@@ -361,6 +367,7 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
                              cudaStream_t stream) {
   uint32_t *status = reinterpret_cast<uint32_t *>(ws);
   uint32_t *counters = reinterpret_cast<uint32_t *>(ws + pl.off_cnt);
+  uint32_t *epochs = reinterpret_cast<uint32_t *>(ws + pl.off_epoch);
   float *ws_lse = reinterpret_cast<float *>(ws + pl.off_lse);
   float *ws_o = reinterpret_cast<float *>(ws + pl.off_o);
   const int32_t D = desc->head_dim;
@@ -415,6 +422,7 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     tp.ws_lse = ws_lse;
     tp.status = status;
     tp.counters = counters;
+    tp.epochs = epochs;
     tp.merge_in_kernel = pl.merge_in_kernel ? 1 : 0;
     tp.split_k = pl.split_k;
     tp.geo = geo;

@@ -131,6 +131,39 @@ __device__ __forceinline__ void tma_load_4d(void *dst_smem, const CUtensorMap *m
       : "memory");
 }
 
+// --------------------------------------------- flagged (value, tag) words
+// A 64-bit word carrying a 32-bit payload in its low half and a tag in its
+// high half.  An aligned 64-bit access is single-copy atomic, so a reader that
+// sees the expected tag also sees the payload stored with it: data and "ready"
+// arrive in one load, with no separate flag or fence (the low-latency protocol
+// of NCCL's LL transport).
+__device__ __forceinline__ void st_tagged(uint64_t *addr, float v, uint32_t tag) {
+  const uint64_t w = (static_cast<uint64_t>(tag) << 32) | __float_as_uint(v);
+  asm volatile("st.volatile.global.u64 [%0], %1;" ::"l"(addr), "l"(w) : "memory");
+}
+
+__device__ __forceinline__ void st_u64_volatile(uint64_t *addr, uint64_t w) {
+  asm volatile("st.volatile.global.u64 [%0], %1;" ::"l"(addr), "l"(w) : "memory");
+}
+
+// Two tagged words (16-byte aligned address).
+__device__ __forceinline__ void ld_tagged2(const uint64_t *addr, uint64_t &a, uint64_t &b) {
+  asm volatile("ld.volatile.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(addr) : "memory");
+}
+
+__device__ __forceinline__ uint64_t ld_u64_volatile(const uint64_t *addr) {
+  uint64_t w;
+  asm volatile("ld.volatile.global.u64 %0, [%1];" : "=l"(w) : "l"(addr) : "memory");
+  return w;
+}
+
+__device__ __forceinline__ uint32_t tag_of(uint64_t w) { return static_cast<uint32_t>(w >> 32); }
+// Tags count calls and never take the value 0 of a cleared word.
+__device__ __forceinline__ uint32_t next_tag(uint32_t epoch) { return epoch + 1 == 0 ? 1 : epoch + 1; }
+__device__ __forceinline__ float payload_of(uint64_t w) {
+  return __uint_as_float(static_cast<uint32_t>(w));
+}
+
 // Atomic add at GPU scope with acquire-release semantics; returns the old value.
 // After a CTA barrier, one thread's release publishes the whole CTA's prior
 // stores; its acquire makes other CTAs' released stores visible to the CTA

@@ -59,6 +59,7 @@ struct TcParams {
   float *ws_lse;          // partial lse [slots][G]
   uint32_t *status;
   uint32_t *counters;     // per unit: parts finished in this call (zero between calls)
+  uint32_t *epochs;       // per unit: tag of the last call's tagged parts (see tc_pair_decode)
   int32_t merge_in_kernel;  // 1: the CTA finishing a unit's last part merges it
   int32_t split_k;        // > 1: unit u is cut into split_k whole-tile parts, part r on
                           // CTA u * split_k + r (units of even length); else flattened chunks

@@ -40,8 +40,15 @@
 //
 // Unit split (p.split_k = k > 1, for units of even length): instead of the
 // flattened chunks, unit u is cut into k whole-tile parts, part r on CTA
-// u * k + r, so no CTA straddles two units.  Every part goes through the merge
-// (an empty part has LSE -inf).
+// u * k + r, so no CTA straddles two units.  The CTA of the last part merges,
+// without counting: the other parts are stored as tagged words (each 64-bit
+// word carries a float and the call's tag for the unit, so a load sees data
+// and readiness at once), and its merge warp polls them while its own last
+// tiles are still running, merging them in part order (the result does not
+// depend on timing).  Its own part arrives through shared memory, so after
+// its last tile no global round trip is left.  Consumed words are cleared;
+// the tag is the unit's epoch + 1, read after the dependency wait and advanced
+// by the merger once it has seen every part.  An empty part has LSE -inf.
 //
 // Warp roles (256 threads): warp 0 TMA, warp 1 QK MMA and TMEM owner, warp 6
 // P.V MMA, warps 2-5 softmax (TMEM sub-partition warp % 4), warp 7 part count
@@ -75,7 +82,9 @@ struct TcPairConfig {
   static constexpr int OFF_P = OFF_Q + 2 * QB;
   static constexpr int OFF_BAR = OFF_P + 2 * PB;
   static constexpr int OFF_RED = OFF_BAR + 256;
-  static constexpr int SMEM = OFF_RED + 2 * 4 * G * 4 + 1024;
+  static constexpr int OFF_PART = OFF_RED + 2 * 4 * G * 4;  // the merger's own part
+  static constexpr int PARTB = G * D * 4 + 64;               // O [G][D], then LSE [G]
+  static constexpr int SMEM = OFF_PART + PARTB + 1024;
   static constexpr int kThreads = 256;
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t S_COL = 0;                // 2 buffers x 4 partial sums x 16 columns
@@ -117,6 +126,9 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
   uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 21);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 22);
   ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 23);  // 48 bytes, ends before +29
+  uint32_t *sh_tag = reinterpret_cast<uint32_t *>(bars + 29);    // this call's tag for the unit
+  float *part_o = reinterpret_cast<float *>(smem + Cfg::OFF_PART);  // merger's own part [G][D]
+  float *part_lse = part_o + G * D;                                  // [G]
   float *redmax = reinterpret_cast<float *>(smem + Cfg::OFF_RED);  // [4 warps][G]
   float *redsum = redmax + 4 * G;                                  // [4 warps][G]
 
@@ -159,6 +171,11 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
   const int32_t split_k = p.split_k > 1 ? p.split_k : 1;
   const bool usplit = split_k > 1;
   const int32_t crank = c % split_k;
+  // Unit split with the merge in this kernel: tagged parts, merged by the last part.
+  const bool tagged = usplit && p.merge_in_kernel;
+  const bool merger = tagged && crank == split_k - 1;
+  uint64_t *tg_o = reinterpret_cast<uint64_t *>(p.ws_o);      // [slots][G][D] tagged words
+  uint64_t *tg_lse = reinterpret_cast<uint64_t *>(p.ws_lse);  // [slots][G] tagged words
   if (warp == 2) {
     if (usplit)
       plan_unit_split(p.geo, c / split_k, crank, split_k, Cfg::TILE, plan);
@@ -403,17 +420,87 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
         }
       };
       if (usplit) {
-        // One part per CTA, part r of unit c / k in slot c + unit.
+        // Part r of unit c / k sits in slot (c / k) * k + unit + r.
         const int32_t unit = c / split_k;
         const int32_t b = unit / p.geo.units_per_seq, x = unit - b * p.geo.units_per_seq;
-        const int64_t slot = static_cast<int64_t>(c) + unit;
-        if (plan->cs < plan->ce) {
-          named_bar_sync(2, 160);  // the softmax warps stored the part
+        const int64_t slot0 = static_cast<int64_t>(unit) * split_k + unit;
+        const bool has_part = plan->cs < plan->ce;
+        uint32_t tag = 0;
+        if (lane == 0) tag = next_tag(__ldcg(p.epochs + unit));
+        tag = __shfl_sync(0xffffffffu, tag, 0);
+        if (!merger) {
+          if (!has_part) {  // an empty part: LSE -inf
+            uint64_t *dst = tg_o + (slot0 + crank) * G * D;
+            for (int e = lane; e < G * D; e += 32) st_tagged(dst + e, 0.f, tag);
+            if (lane < G) st_tagged(tg_lse + (slot0 + crank) * G + lane, -INFINITY, tag);
+          }
         } else {
-          if (lane < G) p.ws_lse[slot * G + lane] = -INFINITY;  // an empty part
-          __syncwarp();
+          // Lane l merges elements [16 l, 16 l + 16) of the unit's G x D outputs.
+          constexpr int PER = G * D / 32;
+          static_assert(PER == 16 && D % PER == 0, "lane mapping");
+          const int h = (PER * lane) / D, d0 = (PER * lane) % D;
+          float m = -INFINITY, z = 0.f, acc[PER];
+#pragma unroll
+          for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+          auto fold = [&](float lse_r, const float (&o)[PER]) {
+            if (lse_r == -INFINITY) return;  // an empty part: weight 0
+            const float mn = fmaxf(m, lse_r);
+            const float r_old = (m == -INFINITY) ? 0.f : __expf(m - mn);
+            const float w = __expf(lse_r - mn);
+            z = z * r_old + w;
+#pragma unroll
+            for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, o[e], acc[e] * r_old);
+            m = mn;
+          };
+          for (int32_t r = 0; r + 1 < split_k; ++r) {
+            uint64_t *src = tg_o + ((slot0 + r) * G + h) * D + d0;
+            uint64_t *lsrc = tg_lse + (slot0 + r) * G + h;
+            uint64_t wv[PER], wl = 0;
+            const long long t0 = clock64();
+            while (true) {
+#pragma unroll
+              for (int e = 0; e < PER; e += 2) ld_tagged2(src + e, wv[e], wv[e + 1]);
+              wl = ld_u64_volatile(lsrc);
+              bool ready = tag_of(wl) == tag;
+#pragma unroll
+              for (int e = 0; e < PER; ++e) ready &= tag_of(wv[e]) == tag;
+              if (__all_sync(0xffffffffu, ready)) break;
+              if (clock64() - t0 > kWaitLimitCycles) {
+                if (lane == 0) atomicOr(p.status, kStatusTimeout);
+                break;
+              }
+            }
+            float o[PER];
+#pragma unroll
+            for (int e = 0; e < PER; ++e) o[e] = payload_of(wv[e]);
+            fold(payload_of(wl), o);
+            // Clear what was consumed, so no later call can mistake it for fresh.
+#pragma unroll
+            for (int e = 0; e < PER; ++e) st_u64_volatile(src + e, 0ull);
+            if ((lane & (D / PER - 1)) == 0) st_u64_volatile(lsrc, 0ull);
+          }
+          if (has_part) {
+            named_bar_sync(2, 160);  // the softmax warps left the own part in shared memory
+            float o[PER];
+#pragma unroll
+            for (int e = 0; e < PER; ++e) o[e] = part_o[h * D + d0 + e];
+            fold(part_lse[h], o);
+          }
+          const float inv_z = (m == -INFINITY) ? 0.f : __fdividef(1.f, z);
+          const int64_t orow = static_cast<int64_t>(b) * p.n_q_heads + x * G + h;
+          uint16_t *dst = p.out + orow * D + d0;
+#pragma unroll
+          for (int e = 0; e < PER; e += 8) {
+            uint4 pk;
+            pk.x = pack_bf16x2(acc[e] * inv_z, acc[e + 1] * inv_z);
+            pk.y = pack_bf16x2(acc[e + 2] * inv_z, acc[e + 3] * inv_z);
+            pk.z = pack_bf16x2(acc[e + 4] * inv_z, acc[e + 5] * inv_z);
+            pk.w = pack_bf16x2(acc[e + 6] * inv_z, acc[e + 7] * inv_z);
+            *reinterpret_cast<uint4 *>(dst + e) = pk;
+          }
+          if (d0 == 0 && p.lse != nullptr) p.lse[orow] = (m == -INFINITY) ? -INFINITY : m + logf(z);
+          if (lane == 0) p.epochs[unit] = tag;  // every part of this call has been read
         }
-        count_and_merge(unit, b, x, slot - crank, split_k);
       } else {
         SegmentIter sit;
         sit.init(p.geo, *plan);
@@ -430,6 +517,9 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
   } else {
     // ---------------------------------------------------------- softmax
     grid_dependency_wait();  // outputs and workspace are written below
+    // This call's tag for the unit (the load completes while the tiles run).
+    uint32_t my_tag = 0;
+    if (tagged && threadIdx.x == 64) my_tag = next_tag(__ldcg(p.epochs + c / split_k));
     // M=64 puts tile token r in TMEM lane (r % 16) + 32 * (r / 16): lanes 0-15 of
     // each warp receive one token's scores.  Lanes 0-15 take head 0 of their
     // token, lanes 16-31 head 1 of the token of lane - 16.
@@ -563,7 +653,9 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
 #pragma unroll
         for (int off = 1; off < 16; off <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
         if ((lane & 15) == 0) redsum[qd * G + hd] = ls;
+        if (threadIdx.x == 64) *sh_tag = my_tag;
         named_bar_sync(1, 128);
+        const uint32_t tag = *sh_tag;
         const Segment &sg = it.seg;
         const bool single = sg.whole() && !usplit;  // a split unit always has parts
         const int64_t slot = static_cast<int64_t>(c) + sg.unit;
@@ -574,12 +666,14 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
           L[h] = (redsum[h] + redsum[G + h]) + (redsum[2 * G + h] + redsum[3 * G + h]);
           inv[h] = __fdividef(1.f, L[h]);
         }
-        if (ok) {
-          tc_fence_after();
+        // A tagged part is stored even after a failed wait, so its merger never
+        // waits for it in vain (the status word reports the failure).
+        if (ok || (tagged && !merger)) {
+          if (ok) tc_fence_after();
 #pragma unroll
           for (int jb = 0; jb < 2; ++jb) {
-            float o[4];
-            tmem_ld4(tmem + lane_base + Cfg::O_COL + jb * 16, o);
+            float o[4] = {0.f, 0.f, 0.f, 0.f};
+            if (ok) tmem_ld4(tmem + lane_base + Cfg::O_COL + jb * 16, o);
             const int d = 128 * jb + 32 * qd + lane;
 #pragma unroll
             for (int h = 0; h < G; ++h) {
@@ -587,13 +681,19 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
               if (single)
                 p.out[(static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + h) * D + d] =
                     f32_to_bf16_rn(val);
+              else if (merger)
+                part_o[h * D + d] = val;
+              else if (tagged)
+                st_tagged(tg_o + (slot * G + h) * D + d, val, tag);
               else
                 p.ws_o[(slot * G + h) * D + d] = val;
             }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(oempty);
+          if (ok) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(oempty);
+          }
           if (qd == 0 && lane < G) {  // LSE of head `lane`
             const float mr = lane ? m_ref[1] : m_ref[0];
             const float Lh = lane ? L[1] : L[0];
@@ -601,13 +701,17 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
             if (single) {
               if (p.lse != nullptr)
                 p.lse[static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + lane] = lse_v;
+            } else if (merger) {
+              part_lse[lane] = lse_v;
+            } else if (tagged) {
+              st_tagged(tg_lse + slot * G + lane, lse_v, tag);
             } else {
               p.ws_lse[slot * G + lane] = lse_v;
             }
           }
         }
-        // Hand a partial over to the merge warp (it counts it after the barrier).
-        if (!single && p.merge_in_kernel) named_bar_sync(2, 160);
+        // Hand a partial over to the merge warp: counted parts, or the merger's own.
+        if (!single && p.merge_in_kernel && (!tagged || merger)) named_bar_sync(2, 160);
       }
       ++i;
     }

@@ -307,3 +307,28 @@ def test_even_unit_split_matches_oracle(name):
     for _ in range(2):
         out, lse = layer.run()
         compare(out, lse, o_ref, l_ref, ulp_floor=True, what=f"{name} k={splits // units}")
+
+
+def test_even_split_workspace_shared_by_two_geometries():
+    """Two even-split layers with different unit counts and part counts take
+    turns on one workspace: per-unit tags and cleared words keep every call's
+    merge on its own parts."""
+    require_gpu()
+    a = workloads.random_case(401, 2, 16, 8, 256, 300, [300, 300], window=300)   # 16 units
+    b = workloads.random_case(402, 1, 4, 2, 256, 1500, [1500], window=0)         # 2 units, more parts
+    refs = [oracle_for(x) for x in (a, b)]
+    layers = [GpuLayer(x) for x in (a, b)]
+    for ly, x in zip(layers, (a, b)):
+        ly.desc = binding.desc_from_spec(x.spec, capacity=x.k.shape[1],
+                                         flags=binding.GDATTN_FLAG_EVEN_UNITS)
+    need = max(binding.workspace_size(ly.B, ly.max_seqlen, ly.desc) for ly in layers)
+    shared = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for ly in layers:
+        ly.ws = shared
+    ks = [binding.plan_splits(ly.B, ly.max_seqlen, ly.desc) // (ly.B * x.spec.n_kv_heads)
+          for ly, x in zip(layers, (a, b))]
+    assert ks[0] != ks[1] and min(ks) >= 2, ks
+    for rep in range(3):
+        for ly, (o_ref, l_ref), name in zip(layers, refs, "ab"):
+            out, lse = ly.run()
+            compare(out, lse, o_ref, l_ref, ulp_floor=True, what=f"{name} round {rep}")
