@@ -284,6 +284,8 @@ EVEN_CASES = {
     "tc16_one_unit": (1, 16, 1, 512, 3000, [3000], 0, 0.0, True),
     "tc16_ragged": (3, 16, 1, 512, 2000, [2000, 100, 1], 0, 0.0, True),
     "tc16_hkv2_softcap": (2, 32, 2, 512, 700, [700, 650], 0, 20.0, True),
+    "tc16_k3_uneven_slices": (40, 16, 1, 512, 192, [192] * 40, 0, 0.0, True),
+    "tc16_many_parts_combine": (1, 16, 1, 512, 4096, [4096], 0, 0.0, True),
 }
 
 
