@@ -429,6 +429,15 @@ def run_ours(args, world, rank, local):
                 "kernel": "sliding layer: tc_pair_decode_kernel (tcgen05; split parts merged in the kernel)",
                 "bytes_per_launch": per_launch_bytes, "us_per_launch": per_launch_ms * 1e3,
                 "traffic": traffic_for("sliding")}
+    if roof is None and ms_gl:  # a workload of global layers only
+        per_launch_ms = ms_gl / len(global_idx)
+        per_launch_bytes = gl_bytes / len(global_idx)
+        ach = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+                "frac": ach / peak, "peak_kind": peak_kind,
+                "kernel": "global layer: tc_decode_kernel (tcgen05) + LSE combine",
+                "bytes_per_launch": per_launch_bytes, "us_per_launch": per_launch_ms * 1e3,
+                "traffic": traffic_for("global")}
     per_type = {}
     if ms_gl:
         ach = gl_bytes / len(global_idx) / (ms_gl / len(global_idx) * 1e-3) / 1e9

@@ -50,10 +50,14 @@
 // the tag is the unit's epoch + 1, read after the dependency wait and advanced
 // by the merger once it has seen every part.  An empty part has LSE -inf.
 //
-// Warp roles (256 threads): warp 0 TMA, warp 1 QK MMA and TMEM owner, warp 6
-// P.V MMA, warps 2-5 softmax (TMEM sub-partition warp % 4), warp 7 part count
-// and merge.  Q is double buffered, so the next segment's Q is loaded while the
-// current one is still in use.  Every wait is bounded.
+// Warp roles (288 threads): warp 0 loads K (and Q), warp 8 loads V, warp 1
+// issues QK and owns TMEM, warp 6 issues P.V, warps 2-5 run the softmax (TMEM
+// sub-partition warp % 4), warp 7 counts and merges parts.  K and V have rings
+// of their own over the same stages: a K tile is released as soon as its QK
+// is done, a V tile after its P.V, so K loads run ahead and the ring turns
+// over faster than with one release per stage.  Q is double buffered, so the
+// next segment's Q is loaded while the current one is still in use.  Every
+// wait is bounded.
 #pragma once
 
 #include <cstdint>
@@ -81,11 +85,11 @@ struct TcPairConfig {
   static constexpr int OFF_Q = NST * STAGEB;          // 2 Q buffers
   static constexpr int OFF_P = OFF_Q + 2 * QB;
   static constexpr int OFF_BAR = OFF_P + 2 * PB;
-  static constexpr int OFF_RED = OFF_BAR + 256;
+  static constexpr int OFF_RED = OFF_BAR + 512;
   static constexpr int OFF_PART = OFF_RED + 2 * 4 * G * 4;  // the merger's own part
   static constexpr int PARTB = G * D * 4 + 64;               // O [G][D], then LSE [G]
   static constexpr int SMEM = OFF_PART + PARTB + 1024;
-  static constexpr int kThreads = 256;
+  static constexpr int kThreads = 288;
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t S_COL = 0;                // 2 buffers x 4 partial sums x 16 columns
   static constexpr uint32_t O_COL = 128;              // 2 d-blocks x 16 columns
@@ -113,8 +117,8 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
   uint8_t *qs = smem + Cfg::OFF_Q;
   uint8_t *ps = smem + Cfg::OFF_P;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
-  uint64_t *full = bars;            // [NST]  TMA -> MMA
-  uint64_t *empty = bars + 3;       // [NST]  P.V -> TMA
+  uint64_t *kfull = bars;           // [NST]  K TMA -> QK
+  uint64_t *kempty = bars + 3;      // [NST]  QK -> K TMA
   uint64_t *qfull = bars + 6;       // [2] TMA -> MMA (Q of segment k in buffer k & 1)
   uint64_t *qempty = bars + 8;      // [2] MMA -> TMA
   uint64_t *sfull = bars + 10;      // [2] MMA -> softmax (S of tile i in buffer i & 1)
@@ -123,10 +127,12 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
   uint64_t *ofull = bars + 16;      // [2] MMA -> softmax: P.V of tile i done (barrier i & 1)
   uint64_t *oempty = bars + 18;     // softmax -> MMA: O of a finished segment read out
   uint64_t *drain = bars + 19;      // [2] QK warp, P.V warp: all their MMAs done
-  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 21);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 22);
-  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 23);  // 48 bytes, ends before +29
-  uint32_t *sh_tag = reinterpret_cast<uint32_t *>(bars + 29);    // this call's tag for the unit
+  uint64_t *vfull = bars + 21;      // [NST]  V TMA -> P.V (and the softmax, for partial tiles)
+  uint64_t *vempty = bars + 24;     // [NST]  P.V -> V TMA
+  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 27);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 28);
+  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 29);  // 48 bytes, ends before +35
+  uint32_t *sh_tag = reinterpret_cast<uint32_t *>(bars + 35);    // this call's tag for the unit
   float *part_o = reinterpret_cast<float *>(smem + Cfg::OFF_PART);  // merger's own part [G][D]
   float *part_lse = part_o + G * D;                                  // [G]
   float *redmax = reinterpret_cast<float *>(smem + Cfg::OFF_RED);  // [4 warps][G]
@@ -138,8 +144,10 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&kfull[s], 1);
+      mbar_init(&kempty[s], 1);
+      mbar_init(&vfull[s], 1);
+      mbar_init(&vempty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&qfull[s], 1);
@@ -262,21 +270,18 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
       }
       const int st = i % NST;
       if (i >= NST) {
-        // The tile in this stage is released after its P.V, which needs its Q.
+        // The K tile in this stage is released after its QK, which needs its Q.
         while (ok && q_issued <= stage_seg[st]) issue_q(true);
-        if (ok && !mbar_wait(&empty[st], ((i / NST) - 1) & 1, abort_flag, p.status)) ok = false;
+        if (ok && !mbar_wait(&kempty[st], ((i / NST) - 1) & 1, abort_flag, p.status)) ok = false;
       }
       if (!__all_sync(0xffffffffu, ok)) break;
       stage_seg[st] = seg_count - 1;
       if (elect_one()) {
         uint8_t *kdst = stages + st * Cfg::STAGEB;
-        mbar_arrive_expect_tx(&full[st], Cfg::STAGEB);
+        mbar_arrive_expect_tx(&kfull[st], Cfg::KB);
 #pragma unroll
-        for (int j = 0; j < D / 64; ++j) {
-          tma_load_4d(kdst + j * Cfg::BOXB, &kmap, 64 * j, it.seg.x, row, it.seg.b, &full[st], pol);
-          tma_load_4d(kdst + Cfg::KB + j * Cfg::BOXB, &vmap, 64 * j, it.seg.x, row, it.seg.b,
-                      &full[st], pol);
-        }
+        for (int j = 0; j < D / 64; ++j)
+          tma_load_4d(kdst + j * Cfg::BOXB, &kmap, 64 * j, it.seg.x, row, it.seg.b, &kfull[st], pol);
       }
       __syncwarp();
       ++i;
@@ -286,7 +291,7 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
     // Drain: never leave with copies in flight into shared memory.
     volatile int no_abort = 0;
     for (uint32_t f = i > NST ? i - NST : 0; f < i; ++f)
-      mbar_wait(&full[f % NST], (f / NST) & 1, &no_abort, p.status);
+      mbar_wait(&kfull[f % NST], (f / NST) & 1, &no_abort, p.status);
     for (uint32_t k = q_issued > 2 ? q_issued - 2 : 0; k < q_issued; ++k)
       mbar_wait(&qfull[k & 1], (k >> 1) & 1, &no_abort, p.status);
   } else if (warp == 1) {
@@ -309,7 +314,7 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
       }
       const uint32_t qb = (nseg - 1) & 1;
       const int st = i % NST, sb = i & 1;
-      if (!mbar_wait(&full[st], (i / NST) & 1, abort_flag, p.status)) ok = false;
+      if (!mbar_wait(&kfull[st], (i / NST) & 1, abort_flag, p.status)) ok = false;
       if (ok && i >= 2 && !mbar_wait(&sempty[sb], ((i >> 1) - 1) & 1, abort_flag, p.status))
         ok = false;
       if (!__all_sync(0xffffffffu, ok)) break;
@@ -326,6 +331,7 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
           }
         }
         tc_commit(&sfull[sb]);
+        tc_commit(&kempty[st]);
         if (last) tc_commit(&qempty[qb]);
       }
       __syncwarp();
@@ -350,6 +356,7 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
     bool first, last;
     while (ok && it.next(C, row, ntok, first, last)) {
       bool w = mbar_wait(&pfull[t & 1], (t >> 1) & 1, abort_flag, p.status);
+      if (w) w = mbar_wait(&vfull[t % NST], (t / NST) & 1, abort_flag, p.status);
       // A segment's first P.V overwrites O: the previous segment must be read out.
       if (w && first && nseg > 0) w = mbar_wait(oempty, (nseg - 1) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, w)) {
@@ -371,7 +378,7 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
           }
         }
         tc_commit(&ofull[t & 1]);
-        tc_commit(&empty[t % NST]);
+        tc_commit(&vempty[t % NST]);
       }
       __syncwarp();
       ++t;
@@ -514,6 +521,41 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
         }
       }
     }
+  } else if (warp == 8) {
+    // ---------------------------------------------------------- V loads
+    // Same schedule and dependency rule as the K loads (warp 0); a V tile is
+    // released by its P.V.
+    const uint64_t pol = l2_evict_first_policy();
+    bool ok = true;
+    uint32_t i = 0;
+    TileIter it;
+    it.init(p.geo, *plan);
+    int32_t row, ntok;
+    bool first, last;
+    bool waited = false;
+    while (ok && it.next(C, row, ntok, first, last)) {
+      if (!waited && (i >= NST || it.newest)) {
+        grid_dependency_wait();
+        waited = true;
+      }
+      const int st = i % NST;
+      if (i >= NST && !mbar_wait(&vempty[st], ((i / NST) - 1) & 1, abort_flag, p.status))
+        ok = false;
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (elect_one()) {
+        uint8_t *vdst = stages + st * Cfg::STAGEB + Cfg::KB;
+        mbar_arrive_expect_tx(&vfull[st], Cfg::KB);
+#pragma unroll
+        for (int j = 0; j < D / 64; ++j)
+          tma_load_4d(vdst + j * Cfg::BOXB, &vmap, 64 * j, it.seg.x, row, it.seg.b, &vfull[st], pol);
+      }
+      __syncwarp();
+      ++i;
+    }
+    // Drain: never leave with copies in flight into shared memory.
+    volatile int no_abort = 0;
+    for (uint32_t f = i > NST ? i - NST : 0; f < i; ++f)
+      mbar_wait(&vfull[f % NST], (f / NST) & 1, &no_abort, p.status);
   } else {
     // ---------------------------------------------------------- softmax
     grid_dependency_wait();  // outputs and workspace are written below
@@ -628,6 +670,11 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
         uint8_t *pbuf = ps + pb * Cfg::PB;
         *reinterpret_cast<uint16_t *>(pbuf + sw128_offset(hd, tok)) = hi;
         *reinterpret_cast<uint16_t *>(pbuf + sw128_offset(G + hd, tok)) = lo;
+      }
+      if (ok && ntok < Cfg::TILE) {
+        // The V tile may still be in flight (it is loaded after K): wait for it.
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&vfull[i % NST], (i / NST) & 1, abort_flag, p.status));
       }
       if (ok && ntok < Cfg::TILE) {
         // V rows past the attended range hold other cache contents (possibly
