@@ -76,6 +76,10 @@ def lib() -> ctypes.CDLL:
         L.gdattn_workspace_init.restype = ctypes.c_int
         L.gdattn_decode.argtypes = [vp, vp, vp, vp, i32, i32, descp, vp, vp, vp, sz, vp]
         L.gdattn_decode.restype = ctypes.c_int
+        if hasattr(L, "gdattn_decode_append"):  # libraries built before it was added lack it
+            L.gdattn_decode_append.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, descp, vp, vp,
+                                               vp, sz, vp]
+            L.gdattn_decode_append.restype = ctypes.c_int
         L.gdattn_decode_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, descp, vp, vp, vp]
         L.gdattn_decode_noalloc.restype = ctypes.c_int
         L.gdattn_combine.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp]
@@ -178,6 +182,29 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor], seqlens:
                     _ptr(lse), _ptr(workspace), workspace.numel(), _stream_handle(stream))
     if st != GDATTN_OK:
         raise GdattnError(st, "gdattn_decode")
+    return out, lse
+
+
+def decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: Optional[torch.Tensor],
+                  k: torch.Tensor, v: Optional[torch.Tensor], seqlens: torch.Tensor,
+                  desc: LayerDesc, max_seqlen: int, out: Optional[torch.Tensor] = None,
+                  lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None):
+    """gdattn_decode_append: write k_new / v_new ([B, Hkv, D]) into slot
+    (L - 1) mod C of the caches, then decode.  Returns (out, lse)."""
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, max_seqlen, desc, q.device, stream)
+    st = int(lib().gdattn_decode_append(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k), _ptr(v),
+                                        _ptr(seqlens), B, int(max_seqlen), ctypes.byref(desc),
+                                        _ptr(out), _ptr(lse), _ptr(workspace),
+                                        workspace.numel(), _stream_handle(stream)))
+    if st != GDATTN_OK:
+        raise GdattnError(st, "gdattn_decode_append")
     return out, lse
 
 

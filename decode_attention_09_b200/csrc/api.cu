@@ -147,8 +147,17 @@ int query_tc(const void *fn, int threads, int smem) {
   using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const TcParams);
   return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
 }
+int query_tc_append(const void *fn, int threads, int smem) {
+  using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const TcParams, const TcAppend);
+  return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
+}
 int query_tc_pair(const void *fn, int threads, int smem) {
   using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const TcParams);
+  return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
+}
+int query_tc_pair_append(const void *fn, int threads, int smem) {
+  using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const TcParams,
+                        const TcAppend);
   return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
 }
 
@@ -202,6 +211,11 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
   } else if (pl.kind == PathKind::kTc) {
     per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_kernel),
                                   TcConfig::kThreads, TcConfig::SMEM, query_tc);
+    // The append entry point shares the configuration (and needs the same
+    // shared-memory attribute, set by the query).
+    if (cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_append_kernel),
+                             TcConfig::kThreads, TcConfig::SMEM, query_tc_append) != per_sm)
+      return GDATTN_ERR_CUDA;
     min_tokens = 2 * TcConfig::TILE;
     pl.align = TcConfig::TILE;
     pl.units_per_seq = d->n_kv_heads;
@@ -209,6 +223,10 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
   } else {
     per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_decode_kernel),
                                   TcPairConfig::kThreads, TcPairConfig::SMEM, query_tc_pair);
+    if (cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_decode_append_kernel),
+                             TcPairConfig::kThreads, TcPairConfig::SMEM,
+                             query_tc_pair_append) != per_sm)
+      return GDATTN_ERR_CUDA;
     min_tokens = 2 * TcPairConfig::TILE;
     pl.align = TcPairConfig::TILE;
     pl.units_per_seq = d->n_kv_heads;
@@ -361,10 +379,12 @@ gdattn_status check_decode_args(const void *q, const void *k_cache, const void *
 
 // Enqueues the decode kernel (and the combine when the plan splits) with the
 // split-KV scratch at `ws`: status word, then partial LSE, then partial O.
+// k_new / v_new (optional): the current token's rows, appended by the kernel.
 gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_cache,
                              const void *v_cache, const int32_t *seqlens, int32_t batch,
                              const gdattn_layer_desc *desc, void *out, float *lse, uint8_t *ws,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, const void *k_new = nullptr,
+                             const void *v_new = nullptr) {
   uint32_t *status = reinterpret_cast<uint32_t *>(ws);
   uint32_t *counters = reinterpret_cast<uint32_t *>(ws + pl.off_cnt);
   uint32_t *epochs = reinterpret_cast<uint32_t *>(ws + pl.off_epoch);
@@ -401,6 +421,8 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     cp.ws_o = ws_o;
     cp.ws_lse = ws_lse;
     cp.status = status;
+    cp.k_new = static_cast<const uint16_t *>(k_new);
+    cp.v_new = static_cast<const uint16_t *>(v_new);
     cp.geo = geo;
     cp.n_q_heads = desc->n_q_heads;
     cp.qscale = qscale;
@@ -421,6 +443,13 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     tp.ws_o = ws_o;
     tp.ws_lse = ws_lse;
     tp.status = status;
+    TcAppend ap;
+    ap.k_new = static_cast<const uint16_t *>(k_new);
+    ap.v_new = static_cast<const uint16_t *>(v_new);
+    ap.k_cache = static_cast<uint16_t *>(const_cast<void *>(k_cache));
+    ap.v_cache = static_cast<uint16_t *>(const_cast<void *>(v_cache));
+    ap.batch_stride = bstride;
+    ap.n_kv_heads = Hkv;
     tp.counters = counters;
     tp.epochs = epochs;
     tp.merge_in_kernel = pl.merge_in_kernel ? 1 : 0;
@@ -432,16 +461,21 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     if (pl.kind == PathKind::kTc) {
       cudaLaunchConfig_t cfg =
           launch_config(dim3(pl.grid), TcConfig::kThreads, TcConfig::SMEM, stream, attr);
-      if (cudaLaunchKernelEx(&cfg, tc_decode_kernel, kmap, qmap, tp) != cudaSuccess)
-        return GDATTN_ERR_CUDA;
+      const cudaError_t e = k_new != nullptr
+                                ? cudaLaunchKernelEx(&cfg, tc_decode_append_kernel, kmap, qmap, tp, ap)
+                                : cudaLaunchKernelEx(&cfg, tc_decode_kernel, kmap, qmap, tp);
+      if (e != cudaSuccess) return GDATTN_ERR_CUDA;
     } else {
       if (!encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, batch, bstride,
                             TcPairConfig::TILE))
         return GDATTN_ERR_CUDA;
       cudaLaunchConfig_t cfg =
           launch_config(dim3(pl.grid), TcPairConfig::kThreads, TcPairConfig::SMEM, stream, attr);
-      if (cudaLaunchKernelEx(&cfg, tc_pair_decode_kernel, kmap, vmap, qmap, tp) != cudaSuccess)
-        return GDATTN_ERR_CUDA;
+      const cudaError_t e =
+          k_new != nullptr
+              ? cudaLaunchKernelEx(&cfg, tc_pair_decode_append_kernel, kmap, vmap, qmap, tp, ap)
+              : cudaLaunchKernelEx(&cfg, tc_pair_decode_kernel, kmap, vmap, qmap, tp);
+      if (e != cudaSuccess) return GDATTN_ERR_CUDA;
     }
   }
   if (pl.needs_combine())
@@ -537,6 +571,28 @@ gdattn_status gdattn_decode(const void *q, const void *k_cache, const void *v_ca
   if (workspace_bytes < pl.bytes) return GDATTN_ERR_WORKSPACE;
   return enqueue_decode(pl, q, k_cache, v_cache, seqlens, batch, desc, out, lse,
                         static_cast<uint8_t *>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+gdattn_status gdattn_decode_append(const void *q, const void *k_new, const void *v_new,
+                                   void *k_cache, void *v_cache, const int32_t *seqlens,
+                                   int32_t batch, int32_t max_seqlen,
+                                   const gdattn_layer_desc *desc, void *out, float *lse,
+                                   void *workspace, size_t workspace_bytes, void *stream) {
+  gdattn_status st = check_decode_args(q, k_cache, v_cache, seqlens, batch, max_seqlen, desc,
+                                       out, lse);
+  if (st != GDATTN_OK) return st;
+  if (k_new == nullptr || (desc->kv_shared == 1) != (v_new == nullptr))
+    return GDATTN_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || (v_new && !aligned16(v_new))) return GDATTN_ERR_MISALIGNED;
+  if (workspace == nullptr) return GDATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GDATTN_ERR_MISALIGNED;
+  LayerPlan pl;
+  st = make_plan(batch, max_seqlen, desc, pl);
+  if (st != GDATTN_OK) return st;
+  if (workspace_bytes < pl.bytes) return GDATTN_ERR_WORKSPACE;
+  return enqueue_decode(pl, q, k_cache, v_cache, seqlens, batch, desc, out, lse,
+                        static_cast<uint8_t *>(workspace), static_cast<cudaStream_t>(stream),
+                        k_new, v_new);
 }
 
 gdattn_status gdattn_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,

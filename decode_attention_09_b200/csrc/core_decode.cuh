@@ -36,6 +36,11 @@ struct CoreParams {
   float *ws_o;            // partial outputs [slots][Hq][D]
   float *ws_lse;          // partial lse [slots][Hq]
   uint32_t *status;       // device status word
+  // Current-token append (k_new non-null): the token row ([Hkv][D] of k_new /
+  // v_new, [B][Hkv][D]) is copied into slot (L - 1) mod C before the stage
+  // holding it is loaded.
+  const uint16_t *k_new;
+  const uint16_t *v_new;  // null when K serves as V
   Geometry geo;           // units_per_seq == 1
   int32_t n_q_heads;
   float qscale;           // folded into q: scale*log2(e), or scale/softcap
@@ -166,6 +171,13 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads, 1)
           const uint32_t bytes = static_cast<uint32_t>(ntok * ROWB);
           const int64_t off = static_cast<int64_t>(s.b) * p.batch_stride +
                               static_cast<int64_t>(runs.start(r) + t0) * (HKV * D);
+          if (p.k_new != nullptr && newest) {  // append the current token's rows first
+            const int64_t row = static_cast<int64_t>(s.b) * p.batch_stride +
+                                static_cast<int64_t>((s.first_pos + s.n - 1) % C) * (HKV * D);
+            const int64_t src = static_cast<int64_t>(s.b) * (HKV * D);
+            append_row(const_cast<uint16_t *>(p.k) + row, p.k_new + src, HKV * D, lane);
+            if (!SHARED) append_row(const_cast<uint16_t *>(p.v) + row, p.v_new + src, HKV * D, lane);
+          }
           if (elect_one()) {
             mbar_arrive_expect_tx(&full[st], bytes * Cfg::NT);
             bulk_g2s(stage_k + st * T * ROWB, p.k + off, bytes, &full[st], pol);

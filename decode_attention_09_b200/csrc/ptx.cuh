@@ -185,6 +185,18 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Current-token append: copy n bf16 elements (16-byte aligned, n % 8 == 0) from
+// src into the cache row at dst with the whole warp, then order those ordinary
+// stores before this warp's later TMA / bulk-copy reads (the async proxy) of
+// the same memory.
+__device__ __forceinline__ void append_row(uint16_t *dst, const uint16_t *src, int32_t n,
+                                           int lane) {
+  for (int32_t e = lane * 8; e < n; e += 256)
+    *reinterpret_cast<uint4 *>(dst + e) = *reinterpret_cast<const uint4 *>(src + e);
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  __syncwarp();
+}
+
 // -------------------------------------------------- programmatic launches
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");

@@ -69,6 +69,20 @@ struct TcParams {
   float post;             // softcap*log2(e), or 0 when soft-cap is off
 };
 
+// Current-token append (k_new non-null): before the tile holding a unit's
+// newest position is loaded, its row is copied from k_new / v_new
+// ([B][Hkv][D]) into slot (L - 1) mod C of k_cache / v_cache.  A parameter of
+// its own: the 16-head kernel without append keeps its smaller parameter block
+// (a larger one measurably slowed that kernel's launches).
+struct TcAppend {
+  const uint16_t *k_new;
+  const uint16_t *v_new;  // null when K serves as V
+  uint16_t *k_cache;
+  uint16_t *v_cache;
+  int64_t batch_stride;   // cache elements from one sequence to the next
+  int32_t n_kv_heads;
+};
+
 struct TcConfig {
   static constexpr int D = 512;
   static constexpr int G = 16;
@@ -154,9 +168,9 @@ __device__ __forceinline__ float warp_reduce_scatter16(float (&r)[16], int lane)
   return MAX ? fmaxf(r[0], got) : r[0] + got;
 }
 
-__global__ void __launch_bounds__(TcConfig::kThreads, 1)
-    tc_decode_kernel(const __grid_constant__ CUtensorMap kmap,
-                     const __grid_constant__ CUtensorMap qmap, const TcParams p) {
+template <bool APPEND>
+__device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CUtensorMap &qmap,
+                                               const TcParams &p, const TcAppend &ap) {
   using Cfg = TcConfig;
   constexpr int G = Cfg::G, D = Cfg::D, NST = Cfg::NST;
 
@@ -311,6 +325,13 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
       }
       if (!__all_sync(0xffffffffu, ok)) break;
       stage_seg[st] = seg_count - 1;
+      if (APPEND && it.newest) {  // append the current token's row (K = V) first
+        const int32_t slot = (it.seg.first_pos + it.seg.n - 1) % C;
+        append_row(ap.k_cache + it.seg.b * ap.batch_stride +
+                       (static_cast<int64_t>(slot) * ap.n_kv_heads + it.seg.x) * D,
+                   ap.k_new + (static_cast<int64_t>(it.seg.b) * ap.n_kv_heads + it.seg.x) * D, D,
+                   lane);
+      }
       if (elect_one()) {
         mbar_arrive_expect_tx(&full[st], Cfg::STAGEB);
 #pragma unroll
@@ -648,6 +669,19 @@ __global__ void __launch_bounds__(TcConfig::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TMEM_COLS);
   }
+}
+
+__global__ void __launch_bounds__(TcConfig::kThreads, 1)
+    tc_decode_kernel(const __grid_constant__ CUtensorMap kmap,
+                     const __grid_constant__ CUtensorMap qmap, const TcParams p) {
+  tc_decode_body<false>(kmap, qmap, p, TcAppend{});
+}
+
+__global__ void __launch_bounds__(TcConfig::kThreads, 1)
+    tc_decode_append_kernel(const __grid_constant__ CUtensorMap kmap,
+                            const __grid_constant__ CUtensorMap qmap, const TcParams p,
+                            const TcAppend ap) {
+  tc_decode_body<true>(kmap, qmap, p, ap);
 }
 
 }  // namespace gdattn

@@ -103,10 +103,11 @@ __device__ __forceinline__ uint32_t sw128_offset(int n, int t) {
   return static_cast<uint32_t>(n * 128 + ((((t >> 3) ^ (n & 7)) << 4) | ((t & 7) << 1)));
 }
 
-__global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
-    tc_pair_decode_kernel(const __grid_constant__ CUtensorMap kmap,
-                          const __grid_constant__ CUtensorMap vmap,
-                          const __grid_constant__ CUtensorMap qmap, const TcParams p) {
+template <bool APPEND>
+__device__ __forceinline__ void tc_pair_decode_body(const CUtensorMap &kmap,
+                                                    const CUtensorMap &vmap,
+                                                    const CUtensorMap &qmap, const TcParams &p,
+                                                    const TcAppend &ap) {
   using Cfg = TcPairConfig;
   constexpr int G = Cfg::G, D = Cfg::D, NST = Cfg::NST;
 
@@ -276,6 +277,13 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
       }
       if (!__all_sync(0xffffffffu, ok)) break;
       stage_seg[st] = seg_count - 1;
+      if (APPEND && it.newest) {  // append the current token's K row first
+        const int32_t slot = (it.seg.first_pos + it.seg.n - 1) % C;
+        append_row(ap.k_cache + it.seg.b * ap.batch_stride +
+                       (static_cast<int64_t>(slot) * ap.n_kv_heads + it.seg.x) * D,
+                   ap.k_new + (static_cast<int64_t>(it.seg.b) * ap.n_kv_heads + it.seg.x) * D, D,
+                   lane);
+      }
       if (elect_one()) {
         uint8_t *kdst = stages + st * Cfg::STAGEB;
         mbar_arrive_expect_tx(&kfull[st], Cfg::KB);
@@ -542,6 +550,13 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
       if (i >= NST && !mbar_wait(&vempty[st], ((i / NST) - 1) & 1, abort_flag, p.status))
         ok = false;
       if (!__all_sync(0xffffffffu, ok)) break;
+      if (APPEND && it.newest) {  // append the current token's V row first
+        const int32_t slot = (it.seg.first_pos + it.seg.n - 1) % C;
+        append_row(ap.v_cache + it.seg.b * ap.batch_stride +
+                       (static_cast<int64_t>(slot) * ap.n_kv_heads + it.seg.x) * D,
+                   ap.v_new + (static_cast<int64_t>(it.seg.b) * ap.n_kv_heads + it.seg.x) * D, D,
+                   lane);
+      }
       if (elect_one()) {
         uint8_t *vdst = stages + st * Cfg::STAGEB + Cfg::KB;
         mbar_arrive_expect_tx(&vfull[st], Cfg::KB);
@@ -770,6 +785,21 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TMEM_COLS);
   }
+}
+
+__global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
+    tc_pair_decode_kernel(const __grid_constant__ CUtensorMap kmap,
+                          const __grid_constant__ CUtensorMap vmap,
+                          const __grid_constant__ CUtensorMap qmap, const TcParams p) {
+  tc_pair_decode_body<false>(kmap, vmap, qmap, p, TcAppend{});
+}
+
+__global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
+    tc_pair_decode_append_kernel(const __grid_constant__ CUtensorMap kmap,
+                                 const __grid_constant__ CUtensorMap vmap,
+                                 const __grid_constant__ CUtensorMap qmap, const TcParams p,
+                                 const TcAppend ap) {
+  tc_pair_decode_body<true>(kmap, vmap, qmap, p, ap);
 }
 
 }  // namespace gdattn

@@ -179,6 +179,28 @@ gdattn_status gdattn_combine(const float *o_partial, const float *lse_partial, i
                              float *lse, void *stream);
 
 /*
+ * gdattn_decode with the current token's append fused in: for every sequence b
+ * the rows k_new[b] (and v_new[b]) are written into cache slot
+ * (seqlens[b] - 1) mod C, then attention runs over the updated cache.  The
+ * result equals writing those rows first and calling gdattn_decode; the
+ * write is done by the CTA that loads that slot, just before it loads it, so
+ * it costs no launch and no extra pass.
+ *
+ *  k_new     bf16 [batch, Hkv, D], device, read only (read after the preceding
+ *            kernel on the stream has completed)
+ *  v_new     bf16 [batch, Hkv, D], or NULL when desc->kv_shared == 1
+ *  k_cache, v_cache: as in gdattn_decode, but written at those slots; nothing
+ *            else in them is written, and the slot of a sequence whose length is
+ *            rejected on the device is left untouched
+ *  other arguments, checks and errors as gdattn_decode
+ */
+gdattn_status gdattn_decode_append(const void *q, const void *k_new, const void *v_new,
+                                   void *k_cache, void *v_cache, const int32_t *seqlens,
+                                   int32_t batch, int32_t max_seqlen,
+                                   const gdattn_layer_desc *desc, void *out, float *lse,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * gdattn_decode without a caller workspace.  A library addition: the paper
  * has no counterpart; it computes exactly what gdattn_decode computes.
  *

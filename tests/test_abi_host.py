@@ -171,3 +171,19 @@ def test_workspace_init_rejects_null(lib):
 def test_combine_rejects_bad_args(lib, args, expect):
     o, l, B, Hq, S, D, out, lse = args
     assert lib.gdattn_combine(o, l, B, Hq, S, D, out, lse, None) == expect
+
+
+def test_decode_append_host_checks(lib):
+    """gdattn_decode_append: the new rows' pointers are checked like the rest."""
+    def app(desc, k_new=A, v_new=A, q=A, k=A, v=A, ws=A):
+        return lib.gdattn_decode_append(q, k_new, v_new, k, v, A, 1, 8, ctypes.byref(desc), A, A,
+                                        ws, 1 << 20, None)
+    d = good_desc()
+    assert app(d, k_new=None) == binding.GDATTN_ERR_INVALID_ARG
+    assert app(d, v_new=None) == binding.GDATTN_ERR_INVALID_ARG      # separate V expected
+    assert app(d, k_new=A + 8) == binding.GDATTN_ERR_MISALIGNED
+    assert app(d, v_new=A + 4) == binding.GDATTN_ERR_MISALIGNED
+    assert app(d, ws=None) == binding.GDATTN_ERR_WORKSPACE
+    shared = good_desc(n_q_heads=16, n_kv_heads=1, head_dim=512, window=0, kv_shared=True)
+    assert app(shared, v=None) == binding.GDATTN_ERR_INVALID_ARG     # K = V: no v_new
+    assert app(shared, v=None, v_new=None, q=None) == binding.GDATTN_ERR_INVALID_ARG
