@@ -598,9 +598,8 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
       if (ok && lane == 0) mbar_arrive(&pfull[pb]);
 
       if (last) {
-        // --- segment end: all of its P.V done, read O out
-        if (i >= 1) ensure_pv(i - 1);
-        ensure_pv(i);
+        // --- segment end: the row sums first (they do not need O), then wait
+        // for the segment's last P.V and read O out
         float r[16];  // this lane's 8 partial sums in their slots, 0 elsewhere
 #pragma unroll
         for (int h = 0; h < 8; ++h) {
@@ -610,6 +609,8 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
         const float ls = warp_reduce_scatter16<false>(r, lane);
         if ((lane & 1) == 0) redsum[qd * G + (lane >> 1)] = ls;
         named_bar_sync(1, 128);
+        if (i >= 1) ensure_pv(i - 1);
+        ensure_pv(i);
         const Segment &sg = it.seg;
         const bool single = sg.whole() && !usplit;  // a split unit always has parts
         const int64_t slot = static_cast<int64_t>(c) + sg.unit;

@@ -708,15 +708,16 @@ __device__ __forceinline__ void tc_pair_decode_body(const CUtensorMap &kmap,
       if (ok && lane == 0) mbar_arrive(&pfull[pb]);
 
       if (last) {
-        // --- segment end: all of its P.V done, read O out
-        if (i >= 1) ensure_pv(i - 1);
-        ensure_pv(i);
+        // --- segment end: the row sums first (they do not need O), then wait
+        // for the segment's last P.V and read O out
         float ls = lpart;
 #pragma unroll
         for (int off = 1; off < 16; off <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
         if ((lane & 15) == 0) redsum[qd * G + hd] = ls;
         if (threadIdx.x == 64) *sh_tag = my_tag;
         named_bar_sync(1, 128);
+        if (i >= 1) ensure_pv(i - 1);
+        ensure_pv(i);
         const uint32_t tag = *sh_tag;
         const Segment &sg = it.seg;
         const bool single = sg.whole() && !usplit;  // a split unit always has parts
