@@ -459,6 +459,37 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     assert torch.equal(out_host[-1], stack.layers[-1]["out"].cpu())  # same result both ways
 
+    # ---- the same step with the current token's K/V append fused in
+    # (gdattn_decode_append): each layer's new rows are written into their ring
+    # slots by the decode kernels.  Last, since it writes into the caches.
+    gen = torch.Generator(device="cpu").manual_seed(7 + rank)
+    new_rows = []
+    for ly in stack.layers:
+        sp = ly["spec"]
+        shape = (w.batch, sp.n_kv_heads, sp.head_dim)
+        kn = torch.randn(shape, generator=gen).to(torch.bfloat16).to(device)
+        vn = None if sp.kv_shared else torch.randn(shape, generator=gen).to(torch.bfloat16).to(device)
+        new_rows.append((kn, vn))
+
+    def append_step():
+        for ly, (kn, vn) in zip(stack.layers, new_rows):
+            binding.decode_append(ly["inp"].q, kn, vn, ly["inp"].k, ly["inp"].v, ly["inp"].seqlens,
+                                  ly["desc"], stack.max_seqlen, out=ly["out"], lse=ly["lse"],
+                                  workspace=ly["ws"], stream=stream)
+
+    g_app = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        append_step()
+        stream.synchronize()
+        with torch.cuda.graph(g_app, stream=stream):
+            append_step()
+    barrier()
+    ms_app = max_over_ranks(time_graph(g_app, stream, args.steps, args.warmup), world)
+    for ly in stack.layers:
+        st = binding.check_device_status(ly["ws"], stream)
+        if st != binding.GDATTN_OK:
+            raise binding.GdattnError(st, "device status after the append step")
+
     # ---- CPU baseline: the oracle over the whole step (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
@@ -473,7 +504,7 @@ def run_ours(args, world, rank, local):
 
     if world > 1:
         import torch.distributed as dist
-        del g_all, g_sl, g_gl, g_e2e
+        del g_all, g_sl, g_gl, g_e2e, g_app
         dist.destroy_process_group()
     if rank != 0:
         return 0
@@ -533,6 +564,11 @@ def run_ours(args, world, rank, local):
                        "CUDA graph and replayed",
                 "eager_value": job_gbs(kv_step, ms_e2e_eager, world),
                 "eager_ms_per_step": ms_e2e_eager},
+        "append": {"value": job_gbs(kv_step, ms_app, world), "unit": "GB/s",
+                   "us_per_step": ms_app * 1e3,
+                   "how": "the same 48 layers through gdattn_decode_append: each layer's "
+                          "current-token K/V rows written into their ring slots by the decode "
+                          "kernels (CUDA graph, device time)"},
         "gpu_launches": stack.launches_per_step(all_idx) * args.steps,
         "clocks": clk,
     }
