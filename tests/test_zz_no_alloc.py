@@ -69,8 +69,9 @@ def test_scratch_size_constant_matches_header():
 
 # ------------------------------------------------------------------ GPU tests
 def _layers():
-    """Two sliding (CUDA-core path) and two global (tcgen05 path) inputs; each
-    pair differs in seed and lengths, so stale scratch would change results."""
+    """Two sliding (tcgen05 pair kernel) and two global (tcgen05 16-head kernel)
+    inputs; each pair differs in seed and lengths, so stale scratch would change
+    results."""
     core = [
         (workloads.random_case(901, 4, 16, 8, 256, 1024, [1500, 700, 1, 4096], window=1024), 0),
         (workloads.random_case(902, 4, 16, 8, 256, 1024, [333, 4000, 1024, 90], window=1024), 37),
@@ -212,3 +213,23 @@ def test_noalloc_graph_replay_matches_workspace_decode():
             assert_same(b, r, f"graph layer {i}")
     assert binding.check_device_status(None) == binding.GDATTN_OK
     del g
+
+
+@pytest.mark.gpu
+def test_noalloc_even_split_matches_workspace_decode():
+    """With the even unit split the pair kernel merges tagged parts, whose
+    per-unit epochs live in the fixed scratch between calls: consecutive
+    no-alloc calls equal gdattn_decode bit for bit."""
+    require_gpu()
+    inp = workloads.random_case(906, 4, 16, 8, 256, 512, [512, 700, 900, 512], window=512)
+    ly = Dev(inp, 0)
+    ly.desc = binding.desc_from_spec(inp.spec, capacity=512, flags=binding.GDATTN_FLAG_EVEN_UNITS)
+    splits = binding.plan_splits(ly.B, ly.max_seqlen, ly.desc)
+    assert splits // (ly.B * 8) >= 2, splits  # the unit split (tagged merge) is in use
+    ref = ly.with_workspace()
+    for rep in range(3):
+        got = ly.outputs()
+        ly.noalloc(*got)
+        torch.cuda.synchronize()
+        assert binding.check_device_status(None) == binding.GDATTN_OK
+        assert_same(got, ref, f"even split call {rep}")
