@@ -34,6 +34,13 @@ class Oracle:
         lib.oracle_decode.argtypes = [u16p, u16p, u16p, i32p, i32, i32, i32, i32, i32, i64, i32,
                                       f64, f64, i32, f64p, f64p]
         lib.oracle_decode.restype = ctypes.c_int
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        f32p = ctypes.POINTER(ctypes.c_float)
+        lib.oracle_decode_fp8.argtypes = [u16p, u8p, u8p, f32p, f32p, i32p, i32, i32, i32, i32,
+                                          i32, i64, i32, f64, f64, i32, f64p, f64p]
+        lib.oracle_decode_fp8.restype = ctypes.c_int
+        lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8, f64p]
+        lib.oracle_e4m3_to_double.restype = ctypes.c_int
         lib.oracle_combine.argtypes = [f64p, f64p, i32, i32, f64p, f64p]
         lib.oracle_combine.restype = None
         lib.oracle_version.restype = ctypes.c_int
@@ -81,6 +88,61 @@ class Oracle:
             self._ptr(out, ctypes.c_double), self._ptr(lse, ctypes.c_double))
         if rc != 0:
             raise ValueError("oracle_decode rejected its arguments")
+        return out, lse
+
+    @staticmethod
+    def _codes(t) -> np.ndarray:
+        """fp8 codes (torch uint8 / float8_e4m3fn tensor or uint8 array) -> contiguous uint8."""
+        if isinstance(t, torch.Tensor):
+            return np.ascontiguousarray(t.detach().cpu().contiguous().view(torch.uint8).numpy())
+        a = np.ascontiguousarray(t)
+        assert a.dtype == np.uint8
+        return a
+
+    @staticmethod
+    def _f32(t) -> np.ndarray:
+        if isinstance(t, torch.Tensor):
+            assert t.dtype == torch.float32, t.dtype
+            return np.ascontiguousarray(t.detach().cpu().contiguous().numpy())
+        return np.ascontiguousarray(np.asarray(t, dtype=np.float32))
+
+    def e4m3_value(self, code: int) -> float:
+        """The value of one e4m3 code, as the oracle decodes it."""
+        v = ctypes.c_double()
+        self.lib.oracle_e4m3_to_double(int(code) & 0xFF, ctypes.byref(v))
+        return v.value
+
+    def decode_fp8(self, q, k_codes, v_codes, k_scale, v_scale, seqlens, window: int,
+                   softcap: float, scale: float):
+        """One decode-attention layer over an fp8 cache.  Returns (out, lse) float64.
+
+        q: bf16 [B,Hq,D]; k_codes (v_codes): e4m3 codes [B,C,Hkv,D]; k_scale (v_scale):
+        float32 [B,Hkv,C] per-row scales.  v_codes=None means K (with its scales) serves as V.
+        """
+        qb, kc = self._bits(q), self._codes(k_codes)
+        B, Hq, D = qb.shape
+        _, C, Hkv, Dk = kc.shape
+        assert Dk == D and kc.shape[0] == B
+        ks = self._f32(k_scale)
+        assert ks.shape == (B, Hkv, C), ks.shape
+        vc = self._codes(v_codes) if v_codes is not None else None
+        vs = self._f32(v_scale) if v_codes is not None else None
+        if vc is not None:
+            assert vc.shape == kc.shape and vs.shape == ks.shape
+        sl = np.ascontiguousarray(np.asarray(seqlens.cpu() if isinstance(seqlens, torch.Tensor)
+                                             else seqlens, dtype=np.int32))
+        out = np.zeros((B, Hq, D), dtype=np.float64)
+        lse = np.zeros((B, Hq), dtype=np.float64)
+        rc = self.lib.oracle_decode_fp8(
+            self._ptr(qb, ctypes.c_uint16), self._ptr(kc, ctypes.c_uint8),
+            self._ptr(vc, ctypes.c_uint8) if vc is not None else None,
+            self._ptr(ks, ctypes.c_float),
+            self._ptr(vs, ctypes.c_float) if vs is not None else None,
+            self._ptr(sl, ctypes.c_int32), B, Hq, Hkv, D, C, C * Hkv * D, int(window),
+            float(softcap), float(scale), 1 if vc is None else 0,
+            self._ptr(out, ctypes.c_double), self._ptr(lse, ctypes.c_double))
+        if rc != 0:
+            raise ValueError("oracle_decode_fp8 rejected its arguments")
         return out, lse
 
     def attend(self, q, k, v, lo: Sequence[int], hi: Sequence[int], softcap: float,

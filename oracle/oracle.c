@@ -24,7 +24,10 @@
  * The soft-cap form cap*tanh(s/cap) applied to the scaled logit, and the
  * natural-log LSE, are the plainest readings where the pages are silent.
  *
- * All inputs are bf16 bit patterns (uint16), widened exactly to double.
+ * Cache rows are bf16 bit patterns (uint16), widened exactly to double, or, in
+ * oracle_decode_fp8, e4m3 codes times a float scale per row (the quantized
+ * rotating cache of "Gemma 4 12B", serviceability join, item 6; the format and
+ * scale layout are spelled out at e4m3_to_double and row_source).  q is bf16.
  *
  * Compile-time ORACLE_MUTATION=n plants one deliberate mistake (used only by the
  * test that shows the pins catch plausible mistakes); 0 (default) is the oracle.
@@ -45,43 +48,113 @@ static double bf16_to_double(uint16_t bits) {
   return (double)f;
 }
 
-/* Address of element d of KV head `kv` in cache slot `slot` of sequence b.
- * Cache layout: sequence b starts at b * batch_stride elements; within it
- * [C][Hkv][D] token-major, D contiguous. */
-static const uint16_t *kv_row(const uint16_t *cache, int64_t batch_stride, int32_t Hkv, int32_t D,
-                              int32_t b, int32_t slot, int32_t kv) {
-  return cache + (int64_t)b * batch_stride + ((int64_t)slot * Hkv + kv) * D;
+/*
+ * An fp8 code in the OCP 8-bit floating point format E4M3 (the "e4m3" of the
+ * fp8 KV caches the pages speak of): sign bit, 4 exponent bits with bias 7, 3
+ * mantissa bits; exponent field 0 holds the subnormals m/8 * 2^-6; no
+ * infinities, and S.1111.111 is NaN (largest finite magnitude 448).
+ */
+static double e4m3_to_double(uint8_t code) {
+  int sign = code >> 7, e = (code >> 3) & 0xF, m = code & 7;
+  int bias = 7;
+#if ORACLE_MUTATION == 9
+  bias = 8; /* exponent bias off by one */
+#endif
+  if (e == 15 && m == 7) return NAN;
+  double mag = (e == 0) ? ldexp((double)m / 8.0, 1 - bias) : ldexp(1.0 + (double)m / 8.0, e - bias);
+  return sign ? -mag : mag;
+}
+
+int oracle_e4m3_to_double(uint8_t code, double *value) {
+  *value = e4m3_to_double(code);
+  return 0;
+}
+
+/*
+ * Where the cache rows come from.  Layout of both caches: sequence b starts at
+ * b * batch_stride elements; within it [C][Hkv][D] token-major, D contiguous.
+ *  bf16: rows of bf16 bit patterns, widened exactly to double.
+ *  fp8:  rows of e4m3 codes; row (b, kv, slot) has one float scale at
+ *        scale[(b * Hkv + kv) * C + slot], and its values are code * scale
+ *        (the per-row scales of a quantized rotating cache: "Gemma 4 12B",
+ *        serviceability join, item 6).
+ */
+typedef struct row_source {
+  int fp8;
+  const uint16_t *k, *v;     /* bf16 */
+  const uint8_t *kc, *vc;    /* fp8 codes */
+  const float *ks, *vs;      /* fp8 per-row scales */
+  int64_t batch_stride;
+  int32_t Hkv, D, C, kv_shared;
+} row_source;
+
+/* The D values of row (b, slot, kv) of K (value == 0) or of the value tensor
+ * (value == 1: V, or K when K serves as V). */
+static void fetch_row(const row_source *src, int32_t b, int32_t slot, int32_t kv, int value,
+                      double *row) {
+  const int use_v = value && !src->kv_shared;
+  const int64_t off = (int64_t)b * src->batch_stride + ((int64_t)slot * src->Hkv + kv) * src->D;
+  if (!src->fp8) {
+    const uint16_t *r = (use_v ? src->v : src->k) + off;
+    for (int32_t d = 0; d < src->D; ++d) row[d] = bf16_to_double(r[d]);
+    return;
+  }
+  const uint8_t *r = (use_v ? src->vc : src->kc) + off;
+  const float *scales = use_v ? src->vs : src->ks;
+#if ORACLE_MUTATION == 10
+  scales = src->ks; /* V rows scaled by the K scales */
+#endif
+  int64_t si = ((int64_t)b * src->Hkv + kv) * src->C + slot;
+#if ORACLE_MUTATION == 12
+  si = ((int64_t)b * src->C + slot) * src->Hkv + kv; /* scales read token-major */
+#endif
+  double sc = (double)scales[si];
+#if ORACLE_MUTATION == 11
+  sc = sc * sc; /* scale applied twice */
+#endif
+  for (int32_t d = 0; d < src->D; ++d) row[d] = e4m3_to_double(r[d]) * sc;
 }
 
 int oracle_version(void) { return 1 + 1000 * ORACLE_MUTATION; }
 
 /*
  * Attention of every query head over an explicit logical position range
- * [lo[b], hi[b]) per sequence.  An empty range yields LSE = -inf and out = 0.
- * q: [B][Hq][D]; k, v: caches as above (v ignored when kv_shared != 0);
- * out: [B][Hq][D] doubles; lse: [B][Hq] doubles.  Returns 0, or -1 on bad input.
+ * [lo[b], hi[b]) per sequence, with cache rows from `src`.  An empty range
+ * yields LSE = -inf and out = 0.  q: [B][Hq][D]; out: [B][Hq][D] doubles;
+ * lse: [B][Hq] doubles.  Returns 0, or -1 on bad input.
  */
-int oracle_attend(const uint16_t *q, const uint16_t *k, const uint16_t *v, int32_t B, int32_t Hq,
-                  int32_t Hkv, int32_t D, int32_t C, int64_t batch_stride, const int32_t *lo,
-                  const int32_t *hi, double softcap, double scale, int32_t kv_shared, double *out,
+static int attend(const uint16_t *q, int32_t B, int32_t Hq, const int32_t *lo, const int32_t *hi,
+                  double softcap, double scale, const row_source *src, double *out,
                   double *lse) {
+  const int32_t Hkv = src->Hkv, D = src->D, C = src->C;
   if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || C <= 0 || Hq % Hkv != 0) return -1;
-  if (!kv_shared && v == NULL) return -1;
   const int32_t G = Hq / Hkv;
-  const uint16_t *vals = kv_shared ? k : v;
+  int value_tensor = 1;
 #if ORACLE_MUTATION == 6
-  vals = k; /* values taken from K even when a separate V exists */
+  value_tensor = 0; /* values taken from K even when a separate V exists */
 #endif
+  double *qd = (double *)malloc(sizeof(double) * (size_t)D);
+  double *row = (double *)malloc(sizeof(double) * (size_t)D);
+  if (!qd || !row) {
+    free(qd);
+    free(row);
+    return -1;
+  }
   for (int32_t b = 0; b < B; ++b) {
     const int32_t n = hi[b] - lo[b];
     double *s = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
-    if (!s) return -1;
+    if (!s) {
+      free(qd);
+      free(row);
+      return -1;
+    }
     for (int32_t h = 0; h < Hq; ++h) {
       int32_t kv = h / G;
 #if ORACLE_MUTATION == 2
       kv = h % Hkv; /* interleaved instead of contiguous GQA groups */
 #endif
       const uint16_t *qh = q + ((int64_t)b * Hq + h) * D;
+      for (int32_t d = 0; d < D; ++d) qd[d] = bf16_to_double(qh[d]);
       double *o = out + ((int64_t)b * Hq + h) * D;
       for (int32_t d = 0; d < D; ++d) o[d] = 0.0;
       if (n <= 0) {
@@ -95,9 +168,9 @@ int oracle_attend(const uint16_t *q, const uint16_t *k, const uint16_t *v, int32
 #if ORACLE_MUTATION == 7
         slot = (j + 1) % C; /* ring index off by one */
 #endif
-        const uint16_t *kr = kv_row(k, batch_stride, Hkv, D, b, slot, kv);
+        fetch_row(src, b, slot, kv, 0, row);
         double dot = 0.0;
-        for (int32_t d = 0; d < D; ++d) dot += bf16_to_double(qh[d]) * bf16_to_double(kr[d]);
+        for (int32_t d = 0; d < D; ++d) dot += qd[d] * row[d];
         double x = scale * dot;
 #if ORACLE_MUTATION == 8
         x = dot; /* scale dropped */
@@ -130,31 +203,22 @@ int oracle_attend(const uint16_t *q, const uint16_t *k, const uint16_t *v, int32
 #if ORACLE_MUTATION == 5
         p = exp(s[j - lo[b]] - m); /* weights not normalised */
 #endif
-        const uint16_t *vr = kv_row(vals, batch_stride, Hkv, D, b, slot, kv);
-        for (int32_t d = 0; d < D; ++d) o[d] += p * bf16_to_double(vr[d]);
+        fetch_row(src, b, slot, kv, value_tensor, row);
+        for (int32_t d = 0; d < D; ++d) o[d] += p * row[d];
       }
     }
     free(s);
   }
+  free(qd);
+  free(row);
   return 0;
 }
 
-/*
- * Decode attention for one layer: the position range follows from the context
- * length L_b (current token included) and the window.  window == 0 attends the
- * whole context.  Returns -1 when a range needs more slots than the cache has.
- */
-int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *seqlens,
-                  int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t C, int64_t batch_stride,
-                  int32_t window, double softcap, double scale, int32_t kv_shared, double *out,
-                  double *lse) {
-  int32_t *lo = (int32_t *)malloc(sizeof(int32_t) * (size_t)(B > 0 ? B : 1));
-  int32_t *hi = (int32_t *)malloc(sizeof(int32_t) * (size_t)(B > 0 ? B : 1));
-  if (!lo || !hi) {
-    free(lo);
-    free(hi);
-    return -1;
-  }
+/* Position range [lo_b, hi_b) of one decode step: the last `window` positions
+ * of the context L_b (window 0: all of it).  -1 when a range needs more slots
+ * than the cache has, or L_b < 1. */
+static int decode_ranges(const int32_t *seqlens, int32_t B, int32_t window, int32_t C,
+                         int32_t *lo, int32_t *hi) {
   int rc = 0;
   for (int32_t b = 0; b < B; ++b) {
     int32_t L = seqlens[b];
@@ -167,12 +231,66 @@ int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
     hi[b] = L;
     if (L < 1 || L - start > C) rc = -1;
   }
-  if (rc == 0)
-    rc = oracle_attend(q, k, v, B, Hq, Hkv, D, C, batch_stride, lo, hi, softcap, scale, kv_shared,
-                       out, lse);
+  return rc;
+}
+
+static int decode_with(const int32_t *seqlens, const uint16_t *q, int32_t B, int32_t Hq,
+                       int32_t window, double softcap, double scale, const row_source *src,
+                       double *out, double *lse) {
+  int32_t *lo = (int32_t *)malloc(sizeof(int32_t) * (size_t)(B > 0 ? B : 1));
+  int32_t *hi = (int32_t *)malloc(sizeof(int32_t) * (size_t)(B > 0 ? B : 1));
+  if (!lo || !hi) {
+    free(lo);
+    free(hi);
+    return -1;
+  }
+  int rc = decode_ranges(seqlens, B, window, src->C, lo, hi);
+  if (rc == 0) rc = attend(q, B, Hq, lo, hi, softcap, scale, src, out, lse);
   free(lo);
   free(hi);
   return rc;
+}
+
+/*
+ * Attention over explicit ranges with a bf16 cache (k; v, or K as V when
+ * kv_shared != 0).
+ */
+int oracle_attend(const uint16_t *q, const uint16_t *k, const uint16_t *v, int32_t B, int32_t Hq,
+                  int32_t Hkv, int32_t D, int32_t C, int64_t batch_stride, const int32_t *lo,
+                  const int32_t *hi, double softcap, double scale, int32_t kv_shared, double *out,
+                  double *lse) {
+  if (!kv_shared && v == NULL) return -1;
+  row_source src = {0, k, v, NULL, NULL, NULL, NULL, batch_stride, Hkv, D, C, kv_shared};
+  return attend(q, B, Hq, lo, hi, softcap, scale, &src, out, lse);
+}
+
+/*
+ * Decode attention for one layer over a bf16 cache: the position range
+ * follows from the context length L_b (current token included) and the
+ * window.  window == 0 attends the whole context.  Returns -1 when a range
+ * needs more slots than the cache has.
+ */
+int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *seqlens,
+                  int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t C, int64_t batch_stride,
+                  int32_t window, double softcap, double scale, int32_t kv_shared, double *out,
+                  double *lse) {
+  if (!kv_shared && v == NULL) return -1;
+  row_source src = {0, k, v, NULL, NULL, NULL, NULL, batch_stride, Hkv, D, C, kv_shared};
+  return decode_with(seqlens, q, B, Hq, window, softcap, scale, &src, out, lse);
+}
+
+/*
+ * oracle_decode over an fp8 cache: codes kc (vc) in e4m3 with per-row scales
+ * ks (vs), [B][Hkv][C] floats; values are code * scale.  vc and vs are ignored
+ * when kv_shared != 0 (K, with its scales, serves as V).
+ */
+int oracle_decode_fp8(const uint16_t *q, const uint8_t *kc, const uint8_t *vc, const float *ks,
+                      const float *vs, const int32_t *seqlens, int32_t B, int32_t Hq, int32_t Hkv,
+                      int32_t D, int32_t C, int64_t batch_stride, int32_t window, double softcap,
+                      double scale, int32_t kv_shared, double *out, double *lse) {
+  if (!kv_shared && (vc == NULL || vs == NULL)) return -1;
+  row_source src = {1, NULL, NULL, kc, vc, ks, vs, batch_stride, Hkv, D, C, kv_shared};
+  return decode_with(seqlens, q, B, Hq, window, softcap, scale, &src, out, lse);
 }
 
 /*

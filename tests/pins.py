@@ -319,10 +319,108 @@ def pin_separate_v(orc):
            "shared K=V mean")
 
 
+# --------------------------------------------------------------------------
+# fp8 e4m3 caches with per-row scales
+# --------------------------------------------------------------------------
+
+
+def e4m3_reference(codes) -> np.ndarray:
+    """Values of e4m3 codes by torch's float8_e4m3fn decoding (a library routine)."""
+    t = torch.as_tensor(np.asarray(codes, dtype=np.uint8))
+    return t.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def dequantize(codes: torch.Tensor, scales: torch.Tensor) -> torch.Tensor:
+    """codes [B, C, Hkv, D] e4m3, scales [B, Hkv, C] -> float64 values [B, C, Hkv, D]."""
+    vals = codes.view(torch.float8_e4m3fn).to(torch.float64)
+    return vals * scales.to(torch.float64).permute(0, 2, 1).unsqueeze(-1)
+
+
+def pin_e4m3_codes(orc):
+    """Every one of the 256 e4m3 codes decodes as torch's float8_e4m3fn does, and the
+    format's landmarks hold: 1.0, the largest finite 448, the smallest normal 2^-6 and
+    subnormal 2^-9, sign symmetry, NaN only at S.1111.111."""
+    ref = e4m3_reference(np.arange(256))
+    got = np.array([orc.e4m3_value(c) for c in range(256)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref)), "e4m3 NaN codes differ"
+    fin = ~np.isnan(ref)
+    assert np.array_equal(got[fin], ref[fin]), "e4m3 decoding differs from float8_e4m3fn"
+    landmarks = {0x38: 1.0, 0x7E: 448.0, 0x08: 2.0 ** -6, 0x01: 2.0 ** -9, 0x00: 0.0,
+                 0xB8: -1.0, 0x40: 2.0, 0x3C: 1.5}
+    for code, val in landmarks.items():
+        assert orc.e4m3_value(code) == val, f"e4m3 code {code:#04x}"
+    assert np.isnan(orc.e4m3_value(0x7F)) and np.isnan(orc.e4m3_value(0xFF))
+
+
+# (B, Hq, Hkv, D, C, seqlens, window, softcap, kv_shared)
+FP8_CASES = [
+    (2, 4, 2, 16, 12, [37, 12], 12, 0.0, False),  # ring wraps
+    (2, 16, 8, 32, 10, [33, 7], 10, 30.0, False),
+    (1, 16, 1, 32, 30, [30], 0, 0.0, True),  # K serves as V
+    (2, 4, 2, 8, 20, [20, 3], 0, 5.0, False),
+]
+
+
+def pin_fp8_equals_bf16_when_exact(orc):
+    """With power-of-two row scales every value code * scale is a bf16 number, so
+    the fp8 decode must equal the (separately pinned) bf16 decode of those values,
+    exactly.  K and V scales differ and vary per (sequence, head, slot)."""
+    for i, (B, Hq, Hkv, D, C, sl, w, cap, shared) in enumerate(FP8_CASES):
+        inp = workloads.random_fp8_case(2000 + i, B, Hq, Hkv, D, C, sl, window=w, softcap=cap,
+                                        kv_shared=shared)
+        g = torch.Generator().manual_seed(3000 + i)
+        pow2 = lambda: torch.exp2(torch.randint(-4, 5, (B, Hkv, C), generator=g).float())
+        ks, vs = pow2(), pow2()
+        k_bf = dequantize(inp.k_codes, ks).to(torch.bfloat16)
+        assert torch.equal(k_bf.to(torch.float64), dequantize(inp.k_codes, ks)), "not exact"
+        v_bf = None
+        if not shared:
+            v_bf = dequantize(inp.v_codes, vs).to(torch.bfloat16)
+        s = inp.spec
+        o1, l1 = orc.decode_fp8(inp.q, inp.k_codes, inp.v_codes if not shared else None, ks,
+                                vs if not shared else None, inp.seqlens, s.window, s.softcap,
+                                s.scale)
+        o2, l2 = orc.decode(inp.q, k_bf, v_bf, inp.seqlens, s.window, s.softcap, s.scale)
+        _close(o1, o2, 0.0, f"fp8 vs bf16 out, case {i}")
+        _close(l1, l2, 0.0, f"fp8 vs bf16 lse, case {i}")
+
+
+def pin_fp8_brute_force(orc):
+    """fp8 decode == the numpy brute force over values dequantized with torch's e4m3
+    decoding and the row scales (arbitrary float scales, soft-cap on and off)."""
+    for i, (B, Hq, Hkv, D, C, sl, w, cap, shared) in enumerate(FP8_CASES):
+        inp = workloads.random_fp8_case(2100 + i, B, Hq, Hkv, D, C, sl, window=w, softcap=cap,
+                                        kv_shared=shared, spread=3.0)
+        s = inp.spec
+        o1, l1 = orc.decode_fp8(inp.q, inp.k_codes, inp.v_codes, inp.k_scale, inp.v_scale,
+                                inp.seqlens, s.window, s.softcap, s.scale)
+        kf = dequantize(inp.k_codes, inp.k_scale)
+        vf = None if shared else dequantize(inp.v_codes, inp.v_scale)
+        o2, l2 = brute_force(inp.q, kf, vf, inp.seqlens.numpy(), s.window, s.softcap, s.scale)
+        _close(o1, o2, 1e-12, f"fp8 brute force out, case {i}")
+        _close(l1, l2, 1e-12, f"fp8 brute force lse, case {i}")
+
+
+def pin_fp8_zero_scale_row(orc):
+    """A row whose scale is 0 has value 0 whatever its codes: with q = 0 the output
+    is the mean of V over the attended rows, counting the zero rows as zeros."""
+    inp = workloads.random_fp8_case(2200, 1, 2, 1, 8, 6, [6], window=0)
+    vs = inp.v_scale.clone()
+    vs[0, 0, 2] = 0.0
+    vs[0, 0, 4] = 0.0
+    o, l = orc.decode_fp8(torch.zeros_like(inp.q), inp.k_codes, inp.v_codes, inp.k_scale, vs,
+                          inp.seqlens, 0, 0.0, 1.0)
+    vf = dequantize(inp.v_codes, vs).numpy()[0, :, 0, :]
+    assert np.all(vf[2] == 0) and np.all(vf[4] == 0)
+    _close(o[0, 0], vf.mean(axis=0), 1e-12, "zero-scale rows out")
+    _close(l[0], np.full(2, math.log(6)), 1e-12, "zero-scale rows lse")
+
+
 ALL_PINS = [pin_brute_force, pin_sdpa, pin_window_covers_context, pin_cap_to_infinity,
             pin_identical_keys, pin_zero_query, pin_single_position, pin_two_positions,
             pin_softcap_bound, pin_sliding_ignores_old_positions, pin_ring_equals_linear,
-            pin_split_recombine, pin_combine_closed_form, pin_separate_v]
+            pin_split_recombine, pin_combine_closed_form, pin_separate_v, pin_e4m3_codes,
+            pin_fp8_equals_bf16_when_exact, pin_fp8_brute_force, pin_fp8_zero_scale_row]
 
 
 def failing_pins(orc):

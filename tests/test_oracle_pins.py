@@ -17,6 +17,10 @@ MUTATIONS = {
     6: "values read from K when a separate V exists",
     7: "ring slot off by one",
     8: "scale dropped",
+    9: "e4m3 exponent bias off by one",
+    10: "V rows scaled by the K scales",
+    11: "row scale applied twice",
+    12: "row scales read token-major",
 }
 
 

@@ -16,6 +16,12 @@ Every tensor is bf16 drawn from N(0, 1) with a torch.Generator seeded as stated,
 except the per-sequence context lengths of the ragged workload (uniform integers)
 and the heavy-row stress of the long-context workload (a Bernoulli row mask whose
 rows are multiplied by a constant before rounding to bf16).
+
+fp8 caches (``fp8_layer_inputs``): each cache row (one token of one KV head) is
+N(0, 1) times a per-row spread 2^u, u uniform in [-spread, spread], then stored
+the way a quantizing cache writer would store it: scale = the row's largest
+|value| / 448 and codes = value / scale rounded to e4m3 (torch's float8_e4m3fn
+conversion).  The decode under test only reads the codes and scales.
 """
 from __future__ import annotations
 
@@ -197,3 +203,65 @@ def random_case(seed: int, batch: int, n_q_heads: int, n_kv_heads: int, head_dim
                      kv_shared, capacity)
     sl = torch.as_tensor(seqlens, dtype=torch.int32).reshape(batch)
     return layer_inputs(spec, batch, sl, seed, device=device)
+
+
+# --------------------------------------------------------------------------
+# fp8 e4m3 caches with per-row scales
+# --------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+@dataclass
+class Fp8LayerInputs:
+    q: torch.Tensor  # bf16 [B, Hq, D]
+    k_codes: torch.Tensor  # uint8 e4m3 codes [B, C, Hkv, D]
+    v_codes: Optional[torch.Tensor]  # uint8 [B, C, Hkv, D] or None when K serves as V
+    k_scale: torch.Tensor  # float32 [B, Hkv, C]: scale of row (b, kv, slot)
+    v_scale: Optional[torch.Tensor]  # float32 [B, Hkv, C] or None
+    seqlens: torch.Tensor  # int32 [B]
+    spec: LayerSpec = field(repr=False, default=None)
+
+
+def quantize_rows_e4m3(x: torch.Tensor):
+    """Rows of x [B, C, Hkv, D] (float32) -> (codes uint8 [B, C, Hkv, D], scales float32
+    [B, Hkv, C]) with scale = row max |x| / 448 (1 for an all-zero row)."""
+    amax = x.abs().amax(dim=-1)  # [B, C, Hkv]
+    scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+    codes = (x / scale.unsqueeze(-1)).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), scale.permute(0, 2, 1).contiguous()
+
+
+def fp8_layer_inputs(spec: LayerSpec, batch: int, seqlens: torch.Tensor, seed: int,
+                     device="cpu", capacity: Optional[int] = None,
+                     spread: float = 1.5) -> Fp8LayerInputs:
+    """q as in ``layer_inputs``; K (and V unless K serves as V) rows N(0, 1) * 2^u,
+    u ~ U(-spread, spread) per row, quantized per row to e4m3 codes and a scale."""
+    C = int(capacity if capacity is not None else spec.capacity)
+    g = _gen(seed, device)
+    B, Hq, Hkv, D = batch, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
+    q = torch.randn((B, Hq, D), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+    def rows():
+        x = torch.randn((B, C, Hkv, D), generator=g, device=device, dtype=torch.float32)
+        u = (torch.rand((B, C, Hkv, 1), generator=g, device=device) * 2 - 1) * spread
+        return quantize_rows_e4m3(x * torch.exp2(u))
+
+    k_codes, k_scale = rows()
+    v_codes = v_scale = None
+    if not spec.kv_shared:
+        v_codes, v_scale = rows()
+    return Fp8LayerInputs(q, k_codes, v_codes, k_scale, v_scale,
+                          seqlens.to(torch.int32).to(device), spec)
+
+
+def random_fp8_case(seed: int, batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
+                    capacity: int, seqlens, window: int = 0, softcap: float = 0.0,
+                    scale: Optional[float] = None, kv_shared: bool = False, spread: float = 1.5,
+                    device="cpu") -> Fp8LayerInputs:
+    """A small seeded fp8-cache case of arbitrary geometry."""
+    spec = LayerSpec("sliding" if window > 0 else "global", n_q_heads, n_kv_heads, head_dim,
+                     window, softcap, (1.0 / math.sqrt(head_dim)) if scale is None else scale,
+                     kv_shared, capacity)
+    sl = torch.as_tensor(seqlens, dtype=torch.int32).reshape(batch)
+    return fp8_layer_inputs(spec, batch, sl, seed, device=device, spread=spread)
