@@ -80,6 +80,10 @@ def lib() -> ctypes.CDLL:
             L.gdattn_decode_append.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, descp, vp, vp,
                                                vp, sz, vp]
             L.gdattn_decode_append.restype = ctypes.c_int
+        if hasattr(L, "gdattn_decode_fp8"):
+            L.gdattn_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, descp, vp, vp, vp,
+                                            sz, vp]
+            L.gdattn_decode_fp8.restype = ctypes.c_int
         L.gdattn_decode_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, descp, vp, vp, vp]
         L.gdattn_decode_noalloc.restype = ctypes.c_int
         L.gdattn_combine.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp]
@@ -205,6 +209,39 @@ def decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: Optional[torch.Te
                                         workspace.numel(), _stream_handle(stream)))
     if st != GDATTN_OK:
         raise GdattnError(st, "gdattn_decode_append")
+    return out, lse
+
+
+def decode_fp8_raw(q, k_codes, v_codes, k_scale, v_scale, seqlens, batch, max_seqlen, desc, out,
+                   lse, workspace, workspace_bytes, stream) -> int:
+    """gdattn_decode_fp8 on raw addresses (ints); returns the status code."""
+    return int(lib().gdattn_decode_fp8(q, k_codes, v_codes, k_scale, v_scale, seqlens,
+                                       int(batch), int(max_seqlen), ctypes.byref(desc), out, lse,
+                                       workspace, int(workspace_bytes), stream))
+
+
+def decode_fp8(q: torch.Tensor, k_codes: torch.Tensor, v_codes: torch.Tensor,
+               k_scale: torch.Tensor, v_scale: torch.Tensor, seqlens: torch.Tensor,
+               desc: LayerDesc, max_seqlen: int, out: Optional[torch.Tensor] = None,
+               lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+               stream=None):
+    """One layer over an fp8 e4m3 cache through gdattn_decode_fp8.  Returns (out, lse).
+
+    k_codes / v_codes: uint8 (or float8_e4m3fn) [B, C, Hkv, D]; k_scale / v_scale:
+    float32 [B, Hkv, C], the scale of each cache row.
+    """
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, max_seqlen, desc, q.device, stream)
+    st = decode_fp8_raw(_ptr(q), _ptr(k_codes), _ptr(v_codes), _ptr(k_scale), _ptr(v_scale),
+                        _ptr(seqlens), B, max_seqlen, desc, _ptr(out), _ptr(lse),
+                        _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    if st != GDATTN_OK:
+        raise GdattnError(st, "gdattn_decode_fp8")
     return out, lse
 
 

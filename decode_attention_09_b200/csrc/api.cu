@@ -15,6 +15,7 @@
 #include "core_decode.cuh"
 #include "tc_decode.cuh"
 #include "tc_pair_decode.cuh"
+#include "tc_pair_fp8_decode.cuh"
 
 using namespace gdattn;
 
@@ -155,6 +156,11 @@ int query_tc_pair(const void *fn, int threads, int smem) {
   using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const TcParams);
   return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
 }
+int query_tc_pair_fp8(const void *fn, int threads, int smem) {
+  using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const TcParams,
+                        const Fp8Scales);
+  return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
+}
 int query_tc_pair_append(const void *fn, int threads, int smem) {
   using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const TcParams,
                         const TcAppend);
@@ -188,13 +194,15 @@ PathKind choose_path(const gdattn_layer_desc *d) {
   return PathKind::kNone;
 }
 
+// fp8: plan for the fp8 cache kernel of the same path (only the pair path has one).
 gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *d,
-                        LayerPlan &pl) {
+                        LayerPlan &pl, bool fp8 = false) {
   gdattn_status st = check_desc(d);
   if (st != GDATTN_OK) return st;
   if (batch <= 0 || max_seqlen <= 0) return GDATTN_ERR_INVALID_ARG;
   pl.kind = choose_path(d);
-  if (pl.kind == PathKind::kNone) return GDATTN_ERR_UNSUPPORTED;
+  if (pl.kind == PathKind::kNone || (fp8 && pl.kind != PathKind::kTcPair))
+    return GDATTN_ERR_UNSUPPORTED;
   const int nsm = sm_count();
   if (nsm <= 0) return GDATTN_ERR_CUDA;
   int per_sm = 1, min_tokens = 64;
@@ -220,6 +228,14 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
     pl.align = TcConfig::TILE;
     pl.units_per_seq = d->n_kv_heads;
     pl.heads_per_unit = TcConfig::G;
+  } else if (fp8) {
+    per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_fp8_decode_kernel),
+                                  TcPairFp8Config::kThreads, TcPairFp8Config::SMEM,
+                                  query_tc_pair_fp8);
+    min_tokens = 2 * TcPairFp8Config::TILE;
+    pl.align = TcPairFp8Config::TILE;
+    pl.units_per_seq = d->n_kv_heads;
+    pl.heads_per_unit = TcPairFp8Config::G;
   } else {
     per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_decode_kernel),
                                   TcPairConfig::kThreads, TcPairConfig::SMEM, query_tc_pair);
@@ -309,19 +325,36 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// K or V cache [B][C][Hkv][D] bf16 as a 4-D tensor map {D, Hkv, C, B} read in
-// 64-d x 1-head x 64-token boxes with 128-byte swizzle.
+// K or V cache [B][C][Hkv][D] as a 4-D tensor map {D, Hkv, C, B} read in
+// 128-byte x 1-head x 64-token boxes with 128-byte swizzle: 64 bf16 elements,
+// or 128 e4m3 codes (fp8), per box row.
 bool encode_cache_map(EncodeTiledFn enc, CUtensorMap *map, const void *base, int32_t D,
-                      int32_t Hkv, int32_t C, int32_t batch, int64_t bstride, uint32_t tile) {
+                      int32_t Hkv, int32_t C, int32_t batch, int64_t bstride, uint32_t tile,
+                      bool fp8 = false) {
+  const cuuint64_t esz = fp8 ? 1 : 2;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv),
                               static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(batch)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2,
-                                 static_cast<cuuint64_t>(Hkv) * D * 2,
-                                 static_cast<cuuint64_t>(bstride) * 2};
-  const cuuint32_t box[4] = {64, 1, tile, 1};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * esz,
+                                 static_cast<cuuint64_t>(Hkv) * D * esz,
+                                 static_cast<cuuint64_t>(bstride) * esz};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / esz), 1, tile, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+             const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// q [B * Hq][D] bf16 as a 2-D tensor map read in whole-row boxes of `rows`
+// rows, unswizzled (row-major in shared memory).
+bool encode_q_rows_map(EncodeTiledFn enc, CUtensorMap *map, const void *q, int32_t D,
+                       int64_t total_rows, uint32_t rows) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(total_rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(D), rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(q), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -483,6 +516,60 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
   return GDATTN_OK;
 }
 
+// Enqueues the fp8-cache pair kernel (it merges split units itself).
+gdattn_status enqueue_decode_fp8(const LayerPlan &pl, const void *q, const void *k_codes,
+                                 const void *v_codes, const float *k_scale, const float *v_scale,
+                                 const int32_t *seqlens, int32_t batch,
+                                 const gdattn_layer_desc *desc, void *out, float *lse,
+                                 uint8_t *ws, cudaStream_t stream) {
+  const int32_t D = desc->head_dim;
+  const int32_t Hkv = desc->n_kv_heads;
+  const int64_t bstride = desc->cache_batch_stride != 0
+                              ? desc->cache_batch_stride
+                              : static_cast<int64_t>(desc->cache_capacity) * Hkv * D;
+  const float log2e = 1.4426950408889634f;
+  EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return GDATTN_ERR_CUDA;
+  CUtensorMap kmap, vmap, qmap;
+  if (!encode_cache_map(enc, &kmap, k_codes, D, Hkv, desc->cache_capacity, batch, bstride,
+                        TcPairFp8Config::TILE, true) ||
+      !encode_cache_map(enc, &vmap, v_codes, D, Hkv, desc->cache_capacity, batch, bstride,
+                        TcPairFp8Config::TILE, true) ||
+      !encode_q_rows_map(enc, &qmap, q, D, static_cast<int64_t>(batch) * desc->n_q_heads,
+                         TcPairFp8Config::G))
+    return GDATTN_ERR_CUDA;
+  TcParams tp;
+  tp.out = static_cast<uint16_t *>(out);
+  tp.lse = lse;
+  tp.ws_o = reinterpret_cast<float *>(ws + pl.off_o);
+  tp.ws_lse = reinterpret_cast<float *>(ws + pl.off_lse);
+  tp.status = reinterpret_cast<uint32_t *>(ws);
+  tp.counters = reinterpret_cast<uint32_t *>(ws + pl.off_cnt);
+  tp.epochs = reinterpret_cast<uint32_t *>(ws + pl.off_epoch);
+  tp.merge_in_kernel = 1;
+  tp.split_k = pl.split_k;
+  tp.geo.seqlens = seqlens;
+  tp.geo.batch = batch;
+  tp.geo.units_per_seq = pl.units_per_seq;
+  tp.geo.window = desc->window;
+  tp.geo.capacity = desc->cache_capacity;
+  tp.geo.nchunks = pl.grid;
+  tp.geo.align = pl.align;
+  tp.n_q_heads = desc->n_q_heads;
+  tp.qscale = desc->softcap > 0.f ? desc->scale / desc->softcap : desc->scale * log2e;
+  tp.post = desc->softcap > 0.f ? desc->softcap * log2e : 0.f;
+  Fp8Scales sc;
+  sc.k_scale = k_scale;
+  sc.v_scale = v_scale;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = launch_config(dim3(pl.grid), TcPairFp8Config::kThreads,
+                                         TcPairFp8Config::SMEM, stream, attr);
+  return cudaLaunchKernelEx(&cfg, tc_pair_fp8_decode_kernel, kmap, vmap, qmap, tp, sc) ==
+                 cudaSuccess
+             ? GDATTN_OK
+             : GDATTN_ERR_CUDA;
+}
+
 // -------------------------------------------------- fixed scratch (no alloc)
 constexpr int kMaxDevices = 64;
 
@@ -593,6 +680,34 @@ gdattn_status gdattn_decode_append(const void *q, const void *k_new, const void 
   return enqueue_decode(pl, q, k_cache, v_cache, seqlens, batch, desc, out, lse,
                         static_cast<uint8_t *>(workspace), static_cast<cudaStream_t>(stream),
                         k_new, v_new);
+}
+
+gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *v_codes,
+                                const float *k_scale, const float *v_scale,
+                                const int32_t *seqlens, int32_t batch, int32_t max_seqlen,
+                                const gdattn_layer_desc *desc, void *out, float *lse,
+                                void *workspace, size_t workspace_bytes, void *stream) {
+  if (q == nullptr || k_codes == nullptr || v_codes == nullptr || k_scale == nullptr ||
+      v_scale == nullptr || seqlens == nullptr || out == nullptr || desc == nullptr)
+    return GDATTN_ERR_INVALID_ARG;
+  gdattn_status st = check_desc(desc);
+  if (st != GDATTN_OK) return st;
+  if (batch <= 0 || max_seqlen <= 0) return GDATTN_ERR_INVALID_ARG;
+  if (choose_path(desc) != PathKind::kTcPair) return GDATTN_ERR_UNSUPPORTED;
+  if (desc->cache_batch_stride % 16 != 0) return GDATTN_ERR_MISALIGNED;  // TMA strides, bytes
+  if (!aligned16(q) || !aligned16(k_codes) || !aligned16(v_codes) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return GDATTN_ERR_MISALIGNED;
+  if (workspace == nullptr) return GDATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GDATTN_ERR_MISALIGNED;
+  LayerPlan pl;
+  st = make_plan(batch, max_seqlen, desc, pl, true);
+  if (st != GDATTN_OK) return st;
+  if (workspace_bytes < pl.bytes) return GDATTN_ERR_WORKSPACE;
+  return enqueue_decode_fp8(pl, q, k_codes, v_codes, k_scale, v_scale, seqlens, batch, desc, out,
+                            lse, static_cast<uint8_t *>(workspace),
+                            static_cast<cudaStream_t>(stream));
 }
 
 gdattn_status gdattn_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,

@@ -103,6 +103,168 @@ __device__ __forceinline__ uint32_t sw128_offset(int n, int t) {
   return static_cast<uint32_t>(n * 128 + ((((t >> 3) ^ (n & 7)) << 4) | ((t & 7) << 1)));
 }
 
+// One warp, when the planner saw an impossible sequence length (L < 1, or a
+// range longer than the cache): flag it in the status word and give every
+// sequence that attends nothing a zero output and LSE -inf.
+template <int D>
+__device__ __forceinline__ void report_bad_seqlens(const TcParams &p, int lane) {
+  grid_dependency_wait();
+  if (lane == 0) atomicOr(p.status, kStatusSeqlen);
+  for (int32_t b = 0; b < p.geo.batch; ++b) {
+    bool dummy = false;
+    if (attended_count(__ldg(p.geo.seqlens + b), p.geo.window, p.geo.capacity, dummy) != 0)
+      continue;
+    for (int i = lane; i < p.n_q_heads * D; i += 32)
+      p.out[static_cast<int64_t>(b) * p.n_q_heads * D + i] = 0;
+    if (p.lse != nullptr)
+      for (int i = lane; i < p.n_q_heads; i += 32)
+        p.lse[static_cast<int64_t>(b) * p.n_q_heads + i] = -INFINITY;
+  }
+}
+
+// Warp 7 of a pair kernel: counts split parts and merges them (see the file
+// comment).  Shared by the bf16 and fp8 pair kernels, whose partial layouts
+// are the same: normalised O [G][D] and LSE [G] per part.
+template <int G, int D>
+__device__ __forceinline__ void pair_merge_warp(const TcParams &p, const ChunkPlan *plan, int c,
+                                                int lane, int32_t split_k, bool usplit,
+                                                bool merger, uint64_t *tg_o, uint64_t *tg_lse,
+                                                const float *part_o, const float *part_lse) {
+  // -------------------------------------------------- part count, merge
+  // Segment by segment in the softmax warps' order: after a partial is
+  // stored (barrier 2), count it with one acq_rel atomic; the CTA whose count
+  // completes the unit merges all of its parts (lane c takes float4 columns
+  // c, c + 32, c + 64, c + 96) and resets the counter.  Parts are counted
+  // after a failed wait too, so the counters always return to zero.
+  if (p.merge_in_kernel) {
+    grid_dependency_wait();  // counters, workspace and outputs
+    // Count one part of unit `unit` (parts in slots slot0 .. slot0 + np - 1);
+    // the last one merges.
+    auto count_and_merge = [&](int32_t unit, int32_t b, int32_t x, int64_t slot0, int32_t np) {
+      uint32_t done = 0;
+      if (lane == 0) done = atomic_add_acq_rel_gpu(p.counters + unit, 1u);
+      done = __shfl_sync(0xffffffffu, done, 0);
+      __syncwarp();  // lane 0's acquire before every lane's reads
+      if (done != static_cast<uint32_t>(np - 1)) return;
+      if (lane == 0) p.counters[unit] = 0u;
+      constexpr int NC = G * D / 4 / 32;  // float4 columns per lane
+      const float *o_col[NC];
+      const float *l_col[NC];
+#pragma unroll
+      for (int k = 0; k < NC; ++k) {
+        const int e = lane + 32 * k, h = e / (D / 4), d = (e % (D / 4)) * 4;
+        o_col[k] = p.ws_o + (slot0 * G + h) * D + d;
+        l_col[k] = p.ws_lse + slot0 * G + h;
+      }
+      float4 res[NC];
+      float m[NC], z[NC];
+      merge_columns<NC, 4>(o_col, l_col, G * D, G, np, true, res, m, z);
+#pragma unroll
+      for (int k = 0; k < NC; ++k) {
+        const int e = lane + 32 * k, h = e / (D / 4), d = (e % (D / 4)) * 4;
+        const int64_t orow = static_cast<int64_t>(b) * p.n_q_heads + x * G + h;
+        store_bf16x4(p.out + orow * D + d, res[k]);
+        if (d == 0 && p.lse != nullptr)
+          p.lse[orow] = (m[k] == -INFINITY) ? -INFINITY : m[k] + logf(z[k]);
+      }
+    };
+    if (usplit) {
+      // Part r of unit c / k sits in slot (c / k) * k + unit + r.
+      const int32_t unit = c / split_k, crank = c % split_k;
+      const int32_t b = unit / p.geo.units_per_seq, x = unit - b * p.geo.units_per_seq;
+      const int64_t slot0 = static_cast<int64_t>(unit) * split_k + unit;
+      const bool has_part = plan->cs < plan->ce;
+      uint32_t tag = 0;
+      if (lane == 0) tag = next_tag(__ldcg(p.epochs + unit));
+      tag = __shfl_sync(0xffffffffu, tag, 0);
+      if (!merger) {
+        if (!has_part) {  // an empty part: LSE -inf
+          uint64_t *dst = tg_o + (slot0 + crank) * G * D;
+          for (int e = lane; e < G * D; e += 32) st_tagged(dst + e, 0.f, tag);
+          if (lane < G) st_tagged(tg_lse + (slot0 + crank) * G + lane, -INFINITY, tag);
+        }
+      } else {
+        // Lane l merges elements [16 l, 16 l + 16) of the unit's G x D outputs.
+        constexpr int PER = G * D / 32;
+        static_assert(PER == 16 && D % PER == 0, "lane mapping");
+        const int h = (PER * lane) / D, d0 = (PER * lane) % D;
+        float m = -INFINITY, z = 0.f, acc[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+        auto fold = [&](float lse_r, const float (&o)[PER]) {
+          if (lse_r == -INFINITY) return;  // an empty part: weight 0
+          const float mn = fmaxf(m, lse_r);
+          const float r_old = (m == -INFINITY) ? 0.f : __expf(m - mn);
+          const float w = __expf(lse_r - mn);
+          z = z * r_old + w;
+#pragma unroll
+          for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, o[e], acc[e] * r_old);
+          m = mn;
+        };
+        for (int32_t r = 0; r + 1 < split_k; ++r) {
+          uint64_t *src = tg_o + ((slot0 + r) * G + h) * D + d0;
+          uint64_t *lsrc = tg_lse + (slot0 + r) * G + h;
+          uint64_t wv[PER], wl = 0;
+          const long long t0 = clock64();
+          while (true) {
+#pragma unroll
+            for (int e = 0; e < PER; e += 2) ld_tagged2(src + e, wv[e], wv[e + 1]);
+            wl = ld_u64_volatile(lsrc);
+            bool ready = tag_of(wl) == tag;
+#pragma unroll
+            for (int e = 0; e < PER; ++e) ready &= tag_of(wv[e]) == tag;
+            if (__all_sync(0xffffffffu, ready)) break;
+            if (clock64() - t0 > kWaitLimitCycles) {
+              if (lane == 0) atomicOr(p.status, kStatusTimeout);
+              break;
+            }
+          }
+          float o[PER];
+#pragma unroll
+          for (int e = 0; e < PER; ++e) o[e] = payload_of(wv[e]);
+          fold(payload_of(wl), o);
+          // Clear what was consumed, so no later call can mistake it for fresh.
+#pragma unroll
+          for (int e = 0; e < PER; ++e) st_u64_volatile(src + e, 0ull);
+          if ((lane & (D / PER - 1)) == 0) st_u64_volatile(lsrc, 0ull);
+        }
+        if (has_part) {
+          named_bar_sync(2, 160);  // the softmax warps left the own part in shared memory
+          float o[PER];
+#pragma unroll
+          for (int e = 0; e < PER; ++e) o[e] = part_o[h * D + d0 + e];
+          fold(part_lse[h], o);
+        }
+        const float inv_z = (m == -INFINITY) ? 0.f : __fdividef(1.f, z);
+        const int64_t orow = static_cast<int64_t>(b) * p.n_q_heads + x * G + h;
+        uint16_t *dst = p.out + orow * D + d0;
+#pragma unroll
+        for (int e = 0; e < PER; e += 8) {
+          uint4 pk;
+          pk.x = pack_bf16x2(acc[e] * inv_z, acc[e + 1] * inv_z);
+          pk.y = pack_bf16x2(acc[e + 2] * inv_z, acc[e + 3] * inv_z);
+          pk.z = pack_bf16x2(acc[e + 4] * inv_z, acc[e + 5] * inv_z);
+          pk.w = pack_bf16x2(acc[e + 6] * inv_z, acc[e + 7] * inv_z);
+          *reinterpret_cast<uint4 *>(dst + e) = pk;
+        }
+        if (d0 == 0 && p.lse != nullptr) p.lse[orow] = (m == -INFINITY) ? -INFINITY : m + logf(z);
+        if (lane == 0) p.epochs[unit] = tag;  // every part of this call has been read
+      }
+    } else {
+      SegmentIter sit;
+      sit.init(p.geo, *plan);
+      Segment sg;
+      while (sit.next(sg)) {
+        if (sg.whole()) continue;
+        named_bar_sync(2, 160);
+        int32_t cf, cl;
+        unit_chunks(sg.unit_start, sg.n, plan->chunk, cf, cl);
+        count_and_merge(sg.unit, sg.b, sg.x, static_cast<int64_t>(cf) + sg.unit, cl - cf + 1);
+      }
+    }
+  }
+}
+
 template <bool APPEND>
 __device__ __forceinline__ void tc_pair_decode_body(const CUtensorMap &kmap,
                                                     const CUtensorMap &vmap,
@@ -196,20 +358,7 @@ __device__ __forceinline__ void tc_pair_decode_body(const CUtensorMap &kmap,
   tc_fence_after();
   const uint32_t tmem = *tmem_base_smem;
 
-  if (c == 0 && warp == 2 && plan->bad) {
-    grid_dependency_wait();
-    if (lane == 0) atomicOr(p.status, kStatusSeqlen);
-    for (int32_t b = 0; b < p.geo.batch; ++b) {
-      bool dummy = false;
-      if (attended_count(__ldg(p.geo.seqlens + b), p.geo.window, p.geo.capacity, dummy) != 0)
-        continue;
-      for (int i = lane; i < p.n_q_heads * D; i += 32)
-        p.out[static_cast<int64_t>(b) * p.n_q_heads * D + i] = 0;
-      if (p.lse != nullptr)
-        for (int i = lane; i < p.n_q_heads; i += 32)
-          p.lse[static_cast<int64_t>(b) * p.n_q_heads + i] = -INFINITY;
-    }
-  }
+  if (c == 0 && warp == 2 && plan->bad) report_bad_seqlens<D>(p, lane);
 
   const int32_t C = p.geo.capacity;
 
@@ -396,139 +545,8 @@ __device__ __forceinline__ void tc_pair_decode_body(const CUtensorMap &kmap,
     volatile int no_abort = 0;
     mbar_wait(&drain[1], 0, &no_abort, p.status);
   } else if (warp == 7) {
-    // -------------------------------------------------- part count, merge
-    // Segment by segment in the softmax warps' order: after a partial is
-    // stored (barrier 2), count it with one acq_rel atomic; the CTA whose count
-    // completes the unit merges all of its parts (lane c takes float4 columns
-    // c, c + 32, c + 64, c + 96) and resets the counter.  Parts are counted
-    // after a failed wait too, so the counters always return to zero.
-    if (p.merge_in_kernel) {
-      grid_dependency_wait();  // counters, workspace and outputs
-      // Count one part of unit `unit` (parts in slots slot0 .. slot0 + np - 1);
-      // the last one merges.
-      auto count_and_merge = [&](int32_t unit, int32_t b, int32_t x, int64_t slot0, int32_t np) {
-        uint32_t done = 0;
-        if (lane == 0) done = atomic_add_acq_rel_gpu(p.counters + unit, 1u);
-        done = __shfl_sync(0xffffffffu, done, 0);
-        __syncwarp();  // lane 0's acquire before every lane's reads
-        if (done != static_cast<uint32_t>(np - 1)) return;
-        if (lane == 0) p.counters[unit] = 0u;
-        constexpr int NC = G * D / 4 / 32;  // float4 columns per lane
-        const float *o_col[NC];
-        const float *l_col[NC];
-#pragma unroll
-        for (int k = 0; k < NC; ++k) {
-          const int e = lane + 32 * k, h = e / (D / 4), d = (e % (D / 4)) * 4;
-          o_col[k] = p.ws_o + (slot0 * G + h) * D + d;
-          l_col[k] = p.ws_lse + slot0 * G + h;
-        }
-        float4 res[NC];
-        float m[NC], z[NC];
-        merge_columns<NC, 4>(o_col, l_col, G * D, G, np, true, res, m, z);
-#pragma unroll
-        for (int k = 0; k < NC; ++k) {
-          const int e = lane + 32 * k, h = e / (D / 4), d = (e % (D / 4)) * 4;
-          const int64_t orow = static_cast<int64_t>(b) * p.n_q_heads + x * G + h;
-          store_bf16x4(p.out + orow * D + d, res[k]);
-          if (d == 0 && p.lse != nullptr)
-            p.lse[orow] = (m[k] == -INFINITY) ? -INFINITY : m[k] + logf(z[k]);
-        }
-      };
-      if (usplit) {
-        // Part r of unit c / k sits in slot (c / k) * k + unit + r.
-        const int32_t unit = c / split_k;
-        const int32_t b = unit / p.geo.units_per_seq, x = unit - b * p.geo.units_per_seq;
-        const int64_t slot0 = static_cast<int64_t>(unit) * split_k + unit;
-        const bool has_part = plan->cs < plan->ce;
-        uint32_t tag = 0;
-        if (lane == 0) tag = next_tag(__ldcg(p.epochs + unit));
-        tag = __shfl_sync(0xffffffffu, tag, 0);
-        if (!merger) {
-          if (!has_part) {  // an empty part: LSE -inf
-            uint64_t *dst = tg_o + (slot0 + crank) * G * D;
-            for (int e = lane; e < G * D; e += 32) st_tagged(dst + e, 0.f, tag);
-            if (lane < G) st_tagged(tg_lse + (slot0 + crank) * G + lane, -INFINITY, tag);
-          }
-        } else {
-          // Lane l merges elements [16 l, 16 l + 16) of the unit's G x D outputs.
-          constexpr int PER = G * D / 32;
-          static_assert(PER == 16 && D % PER == 0, "lane mapping");
-          const int h = (PER * lane) / D, d0 = (PER * lane) % D;
-          float m = -INFINITY, z = 0.f, acc[PER];
-#pragma unroll
-          for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-          auto fold = [&](float lse_r, const float (&o)[PER]) {
-            if (lse_r == -INFINITY) return;  // an empty part: weight 0
-            const float mn = fmaxf(m, lse_r);
-            const float r_old = (m == -INFINITY) ? 0.f : __expf(m - mn);
-            const float w = __expf(lse_r - mn);
-            z = z * r_old + w;
-#pragma unroll
-            for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, o[e], acc[e] * r_old);
-            m = mn;
-          };
-          for (int32_t r = 0; r + 1 < split_k; ++r) {
-            uint64_t *src = tg_o + ((slot0 + r) * G + h) * D + d0;
-            uint64_t *lsrc = tg_lse + (slot0 + r) * G + h;
-            uint64_t wv[PER], wl = 0;
-            const long long t0 = clock64();
-            while (true) {
-#pragma unroll
-              for (int e = 0; e < PER; e += 2) ld_tagged2(src + e, wv[e], wv[e + 1]);
-              wl = ld_u64_volatile(lsrc);
-              bool ready = tag_of(wl) == tag;
-#pragma unroll
-              for (int e = 0; e < PER; ++e) ready &= tag_of(wv[e]) == tag;
-              if (__all_sync(0xffffffffu, ready)) break;
-              if (clock64() - t0 > kWaitLimitCycles) {
-                if (lane == 0) atomicOr(p.status, kStatusTimeout);
-                break;
-              }
-            }
-            float o[PER];
-#pragma unroll
-            for (int e = 0; e < PER; ++e) o[e] = payload_of(wv[e]);
-            fold(payload_of(wl), o);
-            // Clear what was consumed, so no later call can mistake it for fresh.
-#pragma unroll
-            for (int e = 0; e < PER; ++e) st_u64_volatile(src + e, 0ull);
-            if ((lane & (D / PER - 1)) == 0) st_u64_volatile(lsrc, 0ull);
-          }
-          if (has_part) {
-            named_bar_sync(2, 160);  // the softmax warps left the own part in shared memory
-            float o[PER];
-#pragma unroll
-            for (int e = 0; e < PER; ++e) o[e] = part_o[h * D + d0 + e];
-            fold(part_lse[h], o);
-          }
-          const float inv_z = (m == -INFINITY) ? 0.f : __fdividef(1.f, z);
-          const int64_t orow = static_cast<int64_t>(b) * p.n_q_heads + x * G + h;
-          uint16_t *dst = p.out + orow * D + d0;
-#pragma unroll
-          for (int e = 0; e < PER; e += 8) {
-            uint4 pk;
-            pk.x = pack_bf16x2(acc[e] * inv_z, acc[e + 1] * inv_z);
-            pk.y = pack_bf16x2(acc[e + 2] * inv_z, acc[e + 3] * inv_z);
-            pk.z = pack_bf16x2(acc[e + 4] * inv_z, acc[e + 5] * inv_z);
-            pk.w = pack_bf16x2(acc[e + 6] * inv_z, acc[e + 7] * inv_z);
-            *reinterpret_cast<uint4 *>(dst + e) = pk;
-          }
-          if (d0 == 0 && p.lse != nullptr) p.lse[orow] = (m == -INFINITY) ? -INFINITY : m + logf(z);
-          if (lane == 0) p.epochs[unit] = tag;  // every part of this call has been read
-        }
-      } else {
-        SegmentIter sit;
-        sit.init(p.geo, *plan);
-        Segment sg;
-        while (sit.next(sg)) {
-          if (sg.whole()) continue;
-          named_bar_sync(2, 160);
-          int32_t cf, cl;
-          unit_chunks(sg.unit_start, sg.n, plan->chunk, cf, cl);
-          count_and_merge(sg.unit, sg.b, sg.x, static_cast<int64_t>(cf) + sg.unit, cl - cf + 1);
-        }
-      }
-    }
+    pair_merge_warp<G, D>(p, plan, c, lane, split_k, usplit, merger, tg_o, tg_lse, part_o,
+                          part_lse);
   } else if (warp == 8) {
     // ---------------------------------------------------------- V loads
     // Same schedule and dependency rule as the K loads (warp 0); a V tile is

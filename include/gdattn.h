@@ -201,6 +201,40 @@ gdattn_status gdattn_decode_append(const void *q, const void *k_new, const void 
                                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * gdattn_decode over an fp8 cache: every cache row (one token of one KV head)
+ * holds D codes in OCP FP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits; no infinities, S.1111.111 is NaN) and one fp32 scale, and its
+ * values are code_d * scale.  The quantized rotating cache is mlx-lm's
+ * RotatingQuantizedKVCache idea ("Gemma 4 12B", serviceability join, item 6);
+ * BF16 queries over an FP8 KV cache at a sliding-window boundary are what
+ * FlashInfer's trtllm kernel got wrong on B200 (same record, item 2).  The
+ * computation is the definition at the top of this file with those values for
+ * K and V; q, out and lse stay bf16 / fp32.
+ *
+ *  k_codes  e4m3 bytes, device, read only; sequence b at k_codes +
+ *           b*cache_batch_stride bytes, laid out [C][Hkv][D] (token-major)
+ *  v_codes  e4m3 bytes, same layout
+ *  k_scale  fp32 [batch][Hkv][C], device, read only: the scale of K row
+ *           (b, kv, slot), contiguous over the slots (4-byte aligned)
+ *  v_scale  fp32 [batch][Hkv][C], the V rows' scales
+ *  other arguments as gdattn_decode.  cache_batch_stride counts bytes here and
+ *  must be a multiple of 16 (0 = C*Hkv*D).  The workspace is sized by
+ *  gdattn_workspace_size for the same desc.
+ *
+ * Supported geometry: G == 2, D == 256, separate V (the sliding layers), any
+ * Hkv; others return GDATTN_ERR_UNSUPPORTED.  Scales must be finite; a zero
+ * scale makes its row zero.  The kernel multiplies fp8 codes on the tensor
+ * cores against q and the softmax weights each split into three e4m3 pieces;
+ * the result matches the float64 definition to about 2^-12 relative to the
+ * largest weight (see the kernel source for the error bound).
+ */
+gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *v_codes,
+                                const float *k_scale, const float *v_scale,
+                                const int32_t *seqlens, int32_t batch, int32_t max_seqlen,
+                                const gdattn_layer_desc *desc, void *out, float *lse,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * gdattn_decode without a caller workspace.  A library addition: the paper
  * has no counterpart; it computes exactly what gdattn_decode computes.
  *

@@ -28,12 +28,13 @@ def lib():
 
 def declared_functions():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"\b(gdattn_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(gdattn_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_api():
     names = declared_functions()
-    for n in ("gdattn_decode", "gdattn_combine", "gdattn_workspace_size", "gdattn_workspace_init",
+    for n in ("gdattn_decode", "gdattn_decode_fp8", "gdattn_combine", "gdattn_workspace_size",
+              "gdattn_workspace_init",
               "gdattn_plan_splits", "gdattn_plan_launches",
               "gdattn_check_device_status", "gdattn_status_string", "gdattn_version"):
         assert n in names
@@ -187,3 +188,46 @@ def test_decode_append_host_checks(lib):
     shared = good_desc(n_q_heads=16, n_kv_heads=1, head_dim=512, window=0, kv_shared=True)
     assert app(shared, v=None) == binding.GDATTN_ERR_INVALID_ARG     # K = V: no v_new
     assert app(shared, v=None, v_new=None, q=None) == binding.GDATTN_ERR_INVALID_ARG
+
+
+def fp8_call(desc, q=A, kc=A, vc=A, ks=A, vs=A, seqlens=A, batch=1, max_seqlen=8, out=A, lse=A,
+             ws=A, ws_bytes=1 << 20):
+    return binding.decode_fp8_raw(q, kc, vc, ks, vs, seqlens, batch, max_seqlen, desc, out, lse,
+                                  ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(q=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(kc=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(vc=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(ks=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(vs=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(seqlens=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(out=None), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(batch=0), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(max_seqlen=0), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(q=A + 8), binding.GDATTN_ERR_MISALIGNED),
+    (dict(kc=A + 1), binding.GDATTN_ERR_MISALIGNED),
+    (dict(vc=A + 8), binding.GDATTN_ERR_MISALIGNED),
+    (dict(ks=A + 2), binding.GDATTN_ERR_MISALIGNED),
+    (dict(vs=A + 1), binding.GDATTN_ERR_MISALIGNED),
+    (dict(out=A + 8), binding.GDATTN_ERR_MISALIGNED),
+    (dict(lse=A + 2), binding.GDATTN_ERR_MISALIGNED),
+    (dict(ws=None), binding.GDATTN_ERR_WORKSPACE),
+    (dict(ws=A + 8), binding.GDATTN_ERR_MISALIGNED),
+])
+def test_decode_fp8_rejects_bad_pointers(lib, case, expect):
+    """gdattn_decode_fp8: the codes need 16-byte alignment (TMA), the scales 4."""
+    assert fp8_call(good_desc(), **case) == expect
+
+
+@pytest.mark.parametrize("desc_kw,expect", [
+    (dict(n_q_heads=16, n_kv_heads=1, head_dim=512, window=0, kv_shared=True),
+     binding.GDATTN_ERR_UNSUPPORTED),                       # global geometry: bf16 only
+    (dict(n_q_heads=8, n_kv_heads=8), binding.GDATTN_ERR_UNSUPPORTED),  # G = 1
+    (dict(head_dim=512), binding.GDATTN_ERR_UNSUPPORTED),
+    (dict(n_q_heads=12), binding.GDATTN_ERR_INVALID_ARG),
+    (dict(cache_batch_stride=1024 * 8 * 256 + 8), binding.GDATTN_ERR_MISALIGNED),  # bytes % 16
+])
+def test_decode_fp8_rejects_bad_desc(lib, desc_kw, expect):
+    assert fp8_call(good_desc(**desc_kw)) == expect
