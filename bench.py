@@ -490,6 +490,50 @@ def run_ours(args, world, rank, local):
         if st != binding.GDATTN_OK:
             raise binding.GdattnError(st, "device status after the append step")
 
+    # ---- fp8 KV cache (gdattn_decode_fp8) on the sliding layers: the same
+    # geometry and lengths with e4m3 codes and per-row scales; the global layers
+    # (no fp8 kernel) stay bf16 in the mixed step.
+    fp8_layers = {}
+    for i in sliding_idx:
+        sp = w.layers[i]
+        inp8 = workloads.fp8_layer_inputs(sp, w.batch, w.seqlens(),
+                                          w.seed * 1000 + 500 + i + rank_seed_offset(rank),
+                                          device=device)
+        fp8_layers[i] = dict(inp=inp8, desc=stack.layers[i]["desc"],
+                             ws=binding.alloc_workspace(w.batch, stack.max_seqlen,
+                                                        stack.layers[i]["desc"], device))
+
+    def launch_fp8(i):
+        f = fp8_layers[i]
+        x, ly = f["inp"], stack.layers[i]
+        binding.decode_fp8(x.q, x.k_codes, x.v_codes, x.k_scale, x.v_scale, x.seqlens, f["desc"],
+                           stack.max_seqlen, out=ly["out"], lse=ly["lse"], workspace=f["ws"],
+                           stream=stream)
+
+    def fp8_graph(indices):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            for i in indices:
+                launch_fp8(i) if i in fp8_layers else stack.launch(i, stream)
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                for i in indices:
+                    launch_fp8(i) if i in fp8_layers else stack.launch(i, stream)
+        return g
+
+    ms_fp8_sl = ms_fp8_step = None
+    if fp8_layers:
+        g_f8 = fp8_graph(sliding_idx)
+        g_f8_step = fp8_graph(all_idx)
+        barrier()
+        ms_fp8_sl = max_over_ranks(time_graph(g_f8, stream, args.steps, 3), world)
+        ms_fp8_step = max_over_ranks(time_graph(g_f8_step, stream, args.steps, 3), world)
+        for f in fp8_layers.values():
+            st = binding.check_device_status(f["ws"], stream)
+            if st != binding.GDATTN_OK:
+                raise binding.GdattnError(st, "device status after the fp8 step")
+        del g_f8, g_f8_step
+
     # ---- CPU baseline: the oracle over the whole step (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
@@ -544,6 +588,24 @@ def run_ours(args, world, rank, local):
     if ms_sl:
         per_type["sliding"] = {"achieved_gbs": roof["achieved"], "frac": roof["frac"],
                                "us_per_layer": roof["us_per_launch"]}
+    fp8_summary = None
+    if ms_fp8_sl:
+        seq = w.seqlens().tolist()
+        b8 = sum(accounting.layer_fp8_kv_bytes(w.layers[i], seq) for i in sliding_idx)
+        step8 = b8 + gl_bytes
+        ach8 = b8 / (ms_fp8_sl * 1e-3) / 1e9
+        fp8_summary = {
+            "kernel": "tc_pair_fp8_decode_kernel (tcgen05 kind::f8f6f4; e4m3 codes, per-row "
+                      "fp32 scales)",
+            "sliding_us_per_layer": ms_fp8_sl / len(sliding_idx) * 1e3,
+            "sliding_achieved_gbs": ach8, "sliding_frac": ach8 / peak, "peak_kind": peak_kind,
+            "sliding_bytes_per_launch": b8 / len(sliding_idx),
+            "traffic": traffic_for("fp8_sliding"),
+            "step_us": ms_fp8_step * 1e3, "step_kv_bytes": step8,
+            "step_gbs": job_gbs(step8, ms_fp8_step, world),
+            "how": "the sliding layers' caches as e4m3 codes + one fp32 scale per row "
+                   "(gdattn_decode_fp8); the mixed step keeps the 8 global layers bf16; "
+                   "bytes = codes + scales actually read; CUDA graphs, device time"}
     line = {
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "us_per_step": ms_step * 1e3,
@@ -569,6 +631,7 @@ def run_ours(args, world, rank, local):
                    "how": "the same 48 layers through gdattn_decode_append: each layer's "
                           "current-token K/V rows written into their ring slots by the decode "
                           "kernels (CUDA graph, device time)"},
+        "fp8_kv": fp8_summary,
         "gpu_launches": stack.launches_per_step(all_idx) * args.steps,
         "clocks": clk,
     }

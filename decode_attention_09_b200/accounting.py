@@ -8,6 +8,8 @@ and split partials are overhead and are not counted.
 
 The per-token formula of the "Gemma 4 12B" record (KV GEOMETRY paragraph) counts
 K and V for every layer; ``count_shared_twice=True`` reproduces that figure.
+
+An fp8 cache row is ``head_dim`` one-byte e4m3 codes plus its 4-byte scale.
 """
 from __future__ import annotations
 
@@ -28,4 +30,19 @@ def attended_positions(spec, seqlen: int) -> int:
 def layer_kv_bytes(spec, seqlens) -> int:
     """Algorithmic KV bytes for one decode step of one layer over a batch."""
     per = kv_bytes_per_position(spec)
+    return sum(attended_positions(spec, int(L)) * per for L in seqlens)
+
+
+FP8_ROW_EXTRA = 4  # the fp32 scale stored with every fp8 cache row
+
+
+def fp8_kv_bytes_per_position(spec) -> int:
+    """fp8-cache bytes read for one attended position of one sequence in one layer."""
+    tensors = 1 if spec.kv_shared else 2
+    return spec.n_kv_heads * (spec.head_dim + FP8_ROW_EXTRA) * tensors
+
+
+def layer_fp8_kv_bytes(spec, seqlens) -> int:
+    """Algorithmic fp8-cache bytes (codes and row scales) for one decode step of one layer."""
+    per = fp8_kv_bytes_per_position(spec)
     return sum(attended_positions(spec, int(L)) * per for L in seqlens)

@@ -264,7 +264,7 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
   // with all units * k CTAs resident at once.  No CTA then straddles two units.
   pl.split_k = 1;
   if ((d->flags & GDATTN_FLAG_EVEN_UNITS) && d->split_ctas == 0 && pl.kind != PathKind::kCore) {
-    const int64_t tiles = (per_unit + 63) / 64;
+    const int64_t tiles = (per_unit + pl.align - 1) / pl.align;
     int64_t best = tiles;
     for (int64_t k = 2; k <= tiles && units * k <= cap && k <= 64; ++k) {
       const int64_t most = (tiles + k - 1) / k;

@@ -108,7 +108,8 @@ struct TcConfig {
 constexpr float kTau = 8.f;
 
 // Tiles of one CTA, in order, across its segments.
-struct TileIter {
+template <int TILE>
+struct TileIterT {
   SegmentIter seg_it;
   Segment seg;
   SlotRuns runs;
@@ -134,9 +135,9 @@ struct TileIter {
       first = true;
     }
     row = runs.start(run) + t0;
-    ntok = min(TcConfig::TILE, runs.len(run) - t0);
+    ntok = min(TILE, runs.len(run) - t0);
     newest = seg.lo + (run == 1 ? runs.len0 : 0) + t0 + ntok == seg.n;
-    t0 += TcConfig::TILE;
+    t0 += TILE;
     if (t0 >= runs.len(run)) {
       ++run;
       t0 = 0;
@@ -146,6 +147,8 @@ struct TileIter {
     return true;
   }
 };
+
+using TileIter = TileIterT<TcConfig::TILE>;
 
 // Reduce 16 per-lane values over the warp (op = max or sum): after it, lane l
 // holds the reduction for value index (l >> 1) & 15.

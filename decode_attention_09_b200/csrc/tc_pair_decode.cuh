@@ -265,6 +265,98 @@ __device__ __forceinline__ void pair_merge_warp(const TcParams &p, const ChunkPl
   }
 }
 
+// ------------------------------------------------- merging in the softmax
+// Helpers for a kernel whose softmax threads merge split parts themselves,
+// each for the output elements it computed, after its own last tile (the fp8
+// pair kernel: a merge warp kept alive through its main loop slowed the
+// merging CTA's whole pipeline there).
+
+// Running LSE merge of normalised parts for one output element (natural log).
+struct PartMerge {
+  float m = -INFINITY, z = 0.f, acc = 0.f;
+  __device__ __forceinline__ void add(float lse, float o) {
+    if (lse == -INFINITY) return;  // an empty part: weight 0
+    const float mn = fmaxf(m, lse);
+    const float r_old = (m == -INFINITY) ? 0.f : __expf(m - mn);
+    const float w = __expf(lse - mn);
+    z = z * r_old + w;
+    acc = fmaf(w, o, acc * r_old);
+    m = mn;
+  }
+  __device__ __forceinline__ float out() const {
+    return m == -INFINITY ? 0.f : __fdividef(acc, z);
+  }
+  __device__ __forceinline__ float lse() const { return m == -INFINITY ? -INFINITY : m + logf(z); }
+};
+
+// Payloads of N tagged words once each carries `tag`: all loads are issued
+// together, then the stragglers re-polled.  After kWaitLimitCycles (SM clock)
+// it latches kStatusTimeout in *status and returns what it has.
+template <int N>
+__device__ __forceinline__ void await_tagged(const uint64_t *const (&addr)[N], uint32_t tag,
+                                             float (&val)[N], uint32_t *status) {
+  uint64_t w[N];
+#pragma unroll
+  for (int e = 0; e < N; ++e) w[e] = ld_u64_volatile(addr[e]);
+  const long long t0 = clock64();
+  while (true) {
+    bool ready = true;
+#pragma unroll
+    for (int e = 0; e < N; ++e) ready &= tag_of(w[e]) == tag;
+    if (ready) break;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicOr(status, kStatusTimeout);
+      break;
+    }
+#pragma unroll
+    for (int e = 0; e < N; ++e)
+      if (tag_of(w[e]) != tag) w[e] = ld_u64_volatile(addr[e]);
+  }
+#pragma unroll
+  for (int e = 0; e < N; ++e) val[e] = payload_of(w[e]);
+}
+
+// The other parts of a tagged unit (all but the last, which merges): the
+// elements (head h[e], dim d[e]) of part r are tagged words at
+// tg_o[((slot0 + r) * G + h) * D + d], its LSEs at tg_lse[(slot0 + r) * G + h].
+// Folds parts 0 .. k-2 in part order into mg[], clearing the O words it read.
+template <int G, int D, int NE>
+__device__ __forceinline__ void merge_tagged_parts(uint64_t *tg_o, uint64_t *tg_lse,
+                                                   int64_t slot0, int32_t k, uint32_t tag,
+                                                   const int (&h)[NE], const int (&d)[NE],
+                                                   PartMerge (&mg)[NE], uint32_t *status) {
+  for (int32_t r = 0; r + 1 < k; ++r) {
+    const uint64_t *addr[2 * NE];
+    float v[2 * NE];
+#pragma unroll
+    for (int e = 0; e < NE; ++e) {
+      addr[e] = tg_o + ((slot0 + r) * G + h[e]) * D + d[e];
+      addr[NE + e] = tg_lse + (slot0 + r) * G + h[e];
+    }
+    await_tagged<2 * NE>(addr, tag, v, status);
+#pragma unroll
+    for (int e = 0; e < NE; ++e) {
+      mg[e].add(v[NE + e], v[e]);
+      st_u64_volatile(const_cast<uint64_t *>(addr[e]), 0ull);  // consumed: never mistaken later
+    }
+  }
+}
+
+// Counted merge of a unit whose parts are plain partials in slots slot0 ..
+// slot0 + np - 1 (normalised O [slot][G][D], LSE [slot][G]): the element
+// (h[e], d[e]) of every part, in part order.
+template <int G, int D, int NE>
+__device__ __forceinline__ void merge_counted_parts(const float *ws_o, const float *ws_lse,
+                                                    int64_t slot0, int32_t np,
+                                                    const int (&h)[NE], const int (&d)[NE],
+                                                    PartMerge (&mg)[NE]) {
+  for (int32_t r = 0; r < np; ++r)
+#pragma unroll
+    for (int e = 0; e < NE; ++e)
+      mg[e].add(__ldcg(ws_lse + (slot0 + r) * G + h[e]),
+                __ldcg(ws_o + ((slot0 + r) * G + h[e]) * D + d[e]));
+}
+
 template <bool APPEND>
 __device__ __forceinline__ void tc_pair_decode_body(const CUtensorMap &kmap,
                                                     const CUtensorMap &vmap,
