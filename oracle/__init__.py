@@ -41,6 +41,9 @@ class Oracle:
         lib.oracle_decode_fp8.restype = ctypes.c_int
         lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8, f64p]
         lib.oracle_e4m3_to_double.restype = ctypes.c_int
+        lib.oracle_decode_multi.argtypes = [u16p, u16p, u16p, i32p, i32, i32, i32, i32, i32, i32,
+                                            i64, i32, f64, f64, i32, f64p, f64p]
+        lib.oracle_decode_multi.restype = ctypes.c_int
         lib.oracle_combine.argtypes = [f64p, f64p, i32, i32, f64p, f64p]
         lib.oracle_combine.restype = None
         lib.oracle_version.restype = ctypes.c_int
@@ -187,6 +190,28 @@ class Oracle:
             out[i] = oo
             lse[i] = ll[0]
         return out.reshape(*lead, D), lse.reshape(lead)
+
+    def decode_multi(self, q, k, v, seqlens, window: int, softcap: float, scale: float):
+        """Multi-query decode: q bf16 [T,B,Hq,D], query t of sequence b at position
+        L_b - T + t, attending causally.  Returns (out [T,B,Hq,D], lse [T,B,Hq]) float64."""
+        qb, kb = self._bits(q), self._bits(k)
+        T, B, Hq, D = qb.shape
+        _, C, Hkv, Dk = kb.shape
+        assert Dk == D and kb.shape[0] == B
+        vb = self._bits(v) if v is not None else None
+        sl = np.ascontiguousarray(np.asarray(seqlens.cpu() if isinstance(seqlens, torch.Tensor)
+                                             else seqlens, dtype=np.int32))
+        out = np.zeros((T, B, Hq, D), dtype=np.float64)
+        lse = np.zeros((T, B, Hq), dtype=np.float64)
+        rc = self.lib.oracle_decode_multi(
+            self._ptr(qb, ctypes.c_uint16), self._ptr(kb, ctypes.c_uint16),
+            self._ptr(vb, ctypes.c_uint16) if vb is not None else None,
+            self._ptr(sl, ctypes.c_int32), T, B, Hq, Hkv, D, C, C * Hkv * D, int(window),
+            float(softcap), float(scale), 1 if vb is None else 0,
+            self._ptr(out, ctypes.c_double), self._ptr(lse, ctypes.c_double))
+        if rc != 0:
+            raise ValueError("oracle_decode_multi rejected its arguments")
+        return out, lse
 
     def decode_layer(self, inputs):
         """Convenience: run ``decode`` on a ``workloads.LayerInputs``."""

@@ -294,6 +294,50 @@ int oracle_decode_fp8(const uint16_t *q, const uint8_t *kc, const uint8_t *vc, c
 }
 
 /*
+ * Multi-query decode over a bf16 cache: T query tokens per sequence, the
+ * sequence's last T positions.  Query t of sequence b sits at position
+ * p = L_b - T + t and attends [max(0, p + 1 - window), p + 1) (window 0: [0, p + 1)),
+ * causally, as a speculative-decoding verify step does.  q: [T][B][Hq][D]; out:
+ * [T][B][Hq][D]; lse: [T][B][Hq].  Returns -1 when a query's range is empty, or
+ * reaches a position the ring no longer holds (older than L_b - C).
+ */
+int oracle_decode_multi(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        const int32_t *seqlens, int32_t T, int32_t B, int32_t Hq, int32_t Hkv,
+                        int32_t D, int32_t C, int64_t batch_stride, int32_t window, double softcap,
+                        double scale, int32_t kv_shared, double *out, double *lse) {
+  if (T < 1 || B < 0) return -1;
+  if (!kv_shared && v == NULL) return -1;
+  int32_t *lo = (int32_t *)malloc(sizeof(int32_t) * (size_t)(B > 0 ? B : 1));
+  int32_t *hi = (int32_t *)malloc(sizeof(int32_t) * (size_t)(B > 0 ? B : 1));
+  if (!lo || !hi) {
+    free(lo);
+    free(hi);
+    return -1;
+  }
+  row_source src = {0, k, v, NULL, NULL, NULL, NULL, batch_stride, Hkv, D, C, kv_shared};
+  int rc = 0;
+  for (int32_t t = 0; t < T && rc == 0; ++t) {
+    for (int32_t b = 0; b < B; ++b) {
+      const int32_t L = seqlens[b];
+      int32_t end = L - T + t + 1; /* one past this query's position */
+#if ORACLE_MUTATION == 13
+      end = L; /* every query sees all T new tokens (not causal) */
+#endif
+      const int32_t start = (window > 0 && end > window) ? end - window : 0;
+      lo[b] = start;
+      hi[b] = end;
+      if (end < 1 || start < L - C) rc = -1;
+    }
+    if (rc == 0)
+      rc = attend(q + (int64_t)t * B * Hq * D, B, Hq, lo, hi, softcap, scale, &src,
+                  out + (int64_t)t * B * Hq * D, lse + (int64_t)t * B * Hq);
+  }
+  free(lo);
+  free(hi);
+  return rc;
+}
+
+/*
  * Merge n partial results of one query head, each normalised over its own part
  * of the position range: LSE = log sum_s exp(LSE_s), out = sum_s exp(LSE_s - LSE) o_s.
  * Parts with LSE_s = -inf contribute nothing; if all are -inf the result is

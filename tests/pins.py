@@ -416,11 +416,76 @@ def pin_fp8_zero_scale_row(orc):
     _close(l[0], np.full(2, math.log(6)), 1e-12, "zero-scale rows lse")
 
 
+# --------------------------------------------------------------------------
+# Multi-query decode (T query tokens per sequence, causal)
+# --------------------------------------------------------------------------
+
+# (T, B, Hq, Hkv, D, C, seqlens, window, softcap, kv_shared)
+MULTI_CASES = [
+    (3, 2, 4, 2, 16, 12, [37, 12], 10, 0.0, False),  # ring wraps, C = w + T - 1
+    (4, 2, 16, 1, 32, 40, [40, 9], 0, 0.0, True),    # whole context, K = V
+    (2, 2, 4, 2, 8, 20, [20, 3], 0, 5.0, False),
+]
+
+
+def multi_inputs(i, case):
+    T, B, Hq, Hkv, D, C, sl, w, cap, shared = case
+    inp = workloads.random_case(4000 + i, B, Hq, Hkv, D, C, sl, window=w, softcap=cap,
+                                kv_shared=shared)
+    g = torch.Generator().manual_seed(4100 + i)
+    q = torch.randn((T, B, Hq, D), generator=g).to(torch.bfloat16)
+    return q, inp
+
+
+def pin_multi_brute_force(orc):
+    """Query t of a T-token step equals the numpy brute force at context length
+    L - (T - 1 - t): it attends causally up to its own position."""
+    for i, case in enumerate(MULTI_CASES):
+        T = case[0]
+        q, inp = multi_inputs(i, case)
+        s = inp.spec
+        o, l = orc.decode_multi(q, inp.k, inp.v, inp.seqlens, s.window, s.softcap, s.scale)
+        for t in range(T):
+            sl = inp.seqlens.numpy() - (T - 1 - t)
+            o2, l2 = brute_force(q[t], inp.k, inp.v, sl, s.window, s.softcap, s.scale)
+            _close(o[t], o2, 1e-12, f"multi brute force out, case {i} token {t}")
+            _close(l[t], l2, 1e-12, f"multi brute force lse, case {i} token {t}")
+
+
+def pin_multi_reduces_to_decode(orc):
+    """T = 1 is single-token decode, and the last of T tokens sees what a single
+    token at L sees (exactly)."""
+    q, inp = multi_inputs(0, MULTI_CASES[0])
+    s = inp.spec
+    o1, l1 = orc.decode_multi(q[-1:], inp.k, inp.v, inp.seqlens, s.window, s.softcap, s.scale)
+    o2, l2 = orc.decode(q[-1], inp.k, inp.v, inp.seqlens, s.window, s.softcap, s.scale)
+    _close(o1[0], o2, 0.0, "T=1 out")
+    _close(l1[0], l2, 0.0, "T=1 lse")
+    o3, l3 = orc.decode_multi(q, inp.k, inp.v, inp.seqlens, s.window, s.softcap, s.scale)
+    _close(o3[-1], o2, 0.0, "last token out")
+    _close(l3[-1], l2, 0.0, "last token lse")
+
+
+def pin_multi_ring_capacity(orc):
+    """A ring of C slots holds positions [L - C, L): with a window w, T tokens
+    need C >= w + T - 1, else the first token's oldest position is gone."""
+    q, inp = multi_inputs(0, MULTI_CASES[0])  # C = 12 = w + T - 1
+    s = inp.spec
+    orc.decode_multi(q, inp.k, inp.v, inp.seqlens, s.window, s.softcap, s.scale)
+    q4 = torch.cat([q, q[:1]], dim=0)  # T = 4 > C - w + 1
+    try:
+        orc.decode_multi(q4, inp.k, inp.v, inp.seqlens, s.window, s.softcap, s.scale)
+    except ValueError:
+        return
+    raise AssertionError("a query reaching an overwritten slot was accepted")
+
+
 ALL_PINS = [pin_brute_force, pin_sdpa, pin_window_covers_context, pin_cap_to_infinity,
             pin_identical_keys, pin_zero_query, pin_single_position, pin_two_positions,
             pin_softcap_bound, pin_sliding_ignores_old_positions, pin_ring_equals_linear,
             pin_split_recombine, pin_combine_closed_form, pin_separate_v, pin_e4m3_codes,
-            pin_fp8_equals_bf16_when_exact, pin_fp8_brute_force, pin_fp8_zero_scale_row]
+            pin_fp8_equals_bf16_when_exact, pin_fp8_brute_force, pin_fp8_zero_scale_row,
+            pin_multi_brute_force, pin_multi_reduces_to_decode, pin_multi_ring_capacity]
 
 
 def failing_pins(orc):

@@ -21,6 +21,7 @@ MUTATIONS = {
     10: "V rows scaled by the K scales",
     11: "row scale applied twice",
     12: "row scales read token-major",
+    13: "multi-query tokens not causal",
 }
 
 
