@@ -60,9 +60,11 @@ def measured_peak_gbs():
 
 
 def kernel_source_hash():
+    """Hash of the device code of the profiled kernels: every kernel lives in a
+    csrc/*.cuh header (api.cu holds the host-side launches)."""
     h = hashlib.sha256()
     for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh")):
+        if name.endswith(".cuh"):
             with open(os.path.join(CSRC, name), "rb") as f:
                 h.update(name.encode())
                 h.update(f.read())

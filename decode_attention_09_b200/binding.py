@@ -80,6 +80,12 @@ def lib() -> ctypes.CDLL:
             L.gdattn_decode_append.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, descp, vp, vp,
                                                vp, sz, vp]
             L.gdattn_decode_append.restype = ctypes.c_int
+        if hasattr(L, "gdattn_decode_multi"):
+            L.gdattn_multi_workspace_size.argtypes = [i32, i32, i32, descp]
+            L.gdattn_multi_workspace_size.restype = sz
+            L.gdattn_decode_multi.argtypes = [vp, vp, vp, vp, i32, i32, i32, descp, vp, vp, vp,
+                                              sz, vp]
+            L.gdattn_decode_multi.restype = ctypes.c_int
         if hasattr(L, "gdattn_decode_fp8"):
             L.gdattn_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, descp, vp, vp, vp,
                                             sz, vp]
@@ -242,6 +248,44 @@ def decode_fp8(q: torch.Tensor, k_codes: torch.Tensor, v_codes: torch.Tensor,
                         _ptr(workspace), workspace.numel(), _stream_handle(stream))
     if st != GDATTN_OK:
         raise GdattnError(st, "gdattn_decode_fp8")
+    return out, lse
+
+
+def multi_workspace_size(batch: int, n_tokens: int, max_seqlen: int, desc: LayerDesc) -> int:
+    return int(lib().gdattn_multi_workspace_size(int(batch), int(n_tokens), int(max_seqlen),
+                                                 ctypes.byref(desc)))
+
+
+def decode_multi_raw(q, k, v, seqlens, batch, n_tokens, max_seqlen, desc, out, lse, workspace,
+                     workspace_bytes, stream) -> int:
+    """gdattn_decode_multi on raw addresses (ints); returns the status code."""
+    return int(lib().gdattn_decode_multi(q, k, v, seqlens, int(batch), int(n_tokens),
+                                         int(max_seqlen), ctypes.byref(desc), out, lse, workspace,
+                                         int(workspace_bytes), stream))
+
+
+def decode_multi(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor],
+                 seqlens: torch.Tensor, desc: LayerDesc, max_seqlen: int,
+                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """Multi-query decode through gdattn_decode_multi.  q bf16 [T, B, Hq, D]: token t
+    of sequence b at position L_b - T + t, attending causally.  Returns (out, lse)."""
+    T, B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty((T, B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((T, B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = multi_workspace_size(B, T, max_seqlen, desc)
+        if n == 0:
+            raise GdattnError(GDATTN_ERR_INVALID_ARG, "gdattn_multi_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+        workspace_init(workspace, stream)
+    st = decode_multi_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(seqlens), B, T, max_seqlen, desc,
+                          _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                          _stream_handle(stream))
+    if st != GDATTN_OK:
+        raise GdattnError(st, "gdattn_decode_multi")
     return out, lse
 
 

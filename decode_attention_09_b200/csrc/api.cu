@@ -292,7 +292,7 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
 
 // --------------------------------------------------------------- launching
 cudaLaunchConfig_t launch_config(dim3 grid, int threads, int smem, cudaStream_t stream,
-                                 cudaLaunchAttribute *attr) {
+                                 cudaLaunchAttribute *attr, bool pdl = true) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(threads);
@@ -303,7 +303,7 @@ cudaLaunchConfig_t launch_config(dim3 grid, int threads, int smem, cudaStream_t 
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 1 : 0;
   return cfg;
 }
 
@@ -413,11 +413,14 @@ gdattn_status check_decode_args(const void *q, const void *k_cache, const void *
 // Enqueues the decode kernel (and the combine when the plan splits) with the
 // split-KV scratch at `ws`: status word, then partial LSE, then partial O.
 // k_new / v_new (optional): the current token's rows, appended by the kernel.
+// pdl = false: a plain launch, for a decode that reads lengths the kernel just
+// before it on the stream wrote (the kernels read seqlens before their
+// dependency wait).
 gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_cache,
                              const void *v_cache, const int32_t *seqlens, int32_t batch,
                              const gdattn_layer_desc *desc, void *out, float *lse, uint8_t *ws,
                              cudaStream_t stream, const void *k_new = nullptr,
-                             const void *v_new = nullptr) {
+                             const void *v_new = nullptr, bool pdl = true) {
   uint32_t *status = reinterpret_cast<uint32_t *>(ws);
   uint32_t *counters = reinterpret_cast<uint32_t *>(ws + pl.off_cnt);
   uint32_t *epochs = reinterpret_cast<uint32_t *>(ws + pl.off_epoch);
@@ -460,7 +463,8 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     cp.n_q_heads = desc->n_q_heads;
     cp.qscale = qscale;
     cp.post = post;
-    cudaLaunchConfig_t cfg = launch_config(dim3(pl.grid), ck.threads, ck.smem, stream, attr);
+    cudaLaunchConfig_t cfg =
+        launch_config(dim3(pl.grid), ck.threads, ck.smem, stream, attr, pdl);
     if (cudaLaunchKernelEx(&cfg, ck.fn, cp) != cudaSuccess) return GDATTN_ERR_CUDA;
   } else {
     EncodeTiledFn enc = encode_tiled();
@@ -493,7 +497,7 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     tp.post = post;
     if (pl.kind == PathKind::kTc) {
       cudaLaunchConfig_t cfg =
-          launch_config(dim3(pl.grid), TcConfig::kThreads, TcConfig::SMEM, stream, attr);
+          launch_config(dim3(pl.grid), TcConfig::kThreads, TcConfig::SMEM, stream, attr, pdl);
       const cudaError_t e = k_new != nullptr
                                 ? cudaLaunchKernelEx(&cfg, tc_decode_append_kernel, kmap, qmap, tp, ap)
                                 : cudaLaunchKernelEx(&cfg, tc_decode_kernel, kmap, qmap, tp);
@@ -502,8 +506,8 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
       if (!encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, batch, bstride,
                             TcPairConfig::TILE))
         return GDATTN_ERR_CUDA;
-      cudaLaunchConfig_t cfg =
-          launch_config(dim3(pl.grid), TcPairConfig::kThreads, TcPairConfig::SMEM, stream, attr);
+      cudaLaunchConfig_t cfg = launch_config(dim3(pl.grid), TcPairConfig::kThreads,
+                                             TcPairConfig::SMEM, stream, attr, pdl);
       const cudaError_t e =
           k_new != nullptr
               ? cudaLaunchKernelEx(&cfg, tc_pair_decode_append_kernel, kmap, vmap, qmap, tp, ap)
@@ -568,6 +572,25 @@ gdattn_status enqueue_decode_fp8(const LayerPlan &pl, const void *q, const void 
                  cudaSuccess
              ? GDATTN_OK
              : GDATTN_ERR_CUDA;
+}
+
+// ------------------------------------------------------ multi-query decode
+// Per-token context lengths of a T-token step: lens[t][b] = seqlens[b] - (T - 1 - t).
+__global__ void multi_lengths_kernel(const int32_t *seqlens, int32_t batch, int32_t T,
+                                     int32_t *lens) {
+  for (int32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < T * batch;
+       i += gridDim.x * blockDim.x) {
+    const int32_t t = i / batch, b = i - t * batch;
+    lens[i] = seqlens[b] - (T - 1 - t);
+  }
+}
+
+constexpr int32_t kMaxMultiTokens = 64;
+
+// Workspace of a multi-query step: the decode plan's, then the lengths [T][B].
+size_t multi_lens_offset(const LayerPlan &pl) { return align256(pl.bytes); }
+size_t multi_bytes(const LayerPlan &pl, int32_t batch, int32_t T) {
+  return align256(multi_lens_offset(pl) + static_cast<size_t>(T) * batch * 4);
 }
 
 // -------------------------------------------------- fixed scratch (no alloc)
@@ -708,6 +731,54 @@ gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *
   return enqueue_decode_fp8(pl, q, k_codes, v_codes, k_scale, v_scale, seqlens, batch, desc, out,
                             lse, static_cast<uint8_t *>(workspace),
                             static_cast<cudaStream_t>(stream));
+}
+
+size_t gdattn_multi_workspace_size(int32_t batch, int32_t n_tokens, int32_t max_seqlen,
+                                   const gdattn_layer_desc *desc) {
+  if (n_tokens < 1 || n_tokens > kMaxMultiTokens) return 0;
+  LayerPlan pl;
+  if (make_plan(batch, max_seqlen, desc, pl) != GDATTN_OK) return 0;
+  return multi_bytes(pl, batch, n_tokens);
+}
+
+gdattn_status gdattn_decode_multi(const void *q, const void *k_cache, const void *v_cache,
+                                  const int32_t *seqlens, int32_t batch, int32_t n_tokens,
+                                  int32_t max_seqlen, const gdattn_layer_desc *desc, void *out,
+                                  float *lse, void *workspace, size_t workspace_bytes,
+                                  void *stream_) {
+  gdattn_status st = check_decode_args(q, k_cache, v_cache, seqlens, batch, max_seqlen, desc,
+                                       out, lse);
+  if (st != GDATTN_OK) return st;
+  if (n_tokens < 1 || n_tokens > kMaxMultiTokens || n_tokens > max_seqlen)
+    return GDATTN_ERR_INVALID_ARG;
+  // A ring holds positions [L - C, L): the first token's window must still be in it.
+  if (desc->window > 0 && desc->cache_capacity < max_seqlen &&
+      static_cast<int64_t>(desc->cache_capacity) <
+          static_cast<int64_t>(desc->window) + n_tokens - 1)
+    return GDATTN_ERR_INVALID_ARG;
+  if (workspace == nullptr) return GDATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GDATTN_ERR_MISALIGNED;
+  LayerPlan pl;
+  st = make_plan(batch, max_seqlen, desc, pl);
+  if (st != GDATTN_OK) return st;
+  if (workspace_bytes < multi_bytes(pl, batch, n_tokens)) return GDATTN_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int32_t *lens = reinterpret_cast<int32_t *>(ws + multi_lens_offset(pl));
+  const int32_t total = n_tokens * batch;
+  multi_lengths_kernel<<<(total + 255) / 256, 256, 0, stream>>>(seqlens, batch, n_tokens, lens);
+  if (cudaGetLastError() != cudaSuccess) return GDATTN_ERR_CUDA;
+  const int64_t rows = static_cast<int64_t>(batch) * desc->n_q_heads;
+  for (int32_t t = 0; t < n_tokens; ++t) {
+    const int64_t off = static_cast<int64_t>(t) * rows * desc->head_dim;
+    st = enqueue_decode(pl, static_cast<const uint16_t *>(q) + off, k_cache, v_cache,
+                        lens + static_cast<int64_t>(t) * batch, batch, desc,
+                        static_cast<uint16_t *>(out) + off,
+                        lse != nullptr ? lse + t * rows : nullptr, ws, stream, nullptr, nullptr,
+                        t > 0);
+    if (st != GDATTN_OK) return st;
+  }
+  return GDATTN_OK;
 }
 
 gdattn_status gdattn_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,

@@ -235,6 +235,39 @@ gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *
                                 void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Multi-query decode: T query tokens per sequence, the last T positions of its
+ * context, each attending causally: the verify step of speculative decoding,
+ * which "Gemma 4 12B" (serviceability join, item 2) runs with 7 draft tokens on
+ * the sliding-window stack.  Query token t of sequence b sits at position
+ * p = L_b - T + t and attends
+ * [max(0, p + 1 - window), p + 1) (window 0: [0, p + 1)); the cache already
+ * holds the rows of all T tokens.  Each token's result is exactly what
+ * gdattn_decode gives for context length L_b - (T - 1 - t).
+ *
+ *  q         bf16 [T, batch, Hq, D] (token-major), device, read only
+ *  out       bf16 [T, batch, Hq, D];  lse: fp32 [T, batch, Hq] or NULL
+ *  n_tokens  T, 1 <= T <= 64;  seqlens: L_b >= T, the length with all T tokens
+ *  workspace at least gdattn_multi_workspace_size bytes (zeroed once by
+ *            gdattn_workspace_init)
+ *  other arguments, geometries and device-side errors as gdattn_decode.
+ *
+ * A ring cache holds positions [L_b - C, L_b), so with a window the first token
+ * needs C >= window + T - 1 unless the cache never wraps (C >= max_seqlen);
+ * otherwise GDATTN_ERR_INVALID_ARG.  The step is one small kernel that writes
+ * the T per-token lengths into the workspace, then T decode launches over the
+ * same cache: every token's window is streamed again (the KV bytes are T times
+ * a single-token step's).
+ */
+size_t gdattn_multi_workspace_size(int32_t batch, int32_t n_tokens, int32_t max_seqlen,
+                                   const gdattn_layer_desc *desc);
+
+gdattn_status gdattn_decode_multi(const void *q, const void *k_cache, const void *v_cache,
+                                  const int32_t *seqlens, int32_t batch, int32_t n_tokens,
+                                  int32_t max_seqlen, const gdattn_layer_desc *desc, void *out,
+                                  float *lse, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/*
  * gdattn_decode without a caller workspace.  A library addition: the paper
  * has no counterpart; it computes exactly what gdattn_decode computes.
  *

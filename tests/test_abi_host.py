@@ -33,7 +33,8 @@ def declared_functions():
 
 def test_header_declares_the_api():
     names = declared_functions()
-    for n in ("gdattn_decode", "gdattn_decode_fp8", "gdattn_combine", "gdattn_workspace_size",
+    for n in ("gdattn_decode", "gdattn_decode_fp8", "gdattn_decode_multi", "gdattn_combine",
+              "gdattn_workspace_size", "gdattn_multi_workspace_size",
               "gdattn_workspace_init",
               "gdattn_plan_splits", "gdattn_plan_launches",
               "gdattn_check_device_status", "gdattn_status_string", "gdattn_version"):
@@ -231,3 +232,19 @@ def test_decode_fp8_rejects_bad_pointers(lib, case, expect):
 ])
 def test_decode_fp8_rejects_bad_desc(lib, desc_kw, expect):
     assert fp8_call(good_desc(**desc_kw)) == expect
+
+
+def test_decode_multi_host_checks(lib):
+    """gdattn_decode_multi: token count, ring capacity and workspace checked on the host."""
+    def multi(desc, T=2, max_seqlen=2048, ws=A, ws_bytes=1 << 24, q=A):
+        return binding.decode_multi_raw(q, A, A, A, 1, T, max_seqlen, desc, A, A, ws, ws_bytes,
+                                        None)
+    d = good_desc(cache_capacity=1030)  # window 1024: room for T <= 7
+    assert multi(d, T=0) == binding.GDATTN_ERR_INVALID_ARG
+    assert multi(d, T=65) == binding.GDATTN_ERR_INVALID_ARG
+    assert multi(d, T=8) == binding.GDATTN_ERR_INVALID_ARG      # C < w + T - 1
+    assert multi(good_desc(), T=2) == binding.GDATTN_ERR_INVALID_ARG  # C = w: no room
+    assert multi(d, T=2, ws=None) == binding.GDATTN_ERR_WORKSPACE
+    assert multi(d, T=2, q=None) == binding.GDATTN_ERR_INVALID_ARG
+    assert multi(d, T=2, q=A + 8) == binding.GDATTN_ERR_MISALIGNED
+    assert binding.multi_workspace_size(1, 0, 8, good_desc()) == 0
