@@ -536,6 +536,46 @@ def run_ours(args, world, rank, local):
                 raise binding.GdattnError(st, "device status after the fp8 step")
         del g_f8, g_f8_step
 
+    # ---- multi-query decode (gdattn_decode_multi): a 4-token verify step over the
+    # global layers (whole-context caches, so every token's range is resident)
+    t_multi, ms_multi = 4, None
+    if global_idx:
+        gen_mq = torch.Generator(device="cpu").manual_seed(11 + rank)
+        mq = {}
+        for i in global_idx:
+            ly = stack.layers[i]
+            sp = ly["spec"]
+            q4 = torch.randn((t_multi, w.batch, sp.n_q_heads, sp.head_dim),
+                             generator=gen_mq).to(torch.bfloat16).to(device)
+            ws4 = torch.empty(binding.multi_workspace_size(w.batch, t_multi, stack.max_seqlen,
+                                                           ly["desc"]),
+                              dtype=torch.uint8, device=device)
+            binding.workspace_init(ws4, stream)
+            mq[i] = (q4, ws4, torch.empty_like(q4),
+                     torch.empty((t_multi, w.batch, sp.n_q_heads), device=device))
+
+        def multi_step():
+            for i in global_idx:
+                q4, ws4, o4, l4 = mq[i]
+                inp = stack.layers[i]["inp"]
+                binding.decode_multi(q4, inp.k, inp.v, inp.seqlens, stack.layers[i]["desc"],
+                                     stack.max_seqlen, out=o4, lse=l4, workspace=ws4,
+                                     stream=stream)
+
+        g_mq = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            multi_step()
+            stream.synchronize()
+            with torch.cuda.graph(g_mq, stream=stream):
+                multi_step()
+        barrier()
+        ms_multi = max_over_ranks(time_graph(g_mq, stream, args.steps, 3), world)
+        for q4, ws4, o4, l4 in mq.values():
+            st = binding.check_device_status(ws4, stream)
+            if st != binding.GDATTN_OK:
+                raise binding.GdattnError(st, "device status after the multi-query step")
+        del g_mq
+
     # ---- CPU baseline: the oracle over the whole step (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
@@ -634,6 +674,15 @@ def run_ours(args, world, rank, local):
                           "current-token K/V rows written into their ring slots by the decode "
                           "kernels (CUDA graph, device time)"},
         "fp8_kv": fp8_summary,
+        "multi_query": None if ms_multi is None else {
+            "tokens": t_multi,
+            "global_us_per_layer": ms_multi / len(global_idx) * 1e3,
+            "single_token_global_us_per_layer": ms_gl / len(global_idx) * 1e3,
+            "kv_gbs": t_multi * gl_bytes / (ms_multi * 1e-3) / 1e9,
+            "how": "the 8 global layers through gdattn_decode_multi with 4 query tokens per "
+                   "sequence (a speculative-decoding verify step): a lengths kernel, then one "
+                   "decode launch per token, each streaming its own window (KV bytes 4x a "
+                   "single-token step); CUDA graph, device time"},
         "gpu_launches": stack.launches_per_step(all_idx) * args.steps,
         "clocks": clk,
     }
