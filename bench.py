@@ -681,8 +681,9 @@ def run_ours(args, world, rank, local):
             "kv_gbs": t_multi * gl_bytes / (ms_multi * 1e-3) / 1e9,
             "how": "the 8 global layers through gdattn_decode_multi with 4 query tokens per "
                    "sequence (a speculative-decoding verify step): a lengths kernel, then one "
-                   "decode launch per token, each streaming its own window (KV bytes 4x a "
-                   "single-token step); CUDA graph, device time"},
+                   "decode launch over 4 x 8 query sequences that read the 8 caches (the "
+                   "tokens of a sequence share its rows through L2); kv_gbs counts each "
+                   "token's window; CUDA graph, device time"},
         "gpu_launches": stack.launches_per_step(all_idx) * args.steps,
         "clocks": clk,
     }

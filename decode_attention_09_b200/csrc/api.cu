@@ -416,11 +416,15 @@ gdattn_status check_decode_args(const void *q, const void *k_cache, const void *
 // pdl = false: a plain launch, for a decode that reads lengths the kernel just
 // before it on the stream wrote (the kernels read seqlens before their
 // dependency wait).
+// cache_batch (> 0): sequences in the caches when it differs from batch (a
+// multi-token step: query sequence b reads cache sequence b % cache_batch).
 gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_cache,
                              const void *v_cache, const int32_t *seqlens, int32_t batch,
                              const gdattn_layer_desc *desc, void *out, float *lse, uint8_t *ws,
                              cudaStream_t stream, const void *k_new = nullptr,
-                             const void *v_new = nullptr, bool pdl = true) {
+                             const void *v_new = nullptr, bool pdl = true,
+                             int32_t cache_batch = 0) {
+  if (cache_batch <= 0) cache_batch = batch;
   uint32_t *status = reinterpret_cast<uint32_t *>(ws);
   uint32_t *counters = reinterpret_cast<uint32_t *>(ws + pl.off_cnt);
   uint32_t *epochs = reinterpret_cast<uint32_t *>(ws + pl.off_epoch);
@@ -441,8 +445,8 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
   geo.units_per_seq = pl.units_per_seq;
   geo.window = desc->window;
   geo.capacity = desc->cache_capacity;
-  geo.nchunks = pl.grid;
-  geo.align = pl.align;
+  geo.nchunks_align = pl.grid | (pl.align << 16);  // grid < 2^16, align <= 128
+  geo.cache_batch = cache_batch;
 
   cudaLaunchAttribute attr[1];
   if (pl.kind == PathKind::kCore) {
@@ -470,8 +474,8 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     EncodeTiledFn enc = encode_tiled();
     if (enc == nullptr) return GDATTN_ERR_CUDA;
     CUtensorMap kmap, vmap, qmap;
-    if (!encode_cache_map(enc, &kmap, k_cache, D, Hkv, desc->cache_capacity, batch, bstride,
-                          TcConfig::TILE) ||
+    if (!encode_cache_map(enc, &kmap, k_cache, D, Hkv, desc->cache_capacity, cache_batch,
+                          bstride, TcConfig::TILE) ||
         !encode_q_map(enc, &qmap, q, D, static_cast<int64_t>(batch) * desc->n_q_heads))
       return GDATTN_ERR_CUDA;
     TcParams tp;
@@ -503,8 +507,8 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
                                 : cudaLaunchKernelEx(&cfg, tc_decode_kernel, kmap, qmap, tp);
       if (e != cudaSuccess) return GDATTN_ERR_CUDA;
     } else {
-      if (!encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, batch, bstride,
-                            TcPairConfig::TILE))
+      if (!encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, cache_batch,
+                            bstride, TcPairConfig::TILE))
         return GDATTN_ERR_CUDA;
       cudaLaunchConfig_t cfg = launch_config(dim3(pl.grid), TcPairConfig::kThreads,
                                              TcPairConfig::SMEM, stream, attr, pdl);
@@ -557,8 +561,8 @@ gdattn_status enqueue_decode_fp8(const LayerPlan &pl, const void *q, const void 
   tp.geo.units_per_seq = pl.units_per_seq;
   tp.geo.window = desc->window;
   tp.geo.capacity = desc->cache_capacity;
-  tp.geo.nchunks = pl.grid;
-  tp.geo.align = pl.align;
+  tp.geo.nchunks_align = pl.grid | (pl.align << 16);
+  tp.geo.cache_batch = batch;
   tp.n_q_heads = desc->n_q_heads;
   tp.qscale = desc->softcap > 0.f ? desc->scale / desc->softcap : desc->scale * log2e;
   tp.post = desc->softcap > 0.f ? desc->softcap * log2e : 0.f;
@@ -735,9 +739,9 @@ gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *
 
 size_t gdattn_multi_workspace_size(int32_t batch, int32_t n_tokens, int32_t max_seqlen,
                                    const gdattn_layer_desc *desc) {
-  if (n_tokens < 1 || n_tokens > kMaxMultiTokens) return 0;
+  if (n_tokens < 1 || n_tokens > kMaxMultiTokens || batch <= 0) return 0;
   LayerPlan pl;
-  if (make_plan(batch, max_seqlen, desc, pl) != GDATTN_OK) return 0;
+  if (make_plan(batch * n_tokens, max_seqlen, desc, pl) != GDATTN_OK) return 0;
   return multi_bytes(pl, batch, n_tokens);
 }
 
@@ -758,27 +762,20 @@ gdattn_status gdattn_decode_multi(const void *q, const void *k_cache, const void
     return GDATTN_ERR_INVALID_ARG;
   if (workspace == nullptr) return GDATTN_ERR_WORKSPACE;
   if (!aligned16(workspace)) return GDATTN_ERR_MISALIGNED;
+  // One decode over T x B query sequences, token-major (q, out, lse and the
+  // lengths are [T][B] ...): query sequence t * B + b reads cache sequence b.
+  const int32_t total = n_tokens * batch;
   LayerPlan pl;
-  st = make_plan(batch, max_seqlen, desc, pl);
+  st = make_plan(total, max_seqlen, desc, pl);
   if (st != GDATTN_OK) return st;
   if (workspace_bytes < multi_bytes(pl, batch, n_tokens)) return GDATTN_ERR_WORKSPACE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   int32_t *lens = reinterpret_cast<int32_t *>(ws + multi_lens_offset(pl));
-  const int32_t total = n_tokens * batch;
   multi_lengths_kernel<<<(total + 255) / 256, 256, 0, stream>>>(seqlens, batch, n_tokens, lens);
   if (cudaGetLastError() != cudaSuccess) return GDATTN_ERR_CUDA;
-  const int64_t rows = static_cast<int64_t>(batch) * desc->n_q_heads;
-  for (int32_t t = 0; t < n_tokens; ++t) {
-    const int64_t off = static_cast<int64_t>(t) * rows * desc->head_dim;
-    st = enqueue_decode(pl, static_cast<const uint16_t *>(q) + off, k_cache, v_cache,
-                        lens + static_cast<int64_t>(t) * batch, batch, desc,
-                        static_cast<uint16_t *>(out) + off,
-                        lse != nullptr ? lse + t * rows : nullptr, ws, stream, nullptr, nullptr,
-                        t > 0);
-    if (st != GDATTN_OK) return st;
-  }
-  return GDATTN_OK;
+  return enqueue_decode(pl, q, k_cache, v_cache, lens, total, desc, out, lse, ws, stream, nullptr,
+                        nullptr, false, batch);
 }
 
 gdattn_status gdattn_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,

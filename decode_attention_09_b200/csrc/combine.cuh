@@ -60,7 +60,8 @@ __device__ void unit_position(const Geometry &g, int32_t b, int32_t x, int64_t &
   before = warp_sum_i64(before);
   n = attended_count(__ldg(g.seqlens + b), g.window, g.capacity, bad);
   unit_start = before + static_cast<int64_t>(x) * n;
-  chunk = total > 0 ? ceil_div64(ceil_div64(total, g.nchunks), g.align) * g.align : 1;
+  chunk = total > 0 ? ceil_div64(ceil_div64(total, geo_nchunks(g)), geo_align(g)) * geo_align(g)
+                    : 1;
 }
 
 // Merges np parts for NC float4 columns at once: for column c, part s holds

@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads, 1)
             break;
           }
           const uint32_t bytes = static_cast<uint32_t>(ntok * ROWB);
-          const int64_t off = static_cast<int64_t>(s.b) * p.batch_stride +
+          const int64_t off = static_cast<int64_t>(cache_seq(p.geo, s.b)) * p.batch_stride +
                               static_cast<int64_t>(runs.start(r) + t0) * (HKV * D);
           if (p.k_new != nullptr && newest) {  // append the current token's rows first
             const int64_t row = static_cast<int64_t>(s.b) * p.batch_stride +

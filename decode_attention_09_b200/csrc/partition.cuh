@@ -30,9 +30,23 @@ struct Geometry {
   int32_t units_per_seq;
   int32_t window;
   int32_t capacity;
-  int32_t nchunks;  // P = gridDim.x of the decode kernel
-  int32_t align;    // chunk sizes are rounded up to a multiple of this (tokens)
+  // Low 16 bits: P = gridDim.x of the decode kernel (< 2^16); high 16 bits: the
+  // chunk alignment in tokens (chunk sizes are rounded up to a multiple of it).
+  // Packed so the kernels' parameter block keeps its size.
+  int32_t nchunks_align;
+  int32_t cache_batch;  // sequences in the cache: query sequence b reads cache b % cache_batch
 };
+
+__device__ __forceinline__ int32_t geo_nchunks(const Geometry &g) {
+  return g.nchunks_align & 0xFFFF;
+}
+__device__ __forceinline__ int32_t geo_align(const Geometry &g) { return g.nchunks_align >> 16; }
+
+// The cache sequence query sequence b reads (several query sequences share one
+// cache sequence in a multi-token step, laid out token-major).
+__device__ __forceinline__ int32_t cache_seq(const Geometry &g, int32_t b) {
+  return b < g.cache_batch ? b : b % g.cache_batch;  // no division in a single-token step
+}
 
 // Positions one decode step attends for context length L (clamped to the cache;
 // an impossible L yields 0 and `bad`).
@@ -87,7 +101,8 @@ __device__ void plan_chunk(const Geometry &g, int32_t c, ChunkPlan *plan) {
     acc += attended_count(__ldg(g.seqlens + b), g.window, g.capacity, bad);
   const int64_t total = warp_sum_i64(acc) * g.units_per_seq;
   const int anybad = __any_sync(0xffffffffu, bad);
-  const int64_t chunk = total > 0 ? ceil_div64(ceil_div64(total, g.nchunks), g.align) * g.align : 1;
+  const int64_t chunk =
+      total > 0 ? ceil_div64(ceil_div64(total, geo_nchunks(g)), geo_align(g)) * geo_align(g) : 1;
   const int64_t cs = imin64(static_cast<int64_t>(c) * chunk, total);
   const int64_t ce = imin64(cs + chunk, total);
   // First sequence whose flattened range ends after cs.

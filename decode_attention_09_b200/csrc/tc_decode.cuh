@@ -340,7 +340,7 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
 #pragma unroll
         for (int j = 0; j < D / 64; ++j)
           tma_load_4d(stages + st * Cfg::STAGEB + j * Cfg::BOXB, &kmap, 64 * j, it.seg.x, row,
-                      it.seg.b, &full[st], pol);
+                      cache_seq(p.geo, it.seg.b), &full[st], pol);
       }
       __syncwarp();
       ++i;

@@ -525,12 +525,13 @@ __device__ __forceinline__ void tc_pair_decode_body(const CUtensorMap &kmap,
                    ap.k_new + (static_cast<int64_t>(it.seg.b) * ap.n_kv_heads + it.seg.x) * D, D,
                    lane);
       }
+      const int32_t cb = cache_seq(p.geo, it.seg.b);
       if (elect_one()) {
         uint8_t *kdst = stages + st * Cfg::STAGEB;
         mbar_arrive_expect_tx(&kfull[st], Cfg::KB);
 #pragma unroll
         for (int j = 0; j < D / 64; ++j)
-          tma_load_4d(kdst + j * Cfg::BOXB, &kmap, 64 * j, it.seg.x, row, it.seg.b, &kfull[st], pol);
+          tma_load_4d(kdst + j * Cfg::BOXB, &kmap, 64 * j, it.seg.x, row, cb, &kfull[st], pol);
       }
       __syncwarp();
       ++i;
@@ -667,12 +668,13 @@ __device__ __forceinline__ void tc_pair_decode_body(const CUtensorMap &kmap,
                    ap.v_new + (static_cast<int64_t>(it.seg.b) * ap.n_kv_heads + it.seg.x) * D, D,
                    lane);
       }
+      const int32_t cb = cache_seq(p.geo, it.seg.b);
       if (elect_one()) {
         uint8_t *vdst = stages + st * Cfg::STAGEB + Cfg::KB;
         mbar_arrive_expect_tx(&vfull[st], Cfg::KB);
 #pragma unroll
         for (int j = 0; j < D / 64; ++j)
-          tma_load_4d(vdst + j * Cfg::BOXB, &vmap, 64 * j, it.seg.x, row, it.seg.b, &vfull[st], pol);
+          tma_load_4d(vdst + j * Cfg::BOXB, &vmap, 64 * j, it.seg.x, row, cb, &vfull[st], pol);
       }
       __syncwarp();
       ++i;

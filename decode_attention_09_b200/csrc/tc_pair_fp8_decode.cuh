@@ -298,7 +298,8 @@ __global__ void __launch_bounds__(TcPairFp8Config::kThreads, 1)
         mbar_arrive_expect_tx(&kfull[st], Cfg::KB);
 #pragma unroll
         for (int j = 0; j < D / 128; ++j)
-          tma_load_4d(kdst + j * Cfg::BOXB, &kmap, 128 * j, it.seg.x, row, it.seg.b, &kfull[st],
+          tma_load_4d(kdst + j * Cfg::BOXB, &kmap, 128 * j, it.seg.x, row,
+                      cache_seq(p.geo, it.seg.b), &kfull[st],
                       pol);
       }
       __syncwarp();
@@ -427,7 +428,8 @@ __global__ void __launch_bounds__(TcPairFp8Config::kThreads, 1)
       if (i >= NST && !mbar_wait(&vempty[st], ((i / NST) - 1) & 1, abort_flag, p.status))
         ok = false;
       if (!__all_sync(0xffffffffu, ok)) break;
-      const int64_t srow = (static_cast<int64_t>(it.seg.b) * Hkv + it.seg.x) * C + row;
+      const int32_t cb = cache_seq(p.geo, it.seg.b);
+      const int64_t srow = (static_cast<int64_t>(cb) * Hkv + it.seg.x) * C + row;
       float *dst = scl + st * 2 * TILE;
 #pragma unroll
       for (int j = lane; j < TILE; j += 32)
@@ -442,7 +444,7 @@ __global__ void __launch_bounds__(TcPairFp8Config::kThreads, 1)
         mbar_arrive_expect_tx(&vfull[st], Cfg::KB);
 #pragma unroll
         for (int j = 0; j < D / 128; ++j)
-          tma_load_4d(vdst + j * Cfg::BOXB, &vmap, 128 * j, it.seg.x, row, it.seg.b, &vfull[st],
+          tma_load_4d(vdst + j * Cfg::BOXB, &vmap, 128 * j, it.seg.x, row, cb, &vfull[st],
                       pol);
       }
       __syncwarp();

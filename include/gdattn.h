@@ -254,9 +254,11 @@ gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *
  * A ring cache holds positions [L_b - C, L_b), so with a window the first token
  * needs C >= window + T - 1 unless the cache never wraps (C >= max_seqlen);
  * otherwise GDATTN_ERR_INVALID_ARG.  The step is one small kernel that writes
- * the T per-token lengths into the workspace, then T decode launches over the
- * same cache: every token's window is streamed again (the KV bytes are T times
- * a single-token step's).
+ * the T per-token lengths into the workspace, then one decode launch over
+ * T x batch query sequences (token-major) in which query sequence t * batch + b
+ * reads cache sequence b.  The T tokens of a sequence read the same cache rows
+ * from different CTAs at about the same time, so much of the repetition is
+ * served from L2 rather than HBM.
  */
 size_t gdattn_multi_workspace_size(int32_t batch, int32_t n_tokens, int32_t max_seqlen,
                                    const gdattn_layer_desc *desc);

@@ -60,16 +60,25 @@ def test_multi_matches_oracle(name):
                     what=f"{name} token {t} call {rep}")
 
 
-def test_multi_last_token_equals_decode():
-    """The last of T tokens is bit-identical to gdattn_decode at the full length."""
+def test_multi_tokens_before_the_context_are_reported():
+    """A sequence shorter than T: its tokens at positions below 0 attend nothing;
+    the device reports it, gives them zero output and LSE -inf, and the other
+    tokens are still right."""
     require_gpu()
-    q, inp = case_inputs("pair_ring_t4")
+    q, inp = case_inputs("core_g4_t3")  # T = 3
+    inp.seqlens[1] = 2                  # token 0 of sequence 1 would sit at position -1
     s = inp.spec
     dev = "cuda"
     desc = binding.desc_from_spec(s, capacity=inp.k.shape[1])
-    k, v, sl = inp.k.to(dev), inp.v.to(dev), inp.seqlens.to(dev)
-    out, lse = binding.decode_multi(q.to(dev), k, v, sl, desc, int(inp.seqlens.max()))
-    o1, l1 = binding.decode(q[-1].to(dev).contiguous(), k, v, sl, desc, int(inp.seqlens.max()))
-    torch.cuda.synchronize()
-    assert torch.equal(out[-1].view(torch.int16), o1.view(torch.int16))
-    assert torch.equal(lse[-1].view(torch.int32), l1.view(torch.int32))
+    T = q.shape[0]
+    ws = torch.empty(binding.multi_workspace_size(2, T, 90, desc), dtype=torch.uint8, device=dev)
+    binding.workspace_init(ws)
+    out, lse = binding.decode_multi(q.to(dev), inp.k.to(dev), inp.v.to(dev), inp.seqlens.to(dev),
+                                    desc, 90, workspace=ws)
+    assert binding.check_device_status(ws) == binding.GDATTN_ERR_DEVICE_SEQLEN
+    assert torch.all(out[0, 1] == 0) and torch.all(torch.isneginf(lse[0, 1]))
+    o_ref, l_ref = oracle.get().decode_multi(q[1:, 0:1], inp.k[0:1], inp.v[0:1],
+                                             inp.seqlens[0:1], s.window, s.softcap, s.scale)
+    for t in range(1, T):
+        compare(out[t, 0:1], lse[t, 0:1], o_ref[t - 1], l_ref[t - 1], ulp_floor=True,
+                what=f"token {t} of the full-length sequence")
