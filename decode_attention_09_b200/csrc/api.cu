@@ -241,7 +241,9 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
                                   TcPairConfig::kThreads, TcPairConfig::SMEM, query_tc_pair);
     if (cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_decode_append_kernel),
                              TcPairConfig::kThreads, TcPairConfig::SMEM,
-                             query_tc_pair_append) != per_sm)
+                             query_tc_pair_append) != per_sm ||
+        cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_decode_multi_kernel),
+                             TcPairConfig::kThreads, TcPairConfig::SMEM, query_tc_pair) != per_sm)
       return GDATTN_ERR_CUDA;
     min_tokens = 2 * TcPairConfig::TILE;
     pl.align = TcPairConfig::TILE;
@@ -515,6 +517,8 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
       const cudaError_t e =
           k_new != nullptr
               ? cudaLaunchKernelEx(&cfg, tc_pair_decode_append_kernel, kmap, vmap, qmap, tp, ap)
+          : cache_batch != batch
+              ? cudaLaunchKernelEx(&cfg, tc_pair_decode_multi_kernel, kmap, vmap, qmap, tp)
               : cudaLaunchKernelEx(&cfg, tc_pair_decode_kernel, kmap, vmap, qmap, tp);
       if (e != cudaSuccess) return GDATTN_ERR_CUDA;
     }

@@ -357,7 +357,9 @@ __device__ __forceinline__ void merge_counted_parts(const float *ws_o, const flo
                 __ldcg(ws_o + ((slot0 + r) * G + h[e]) * D + d[e]));
 }
 
-template <bool APPEND>
+// MULTI: a multi-token step, whose query sequence b reads cache sequence
+// cache_seq(b); the single-token entry points read cache sequence b directly.
+template <bool APPEND, bool MULTI>
 __device__ __forceinline__ void tc_pair_decode_body(const CUtensorMap &kmap,
                                                     const CUtensorMap &vmap,
                                                     const CUtensorMap &qmap, const TcParams &p,
@@ -525,7 +527,7 @@ __device__ __forceinline__ void tc_pair_decode_body(const CUtensorMap &kmap,
                    ap.k_new + (static_cast<int64_t>(it.seg.b) * ap.n_kv_heads + it.seg.x) * D, D,
                    lane);
       }
-      const int32_t cb = cache_seq(p.geo, it.seg.b);
+      const int32_t cb = MULTI ? cache_seq(p.geo, it.seg.b) : it.seg.b;
       if (elect_one()) {
         uint8_t *kdst = stages + st * Cfg::STAGEB;
         mbar_arrive_expect_tx(&kfull[st], Cfg::KB);
@@ -668,7 +670,7 @@ __device__ __forceinline__ void tc_pair_decode_body(const CUtensorMap &kmap,
                    ap.v_new + (static_cast<int64_t>(it.seg.b) * ap.n_kv_heads + it.seg.x) * D, D,
                    lane);
       }
-      const int32_t cb = cache_seq(p.geo, it.seg.b);
+      const int32_t cb = MULTI ? cache_seq(p.geo, it.seg.b) : it.seg.b;
       if (elect_one()) {
         uint8_t *vdst = stages + st * Cfg::STAGEB + Cfg::KB;
         mbar_arrive_expect_tx(&vfull[st], Cfg::KB);
@@ -904,7 +906,14 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
     tc_pair_decode_kernel(const __grid_constant__ CUtensorMap kmap,
                           const __grid_constant__ CUtensorMap vmap,
                           const __grid_constant__ CUtensorMap qmap, const TcParams p) {
-  tc_pair_decode_body<false>(kmap, vmap, qmap, p, TcAppend{});
+  tc_pair_decode_body<false, false>(kmap, vmap, qmap, p, TcAppend{});
+}
+
+__global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
+    tc_pair_decode_multi_kernel(const __grid_constant__ CUtensorMap kmap,
+                                const __grid_constant__ CUtensorMap vmap,
+                                const __grid_constant__ CUtensorMap qmap, const TcParams p) {
+  tc_pair_decode_body<false, true>(kmap, vmap, qmap, p, TcAppend{});
 }
 
 __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
@@ -912,7 +921,7 @@ __global__ void __launch_bounds__(TcPairConfig::kThreads, 1)
                                  const __grid_constant__ CUtensorMap vmap,
                                  const __grid_constant__ CUtensorMap qmap, const TcParams p,
                                  const TcAppend ap) {
-  tc_pair_decode_body<true>(kmap, vmap, qmap, p, ap);
+  tc_pair_decode_body<true, false>(kmap, vmap, qmap, p, ap);
 }
 
 }  // namespace gdattn
