@@ -90,15 +90,21 @@ def test_single_global_layer():
     compare(out, lse, o_ref, l_ref, what=w.name)
 
 
+@pytest.mark.parametrize("flags", [0, binding.GDATTN_FLAG_EVEN_UNITS])
 @pytest.mark.parametrize("layer", [0, 5])
-def test_gemma4_12b_stack_layers(layer):
-    """Batch 8, context 8192: one sliding layer (ring of 1024) and one global K=V layer."""
+def test_gemma4_12b_stack_layers(layer, flags):
+    """Batch 8, context 8192: one sliding layer (ring of 1024) and one global K=V
+    layer, with the default planner and with the even unit split the bench uses."""
     require_gpu()
     w = workloads.gemma4_12b_b8_l8192()
     inp = workloads.workload_layer_inputs(w, layer)
     o_ref, l_ref = oracle_for(inp)
-    out, lse = GpuLayer(inp).run()
-    compare(out, lse, o_ref, l_ref, what=f"{w.name} layer {layer}")
+    layer_gpu = GpuLayer(inp)
+    if flags:
+        layer_gpu.desc = binding.desc_from_spec(inp.spec, flags=flags)
+        layer_gpu.ws = binding.alloc_workspace(w.batch, layer_gpu.max_seqlen, layer_gpu.desc)
+    out, lse = layer_gpu.run()
+    compare(out, lse, o_ref, l_ref, what=f"{w.name} layer {layer} flags {flags}")
 
 
 @pytest.mark.parametrize("layer", [0, 1])
