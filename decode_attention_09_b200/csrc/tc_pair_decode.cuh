@@ -122,9 +122,10 @@ __device__ __forceinline__ void report_bad_seqlens(const TcParams &p, int lane) 
   }
 }
 
-// Warp 7 of a pair kernel: counts split parts and merges them (see the file
-// comment).  Shared by the bf16 and fp8 pair kernels, whose partial layouts
-// are the same: normalised O [G][D] and LSE [G] per part.
+// Warp 7 of the bf16 pair kernel: counts split parts and merges them (see the
+// file comment).  Partials are normalised O [G][D] and LSE [G] per part.  (The
+// fp8 pair kernel merges in its softmax threads instead, with the helpers
+// below.)
 template <int G, int D>
 __device__ __forceinline__ void pair_merge_warp(const TcParams &p, const ChunkPlan *plan, int c,
                                                 int lane, int32_t split_k, bool usplit,
