@@ -225,8 +225,11 @@ gdattn_status gdattn_decode_append(const void *q, const void *k_new, const void 
  * Hkv; others return GDATTN_ERR_UNSUPPORTED.  Scales must be finite; a zero
  * scale makes its row zero.  The kernel multiplies fp8 codes on the tensor
  * cores against q and the softmax weights each split into three e4m3 pieces;
- * the result matches the float64 definition to about 2^-12 relative to the
- * largest weight (see the kernel source for the error bound).
+ * the q split is exact for bf16 elements down to 2^-6 of the head's largest,
+ * and the weight split's error is below 2^-13 relative (2^-17 absolute for the
+ * smallest scaled weights); against the float64 definition of the dequantised
+ * attention the output meets the bf16 entry points' gates (|dout| <= 8e-3, with a
+ * one-bf16-ulp floor for outputs above 1, and |dlse| <= 1e-3).
  */
 gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *v_codes,
                                 const float *k_scale, const float *v_scale,
