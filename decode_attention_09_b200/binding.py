@@ -1,7 +1,10 @@
 """ctypes binding of libgdattn's C ABI (include/gdattn.h).
 
 Argument marshalling only: every step of decode attention runs in the CUDA
-kernels of libgdattn.so.  Torch supplies device memory and streams.  There is no
+kernels of libgdattn.so.  The tensor wrappers check what the C ABI cannot see
+(dtype, contiguity, that each tensor reaches as far as the call reads or
+writes, and its device) and raise ValueError before anything is enqueued; the
+``*_raw`` functions pass addresses through unchecked.  Torch supplies device memory and streams.  There is no
 fallback: if the library has not been built, loading it raises.
 """
 from __future__ import annotations
@@ -118,6 +121,111 @@ def _stream_handle(stream) -> Optional[int]:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def _dense(t: torch.Tensor, name: str, dtypes, numel: int, device) -> None:
+    """A dense tensor argument: one of ``dtypes``, contiguous, holding at least
+    ``numel`` elements (what the call reads or writes through its pointer), on
+    the CUDA device of the call.  The C ABI sees only the address, so a tensor
+    that is too small would be read or written past its end on the device."""
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {' or '.join(map(str, dtypes))}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name}: {t.numel()} elements, the call reaches {numel}")
+    _on(t, name, device)
+
+
+def _extent(t: torch.Tensor, name: str, dtypes, numel: int, device) -> None:
+    """A strided cache argument: one of ``dtypes``, with at least ``numel``
+    elements of storage from its first element on (the rows the call may reach
+    through ``cache_batch_stride``), on the CUDA device of the call."""
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {' or '.join(map(str, dtypes))}")
+    have = t.untyped_storage().nbytes() // t.element_size() - t.storage_offset()
+    if have < numel:
+        raise ValueError(f"{name}: storage holds {have} elements, the call reaches {numel}")
+    _on(t, name, device)
+
+
+def _on(t: torch.Tensor, name: str, device) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: on {t.device}, the call runs on {device}")
+
+
+def _cache_elems(batch: int, desc: "LayerDesc") -> int:
+    """Elements of a cache that sequences 0..batch-1 span: sequence b starts at
+    b * cache_batch_stride (0 = C * Hkv * D) and holds C * Hkv * D."""
+    rows = int(desc.cache_capacity) * int(desc.n_kv_heads) * int(desc.head_dim)
+    stride = int(desc.cache_batch_stride) or rows
+    return (batch - 1) * stride + rows if batch > 0 else 0
+
+
+_BF16 = (torch.bfloat16,)
+_F32 = (torch.float32,)
+_I32 = (torch.int32,)
+_CODES = (torch.uint8, torch.float8_e4m3fn)
+
+
+def _check_layer(q, k, v, seqlens, out, lse, desc, n_seq: int, n_cache: int) -> None:
+    """The arguments every decode entry point shares: q and out are bf16
+    [n_seq, Hq, D] (possibly with a leading token axis folded into n_seq), lse fp32
+    [n_seq, Hq] or None, seqlens int32 [n_cache], and bf16 K / V caches spanning
+    n_cache sequences."""
+    dev = q.device
+    hq, d = int(desc.n_q_heads), int(desc.head_dim)
+    _dense(q, "q", _BF16, n_seq * hq * d, dev)
+    _extent(k, "k", _BF16, _cache_elems(n_cache, desc), dev)
+    if v is not None:
+        _extent(v, "v", _BF16, _cache_elems(n_cache, desc), dev)
+    _dense(seqlens, "seqlens", _I32, n_cache, dev)
+    _dense(out, "out", _BF16, n_seq * hq * d, dev)
+    if lse is not None:
+        _dense(lse, "lse", _F32, n_seq * hq, dev)
+
+
+def _check_new_rows(k_new, v_new, desc, batch: int, device) -> None:
+    """gdattn_decode_append's rows: bf16 [batch, Hkv, D] (v_new None when K = V)."""
+    rows = batch * int(desc.n_kv_heads) * int(desc.head_dim)
+    _dense(k_new, "k_new", _BF16, rows, device)
+    if v_new is not None:
+        _dense(v_new, "v_new", _BF16, rows, device)
+
+
+def _check_fp8(q, k_codes, v_codes, k_scale, v_scale, seqlens, out, lse, desc,
+               batch: int) -> None:
+    """gdattn_decode_fp8's arguments: e4m3 code caches (uint8 or float8_e4m3fn)
+    spanning ``batch`` sequences, fp32 scales [batch, Hkv, C], the rest as for
+    gdattn_decode."""
+    dev = q.device
+    hq, d = int(desc.n_q_heads), int(desc.head_dim)
+    _dense(q, "q", _BF16, batch * hq * d, dev)
+    n_scales = batch * int(desc.n_kv_heads) * int(desc.cache_capacity)
+    _extent(k_codes, "k_codes", _CODES, _cache_elems(batch, desc), dev)
+    _dense(k_scale, "k_scale", _F32, n_scales, dev)
+    if v_codes is not None:  # None is the C ABI's to refuse (no fp8 path for K = V)
+        _extent(v_codes, "v_codes", _CODES, _cache_elems(batch, desc), dev)
+    if v_scale is not None:
+        _dense(v_scale, "v_scale", _F32, n_scales, dev)
+    _dense(seqlens, "seqlens", _I32, batch, dev)
+    _dense(out, "out", _BF16, batch * hq * d, dev)
+    if lse is not None:
+        _dense(lse, "lse", _F32, batch * hq, dev)
+
+
+def _check_combine(o_partial, lse_partial, out, lse) -> None:
+    """gdattn_combine's arguments: fp32 partials [B, Hq, S, D] and [B, Hq, S],
+    bf16 out [B, Hq, D], fp32 lse [B, Hq]."""
+    B, Hq, S, D = o_partial.shape
+    dev = o_partial.device
+    _dense(o_partial, "o_partial", _F32, B * Hq * S * D, dev)
+    _dense(lse_partial, "lse_partial", _F32, B * Hq * S, dev)
+    _dense(out, "out", _BF16, B * Hq * D, dev)
+    if lse is not None:
+        _dense(lse, "lse", _F32, B * Hq, dev)
+
+
 GDATTN_FLAG_EVEN_UNITS = 1
 
 
@@ -186,8 +294,10 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor], seqlens:
         out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _check_layer(q, k, v, seqlens, out, lse, desc, B, B)
     if workspace is None:
         workspace = alloc_workspace(B, max_seqlen, desc, q.device, stream)
+    _on(workspace, "workspace", q.device)
     st = decode_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(seqlens), B, max_seqlen, desc, _ptr(out),
                     _ptr(lse), _ptr(workspace), workspace.numel(), _stream_handle(stream))
     if st != GDATTN_OK:
@@ -207,8 +317,11 @@ def decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: Optional[torch.Te
         out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _check_layer(q, k, v, seqlens, out, lse, desc, B, B)
+    _check_new_rows(k_new, v_new, desc, B, q.device)
     if workspace is None:
         workspace = alloc_workspace(B, max_seqlen, desc, q.device, stream)
+    _on(workspace, "workspace", q.device)
     st = int(lib().gdattn_decode_append(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k), _ptr(v),
                                         _ptr(seqlens), B, int(max_seqlen), ctypes.byref(desc),
                                         _ptr(out), _ptr(lse), _ptr(workspace),
@@ -241,8 +354,10 @@ def decode_fp8(q: torch.Tensor, k_codes: torch.Tensor, v_codes: torch.Tensor,
         out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _check_fp8(q, k_codes, v_codes, k_scale, v_scale, seqlens, out, lse, desc, B)
     if workspace is None:
         workspace = alloc_workspace(B, max_seqlen, desc, q.device, stream)
+    _on(workspace, "workspace", q.device)
     st = decode_fp8_raw(_ptr(q), _ptr(k_codes), _ptr(v_codes), _ptr(k_scale), _ptr(v_scale),
                         _ptr(seqlens), B, max_seqlen, desc, _ptr(out), _ptr(lse),
                         _ptr(workspace), workspace.numel(), _stream_handle(stream))
@@ -275,12 +390,14 @@ def decode_multi(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor],
         out = torch.empty((T, B, Hq, D), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((T, B, Hq), dtype=torch.float32, device=q.device)
+    _check_layer(q, k, v, seqlens, out, lse, desc, T * B, B)
     if workspace is None:
         n = multi_workspace_size(B, T, max_seqlen, desc)
         if n == 0:
             raise GdattnError(GDATTN_ERR_INVALID_ARG, "gdattn_multi_workspace_size")
         workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
         workspace_init(workspace, stream)
+    _on(workspace, "workspace", q.device)
     st = decode_multi_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(seqlens), B, T, max_seqlen, desc,
                           _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
                           _stream_handle(stream))
@@ -307,6 +424,7 @@ def decode_noalloc(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor],
     Calls that can overlap in time on one device race on the shared scratch.
     """
     B = q.shape[0]
+    _check_layer(q, k, v, seqlens, out, lse, desc, B, B)
     st = decode_noalloc_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(seqlens), B, max_seqlen, desc,
                             _ptr(out), _ptr(lse), _stream_handle(stream))
     if st != GDATTN_OK:
@@ -322,6 +440,7 @@ def combine(o_partial: torch.Tensor, lse_partial: torch.Tensor, out: Optional[to
         out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=o_partial.device)
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=o_partial.device)
+    _check_combine(o_partial, lse_partial, out, lse)
     st = lib().gdattn_combine(_ptr(o_partial), _ptr(lse_partial), B, Hq, S, D, _ptr(out), _ptr(lse),
                               _stream_handle(stream))
     if st != GDATTN_OK:
