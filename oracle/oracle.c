@@ -355,11 +355,19 @@ void oracle_combine(const double *o_parts, const double *lse_parts, int32_t n, i
   }
   double z = 0.0;
   for (int32_t s = 0; s < n; ++s) z += exp(lse_parts[s] - m);
+#if ORACLE_MUTATION == 14
+  double L = m;
+#else
   double L = m + log(z);
+#endif
   *lse = L;
   for (int32_t s = 0; s < n; ++s) {
     if (lse_parts[s] == -INFINITY) continue;
+#if ORACLE_MUTATION == 15
+    double w = exp(lse_parts[s] - m);
+#else
     double w = exp(lse_parts[s] - L);
+#endif
     for (int32_t d = 0; d < D; ++d) out[d] += w * o_parts[(int64_t)s * D + d];
   }
 }

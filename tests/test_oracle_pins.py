@@ -22,6 +22,8 @@ MUTATIONS = {
     11: "row scale applied twice",
     12: "row scales read token-major",
     13: "multi-query tokens not causal",
+    14: "merged LSE is the largest part's",
+    15: "merge weights relative to the largest part, not normalised",
 }
 
 
