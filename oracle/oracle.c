@@ -62,6 +62,9 @@ static double e4m3_to_double(uint8_t code) {
 #endif
   if (e == 15 && m == 7) return NAN;
   double mag = (e == 0) ? ldexp((double)m / 8.0, 1 - bias) : ldexp(1.0 + (double)m / 8.0, e - bias);
+#if ORACLE_MUTATION == 17
+  if (e == 0) mag = ldexp(1.0 + (double)m / 8.0, -bias); /* subnormals with a leading one */
+#endif
   return sign ? -mag : mag;
 }
 
@@ -180,6 +183,9 @@ static int attend(const uint16_t *q, int32_t B, int32_t Hq, const int32_t *lo, c
           sj = softcap * tanh(x / softcap);
 #if ORACLE_MUTATION == 3
           sj = scale * softcap * tanh(dot / softcap); /* cap before scale */
+#endif
+#if ORACLE_MUTATION == 16
+          sj = tanh(x / softcap); /* outer factor cap dropped */
 #endif
         }
         s[j - lo[b]] = sj;

@@ -24,6 +24,8 @@ MUTATIONS = {
     13: "multi-query tokens not causal",
     14: "merged LSE is the largest part's",
     15: "merge weights relative to the largest part, not normalised",
+    16: "soft-cap without its outer factor",
+    17: "e4m3 subnormals decoded with a leading one",
 }
 
 
