@@ -97,12 +97,41 @@ class ClockSampler:
         self.proc = None
         self.path = None
 
-    def start(self):
+    def _ids(self):
+        """nvidia-smi ids for this process's device: its UUID first (a CUDA index
+        and nvidia-smi's index differ when CUDA_VISIBLE_DEVICES remaps devices),
+        then the CUDA index."""
+        ids = []
         try:
-            self.path = os.path.join(tempfile.gettempdir(), f"gdattn_clocks_{os.getpid()}.csv")
+            u = str(torch.cuda.get_device_properties(self.idx).uuid)
+            if u:
+                ids.append(u if u.startswith("GPU-") else "GPU-" + u)
+        except Exception:  # noqa: BLE001 - a device without a UUID: use the index
+            pass
+        ids.append(str(self.idx))
+        return ids
+
+    def _pick_id(self):
+        """The first id that a one-shot nvidia-smi query accepts, or None."""
+        for gid in self._ids():
+            try:
+                r = subprocess.run(["nvidia-smi", f"--id={gid}", "--query-gpu=index",
+                                    "--format=csv,noheader"], capture_output=True, timeout=20)
+            except (OSError, subprocess.TimeoutExpired):
+                continue
+            if r.returncode == 0 and r.stdout.strip():
+                return gid
+        return None
+
+    def start(self):
+        gid = self._pick_id()
+        if gid is None:
+            return
+        self.path = os.path.join(tempfile.gettempdir(), f"gdattn_clocks_{os.getpid()}.csv")
+        try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
+                ["nvidia-smi", f"--id={gid}", f"--query-gpu={self.QUERY}",
                  "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
                 stderr=subprocess.DEVNULL)
             time.sleep(0.3)
@@ -122,18 +151,20 @@ class ClockSampler:
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
+            lines = f.readlines()
+        os.remove(self.path)
+        for line in lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
         if not sm:
             return None
         top = max(sm)

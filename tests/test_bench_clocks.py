@@ -1,0 +1,81 @@
+"""The bench's clock sampler on the CPU, against a stand-in nvidia-smi.
+
+The stand-in accepts only the ids it is told to (as nvidia-smi refuses an id it
+does not know), answers the one-shot id query, and in loop mode prints sample
+lines in the format of the sampler's query until it is terminated.
+"""
+import os
+import stat
+import sys
+import time
+
+import pytest
+
+import bench
+
+FAKE = """#!{python}
+import sys, time
+args = sys.argv[1:]
+gid = next(a.split("=", 1)[1] for a in args if a.startswith("--id="))
+if gid not in {accepted!r}:
+    print("No devices were found", file=sys.stderr)
+    sys.exit(6)
+query = next(a.split("=", 1)[1] for a in args if a.startswith("--query-gpu="))
+if query == "index":
+    print("0")
+    sys.exit(0)
+rows = {rows!r}
+i = 0
+while True:
+    print(rows[i % len(rows)], flush=True)
+    i += 1
+    time.sleep(0.05)
+"""
+
+ROWS = [
+    "0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+    "0, 1950, 1965, 980.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+    "0, 1965, 1965, 650.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+]
+
+
+@pytest.fixture
+def fake_smi(tmp_path, monkeypatch):
+    def make(accepted):
+        path = tmp_path / "nvidia-smi"
+        path.write_text(FAKE.format(python=sys.executable, accepted=list(accepted), rows=ROWS))
+        path.chmod(path.stat().st_mode | stat.S_IXUSR)
+        monkeypatch.setenv("PATH", f"{tmp_path}{os.pathsep}{os.environ['PATH']}")
+    return make
+
+
+def test_sampler_reads_clocks_and_reasons(fake_smi):
+    fake_smi(["0"])
+    c = bench.ClockSampler(0)
+    c.start()
+    assert c.proc is not None
+    time.sleep(0.5)
+    clk = c.stop()
+    assert clk is not None and clk["samples"] >= 3
+    assert clk["sm_max_mhz"] == 1965.0
+    assert 1950.0 <= clk["sm_mhz"] <= 1965.0
+    assert clk["reasons"] == ["sw_power_cap"]
+    assert not os.path.exists(c.path)  # the sample file is removed
+
+
+def test_sampler_prefers_the_device_uuid(fake_smi, monkeypatch):
+    """With CUDA_VISIBLE_DEVICES remapping, the CUDA index is not nvidia-smi's:
+    the UUID is tried first."""
+    fake_smi(["GPU-1234"])
+    c = bench.ClockSampler(0)
+    monkeypatch.setattr(c, "_ids", lambda: ["GPU-1234", "0"])
+    assert c._pick_id() == "GPU-1234"
+    fake_smi(["0"])  # an id it refuses falls through to the next
+    assert c._pick_id() == "0"
+
+
+def test_sampler_without_nvidia_smi_reports_nothing(fake_smi):
+    fake_smi([])  # refuses every id
+    c = bench.ClockSampler(0)
+    c.start()
+    assert c.proc is None and c.stop() is None
