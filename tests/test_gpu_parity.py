@@ -264,6 +264,27 @@ def test_cuda_graph_replay_matches_eager():
         assert torch.equal(o, eo) and torch.equal(l, el)
 
 
+def test_latched_timeout_is_reported_then_cleared():
+    """Failure detection's host side, with no wait made to run out: a workspace
+    whose status word carries the timeout bit (what a kernel whose bounded wait
+    expired leaves behind) reads as GDATTN_ERR_DEVICE_TIMEOUT.  Kernels only set
+    bits, so the latch survives a later call; the read clears it.  With both bits
+    set, the timeout is the one reported."""
+    require_gpu()
+    inp = workloads.random_case(59, 2, 16, 8, 256, 64, [64, 30], window=64)
+    o_ref, l_ref = oracle_for(inp)
+    layer = GpuLayer(inp)
+    word = layer.ws[:4].view(torch.int32)
+    word.fill_(1)  # the timeout bit
+    out, lse = layer.run(check_status=False)
+    assert binding.check_device_status(layer.ws) == binding.GDATTN_ERR_DEVICE_TIMEOUT
+    assert binding.check_device_status(layer.ws) == binding.GDATTN_OK
+    compare(out, lse, o_ref, l_ref, ulp_floor=True, what="call after a latched timeout")
+    word.fill_(3)  # the timeout and sequence-length bits
+    assert binding.check_device_status(layer.ws) == binding.GDATTN_ERR_DEVICE_TIMEOUT
+    assert binding.check_device_status(layer.ws) == binding.GDATTN_OK
+
+
 @pytest.mark.parametrize("split", [2, 7, 33])
 def test_part_counters_return_to_zero(split):
     """Units merged inside the decode kernel leave their arrival counters at
