@@ -1,9 +1,11 @@
-"""The bench's clock sampler on the CPU, against a stand-in nvidia-smi.
+"""The bench's host-side pieces on the CPU: the clock sampler against a
+stand-in nvidia-smi, the peak and traffic records it reads.
 
 The stand-in accepts only the ids it is told to (as nvidia-smi refuses an id it
 does not know), answers the one-shot id query, and in loop mode prints sample
 lines in the format of the sampler's query until it is terminated.
 """
+import json
 import os
 import stat
 import sys
@@ -79,3 +81,33 @@ def test_sampler_without_nvidia_smi_reports_nothing(fake_smi):
     c = bench.ClockSampler(0)
     c.start()
     assert c.proc is None and c.stop() is None
+
+
+def test_traffic_record_is_used_only_for_the_kernels_it_was_taken_on(tmp_path, monkeypatch):
+    rec = {"source_sha": bench.kernel_source_hash(),
+           "kernels": {"sliding": {"dram_bytes_per_launch": 123}}}
+    path = tmp_path / "traffic.json"
+    path.write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "TRAFFIC_RECORD", str(path))
+    assert bench.traffic_for("sliding") == 123
+    assert bench.traffic_for("global") is None  # no entry
+    rec["source_sha"] = "0" * 16  # kernels changed since the counters were taken
+    path.write_text(json.dumps(rec))
+    assert bench.traffic_for("sliding") is None
+    path.write_text("not json")
+    assert bench.traffic_for("sliding") is None
+
+
+def test_committed_traffic_record_names_every_profiled_kernel():
+    with open(bench.TRAFFIC_RECORD) as f:
+        rec = json.load(f)
+    assert set(rec["kernels"]) >= {"sliding", "global", "combine", "fp8_sliding"}
+    for ent in rec["kernels"].values():
+        assert ent["dram_bytes_per_launch"] > 0
+
+
+def test_peak_falls_back_without_a_measured_record(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_peak_gbs() == (bench.FALLBACK_HBM_GBS, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6450.0}))
+    assert bench.measured_peak_gbs() == (6450.0, "measured")
