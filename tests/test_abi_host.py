@@ -69,6 +69,19 @@ def test_desc_layout_matches_c(tmp_path):
     assert vals == expect
 
 
+def test_plain_c_client_links_and_gets_the_documented_statuses(lib, tmp_path):
+    """tests/abi_client.c: a C99 program that includes only gdattn.h, links the
+    shared library and checks the statuses of calls the host checks refuse."""
+    pkg = os.path.dirname(binding.LIB_PATH)
+    exe = tmp_path / "abi_client"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "abi_client.c"), "-o", str(exe),
+                    f"-L{pkg}", "-lgdattn", f"-Wl,-rpath,{pkg}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
 def test_version_and_status_strings(lib):
     assert binding.version() == 100
     assert binding.status_string(0) == "GDATTN_OK"
