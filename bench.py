@@ -24,8 +24,8 @@ import json
 import os
 import statistics
 import subprocess
-import tempfile
 import sys
+import tempfile
 import time
 
 import torch
