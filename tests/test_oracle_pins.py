@@ -61,3 +61,22 @@ def test_golden_kv_bytes_per_token():
     assert per_tok(stack, True) == g["total_bytes_per_token"]
     # K = V read once: the full layers' term halves.
     assert per_tok(stack, False) == g["sliding_bytes_per_token"] + g["full_bytes_per_token"] // 2
+
+
+def test_step_bytes_of_the_headline_workload():
+    """Algorithmic bytes of one 48-layer step at batch 8, context 8192, written out
+    by hand: each sliding layer reads the last 1024 positions of K and V for 8 KV
+    heads of 256 bf16 values; each global layer reads all 8192 positions of its
+    one K = V tensor of 512 bf16 values.  With fp8 sliding caches a sliding row is
+    256 one-byte codes plus a 4-byte scale."""
+    from decode_attention_09_b200 import accounting
+
+    w = workloads.gemma4_12b_b8_l8192()
+    sl = w.seqlens().tolist()
+    bf16 = sum(accounting.layer_kv_bytes(s, sl) for s in w.layers)
+    sliding = 40 * 8 * 1024 * (8 * 256 * 2) * 2
+    glob = 8 * 8 * 8192 * (1 * 512 * 2)
+    assert bf16 == sliding + glob == 3_221_225_472
+    fp8 = sum(accounting.layer_fp8_kv_bytes(s, sl) for s in w.layers if s.kind == "sliding")
+    assert fp8 == 40 * 8 * 1024 * (8 * (256 + 4)) * 2 == 1_363_148_800
+    assert accounting.layer_kv_bytes(w.layers[0], [5]) == 5 * 8 * 256 * 2 * 2  # L < w
