@@ -9,6 +9,8 @@ anything is enqueued.
 """
 import pytest
 import torch
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
 
 import workloads
 from decode_attention_09_b200 import binding
@@ -179,3 +181,30 @@ def test_headline_stack_layers_pass(any_device):
     f8 = workloads.fp8_layer_inputs(spec, w.batch, sl, 2)
     check_fp8(f8, binding.desc_from_spec(spec), torch.empty_like(f8.q),
               torch.empty(f8.q.shape[:2]))
+
+
+# the fixture only patches out the device check: the same for every example
+@settings(max_examples=30, deadline=None, derandomize=True,
+          suppress_health_check=[HealthCheck.function_scoped_fixture])
+@given(hkv=st.sampled_from([1, 2, 4, 8]), g=st.sampled_from([1, 2, 4, 16]),
+       d=st.sampled_from([256, 512]), cap=st.integers(1, 70), batch=st.integers(1, 4),
+       tokens=st.integers(1, 4), shared=st.booleans(), pad=st.integers(0, 3))
+def test_any_well_formed_call_passes(any_device, hkv, g, d, cap, batch, tokens, shared, pad):
+    """Whatever the geometry, the tensors a caller lays out as the header says pass
+    the checks, with dense caches or with sequences `pad` rows apart."""
+    inp = workloads.random_case(7, batch, hkv * g, hkv, d, cap, [cap] * batch,
+                                kv_shared=shared)
+    desc = binding.desc_from_spec(inp.spec, capacity=cap)
+    if pad:
+        big = torch.zeros((batch, cap + pad, hkv, d), dtype=torch.bfloat16)
+        big[:, :cap] = inp.k
+        desc.cache_batch_stride = (cap + pad) * hkv * d
+        k = big[:, :cap]
+        v = None if shared else big[:, :cap]
+    else:
+        k, v = inp.k, inp.v
+    out = torch.empty((batch, hkv * g, d), dtype=torch.bfloat16)
+    binding._check_layer(inp.q, k, v, inp.seqlens, out, None, desc, batch, batch)
+    q = torch.zeros((tokens, batch, hkv * g, d), dtype=torch.bfloat16)
+    binding._check_layer(q, k, v, inp.seqlens, torch.empty_like(q),
+                         torch.empty((tokens, batch, hkv * g)), desc, tokens * batch, batch)
