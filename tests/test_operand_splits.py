@@ -1,4 +1,10 @@
-"""The error bounds of the fp8 pair kernel's operand splits, checked on the CPU.
+"""The error bounds of the tcgen05 kernels' operand splits, checked on the CPU.
+
+bf16 kernels: an MMA's two operands share one type, and V is bf16, so the fp32
+softmax weights go in as two bf16 pieces, p = p_hi + p_lo with p_hi = bf16(p)
+and p_lo = bf16(p - p_hi), in separate MMA columns summed in fp32.
+
+fp8 kernel:
 
 The kernel multiplies e4m3 cache codes on the tensor cores against q and against
 the softmax weights, each represented as three e4m3 pieces scaled 1, 1/16 and
@@ -72,3 +78,15 @@ def test_pieces_stay_inside_e4m3_range():
     for p in split3(x):
         assert p.abs().max().item() <= 448
         assert torch.isfinite(p).all()
+
+
+def test_bf16_hi_lo_weight_split():
+    """Two bf16 pieces keep an fp32 weight to 2^-17 relative; one piece keeps 2^-8."""
+    g = torch.Generator().manual_seed(2)
+    p = torch.exp2(torch.rand(1_000_000, generator=g, dtype=torch.float64) * 40 - 32).float()
+    hi = p.to(torch.bfloat16).float()
+    lo = (p - hi).to(torch.bfloat16).float()
+    rel = ((hi.double() + lo.double()) - p.double()).abs() / p.double()
+    assert rel.max().item() <= 2.0 ** -17
+    one = (hi.double() - p.double()).abs() / p.double()
+    assert 2.0 ** -9 < one.max().item() <= 2.0 ** -8  # what a single piece would keep
