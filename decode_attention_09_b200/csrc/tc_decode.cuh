@@ -18,7 +18,7 @@
 // bf16), so each weight p is split into p_hi = bf16(p) and p_lo = bf16(p - p_hi):
 // the 32 columns of P^T are the 16 heads' p_hi then their p_lo, and O^T for a head
 // is the sum of its two column blocks.  That keeps the weights to ~2^-17
-// relative error instead of 2^-9, which matters when a few large key rows
+// relative error instead of 2^-8, which matters when a few large key rows
 // dominate the weighted sum of values.
 //
 // K = V: the one 64-token tile in shared memory is the K-major A operand of the
