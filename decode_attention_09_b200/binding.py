@@ -99,6 +99,8 @@ def lib() -> ctypes.CDLL:
         L.gdattn_combine.restype = ctypes.c_int
         L.gdattn_check_device_status.argtypes = [vp, vp]
         L.gdattn_check_device_status.restype = ctypes.c_int
+        L.gdattn_read_probe.argtypes = [vp, sz, i32, vp, vp]
+        L.gdattn_read_probe.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -451,3 +453,15 @@ def combine(o_partial: torch.Tensor, lse_partial: torch.Tensor, out: Optional[to
 def check_device_status(workspace: Optional[torch.Tensor], stream=None) -> int:
     """Read and clear a workspace's status word (None: the no-alloc scratch)."""
     return int(lib().gdattn_check_device_status(_ptr(workspace), _stream_handle(stream)))
+
+
+def read_probe(src: torch.Tensor, mode: int, sink: torch.Tensor, stream=None) -> None:
+    """gdattn_read_probe over the whole of ``src`` (a contiguous device tensor);
+    ``sink``: int32 tensor of 2 elements on the same device."""
+    _on(sink, "sink", src.device)
+    if not src.is_contiguous() or sink.numel() < 2 or sink.dtype != torch.int32:
+        raise ValueError("read_probe: contiguous src and an int32 sink of 2 elements")
+    st = lib().gdattn_read_probe(_ptr(src), src.numel() * src.element_size(), int(mode),
+                                 _ptr(sink), _stream_handle(stream))
+    if st != GDATTN_OK:
+        raise GdattnError(st, "gdattn_read_probe")

@@ -13,6 +13,7 @@
 
 #include "combine.cuh"
 #include "core_decode.cuh"
+#include "read_probe.cuh"
 #include "tc_decode.cuh"
 #include "tc_pair_decode.cuh"
 #include "tc_pair_fp8_decode.cuh"
@@ -20,7 +21,8 @@
 using namespace gdattn;
 
 // Split-KV scratch of gdattn_decode_noalloc: one array per device context,
-// laid out like a caller workspace (status word, partial LSE, partial O).
+// laid out like a caller workspace (the fixed header of status word, part
+// counters and epochs, then partial LSE and partial O).
 // A __device__ array without initialiser occupies no space in the binary.
 constexpr size_t kNoallocScratchBytes = GDATTN_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
@@ -47,6 +49,17 @@ struct LayerPlan {
 };
 
 constexpr size_t kStatusBytes = 256;
+// Every workspace starts with the same header, whatever the plan: the status
+// word, then one part counter and one epoch per unit index below kMaxUnits.
+// Counters must read zero and epochs must hold the last call's tag when a call
+// starts; with fixed offsets no plan's partials ever land on them, so calls
+// with different plans (geometry, batch, split) can take turns on one
+// workspace.  A plan with more units is refused.
+constexpr int64_t kMaxUnits = 16384;
+constexpr size_t kOffCounters = kStatusBytes;
+constexpr size_t kOffEpochs = kOffCounters + 4 * kMaxUnits;
+constexpr size_t kHeaderBytes = kOffEpochs + 4 * kMaxUnits;
+static_assert(kHeaderBytes % 256 == 0, "partials start 256-byte aligned");
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -167,6 +180,11 @@ int query_tc_pair_append(const void *fn, int threads, int smem) {
   return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
 }
 
+int query_probe(const void *fn, int threads, int smem) {
+  return blocks_per_sm(reinterpret_cast<void (*)(const ReadProbeParams)>(const_cast<void *>(fn)),
+                       threads, smem);
+}
+
 // ---------------------------------------------------------------- planning
 gdattn_status check_desc(const gdattn_layer_desc *d) {
   if (d == nullptr) return GDATTN_ERR_INVALID_ARG;
@@ -203,6 +221,11 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
   pl.kind = choose_path(d);
   if (pl.kind == PathKind::kNone || (fp8 && pl.kind != PathKind::kTcPair))
     return GDATTN_ERR_UNSUPPORTED;
+  // Units (query-head groups) of the call: one per sequence on the CUDA-core
+  // path, one per (sequence, KV head) on the tcgen05 paths.
+  const int64_t units =
+      static_cast<int64_t>(batch) * (pl.kind == PathKind::kCore ? 1 : d->n_kv_heads);
+  if (units > kMaxUnits) return GDATTN_ERR_UNSUPPORTED;
   const int nsm = sm_count();
   if (nsm <= 0) return GDATTN_ERR_CUDA;
   int per_sm = 1, min_tokens = 64;
@@ -254,7 +277,6 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
   int64_t per_unit = max_seqlen;
   if (d->window > 0 && d->window < per_unit) per_unit = d->window;
   if (d->cache_capacity < per_unit) per_unit = d->cache_capacity;
-  const int64_t units = static_cast<int64_t>(batch) * pl.units_per_seq;
   const int64_t total = units * per_unit;
   int64_t grid = (total + min_tokens - 1) / min_tokens;
   const int64_t cap = static_cast<int64_t>(nsm) * per_sm;
@@ -283,9 +305,9 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
   pl.merge_in_kernel = pl.kind == PathKind::kTcPair;
   pl.tagged = pl.merge_in_kernel && pl.split_k > 1;
   const size_t elem = pl.tagged ? 8 : 4;
-  pl.off_cnt = kStatusBytes;
-  pl.off_epoch = align256(pl.off_cnt + static_cast<size_t>(units) * 4);
-  pl.off_lse = align256(pl.off_epoch + static_cast<size_t>(units) * 4);
+  pl.off_cnt = kOffCounters;
+  pl.off_epoch = kOffEpochs;
+  pl.off_lse = kHeaderBytes;
   pl.off_o = align256(pl.off_lse + static_cast<size_t>(pl.slots) * pl.heads_per_unit * elem);
   pl.bytes =
       align256(pl.off_o + static_cast<size_t>(pl.slots) * pl.heads_per_unit * d->head_dim * elem);
@@ -604,24 +626,75 @@ size_t multi_bytes(const LayerPlan &pl, int32_t batch, int32_t T) {
 // -------------------------------------------------- fixed scratch (no alloc)
 constexpr int kMaxDevices = 64;
 
-// Address of g_noalloc_scratch on the current device.  The first call on a
-// device looks it up and enqueues a clear of the array on `stream`: the status
-// word and the per-unit part counters must start at zero (every call leaves
-// the counters at zero again); partial slots are written before they are read.
+// Process-unique id of the current CUDA context (cuCtxGetId), so that a
+// context created after a reset is never mistaken for its predecessor even if
+// it reuses the handle.  0 when the driver cannot say.
+unsigned long long current_context_id() {
+  using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+  using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+  static CtxGetCurrentFn get_current = []() -> CtxGetCurrentFn {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  static CtxGetIdFn get_id = []() -> CtxGetIdFn {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<CtxGetIdFn>(p);
+  }();
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS ||
+      ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Address of g_noalloc_scratch in the current device's context.  The first
+// call in a context looks it up and enqueues a clear of the whole array on
+// `stream`: the status word and the part counters must start at zero (every
+// call leaves the counters at zero again); partial slots are written before
+// they are read.  That first call must not be captured (the clear would only
+// run at replay while later eager calls assumed it done): it returns
+// GDATTN_ERR_INVALID_ARG while `stream` is capturing and records nothing.
 gdattn_status noalloc_scratch(cudaStream_t stream, uint8_t **addr) {
+  struct Entry {
+    unsigned long long ctx_id;
+    void *ptr;
+  };
   static std::mutex mu;
-  static void *by_device[kMaxDevices] = {};
+  static Entry by_device[kMaxDevices] = {};
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDATTN_ERR_CUDA;
+  unsigned long long ctx_id = current_context_id();
+  if (ctx_id == 0) {
+    // No current context yet: the runtime creates the device's primary
+    // context (and makes it current) on its first call that needs one.
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return GDATTN_ERR_CUDA;
+    ctx_id = current_context_id();
+    if (ctx_id == 0) return GDATTN_ERR_CUDA;
+  }
   std::lock_guard<std::mutex> lock(mu);
-  if (by_device[dev] == nullptr) {
+  Entry &e = by_device[dev];
+  if (e.ptr == nullptr || e.ctx_id != ctx_id) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return GDATTN_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone) return GDATTN_ERR_INVALID_ARG;
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return GDATTN_ERR_CUDA;
     if (cudaMemsetAsync(p, 0, kNoallocScratchBytes, stream) != cudaSuccess) return GDATTN_ERR_CUDA;
-    by_device[dev] = p;
+    e.ptr = p;
+    e.ctx_id = ctx_id;
   }
-  *addr = static_cast<uint8_t *>(by_device[dev]);
+  *addr = static_cast<uint8_t *>(e.ptr);
   return GDATTN_OK;
 }
 
@@ -827,6 +900,35 @@ gdattn_status gdattn_combine(const float *o_partial, const float *lse_partial, i
                                          static_cast<cudaStream_t>(stream), attr);
   return cudaLaunchKernelEx(&cfg, combine_kernel<false>, cp) == cudaSuccess ? GDATTN_OK
                                                                              : GDATTN_ERR_CUDA;
+}
+
+gdattn_status gdattn_read_probe(const void *src, size_t bytes, int32_t mode, uint32_t *sink,
+                                void *stream_) {
+  if (src == nullptr || sink == nullptr || bytes == 0 || (bytes & 15u) != 0 ||
+      (mode != 0 && mode != 1))
+    return GDATTN_ERR_INVALID_ARG;
+  if (!aligned16(src) || (reinterpret_cast<uintptr_t>(sink) & 3u)) return GDATTN_ERR_MISALIGNED;
+  const int nsm = sm_count();
+  if (nsm <= 0) return GDATTN_ERR_CUDA;
+  ReadProbeParams rp;
+  rp.src = static_cast<const uint8_t *>(src);
+  rp.bytes = static_cast<int64_t>(bytes);
+  rp.sink = sink;
+  rp.status = sink + 1;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (mode == 0) {
+    const int per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(read_probe_ldg_kernel),
+                                            kReadProbeThreads, 0, query_probe);
+    if (per_sm <= 0) return GDATTN_ERR_CUDA;
+    read_probe_ldg_kernel<<<nsm * per_sm, kReadProbeThreads, 0, stream>>>(rp);
+  } else {
+    using Cfg = ReadProbeBulkConfig;
+    if (cached_blocks_per_sm(reinterpret_cast<const void *>(read_probe_bulk_kernel), Cfg::kThreads,
+                             Cfg::SMEM, query_probe) <= 0)
+      return GDATTN_ERR_CUDA;
+    read_probe_bulk_kernel<<<nsm, Cfg::kThreads, Cfg::SMEM, stream>>>(rp);
+  }
+  return cudaGetLastError() == cudaSuccess ? GDATTN_OK : GDATTN_ERR_CUDA;
 }
 
 gdattn_status gdattn_check_device_status(void *workspace, void *stream_) {

@@ -173,8 +173,15 @@ __device__ __forceinline__ uint64_t ld_u64_volatile(const uint64_t *addr) {
 }
 
 __device__ __forceinline__ uint32_t tag_of(uint64_t w) { return static_cast<uint32_t>(w >> 32); }
-// Tags count calls and never take the value 0 of a cleared word.
-__device__ __forceinline__ uint32_t next_tag(uint32_t epoch) { return epoch + 1 == 0 ? 1 : epoch + 1; }
+// Tags count calls.  They are the bit patterns 0x7F800001 .. 0x7FBFFFFE: NaNs
+// with the quiet bit clear, which no arithmetic produces (the GPU's NaN result
+// is 0x7FFFFFFF), so neither a cleared word (0) nor a finite partial that
+// another plan's call left in the same workspace bytes can pass for a tag.
+// Any epoch value, even garbage, yields a valid next tag.
+__device__ __forceinline__ uint32_t next_tag(uint32_t epoch) {
+  const uint32_t n = (epoch & 0x003FFFFFu) + 1u;
+  return 0x7F800000u | (n >= 0x003FFFFFu ? 1u : n);
+}
 __device__ __forceinline__ float payload_of(uint64_t w) {
   return __uint_as_float(static_cast<uint32_t>(w));
 }

@@ -29,7 +29,9 @@
  *
  * Conventions for every entry point:
  *  - All tensors are caller-owned.  The library allocates no device or host
- *    memory and keeps no state between calls; calls are thread-safe.
+ *    memory and keeps no state between calls, and calls are thread-safe, with
+ *    one exception: gdattn_decode_noalloc keeps its scratch in one array per
+ *    device context inside the library, shared by all its calls (see there).
  *  - Device pointers must be 16-byte aligned and rows are contiguous along the
  *    head dimension.  bf16 means IEEE bfloat16, stored as 16-bit words.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
@@ -107,9 +109,16 @@ typedef struct gdattn_layer_desc {
 
 /*
  * Bytes of device workspace gdattn_decode needs for this layer geometry and
- * batch on the current CUDA device (partial results of split ranges plus a
- * 256-byte status word).  max_seqlen is the host's upper bound on seqlens[];
- * it only steers the split count.  Returns 0 on invalid arguments.
+ * batch on the current CUDA device.  max_seqlen is the host's upper bound on
+ * seqlens[]; it only steers the split count.  Returns 0 on invalid arguments.
+ *
+ * Every workspace starts with the same 128 KiB + 256 B header: the status
+ * word, then a part counter and a merge epoch for each (sequence, KV head)
+ * unit index below 16384; the partial results of split ranges follow.  Since
+ * the header never moves, calls with different geometries, batches or splits
+ * may take turns on one workspace (ordered on one stream) if it holds the
+ * largest of their sizes.  A call with batch * n_kv_heads > 16384 (times
+ * n_tokens for gdattn_decode_multi) returns GDATTN_ERR_UNSUPPORTED.
  */
 size_t gdattn_workspace_size(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *desc);
 
@@ -148,8 +157,9 @@ gdattn_status gdattn_workspace_init(void *workspace, size_t workspace_bytes, voi
  *  out      bf16 [batch, Hq, D], device, written
  *  lse      fp32 [batch, Hq], device, written (natural log), or NULL
  *  workspace / workspace_bytes: device scratch of at least gdattn_workspace_size
- *           bytes, status word zeroed once by gdattn_workspace_init.  Calls that
- *           share a workspace must be ordered on one stream.
+ *           bytes, zeroed once by gdattn_workspace_init.  Calls that share a
+ *           workspace must be ordered on one stream; they may differ in
+ *           geometry and batch (see gdattn_workspace_size).
  *
  * Supported geometries (G = Hq / Hkv), by the kernel that runs them:
  *  - G == 2, D == 256, separate V, any Hkv: tcgen05 pair kernel;
@@ -163,6 +173,11 @@ gdattn_status gdattn_decode(const void *q, const void *k_cache, const void *v_ca
                             void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * The log-sum-exp combine of split decode attention ("Gemma support" PR,
+ * Performance: split decode attention for head sizes 256/512; "Gemma 4 12B",
+ * item 4: single-query global layers split the KV range into num_splits parts
+ * whose partial results are merged).
+ *
  * Merge n_splits partial results per (sequence, head), each normalised over its
  * own part of the position range:
  *   lse = log sum_s exp(lse_s),  out = sum_s exp(lse_s - lse) * o_s.
@@ -282,9 +297,16 @@ gdattn_status gdattn_decode_multi(const void *q, const void *k_cache, const void
  * part counters, partial LSE, partial O) is one fixed array inside the library,
  * GDATTN_NOALLOC_SCRATCH_BYTES per device context, reserved when the library's
  * device code is loaded, so no call allocates device or host memory.
- *  - The first call on each device looks the array up (cudaGetSymbolAddress)
- *    and enqueues a clear of the whole array on `stream`; make that first call
- *    outside stream capture.  Later calls only enqueue kernels.
+ *  - The first call in each device context looks the array up
+ *    (cudaGetSymbolAddress) and enqueues a clear of the whole array on
+ *    `stream`; later calls only enqueue kernels.  That first call must not be
+ *    captured into a CUDA graph: made while `stream` is capturing it returns
+ *    GDATTN_ERR_INVALID_ARG and enqueues nothing.  A context created after a
+ *    reset (cudaDeviceReset) counts as new: its first call looks up and clears
+ *    the array again.
+ *  - The array has the workspace layout of gdattn_workspace_size (fixed
+ *    header, then partials), so calls with different geometries and batches
+ *    may follow one another.
  *  - A layer whose gdattn_workspace_size exceeds GDATTN_NOALLOC_SCRATCH_BYTES
  *    returns GDATTN_ERR_WORKSPACE and enqueues nothing; use gdattn_decode.
  *  - One array per device: calls that can overlap in time on one device (on
@@ -309,6 +331,25 @@ gdattn_status gdattn_decode_noalloc(const void *q, const void *k_cache, const vo
  * if none).
  */
 gdattn_status gdattn_check_device_status(void *workspace, void *stream);
+
+/*
+ * Read-only streaming probe: the practical ceiling of HBM read bandwidth for
+ * the loads the decode kernels use, to set their roofline fractions against.
+ * A measurement utility with no counterpart in the pages.
+ *
+ *  src    device buffer of `bytes` bytes (16-byte aligned, bytes a multiple of
+ *         16 and > 0), read once
+ *  mode   0: every thread streams 16-byte vector loads (non-coherent, no L1
+ *         allocation, evict-first in L2), grid of resident CTAs on all SMs;
+ *         1: one CTA per SM copies 32 KiB chunks of its contiguous share into a
+ *         six-stage shared-memory ring with bulk copies (cp.async.bulk)
+ *  sink   uint32_t[2], device: the XOR of the data read is folded into sink[0]
+ *         (so the loads cannot be removed); sink[1] latches the device status
+ *         bits (a bounded wait that expired in mode 1)
+ * One kernel launch on `stream`; time it with events around the call.
+ */
+gdattn_status gdattn_read_probe(const void *src, size_t bytes, int32_t mode, uint32_t *sink,
+                                void *stream);
 
 /* Static, human-readable name of a status code. */
 const char *gdattn_status_string(gdattn_status status);

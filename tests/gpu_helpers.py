@@ -88,3 +88,30 @@ def oracle_for(inp, batch_index=None):
     v = inp.v.index_select(0, idx.to(inp.v.device)).cpu() if inp.v is not None else None
     sl = inp.seqlens.cpu().index_select(0, idx)
     return orc.decode(q, k, v, sl, s.window, s.softcap, s.scale)
+
+
+def oracle_per_sequence(inp, batch_index=None, workers=None):
+    """Oracle result for the listed sequences (all by default), one oracle call
+    per sequence spread over the host cores: the C oracle releases the GIL, so
+    threads run it in parallel.  Each sequence's inputs are copied to the host
+    first (in this thread).  Returns (out [n,Hq,D], lse [n,Hq]) float64 in the
+    order of ``batch_index``."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    orc = oracle.get()
+    s = inp.spec
+    picks = list(range(inp.q.shape[0])) if batch_index is None else list(batch_index)
+    jobs = []
+    for b in picks:
+        q = inp.q[b:b + 1].cpu()
+        k = inp.k[b:b + 1].cpu()
+        v = inp.v[b:b + 1].cpu() if inp.v is not None else None
+        sl = inp.seqlens[b:b + 1].cpu()
+        jobs.append((q, k, v, sl))
+    n = workers or max(1, min(len(jobs), len(os.sched_getaffinity(0))))
+    with ThreadPoolExecutor(max_workers=n) as ex:
+        res = list(ex.map(lambda a: orc.decode(a[0], a[1], a[2], a[3], s.window, s.softcap,
+                                               s.scale), jobs))
+    return (np.concatenate([r[0] for r in res], axis=0),
+            np.concatenate([r[1] for r in res], axis=0))

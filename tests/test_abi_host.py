@@ -155,6 +155,15 @@ def test_tensor_core_path_needs_shared_kv(lib):
     assert call(d) == binding.GDATTN_ERR_UNSUPPORTED
 
 
+def test_unit_count_beyond_the_fixed_header_is_refused(lib):
+    """The workspace header holds counters and epochs for 16384 (sequence, KV
+    head) units; a call with more is refused before anything is enqueued."""
+    assert call(good_desc(), batch=2049) == binding.GDATTN_ERR_UNSUPPORTED  # 16392 units
+    assert binding.workspace_size(2049, 8, good_desc()) == 0
+    core = good_desc(n_q_heads=4, n_kv_heads=1, head_dim=256, window=0)  # one unit per sequence
+    assert call(core, v=A, batch=16385) == binding.GDATTN_ERR_UNSUPPORTED
+
+
 def test_workspace_size_rejects_bad_args(lib):
     assert binding.workspace_size(0, 8, good_desc()) == 0
     assert binding.workspace_size(1, 8, good_desc(head_dim=128)) == 0

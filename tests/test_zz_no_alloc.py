@@ -233,3 +233,97 @@ def test_noalloc_even_split_matches_workspace_decode():
         torch.cuda.synchronize()
         assert binding.check_device_status(None) == binding.GDATTN_OK
         assert_same(got, ref, f"even split call {rep}")
+
+
+def _many_unit_layers():
+    """Plans whose header use and partial areas differ widely, drawn on the GPU
+    (the test compares two library paths, not the oracle): a ragged sliding
+    layer of 512 units (counted merge), a global layer of 64 units (combine
+    kernel, partials right after the header), and even-split sliding layers of
+    136 and 512 units (tagged merge), some with soft-cap."""
+    g = torch.Generator(device="cpu").manual_seed(907)
+    rag = torch.randint(1, 2200, (64,), generator=g).tolist()
+    specs = [
+        # (seed, B, Hq, Hkv, D, C, seqlens, window, cap, shared, flags)
+        (911, 64, 16, 8, 256, 1024, rag, 1024, 50.0, False, 0),
+        (912, 64, 16, 1, 512, 2200, rag, 0, 0.0, True, 0),
+        (913, 17, 16, 8, 256, 512, [1500] * 17, 512, 0.0, False, binding.GDATTN_FLAG_EVEN_UNITS),
+        (914, 64, 16, 8, 256, 1024, [3000] * 64, 1024, 30.0, False,
+         binding.GDATTN_FLAG_EVEN_UNITS),
+        (915, 64, 16, 1, 512, 1024, [1024] * 64, 0, 0.0, True, binding.GDATTN_FLAG_EVEN_UNITS),
+    ]
+    layers = []
+    for seed, B, Hq, Hkv, D, C, sl, w, cap, shared, flags in specs:
+        inp = workloads.random_case(seed, B, Hq, Hkv, D, C, sl, window=w, softcap=cap,
+                                    kv_shared=shared, device="cuda")
+        ly = Dev(inp, 0)
+        ly.desc = binding.desc_from_spec(inp.spec, capacity=C, flags=flags)
+        layers.append(ly)
+    return layers
+
+
+@pytest.mark.gpu
+def test_noalloc_alternating_plans_with_many_units():
+    """Layouts whose unit counts exceed 64 take turns on the fixed scratch, in
+    both orders, twice: every call equals gdattn_decode bit for bit and no
+    device-side error is latched.  (Counters and epochs sit at fixed offsets,
+    so no plan's partials land on another plan's counters.)"""
+    require_gpu()
+    layers = _many_unit_layers()
+    for ly in layers:
+        assert binding.workspace_size(ly.B, ly.max_seqlen, ly.desc) <= \
+            binding.NOALLOC_SCRATCH_BYTES
+    ref = [ly.with_workspace() for ly in layers]
+    order = list(range(len(layers)))
+    for rep, seq in enumerate([order, order[::-1], order, [0, 2, 0, 3, 1, 3, 2]]):
+        for i in seq:
+            got = layers[i].outputs()
+            layers[i].noalloc(*got)  # no synchronisation between the calls
+            torch.cuda.synchronize()
+            assert binding.check_device_status(None) == binding.GDATTN_OK, (rep, i)
+            assert_same(got, ref[i], f"sequence {rep} layer {i}")
+
+
+_FIRST_CALL_CAPTURED = r"""
+import sys, torch
+sys.path.insert(0, sys.argv[1])
+import workloads
+from decode_attention_09_b200 import binding
+inp = workloads.random_case(921, 2, 16, 8, 256, 128, [128, 77], window=128, device="cuda")
+desc = binding.desc_from_spec(inp.spec, capacity=128)
+out = torch.empty_like(inp.q)
+lse = torch.empty(inp.q.shape[:2], device="cuda")
+args = lambda s: (binding._ptr(inp.q), binding._ptr(inp.k), binding._ptr(inp.v),
+                  binding._ptr(inp.seqlens), 2, 128, desc, binding._ptr(out), binding._ptr(lse), s)
+torch.cuda.synchronize()
+s = torch.cuda.Stream()
+g = torch.cuda.CUDAGraph()
+with torch.cuda.stream(s):
+    with torch.cuda.graph(g, stream=s):
+        st_captured = binding.decode_noalloc_raw(*args(s.cuda_stream))
+st_eager = binding.decode_noalloc_raw(*args(None))
+torch.cuda.synchronize()
+ref_out, ref_lse = binding.decode(inp.q, inp.k, inp.v, inp.seqlens, desc, 128)
+torch.cuda.synchronize()
+same = torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
+print(st_captured, st_eager, binding.check_device_status(None), int(same))
+"""
+
+
+@pytest.mark.gpu
+def test_noalloc_first_call_refused_under_capture():
+    """In a fresh process (so the call really is the context's first), a first
+    call made while its stream is capturing returns GDATTN_ERR_INVALID_ARG and
+    enqueues nothing; the next, eager call sets the scratch up and computes
+    gdattn_decode's result."""
+    require_gpu()
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _FIRST_CALL_CAPTURED, root], capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    st_cap, st_eager, st_dev, same = (int(x) for x in r.stdout.split()[-4:])
+    assert st_cap == binding.GDATTN_ERR_INVALID_ARG
+    assert st_eager == binding.GDATTN_OK and st_dev == binding.GDATTN_OK and same == 1
