@@ -204,7 +204,7 @@ gdattn_status check_desc(const gdattn_layer_desc *d) {
 
 PathKind choose_path(const gdattn_layer_desc *d) {
   const int g = d->n_q_heads / d->n_kv_heads;
-  if (g == 16 && d->head_dim == 512 && d->kv_shared == 1) return PathKind::kTc;
+  if ((g == 16 || g == 8) && d->head_dim == 512) return PathKind::kTc;
   if (g == 2 && d->head_dim == 256 && d->kv_shared == 0) return PathKind::kTcPair;
   if ((d->head_dim == 256 || d->head_dim == 512) && (g == 1 || g == 2 || g == 4) &&
       (d->n_kv_heads == 1 || d->n_kv_heads == 2 || d->n_kv_heads == 4 || d->n_kv_heads == 8))
@@ -240,17 +240,31 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
     pl.units_per_seq = 1;
     pl.heads_per_unit = d->n_q_heads;
   } else if (pl.kind == PathKind::kTc) {
-    per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_kernel),
+    // Every instantiation of the 16-head kernel shares one configuration; the
+    // queries also set each one's shared-memory attribute before its launch.
+    per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_kernel<16>),
                                   TcConfig::kThreads, TcConfig::SMEM, query_tc);
-    // The append entry point shares the configuration (and needs the same
-    // shared-memory attribute, set by the query).
-    if (cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_append_kernel),
-                             TcConfig::kThreads, TcConfig::SMEM, query_tc_append) != per_sm)
-      return GDATTN_ERR_CUDA;
+    const int others[] = {
+        cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_kernel<8>),
+                             TcConfig::kThreads, TcConfig::SMEM, query_tc),
+        cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_append_kernel<16>),
+                             TcConfig::kThreads, TcConfig::SMEM, query_tc_append),
+        cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_append_kernel<8>),
+                             TcConfig::kThreads, TcConfig::SMEM, query_tc_append),
+        cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_kv_kernel<16>),
+                             TcConfig::kThreads, TcConfig::SMEM, query_tc_pair),
+        cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_kv_kernel<8>),
+                             TcConfig::kThreads, TcConfig::SMEM, query_tc_pair),
+        cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_kv_append_kernel<16>),
+                             TcConfig::kThreads, TcConfig::SMEM, query_tc_pair_append),
+        cached_blocks_per_sm(reinterpret_cast<const void *>(tc_decode_kv_append_kernel<8>),
+                             TcConfig::kThreads, TcConfig::SMEM, query_tc_pair_append)};
+    for (int nb : others)
+      if (nb != per_sm) return GDATTN_ERR_CUDA;
     min_tokens = 2 * TcConfig::TILE;
     pl.align = TcConfig::TILE;
     pl.units_per_seq = d->n_kv_heads;
-    pl.heads_per_unit = TcConfig::G;
+    pl.heads_per_unit = d->n_q_heads / d->n_kv_heads;  // 8 or 16 (the kernel pads to 16)
   } else if (fp8) {
     per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_fp8_decode_kernel),
                                   TcPairFp8Config::kThreads, TcPairFp8Config::SMEM,
@@ -290,6 +304,9 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
   if ((d->flags & GDATTN_FLAG_EVEN_UNITS) && d->split_ctas == 0 && pl.kind != PathKind::kCore) {
     const int64_t tiles = (per_unit + pl.align - 1) / pl.align;
     int64_t best = tiles;
+    // At most 64 parts per unit: the LSE merge of more parts costs more than the
+    // shorter parts save (one 32 KiB unit of 16 heads merged from 128 parts took
+    // longer than from 64).
     for (int64_t k = 2; k <= tiles && units * k <= cap && k <= 64; ++k) {
       const int64_t most = (tiles + k - 1) / k;
       if (most < best) {
@@ -526,9 +543,27 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     if (pl.kind == PathKind::kTc) {
       cudaLaunchConfig_t cfg =
           launch_config(dim3(pl.grid), TcConfig::kThreads, TcConfig::SMEM, stream, attr, pdl);
-      const cudaError_t e = k_new != nullptr
-                                ? cudaLaunchKernelEx(&cfg, tc_decode_append_kernel, kmap, qmap, tp, ap)
-                                : cudaLaunchKernelEx(&cfg, tc_decode_kernel, kmap, qmap, tp);
+      const bool g8 = pl.heads_per_unit == 8;
+      cudaError_t e;
+      if (v_cache == nullptr) {
+        if (k_new != nullptr)
+          e = g8 ? cudaLaunchKernelEx(&cfg, tc_decode_append_kernel<8>, kmap, qmap, tp, ap)
+                 : cudaLaunchKernelEx(&cfg, tc_decode_append_kernel<16>, kmap, qmap, tp, ap);
+        else
+          e = g8 ? cudaLaunchKernelEx(&cfg, tc_decode_kernel<8>, kmap, qmap, tp)
+                 : cudaLaunchKernelEx(&cfg, tc_decode_kernel<16>, kmap, qmap, tp);
+      } else {
+        if (!encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, cache_batch,
+                              bstride, TcConfig::TILE))
+          return GDATTN_ERR_CUDA;
+        if (k_new != nullptr)
+          e = g8 ? cudaLaunchKernelEx(&cfg, tc_decode_kv_append_kernel<8>, kmap, vmap, qmap, tp, ap)
+                 : cudaLaunchKernelEx(&cfg, tc_decode_kv_append_kernel<16>, kmap, vmap, qmap, tp,
+                                      ap);
+        else
+          e = g8 ? cudaLaunchKernelEx(&cfg, tc_decode_kv_kernel<8>, kmap, vmap, qmap, tp)
+                 : cudaLaunchKernelEx(&cfg, tc_decode_kv_kernel<16>, kmap, vmap, qmap, tp);
+      }
       if (e != cudaSuccess) return GDATTN_ERR_CUDA;
     } else {
       if (!encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, cache_batch,

@@ -1,6 +1,7 @@
 // Split-KV decode attention on the 5th-generation tensor cores (tcgen05), for a
-// GQA group of 16 query heads over one KV head with key == value, head_dim 512:
-// Gemma-4 full-attention layers (attention_k_eq_v).
+// GQA group of 16 (or 8) query heads over one KV head, head_dim 512: Gemma-4
+// full-attention layers, where key == value (attention_k_eq_v), or, for models
+// whose cached K and V differ, with a separate V cache.
 //
 // With 16 query rows per KV row the products are a dense contraction (32 flop
 // per KV byte), far beyond what CUDA-core FMAs sustain at HBM speed, so both
@@ -24,7 +25,14 @@
 // K = V: the one 64-token tile in shared memory is the K-major A operand of the
 // first product and the MN-major A operand of the second, so each cache byte
 // crosses HBM once.  The tile arrives by TMA as eight 64x64 boxes with 128-byte
-// swizzle, the canonical operand layout for both majors.
+// swizzle, the canonical operand layout for both majors.  With a separate V the
+// same ring of 64 KiB stages carries a tile's K and then its V in two
+// consecutive ring slots: the K slot is released by its QK, the V slot by its
+// P.V.
+//
+// A group of 8 query heads per KV head runs the same MMAs: Q rows 8-15 of a
+// unit are the next unit's heads (or TMA zero fill), and their score columns,
+// weights and outputs are computed but never stored.
 //
 // Softmax with a lazily moved reference: P = exp2(s - m_ref) with m_ref a
 // running per-head reference that only moves when some score exceeds it by more
@@ -85,7 +93,7 @@ struct TcAppend {
 
 struct TcConfig {
   static constexpr int D = 512;
-  static constexpr int G = 16;
+  static constexpr int G = 16;                        // QK MMA width: query rows per unit, padded
   static constexpr int TILE = 64;                     // tokens per tile
   static constexpr int NST = 3;                       // KV stages
   static constexpr int BOXB = TILE * 128;             // one 64-token x 64-d box
@@ -171,11 +179,26 @@ __device__ __forceinline__ float warp_reduce_scatter16(float (&r)[16], int lane)
   return MAX ? fmaxf(r[0], got) : r[0] + got;
 }
 
-template <bool APPEND>
-__device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CUtensorMap &qmap,
-                                               const TcParams &p, const TcAppend &ap) {
+// Ring slots of tile t: K = V in one slot (t), or K in slot 2t and V in 2t + 1.
+template <bool SHARED>
+__device__ __forceinline__ uint32_t k_slot(uint32_t t) {
+  return SHARED ? t : 2 * t;
+}
+template <bool SHARED>
+__device__ __forceinline__ uint32_t v_slot(uint32_t t) {
+  return SHARED ? t : 2 * t + 1;
+}
+
+// SHARED: K serves as V (vmap is not read).  GU: query heads per unit (16 or
+// 8; the MMAs always take 16 rows).  APPEND: the current token's rows are
+// written into the cache first (TcAppend).
+template <bool APPEND, bool SHARED, int GU>
+__device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CUtensorMap &vmap,
+                                               const CUtensorMap &qmap, const TcParams &p,
+                                               const TcAppend &ap) {
   using Cfg = TcConfig;
   constexpr int G = Cfg::G, D = Cfg::D, NST = Cfg::NST;
+  static_assert(GU == 16 || GU == 8, "query heads per unit");
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -225,6 +248,7 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
   }
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&kmap);
+    if (!SHARED) prefetch_tensormap(&vmap);
     prefetch_tensormap(&qmap);
   }
   if (warp == 1) {
@@ -274,9 +298,9 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
     // and at the latest before waiting on a stage whose release needs it.
     const uint64_t pol = l2_evict_first_policy();
     bool ok = true;
-    uint32_t i = 0, seg_count = 0, q_issued = 0;
+    uint32_t n = 0, seg_count = 0, q_issued = 0;  // n: ring slots filled
     int32_t qrows[8] = {};       // Q rows of segments whose Q is not issued yet
-    uint32_t stage_seg[NST];     // segment of the tile last loaded into each stage
+    uint32_t stage_seg[NST];     // segment of the tile whose K or V went into each stage
     auto issue_q = [&](bool block) -> bool {  // warp-uniform result
       if (q_issued > 0) {
         bool got = block ? mbar_wait(qempty, (q_issued - 1) & 1, abort_flag, p.status)
@@ -314,42 +338,50 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
     while (ok && it.next(C, row, ntok, first, last)) {
       if (first) {
         // At most NST + 1 segments can be pending (see the wait below), so 8 slots do.
-        qrows[seg_count & 7] = it.seg.b * p.n_q_heads + it.seg.x * G;
+        qrows[seg_count & 7] = it.seg.b * p.n_q_heads + it.seg.x * GU;
         ++seg_count;
       }
-      if (i >= NST || it.newest) ensure_waited();
-      while (ok && waited && q_issued < seg_count && issue_q(false)) {
-      }
-      const int st = i % NST;
-      if (i >= NST) {
-        // The tile in this stage is released after its P.V, which needs its Q.
-        while (ok && q_issued <= stage_seg[st]) issue_q(true);
-        if (ok && !mbar_wait(&empty[st], ((i / NST) - 1) & 1, abort_flag, p.status)) ok = false;
-      }
-      if (!__all_sync(0xffffffffu, ok)) break;
-      stage_seg[st] = seg_count - 1;
-      if (APPEND && it.newest) {  // append the current token's row (K = V) first
-        const int32_t slot = (it.seg.first_pos + it.seg.n - 1) % C;
-        append_row(ap.k_cache + it.seg.b * ap.batch_stride +
-                       (static_cast<int64_t>(slot) * ap.n_kv_heads + it.seg.x) * D,
-                   ap.k_new + (static_cast<int64_t>(it.seg.b) * ap.n_kv_heads + it.seg.x) * D, D,
-                   lane);
-      }
-      if (elect_one()) {
-        mbar_arrive_expect_tx(&full[st], Cfg::STAGEB);
 #pragma unroll
-        for (int j = 0; j < D / 64; ++j)
-          tma_load_4d(stages + st * Cfg::STAGEB + j * Cfg::BOXB, &kmap, 64 * j, it.seg.x, row,
-                      cache_seq(p.geo, it.seg.b), &full[st], pol);
+      for (int part = 0; part < (SHARED ? 1 : 2); ++part) {  // K (= V), then a separate V
+        if (n >= NST || it.newest) ensure_waited();
+        while (ok && waited && q_issued < seg_count && issue_q(false)) {
+        }
+        const int st = n % NST;
+        if (n >= NST) {
+          // The slot in this stage is released by a QK or a P.V, which needs its Q.
+          while (ok && q_issued <= stage_seg[st]) issue_q(true);
+          if (ok && !mbar_wait(&empty[st], ((n / NST) - 1) & 1, abort_flag, p.status)) ok = false;
+        }
+        if (!__all_sync(0xffffffffu, ok)) break;
+        stage_seg[st] = seg_count - 1;
+        if (APPEND && it.newest) {  // append the current token's row first
+          const int32_t slot = (it.seg.first_pos + it.seg.n - 1) % C;
+          const int64_t row_off = it.seg.b * ap.batch_stride +
+                                  (static_cast<int64_t>(slot) * ap.n_kv_heads + it.seg.x) * D;
+          const int64_t new_off =
+              (static_cast<int64_t>(it.seg.b) * ap.n_kv_heads + it.seg.x) * D;
+          if (part == 0)
+            append_row(ap.k_cache + row_off, ap.k_new + new_off, D, lane);
+          else
+            append_row(ap.v_cache + row_off, ap.v_new + new_off, D, lane);
+        }
+        const CUtensorMap *map = part == 0 ? &kmap : &vmap;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&full[st], Cfg::STAGEB);
+#pragma unroll
+          for (int j = 0; j < D / 64; ++j)
+            tma_load_4d(stages + st * Cfg::STAGEB + j * Cfg::BOXB, map, 64 * j, it.seg.x, row,
+                        cache_seq(p.geo, it.seg.b), &full[st], pol);
+        }
+        __syncwarp();
+        ++n;
       }
-      __syncwarp();
-      ++i;
     }
     ensure_waited();
     while (ok && q_issued < seg_count) issue_q(true);
     // Drain: never leave with copies in flight into shared memory.
     volatile int no_abort = 0;
-    for (uint32_t f = i > NST ? i - NST : 0; f < i; ++f)
+    for (uint32_t f = n > NST ? n - NST : 0; f < n; ++f)
       mbar_wait(&full[f % NST], (f / NST) & 1, &no_abort, p.status);
     if (q_issued > 0) mbar_wait(qfull, (q_issued - 1) & 1, &no_abort, p.status);
   } else if (warp == 1) {
@@ -373,8 +405,9 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
         if (!__all_sync(0xffffffffu, ok)) break;
         ++nseg;
       }
-      const int st = i % NST, sb = i & 1;
-      if (!mbar_wait(&full[st], (i / NST) & 1, abort_flag, p.status)) ok = false;
+      const uint32_t ks = k_slot<SHARED>(i);
+      const int st = ks % NST, sb = i & 1;
+      if (!mbar_wait(&full[st], (ks / NST) & 1, abort_flag, p.status)) ok = false;
       if (ok && i >= 2 && !mbar_wait(&sempty[sb], ((i >> 1) - 1) & 1, abort_flag, p.status))
         ok = false;
       if (!__all_sync(0xffffffffu, ok)) break;
@@ -391,6 +424,7 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
           }
         }
         tc_commit(&sfull[sb]);
+        if (!SHARED) tc_commit(&empty[st]);  // a separate K slot: its only reader is done
         if (last) tc_commit(qempty);
       }
       __syncwarp();
@@ -413,7 +447,9 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
     int32_t row, ntok;
     bool first, last;
     while (ok && it.next(C, row, ntok, first, last)) {
+      const uint32_t vs = v_slot<SHARED>(t);
       bool w = mbar_wait(&pfull[t & 1], (t >> 1) & 1, abort_flag, p.status);
+      if (!SHARED && w) w = mbar_wait(&full[vs % NST], (vs / NST) & 1, abort_flag, p.status);
       // A segment's first P.V overwrites O: the previous segment must be read out.
       if (w && first && nseg > 0) w = mbar_wait(oempty, (nseg - 1) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, w)) {
@@ -422,7 +458,7 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
       }
       if (first) ++nseg;
       tc_fence_after();
-      const uint64_t a0 = vdesc + (((t % NST) * Cfg::STAGEB) >> 4);
+      const uint64_t a0 = vdesc + (((vs % NST) * Cfg::STAGEB) >> 4);
       const uint64_t b0 = pdesc + (((t & 1) * Cfg::PB) >> 4);
       if (elect_one()) {
 #pragma unroll
@@ -437,7 +473,7 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
           }
         }
         tc_commit(&ofull[t & 1]);
-        tc_commit(&empty[t % NST]);
+        tc_commit(&empty[vs % NST]);
       }
       __syncwarp();
       ++t;
@@ -585,15 +621,22 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
             make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
       if (ok && ntok < Cfg::TILE) {
-        // Rows past the attended range hold other cache contents (possibly
+        const uint32_t vs = v_slot<SHARED>(i);
+        // A separate V tile may still be in flight (it is loaded after K): wait for it.
+        if (!SHARED)
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(&full[vs % NST], (vs / NST) & 1, abort_flag, p.status));
+        // V rows past the attended range hold other cache contents (possibly
         // NaN); they get weight 0, but 0 * NaN would still reach O, so clear them.
-        uint8_t *tile = stages + (i % NST) * Cfg::STAGEB;
+        uint8_t *tile = stages + (vs % NST) * Cfg::STAGEB;
         const int per_box = (Cfg::TILE - ntok) * 8;  // 16-byte chunks past row ntok
+        if (ok) {
 #pragma unroll 1
-        for (int box = 0; box < D / 64; ++box)
-          for (int e = threadIdx.x - 64; e < per_box; e += 128)
-            *reinterpret_cast<uint4 *>(tile + box * Cfg::BOXB + (ntok + (e >> 3)) * 128 +
-                                       (e & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+          for (int box = 0; box < D / 64; ++box)
+            for (int e = threadIdx.x - 64; e < per_box; e += 128)
+              *reinterpret_cast<uint4 *>(tile + box * Cfg::BOXB + (ntok + (e >> 3)) * 128 +
+                                         (e & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -617,7 +660,7 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
         const Segment &sg = it.seg;
         const bool single = sg.whole() && !usplit;  // a split unit always has parts
         const int64_t slot = static_cast<int64_t>(c) + sg.unit;
-        const int h0 = sg.x * G;
+        const int h0 = sg.x * GU;
         float inv[G];
 #pragma unroll
         for (int h = 0; h < G; ++h)
@@ -631,19 +674,19 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
             tmem_ld16(tmem + lane_base + Cfg::O_COL + jb * 32 + 16, w);
             const int d = 128 * jb + 32 * qd + lane;
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
+            for (int h = 0; h < GU; ++h) {  // columns GU .. 15 are padding
               const float val = (v[h] + w[h]) * inv[h];
               if (single)
                 p.out[(static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + h) * D + d] =
                     f32_to_bf16_rn(val);
               else
-                p.ws_o[(slot * G + h) * D + d] = val;
+                p.ws_o[(slot * GU + h) * D + d] = val;
             }
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(oempty);
-          if (qd == 0 && lane < G) {  // LSE of head `lane`: one store per lane
+          if (qd == 0 && lane < GU) {  // LSE of head `lane`: one store per lane
             float mr = m_ref[0];
 #pragma unroll
             for (int h = 1; h < G; ++h) mr = (lane == h) ? m_ref[h] : mr;
@@ -653,17 +696,17 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
             if (single) {
               if (p.lse != nullptr) p.lse[static_cast<int64_t>(sg.b) * p.n_q_heads + h0 + lane] = lse_v;
             } else {
-              p.ws_lse[slot * G + lane] = lse_v;
+              p.ws_lse[slot * GU + lane] = lse_v;
             }
           }
         }
       }
       ++i;
     }
-    if (usplit && i == 0 && qd == 0 && lane < G) {
+    if (usplit && i == 0 && qd == 0 && lane < GU) {
       // An empty part (the unit is shorter than split_k tiles): LSE -inf.
       const int64_t slot = static_cast<int64_t>(c) + c / split_k;
-      p.ws_lse[slot * G + lane] = -INFINITY;
+      p.ws_lse[slot * GU + lane] = -INFINITY;
     }
   }
 
@@ -675,17 +718,38 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
   }
 }
 
+// K = V (attention_k_eq_v): no V map in the parameter block.
+template <int GU>
 __global__ void __launch_bounds__(TcConfig::kThreads, 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap qmap, const TcParams p) {
-  tc_decode_body<false>(kmap, qmap, p, TcAppend{});
+  tc_decode_body<false, true, GU>(kmap, kmap, qmap, p, TcAppend{});
 }
 
+template <int GU>
 __global__ void __launch_bounds__(TcConfig::kThreads, 1)
     tc_decode_append_kernel(const __grid_constant__ CUtensorMap kmap,
                             const __grid_constant__ CUtensorMap qmap, const TcParams p,
                             const TcAppend ap) {
-  tc_decode_body<true>(kmap, qmap, p, ap);
+  tc_decode_body<true, true, GU>(kmap, kmap, qmap, p, ap);
+}
+
+// Separate K and V caches.
+template <int GU>
+__global__ void __launch_bounds__(TcConfig::kThreads, 1)
+    tc_decode_kv_kernel(const __grid_constant__ CUtensorMap kmap,
+                        const __grid_constant__ CUtensorMap vmap,
+                        const __grid_constant__ CUtensorMap qmap, const TcParams p) {
+  tc_decode_body<false, false, GU>(kmap, vmap, qmap, p, TcAppend{});
+}
+
+template <int GU>
+__global__ void __launch_bounds__(TcConfig::kThreads, 1)
+    tc_decode_kv_append_kernel(const __grid_constant__ CUtensorMap kmap,
+                               const __grid_constant__ CUtensorMap vmap,
+                               const __grid_constant__ CUtensorMap qmap, const TcParams p,
+                               const TcAppend ap) {
+  tc_decode_body<true, false, GU>(kmap, vmap, qmap, p, ap);
 }
 
 }  // namespace gdattn

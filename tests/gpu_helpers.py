@@ -19,11 +19,12 @@ def require_gpu():
 
 
 def uses_tensor_cores(spec) -> bool:
-    """Whether the library runs this geometry on its tcgen05 kernels: 16 query
-    heads per KV head with head_dim 512 and K = V, or pairs of query heads with
-    head_dim 256 and separate V.  Other geometries take the CUDA-core kernel."""
+    """Whether the library runs this geometry on its tcgen05 kernels: 8 or 16
+    query heads per KV head with head_dim 512 (K = V or a separate V), or pairs
+    of query heads with head_dim 256 and separate V.  Other geometries take the
+    CUDA-core kernel."""
     g = spec.n_q_heads // spec.n_kv_heads
-    return ((g == 16 and spec.head_dim == 512 and spec.kv_shared)
+    return ((g in (8, 16) and spec.head_dim == 512)
             or (g == 2 and spec.head_dim == 256 and not spec.kv_shared))
 
 

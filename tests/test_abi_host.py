@@ -150,9 +150,14 @@ def test_kv_shared_requires_null_v(lib):
     assert call(d, v=None) == binding.GDATTN_ERR_INVALID_ARG
 
 
-def test_tensor_core_path_needs_shared_kv(lib):
-    d = good_desc(n_q_heads=16, n_kv_heads=1, head_dim=512, window=0, kv_shared=False)
-    assert call(d) == binding.GDATTN_ERR_UNSUPPORTED
+def test_sixteen_head_groups_need_head_dim_512(lib):
+    """8- and 16-head groups run on the tcgen05 16-head kernel at head_dim 512
+    (K = V or separate V); at other head sizes no kernel serves them."""
+    for g in (8, 16):
+        d = good_desc(n_q_heads=g, n_kv_heads=1, head_dim=256, window=0, kv_shared=False)
+        assert call(d) == binding.GDATTN_ERR_UNSUPPORTED
+    d = good_desc(n_q_heads=12, n_kv_heads=1, head_dim=512, window=0, kv_shared=False)
+    assert call(d) == binding.GDATTN_ERR_UNSUPPORTED  # G = 12
 
 
 def test_unit_count_beyond_the_fixed_header_is_refused(lib):

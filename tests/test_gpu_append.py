@@ -18,6 +18,8 @@ CASES = {
     "pair_forced_split": (2, 16, 8, 256, 200, [450, 130], 200, 0.0, False, 7, 0),
     "tc16_kv_shared": (2, 16, 1, 512, 400, [400, 77], 0, 0.0, True, 0, 0),
     "tc16_even_split": (2, 32, 2, 512, 300, [300, 290], 0, 0.0, True, 0, 1),
+    "tc16_sepv": (2, 16, 1, 512, 400, [400, 77], 0, 0.0, False, 0, 0),
+    "tc8_sepv_ring_even": (2, 16, 2, 512, 128, [300, 128], 128, 30.0, False, 0, 1),
     "core_g4": (2, 8, 2, 256, 90, [90, 33], 0, 0.0, False, 3, 0),
     "core_g2_shared": (2, 16, 8, 256, 70, [150, 70], 70, 5.0, True, 0, 0),
 }

@@ -20,6 +20,9 @@ CASES = {
     # tcgen05 16-head kernel (global, K = V)
     "tc16_t3": (3, 2, 16, 1, 512, 400, [400, 77], 0, 0.0, True, 0),
     "tc16_even_t2": (2, 2, 32, 2, 512, 300, [300, 300], 0, 30.0, True, 1),
+    # tcgen05 16-head kernel with a separate V, and an 8-head group
+    "tc16_sepv_t4": (4, 2, 16, 1, 512, 400, [400, 77], 0, 0.0, False, 0),
+    "tc8_sepv_ring_t3": (3, 2, 16, 2, 512, 130, [500, 130], 128, 0.0, False, 1),
     # CUDA-core kernel
     "core_g4_t3": (3, 2, 8, 2, 256, 90, [90, 33], 0, 0.0, False, 0),
 }

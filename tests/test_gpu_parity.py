@@ -40,6 +40,12 @@ CASES = {
     "tc_hkv2": (2, 32, 2, 512, 150, [150, 65], 0, 0.0, True),
     "tc_window_ring": (2, 16, 1, 512, 96, [150, 96], 96, 0.0, True),
     "tc_softcap": (2, 16, 1, 512, 129, [129, 128], 0, 30.0, True),
+    # tensor-core 16-head kernel with a separate V cache, and 8-head groups
+    "tc16_sepv_multi_tile": (2, 16, 1, 512, 300, [300, 77], 0, 0.0, False),
+    "tc16_sepv_window_ring": (2, 16, 1, 512, 96, [150, 96], 96, 0.0, False),
+    "tc16_sepv_softcap_hkv2": (2, 32, 2, 512, 129, [129, 128], 0, 30.0, False),
+    "tc8_shared_hkv2": (2, 16, 2, 512, 200, [200, 65], 0, 0.0, True),
+    "tc8_sepv_ring_edges": (3, 8, 1, 512, 96, [150, 96, 1], 96, 20.0, False),
 }
 
 _ref_cache = {}
@@ -134,7 +140,8 @@ def test_long_context(layer):
 
 
 @pytest.mark.parametrize("name", ["sliding_g2_window_lt_cap", "sliding_g2_ring_wraps",
-                                  "pair_multi_tile_ring", "tc_multi_tile_tail", "tc_window_ring", "tc_edges"])
+                                  "pair_multi_tile_ring", "tc_multi_tile_tail", "tc_window_ring",
+                                  "tc_edges", "tc16_sepv_window_ring", "tc8_sepv_ring_edges"])
 def test_unattended_slots_never_matter(name):
     """NaN in every cache slot outside the attended range leaves the result unchanged."""
     require_gpu()
@@ -309,6 +316,9 @@ EVEN_CASES = {
     "tc16_hkv2_softcap": (2, 32, 2, 512, 700, [700, 650], 0, 20.0, True),
     "tc16_k3_uneven_slices": (40, 16, 1, 512, 192, [192] * 40, 0, 0.0, True),
     "tc16_many_parts_combine": (1, 16, 1, 512, 4096, [4096], 0, 0.0, True),
+    "tc16_sepv_ragged": (3, 16, 1, 512, 2000, [2000, 100, 1], 0, 0.0, False),
+    "tc8_sepv_softcap": (2, 16, 2, 512, 700, [700, 650], 0, 20.0, False),
+    "tc16_one_unit_148_parts": (1, 16, 1, 512, 32768, [32768], 0, 0.0, True),
 }
 
 
@@ -327,7 +337,7 @@ def test_even_unit_split_matches_oracle(name):
     units = B * Hkv
     splits = binding.plan_splits(B, layer.max_seqlen, layer.desc)
     assert splits % units == 0 and splits // units >= 2, splits  # the unit split was taken
-    expect_launches = 2 if shared else 1  # the 16-head kernel merges in the combine kernel
+    expect_launches = 2 if D == 512 else 1  # the 16-head kernel merges in the combine kernel
     assert binding.launches_per_call(B, layer.max_seqlen, layer.desc) == expect_launches
     for _ in range(2):
         out, lse = layer.run()
