@@ -318,7 +318,7 @@ EVEN_CASES = {
     "tc16_many_parts_combine": (1, 16, 1, 512, 4096, [4096], 0, 0.0, True),
     "tc16_sepv_ragged": (3, 16, 1, 512, 2000, [2000, 100, 1], 0, 0.0, False),
     "tc8_sepv_softcap": (2, 16, 2, 512, 700, [700, 650], 0, 20.0, False),
-    "tc16_one_unit_148_parts": (1, 16, 1, 512, 32768, [32768], 0, 0.0, True),
+    "tc16_one_unit_64_parts": (1, 16, 1, 512, 32768, [32768], 0, 0.0, True),
 }
 
 
