@@ -229,6 +229,7 @@ def _check_combine(o_partial, lse_partial, out, lse) -> None:
 
 
 GDATTN_FLAG_EVEN_UNITS = 1
+GDATTN_FLAG_TEST_WITHHOLD_KV = 2
 
 
 def make_desc(n_q_heads: int, n_kv_heads: int, head_dim: int, window: int, softcap: float,

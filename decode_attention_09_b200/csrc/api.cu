@@ -191,7 +191,8 @@ gdattn_status check_desc(const gdattn_layer_desc *d) {
   if (d->n_q_heads <= 0 || d->n_kv_heads <= 0 || d->head_dim <= 0 || d->cache_capacity <= 0)
     return GDATTN_ERR_INVALID_ARG;
   if (d->n_q_heads % d->n_kv_heads != 0) return GDATTN_ERR_INVALID_ARG;
-  if (d->window < 0 || d->split_ctas < 0 || (d->flags & ~GDATTN_FLAG_EVEN_UNITS) != 0)
+  if (d->window < 0 || d->split_ctas < 0 ||
+      (d->flags & ~(GDATTN_FLAG_EVEN_UNITS | GDATTN_FLAG_TEST_WITHHOLD_KV)) != 0)
     return GDATTN_ERR_INVALID_ARG;
   if (!(d->softcap >= 0.f) || !std::isfinite(d->softcap) || !std::isfinite(d->scale))
     return GDATTN_ERR_INVALID_ARG;
@@ -508,6 +509,7 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     cp.n_q_heads = desc->n_q_heads;
     cp.qscale = qscale;
     cp.post = post;
+    cp.test_withhold = (desc->flags & GDATTN_FLAG_TEST_WITHHOLD_KV) ? 1 : 0;
     cudaLaunchConfig_t cfg =
         launch_config(dim3(pl.grid), ck.threads, ck.smem, stream, attr, pdl);
     if (cudaLaunchKernelEx(&cfg, ck.fn, cp) != cudaSuccess) return GDATTN_ERR_CUDA;
@@ -534,6 +536,7 @@ gdattn_status enqueue_decode(const LayerPlan &pl, const void *q, const void *k_c
     ap.n_kv_heads = Hkv;
     tp.counters = counters;
     tp.epochs = epochs;
+    tp.test_withhold = (desc->flags & GDATTN_FLAG_TEST_WITHHOLD_KV) ? 1 : 0;
     tp.merge_in_kernel = pl.merge_in_kernel ? 1 : 0;
     tp.split_k = pl.split_k;
     tp.geo = geo;
@@ -616,6 +619,7 @@ gdattn_status enqueue_decode_fp8(const LayerPlan &pl, const void *q, const void 
   tp.counters = reinterpret_cast<uint32_t *>(ws + pl.off_cnt);
   tp.epochs = reinterpret_cast<uint32_t *>(ws + pl.off_epoch);
   tp.merge_in_kernel = 1;
+  tp.test_withhold = (desc->flags & GDATTN_FLAG_TEST_WITHHOLD_KV) ? 1 : 0;
   tp.split_k = pl.split_k;
   tp.geo.seqlens = seqlens;
   tp.geo.batch = batch;

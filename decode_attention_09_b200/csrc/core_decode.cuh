@@ -45,6 +45,9 @@ struct CoreParams {
   int32_t n_q_heads;
   float qscale;           // folded into q: scale*log2(e), or scale/softcap
   float post;             // softcap*log2(e), or 0 when soft-cap is off
+  // Test hook (GDATTN_FLAG_TEST_WITHHOLD_KV): every CTA leaves its first stage
+  // unloaded, so the wait for it runs out and the timeout path runs.
+  int32_t test_withhold;
 };
 
 template <int D, int G, int HKV, bool SHARED>
@@ -178,7 +181,7 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads, 1)
             append_row(const_cast<uint16_t *>(p.k) + row, p.k_new + src, HKV * D, lane);
             if (!SHARED) append_row(const_cast<uint16_t *>(p.v) + row, p.v_new + src, HKV * D, lane);
           }
-          if (elect_one()) {
+          if (!(p.test_withhold && fills == 0) && elect_one()) {
             mbar_arrive_expect_tx(&full[st], bytes * Cfg::NT);
             bulk_g2s(stage_k + st * T * ROWB, p.k + off, bytes, &full[st], pol);
             if (!SHARED) bulk_g2s(stage_v + st * T * ROWB, p.v + off, bytes, &full[st], pol);
@@ -191,7 +194,8 @@ __global__ void __launch_bounds__(CoreConfig<D, G, HKV, SHARED>::kThreads, 1)
     // Never leave with copies in flight into this CTA's shared memory.
     for (uint32_t f = fills > NSTAGE ? fills - NSTAGE : 0; f < fills; ++f) {
       volatile int no_abort = 0;
-      mbar_wait(&full[f % NSTAGE], (f / NSTAGE) & 1, &no_abort, p.status);
+      if (!(p.test_withhold && f == 0))
+        mbar_wait(&full[f % NSTAGE], (f / NSTAGE) & 1, &no_abort, p.status);
     }
   } else {
     // ------------------------------------------------------------- compute

@@ -75,7 +75,11 @@ struct TcParams {
   int32_t n_q_heads;
   float qscale;           // multiplies raw scores: scale*log2(e), or scale/softcap
   float post;             // softcap*log2(e), or 0 when soft-cap is off
+  // Test hook (GDATTN_FLAG_TEST_WITHHOLD_KV): every CTA leaves its first KV tile
+  // unloaded, so the wait for it runs out and the timeout path runs.
+  int32_t test_withhold;
 };
+static_assert(sizeof(TcParams) == 112, "the test hook fits the parameter block's padding");
 
 // Current-token append (k_new non-null): before the tile holding a unit's
 // newest position is loaded, its row is copied from k_new / v_new
@@ -366,7 +370,7 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
             append_row(ap.v_cache + row_off, ap.v_new + new_off, D, lane);
         }
         const CUtensorMap *map = part == 0 ? &kmap : &vmap;
-        if (elect_one()) {
+        if (!(p.test_withhold && n == 0) && elect_one()) {
           mbar_arrive_expect_tx(&full[st], Cfg::STAGEB);
 #pragma unroll
           for (int j = 0; j < D / 64; ++j)
@@ -382,7 +386,7 @@ __device__ __forceinline__ void tc_decode_body(const CUtensorMap &kmap, const CU
     // Drain: never leave with copies in flight into shared memory.
     volatile int no_abort = 0;
     for (uint32_t f = n > NST ? n - NST : 0; f < n; ++f)
-      mbar_wait(&full[f % NST], (f / NST) & 1, &no_abort, p.status);
+      if (!(p.test_withhold && f == 0)) mbar_wait(&full[f % NST], (f / NST) & 1, &no_abort, p.status);
     if (q_issued > 0) mbar_wait(qfull, (q_issued - 1) & 1, &no_abort, p.status);
   } else if (warp == 1) {
     // ----------------------------------------------------------- QK MMA

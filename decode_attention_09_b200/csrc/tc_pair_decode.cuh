@@ -529,7 +529,7 @@ __device__ __forceinline__ void tc_pair_decode_body(const CUtensorMap &kmap,
                    lane);
       }
       const int32_t cb = MULTI ? cache_seq(p.geo, it.seg.b) : it.seg.b;
-      if (elect_one()) {
+      if (!(p.test_withhold && i == 0) && elect_one()) {
         uint8_t *kdst = stages + st * Cfg::STAGEB;
         mbar_arrive_expect_tx(&kfull[st], Cfg::KB);
 #pragma unroll
@@ -544,7 +544,7 @@ __device__ __forceinline__ void tc_pair_decode_body(const CUtensorMap &kmap,
     // Drain: never leave with copies in flight into shared memory.
     volatile int no_abort = 0;
     for (uint32_t f = i > NST ? i - NST : 0; f < i; ++f)
-      mbar_wait(&kfull[f % NST], (f / NST) & 1, &no_abort, p.status);
+      if (!(p.test_withhold && f == 0)) mbar_wait(&kfull[f % NST], (f / NST) & 1, &no_abort, p.status);
     for (uint32_t k = q_issued > 2 ? q_issued - 2 : 0; k < q_issued; ++k)
       mbar_wait(&qfull[k & 1], (k >> 1) & 1, &no_abort, p.status);
   } else if (warp == 1) {

@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(TcPairFp8Config::kThreads, 1)
       }
       if (!__all_sync(0xffffffffu, ok)) break;
       stage_seg[st] = seg_count - 1;
-      if (elect_one()) {
+      if (!(p.test_withhold && i == 0) && elect_one()) {
         uint8_t *kdst = stages + st * Cfg::STAGEB;
         mbar_arrive_expect_tx(&kfull[st], Cfg::KB);
 #pragma unroll
@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(TcPairFp8Config::kThreads, 1)
     while (ok && q_issued < seg_count) issue_q(true);
     volatile int no_abort = 0;
     for (uint32_t f = i > NST ? i - NST : 0; f < i; ++f)
-      mbar_wait(&kfull[f % NST], (f / NST) & 1, &no_abort, p.status);
+      if (!(p.test_withhold && f == 0)) mbar_wait(&kfull[f % NST], (f / NST) & 1, &no_abort, p.status);
     for (uint32_t k = q_issued > 2 ? q_issued - 2 : 0; k < q_issued; ++k)
       mbar_wait(&qfull[k & 1], (k >> 1) & 1, &no_abort, p.status);
   } else if (warp == 1) {

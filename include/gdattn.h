@@ -108,6 +108,18 @@ typedef struct gdattn_layer_desc {
 #define GDATTN_FLAG_EVEN_UNITS 1
 
 /*
+ * Test hook for the device-side failure path, not for production calls: every
+ * CTA of the decode kernel leaves its first KV tile unloaded, so the pipeline
+ * wait for it runs out after the bounded wait limit (about 2 s at the maximum
+ * SM clock).  The kernel then drains its copies and tensor-core work, frees
+ * tensor memory and returns; the call latches GDATTN_ERR_DEVICE_TIMEOUT in the
+ * workspace status word and its out and lse are invalid.  After any device
+ * timeout, re-initialise the workspace (gdattn_workspace_init) before reusing
+ * it: split merges may have left part counters set.
+ */
+#define GDATTN_FLAG_TEST_WITHHOLD_KV 2
+
+/*
  * Bytes of device workspace gdattn_decode needs for this layer geometry and
  * batch on the current CUDA device.  max_seqlen is the host's upper bound on
  * seqlens[]; it only steers the split count.  Returns 0 on invalid arguments.

@@ -34,11 +34,54 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
     return np.exp2(np.floor(np.log2(ax)) - 7)
 
 
+GUARD_BYTES = 4096
+GUARD_BYTE = 0xA5
+
+
+class Guarded:
+    """A device tensor with GUARD_BYTES of a known byte pattern on each side, so
+    a kernel that writes past either end of it is caught (``check``).  Write-side
+    bounds checks in place of a memory checker."""
+
+    _all = []
+
+    def __init__(self, shape, dtype, device="cuda", fill=None):
+        n = 1
+        for d in shape:
+            n *= int(d)
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        self.raw = torch.full((GUARD_BYTES + nbytes + GUARD_BYTES,), GUARD_BYTE, dtype=torch.uint8,
+                              device=device)
+        self.nbytes = nbytes
+        self.t = self.raw[GUARD_BYTES:GUARD_BYTES + nbytes].view(dtype).view(*shape)
+        if fill is not None:
+            self.t.fill_(fill)
+        Guarded._all.append(self)
+
+    def check(self, what=""):
+        lo = self.raw[:GUARD_BYTES]
+        hi = self.raw[GUARD_BYTES + self.nbytes:]
+        bad_lo = int((lo != GUARD_BYTE).sum())
+        bad_hi = int((hi != GUARD_BYTE).sum())
+        assert bad_lo == 0 and bad_hi == 0, (
+            f"{what}: {bad_lo} bytes written before and {bad_hi} bytes after the buffer")
+
+
+def guarded_workspace(B, max_seqlen, desc, device="cuda"):
+    n = binding.workspace_size(B, max_seqlen, desc)
+    assert n > 0
+    ws = Guarded((n,), torch.uint8, device)
+    binding.workspace_init(ws.t)
+    return ws
+
+
 class GpuLayer:
-    """Device copies of a layer's inputs plus a workspace."""
+    """Device copies of a layer's inputs plus a workspace.  The outputs, the LSE
+    and the workspace sit between guard bytes that every run checks."""
 
     def __init__(self, inp, split_ctas=0, max_seqlen=None, device="cuda"):
         self.inp = inp
+        self.device = device
         self.q = inp.q.to(device)
         self.k = inp.k.to(device)
         self.v = inp.v.to(device) if inp.v is not None else None
@@ -46,16 +89,32 @@ class GpuLayer:
         self.B = inp.q.shape[0]
         self.max_seqlen = int(max_seqlen or int(inp.seqlens.max()))
         self.desc = binding.desc_from_spec(inp.spec, split_ctas, capacity=inp.k.shape[1])
-        self.ws = binding.alloc_workspace(self.B, self.max_seqlen, self.desc, device)
+        self._ws = None
+        self.ws = None  # set below; replaced by tests that share workspaces
+        self._guard_ws = guarded_workspace(self.B, self.max_seqlen, self.desc, device)
+        self.ws = self._guard_ws.t
+        self._out = Guarded(tuple(self.q.shape), torch.bfloat16, device)
+        self._lse = Guarded((self.B, self.q.shape[1]), torch.float32, device)
+
+    def set_desc(self, desc):
+        """Use another descriptor (and a fresh guarded workspace sized for it)."""
+        self.desc = desc
+        self._guard_ws = guarded_workspace(self.B, self.max_seqlen, desc, self.device)
+        self.ws = self._guard_ws.t
 
     def run(self, check_status=True):
-        out, lse = binding.decode(self.q, self.k, self.v, self.seqlens, self.desc,
-                                  self.max_seqlen, workspace=self.ws)
+        out, lse = self._out.t, self._lse.t
+        binding.decode(self.q, self.k, self.v, self.seqlens, self.desc, self.max_seqlen, out=out,
+                       lse=lse, workspace=self.ws)
         if check_status:
             st = binding.check_device_status(self.ws)
             assert st == binding.GDATTN_OK, binding.status_string(st)
         torch.cuda.synchronize()
-        return out, lse
+        self._out.check("out")
+        self._lse.check("lse")
+        if self.ws is self._guard_ws.t:
+            self._guard_ws.check("workspace")
+        return out.clone(), lse.clone()
 
 
 def compare(out_gpu, lse_gpu, out_ref, lse_ref, ulp_floor=False, what=""):

@@ -146,7 +146,7 @@ def test_decode_rejects_bad_desc(lib, desc_kw, expect):
 def test_kv_shared_requires_null_v(lib):
     d = good_desc(n_q_heads=16, n_kv_heads=1, head_dim=512, window=0, kv_shared=True)
     assert call(d, v=A) == binding.GDATTN_ERR_INVALID_ARG
-    d.flags = 2  # undefined flag bit
+    d.flags = 4  # undefined flag bit
     assert call(d, v=None) == binding.GDATTN_ERR_INVALID_ARG
 
 

@@ -7,7 +7,7 @@ import torch
 
 import workloads
 from decode_attention_09_b200 import binding
-from gpu_helpers import compare, oracle_for, require_gpu
+from gpu_helpers import Guarded, compare, guarded_workspace, oracle_for, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -45,16 +45,33 @@ def test_append_then_decode_matches_oracle(name):
     o_ref, l_ref = oracle_for(ref_inp)
 
     dev = "cuda"
-    k_dev = inp.k.to(dev)
-    v_dev = inp.v.to(dev) if inp.v is not None else None
+    # The caches, outputs, LSE and workspace sit between guard bytes: the append
+    # writes into the caches, so a row written past either end is caught.
+    kg = Guarded(tuple(inp.k.shape), torch.bfloat16, dev)
+    kg.t.copy_(inp.k)
+    k_dev = kg.t
+    vg = None
+    if inp.v is not None:
+        vg = Guarded(tuple(inp.v.shape), torch.bfloat16, dev)
+        vg.t.copy_(inp.v)
+    v_dev = vg.t if vg is not None else None
     desc = binding.desc_from_spec(inp.spec, split, capacity=C, flags=flags)
-    ws = binding.alloc_workspace(B, max(sl), desc)
+    wsg = guarded_workspace(B, max(sl), desc)
+    ws = wsg.t
+    og = Guarded(tuple(inp.q.shape), torch.bfloat16, dev)
+    lg = Guarded((B, Hq), torch.float32, dev)
     for rep in range(2):  # the same rows twice: the second call rewrites them
         out, lse = binding.decode_append(inp.q.to(dev), k_new.to(dev),
                                          v_new.to(dev) if v_new is not None else None, k_dev,
-                                         v_dev, inp.seqlens.to(dev), desc, max(sl), workspace=ws)
+                                         v_dev, inp.seqlens.to(dev), desc, max(sl), out=og.t,
+                                         lse=lg.t, workspace=ws)
         st = binding.check_device_status(ws)
         assert st == binding.GDATTN_OK, binding.status_string(st)
+        torch.cuda.synchronize()
+        for g, what in ((kg, "k cache"), (vg, "v cache"), (wsg, "workspace"), (og, "out"),
+                        (lg, "lse")):
+            if g is not None:
+                g.check(f"{name} call {rep}: {what}")
         compare(out, lse, o_ref, l_ref, ulp_floor=True, what=f"{name} call {rep}")
         assert torch.equal(k_dev.cpu().view(torch.int16), k_after.view(torch.int16))
         if v_dev is not None:

@@ -11,7 +11,7 @@ import torch
 import oracle
 import workloads
 from decode_attention_09_b200 import binding
-from gpu_helpers import compare, require_gpu
+from gpu_helpers import Guarded, compare, guarded_workspace, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -31,16 +31,23 @@ class Fp8Layer:
         self.max_seqlen = int(inp.seqlens.max())
         self.desc = binding.desc_from_spec(inp.spec, split_ctas, capacity=inp.k_codes.shape[1],
                                            flags=flags)
-        self.ws = binding.alloc_workspace(self.B, self.max_seqlen, self.desc, device)
+        # outputs, LSE and workspace between guard bytes checked after every run
+        self._ws = guarded_workspace(self.B, self.max_seqlen, self.desc, device)
+        self.ws = self._ws.t
+        self._out = Guarded(tuple(self.q.shape), torch.bfloat16, device)
+        self._lse = Guarded((self.B, self.q.shape[1]), torch.float32, device)
 
     def run(self, check_status=True):
         out, lse = binding.decode_fp8(self.q, self.kc, self.vc, self.ks, self.vs, self.seqlens,
-                                      self.desc, self.max_seqlen, workspace=self.ws)
+                                      self.desc, self.max_seqlen, out=self._out.t,
+                                      lse=self._lse.t, workspace=self.ws)
         if check_status:
             st = binding.check_device_status(self.ws)
             assert st == binding.GDATTN_OK, binding.status_string(st)
         torch.cuda.synchronize()
-        return out, lse
+        for g, what in ((self._out, "out"), (self._lse, "lse"), (self._ws, "workspace")):
+            g.check(what)
+        return out.clone(), lse.clone()
 
 
 def fp8_ref(inp):

@@ -7,7 +7,7 @@ import torch
 import oracle
 import workloads
 from decode_attention_09_b200 import binding
-from gpu_helpers import compare, require_gpu
+from gpu_helpers import Guarded, compare, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -48,16 +48,21 @@ def test_multi_matches_oracle(name):
                                              s.scale)
     dev = "cuda"
     desc = binding.desc_from_spec(s, capacity=C, flags=flags)
-    ws = torch.empty(binding.multi_workspace_size(B, T, max(sl), desc), dtype=torch.uint8,
-                     device=dev)
+    wsg = Guarded((binding.multi_workspace_size(B, T, max(sl), desc),), torch.uint8, dev)
+    ws = wsg.t
     binding.workspace_init(ws)
+    og = Guarded((T, B, Hq, D), torch.bfloat16, dev)
+    lg = Guarded((T, B, Hq), torch.float32, dev)
     k = inp.k.to(dev)
     v = inp.v.to(dev) if inp.v is not None else None
     for rep in range(2):  # consecutive calls on one workspace
         out, lse = binding.decode_multi(q.to(dev), k, v, inp.seqlens.to(dev), desc, max(sl),
-                                        workspace=ws)
+                                        out=og.t, lse=lg.t, workspace=ws)
         st = binding.check_device_status(ws)
         assert st == binding.GDATTN_OK, binding.status_string(st)
+        torch.cuda.synchronize()
+        for g, what in ((wsg, "workspace"), (og, "out"), (lg, "lse")):
+            g.check(f"{name} call {rep}: {what}")
         for t in range(T):
             compare(out[t], lse[t], o_ref[t], l_ref[t], ulp_floor=True,
                     what=f"{name} token {t} call {rep}")

@@ -108,8 +108,7 @@ def test_gemma4_12b_stack_layers(layer, flags):
     o_ref, l_ref = oracle_for(inp)
     layer_gpu = GpuLayer(inp)
     if flags:
-        layer_gpu.desc = binding.desc_from_spec(inp.spec, flags=flags)
-        layer_gpu.ws = binding.alloc_workspace(w.batch, layer_gpu.max_seqlen, layer_gpu.desc)
+        layer_gpu.set_desc(binding.desc_from_spec(inp.spec, flags=flags))
     out, lse = layer_gpu.run()
     compare(out, lse, o_ref, l_ref, what=f"{w.name} layer {layer} flags {flags}")
 
@@ -332,8 +331,8 @@ def test_even_unit_split_matches_oracle(name):
                                 window=w, softcap=cap, kv_shared=shared)
     o_ref, l_ref = oracle_for(inp)
     layer = GpuLayer(inp)
-    layer.desc = binding.desc_from_spec(inp.spec, capacity=C, flags=binding.GDATTN_FLAG_EVEN_UNITS)
-    layer.ws = binding.alloc_workspace(B, layer.max_seqlen, layer.desc)
+    layer.set_desc(binding.desc_from_spec(inp.spec, capacity=C,
+                                          flags=binding.GDATTN_FLAG_EVEN_UNITS))
     units = B * Hkv
     splits = binding.plan_splits(B, layer.max_seqlen, layer.desc)
     assert splits % units == 0 and splits // units >= 2, splits  # the unit split was taken
@@ -387,8 +386,7 @@ def test_workspace_shared_by_plans_with_many_units():
         inp = workloads.random_case(seed, B, Hq, Hkv, D, C, sl, window=w, softcap=cap,
                                     kv_shared=shared, device="cuda")
         ly = GpuLayer(inp)
-        ly.desc = binding.desc_from_spec(inp.spec, capacity=C, flags=flags)
-        ly.ws = binding.alloc_workspace(ly.B, ly.max_seqlen, ly.desc)
+        ly.set_desc(binding.desc_from_spec(inp.spec, capacity=C, flags=flags))
         layers.append(ly)
     ref = [ly.run() for ly in layers]
     need = max(binding.workspace_size(ly.B, ly.max_seqlen, ly.desc) for ly in layers)
