@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -17,6 +18,7 @@
 #include "tc_decode.cuh"
 #include "tc_pair_decode.cuh"
 #include "tc_pair_fp8_decode.cuh"
+#include "tc_pair_multi_decode.cuh"
 
 using namespace gdattn;
 
@@ -174,6 +176,11 @@ int query_tc_pair_fp8(const void *fn, int threads, int smem) {
                         const Fp8Scales);
   return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
 }
+int query_tc_pair_multi(const void *fn, int threads, int smem) {
+  using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const TcParams,
+                        const MultiTokens);
+  return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
+}
 int query_tc_pair_append(const void *fn, int threads, int smem) {
   using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const TcParams,
                         const TcAppend);
@@ -214,13 +221,15 @@ PathKind choose_path(const gdattn_layer_desc *d) {
 }
 
 // fp8: plan for the fp8 cache kernel of the same path (only the pair path has one).
+// tokens > 0: plan for the single-pass multi-token pair kernel (d's window is
+// already the union window of the step); a unit then has 2 * tokens rows.
 gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_desc *d,
-                        LayerPlan &pl, bool fp8 = false) {
+                        LayerPlan &pl, bool fp8 = false, int32_t tokens = 0) {
   gdattn_status st = check_desc(d);
   if (st != GDATTN_OK) return st;
   if (batch <= 0 || max_seqlen <= 0) return GDATTN_ERR_INVALID_ARG;
   pl.kind = choose_path(d);
-  if (pl.kind == PathKind::kNone || (fp8 && pl.kind != PathKind::kTcPair))
+  if (pl.kind == PathKind::kNone || ((fp8 || tokens > 0) && pl.kind != PathKind::kTcPair))
     return GDATTN_ERR_UNSUPPORTED;
   // Units (query-head groups) of the call: one per sequence on the CUDA-core
   // path, one per (sequence, KV head) on the tcgen05 paths.
@@ -266,6 +275,14 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
     pl.align = TcConfig::TILE;
     pl.units_per_seq = d->n_kv_heads;
     pl.heads_per_unit = d->n_q_heads / d->n_kv_heads;  // 8 or 16 (the kernel pads to 16)
+  } else if (tokens > 0) {
+    per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_multi_decode_kernel),
+                                  TcPairMultiConfig::kThreads, TcPairMultiConfig::SMEM,
+                                  query_tc_pair_multi);
+    min_tokens = 2 * TcPairMultiConfig::TILE;
+    pl.align = TcPairMultiConfig::TILE;
+    pl.units_per_seq = d->n_kv_heads;
+    pl.heads_per_unit = 2 * tokens;  // query rows of a unit: (token, head)
   } else if (fp8) {
     per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_fp8_decode_kernel),
                                   TcPairFp8Config::kThreads, TcPairFp8Config::SMEM,
@@ -320,7 +337,9 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
   if (grid > 65535) return GDATTN_ERR_INVALID_ARG;
   pl.grid = static_cast<int32_t>(grid);
   pl.slots = grid + units;
-  pl.merge_in_kernel = pl.kind == PathKind::kTcPair;
+  // The pair kernels merge split units themselves; the multi-token kernel and
+  // the 16-head kernel leave them to the combine kernel.
+  pl.merge_in_kernel = pl.kind == PathKind::kTcPair && tokens == 0;
   pl.tagged = pl.merge_in_kernel && pl.split_k > 1;
   const size_t elem = pl.tagged ? 8 : 4;
   pl.off_cnt = kOffCounters;
@@ -400,6 +419,22 @@ bool encode_q_rows_map(EncodeTiledFn enc, CUtensorMap *map, const void *q, int32
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// q [T][rows][D] bf16 (rows = B * Hq) as a 3-D tensor map read in
+// {64 d, 2 rows, T tokens} boxes with 128-byte swizzle: the 2T query rows of a
+// pair unit land as 2T consecutive 128-byte rows, token-major.
+bool encode_q_tokens_map(EncodeTiledFn enc, CUtensorMap *map, const void *q, int32_t D,
+                         int64_t rows, int32_t T) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                 static_cast<cuuint64_t>(rows) * D * 2};
+  const cuuint32_t box[3] = {64, 2, static_cast<cuuint32_t>(T)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // q [B * Hq][D] bf16 as a 2-D tensor map read in 64-d x 16-row boxes.
 bool encode_q_map(EncodeTiledFn enc, CUtensorMap *map, const void *q, int32_t D, int64_t rows) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
@@ -411,10 +446,12 @@ bool encode_q_map(EncodeTiledFn enc, CUtensorMap *map, const void *q, int32_t D,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// tokens > 0: the parts of a single-pass multi-token step (token-major out / lse).
 gdattn_status launch_combine_internal(const LayerPlan &pl, const Geometry &geo, const float *ws_lse,
                                       const float *ws_o, const gdattn_layer_desc *d, void *out,
-                                      float *lse, cudaStream_t stream) {
+                                      float *lse, cudaStream_t stream, int32_t tokens = 0) {
   CombineParams cp = {};
+  cp.tokens = tokens;
   cp.parts_o = ws_o;
   cp.parts_lse = ws_lse;
   cp.out = static_cast<uint16_t *>(out);
@@ -656,6 +693,78 @@ __global__ void multi_lengths_kernel(const int32_t *seqlens, int32_t batch, int3
 
 constexpr int32_t kMaxMultiTokens = 64;
 
+// Multi-token steps of the pair geometry with at most 8 tokens run in one pass
+// over the cache (tc_pair_multi_decode.cuh); the others as T x B sequences.
+bool multi_single_pass(const gdattn_layer_desc *d, int32_t T) {
+  return choose_path(d) == PathKind::kTcPair && T <= TcPairMultiConfig::TMAX;
+}
+
+// The layer as the single-pass kernel plans it: the union of the T tokens'
+// windows, w + T - 1 positions (still 0 for a global layer).
+gdattn_layer_desc union_window_desc(const gdattn_layer_desc *d, int32_t T) {
+  gdattn_layer_desc u = *d;
+  if (u.window > 0) u.window = u.window > INT32_MAX - (T - 1) ? INT32_MAX : u.window + (T - 1);
+  return u;
+}
+
+// Enqueues the single-pass multi-token kernel (and the combine when the plan
+// splits units); pl comes from make_plan over union_window_desc(desc, T).
+gdattn_status enqueue_decode_multi_pass(const LayerPlan &pl, const void *q, const void *k_cache,
+                                        const void *v_cache, const int32_t *seqlens,
+                                        int32_t batch, int32_t T, const gdattn_layer_desc *desc,
+                                        void *out, float *lse, uint8_t *ws,
+                                        cudaStream_t stream) {
+  const gdattn_layer_desc ud = union_window_desc(desc, T);
+  const int32_t D = desc->head_dim;
+  const int32_t Hkv = desc->n_kv_heads;
+  const int64_t bstride = desc->cache_batch_stride != 0
+                              ? desc->cache_batch_stride
+                              : static_cast<int64_t>(desc->cache_capacity) * Hkv * D;
+  const float log2e = 1.4426950408889634f;
+  EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return GDATTN_ERR_CUDA;
+  CUtensorMap kmap, vmap, qmap;
+  if (!encode_cache_map(enc, &kmap, k_cache, D, Hkv, desc->cache_capacity, batch, bstride,
+                        TcPairMultiConfig::TILE) ||
+      !encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, batch, bstride,
+                        TcPairMultiConfig::TILE) ||
+      !encode_q_tokens_map(enc, &qmap, q, D, static_cast<int64_t>(batch) * desc->n_q_heads, T))
+    return GDATTN_ERR_CUDA;
+  Geometry geo;
+  geo.seqlens = seqlens;
+  geo.batch = batch;
+  geo.units_per_seq = pl.units_per_seq;
+  geo.window = ud.window;
+  geo.capacity = desc->cache_capacity;
+  geo.nchunks_align = pl.grid | (pl.align << 16);
+  geo.cache_batch = batch;
+  TcParams tp;
+  tp.out = static_cast<uint16_t *>(out);
+  tp.lse = lse;
+  tp.ws_o = reinterpret_cast<float *>(ws + pl.off_o);
+  tp.ws_lse = reinterpret_cast<float *>(ws + pl.off_lse);
+  tp.status = reinterpret_cast<uint32_t *>(ws);
+  tp.counters = reinterpret_cast<uint32_t *>(ws + pl.off_cnt);
+  tp.epochs = reinterpret_cast<uint32_t *>(ws + pl.off_epoch);
+  tp.merge_in_kernel = 0;
+  tp.test_withhold = (desc->flags & GDATTN_FLAG_TEST_WITHHOLD_KV) ? 1 : 0;
+  tp.split_k = pl.split_k;
+  tp.geo = geo;
+  tp.n_q_heads = desc->n_q_heads;
+  tp.qscale = desc->softcap > 0.f ? desc->scale / desc->softcap : desc->scale * log2e;
+  tp.post = desc->softcap > 0.f ? desc->softcap * log2e : 0.f;
+  const MultiTokens mt = {T, desc->window};
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = launch_config(dim3(pl.grid), TcPairMultiConfig::kThreads,
+                                         TcPairMultiConfig::SMEM, stream, attr);
+  if (cudaLaunchKernelEx(&cfg, tc_pair_multi_decode_kernel, kmap, vmap, qmap, tp, mt) !=
+      cudaSuccess)
+    return GDATTN_ERR_CUDA;
+  if (pl.needs_combine())
+    return launch_combine_internal(pl, geo, tp.ws_lse, tp.ws_o, desc, out, lse, stream, T);
+  return GDATTN_OK;
+}
+
 // Workspace of a multi-query step: the decode plan's, then the lengths [T][B].
 size_t multi_lens_offset(const LayerPlan &pl) { return align256(pl.bytes); }
 size_t multi_bytes(const LayerPlan &pl, int32_t batch, int32_t T) {
@@ -855,8 +964,13 @@ gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *
 
 size_t gdattn_multi_workspace_size(int32_t batch, int32_t n_tokens, int32_t max_seqlen,
                                    const gdattn_layer_desc *desc) {
-  if (n_tokens < 1 || n_tokens > kMaxMultiTokens || batch <= 0) return 0;
+  if (n_tokens < 1 || n_tokens > kMaxMultiTokens || batch <= 0 || desc == nullptr) return 0;
   LayerPlan pl;
+  if (multi_single_pass(desc, n_tokens)) {
+    const gdattn_layer_desc ud = union_window_desc(desc, n_tokens);
+    if (make_plan(batch, max_seqlen, &ud, pl, false, n_tokens) != GDATTN_OK) return 0;
+    return pl.bytes;
+  }
   if (make_plan(batch * n_tokens, max_seqlen, desc, pl) != GDATTN_OK) return 0;
   return multi_bytes(pl, batch, n_tokens);
 }
@@ -878,6 +992,16 @@ gdattn_status gdattn_decode_multi(const void *q, const void *k_cache, const void
     return GDATTN_ERR_INVALID_ARG;
   if (workspace == nullptr) return GDATTN_ERR_WORKSPACE;
   if (!aligned16(workspace)) return GDATTN_ERR_MISALIGNED;
+  if (multi_single_pass(desc, n_tokens)) {
+    const gdattn_layer_desc ud = union_window_desc(desc, n_tokens);
+    LayerPlan pl;
+    st = make_plan(batch, max_seqlen, &ud, pl, false, n_tokens);
+    if (st != GDATTN_OK) return st;
+    if (workspace_bytes < pl.bytes) return GDATTN_ERR_WORKSPACE;
+    return enqueue_decode_multi_pass(pl, q, k_cache, v_cache, seqlens, batch, n_tokens, desc, out,
+                                     lse, static_cast<uint8_t *>(workspace),
+                                     static_cast<cudaStream_t>(stream_));
+  }
   // One decode over T x B query sequences, token-major (q, out, lse and the
   // lengths are [T][B] ...): query sequence t * B + b reads cache sequence b.
   const int32_t total = n_tokens * batch;

@@ -36,6 +36,10 @@ struct CombineParams {
   // Internal layout with units cut into split_k parts (> 1): unit u's parts are
   // in slots u * split_k + u .. + split_k - 1, empty ones with LSE -inf.
   int32_t split_k;
+  // Internal layout of a multi-token step (> 0): row r of a unit is query token
+  // r / (heads_per_unit / tokens) of head r % (heads_per_unit / tokens), and
+  // out / lse are token-major [tokens][B][Hq].
+  int32_t tokens;
 };
 
 // Threads per combine CTA: one float4 column of D each, whole warps.
@@ -213,7 +217,14 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
     l_base = p.parts_lse + (static_cast<int64_t>(b) * p.n_q_heads + h) * np;
   }
 
-  uint16_t *dst = p.out + (static_cast<int64_t>(b) * p.n_q_heads + h) * D;
+  int64_t orow = static_cast<int64_t>(b) * p.n_q_heads + h;  // output row of (b, h)
+  if (INTERNAL && p.tokens > 0) {
+    const int32_t gq = p.heads_per_unit / p.tokens;  // query heads of the unit
+    const int32_t t = hh / gq;
+    orow = (static_cast<int64_t>(t) * p.geo.batch + b) * p.n_q_heads + (h - hh) / p.heads_per_unit * gq +
+           hh % gq;
+  }
+  uint16_t *dst = p.out + orow * D;
   const int d = 4 * threadIdx.x;
   const bool owner = d < D;
   float m, z;
@@ -221,7 +232,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
                                         owner, m, z);
   if (owner) store_bf16x4(dst + d, v);
   if (threadIdx.x == 0 && p.lse != nullptr)
-    p.lse[static_cast<int64_t>(b) * p.n_q_heads + h] = (m == -INFINITY) ? -INFINITY : m + logf(z);
+    p.lse[orow] = (m == -INFINITY) ? -INFINITY : m + logf(z);
 }
 
 }  // namespace gdattn

@@ -128,6 +128,7 @@ struct TileIterT {
   int32_t run, t0;
   bool have_seg;
   bool newest;  // the last tile yielded holds the unit's newest position (L - 1)
+  int32_t off;  // offset of the last tile's first token in its unit's attended range
 
   __device__ __forceinline__ void init(const Geometry &g, const ChunkPlan &p) {
     seg_it.init(g, p);
@@ -148,7 +149,8 @@ struct TileIterT {
     }
     row = runs.start(run) + t0;
     ntok = min(TILE, runs.len(run) - t0);
-    newest = seg.lo + (run == 1 ? runs.len0 : 0) + t0 + ntok == seg.n;
+    off = seg.lo + (run == 1 ? runs.len0 : 0) + t0;
+    newest = off + ntok == seg.n;
     t0 += TILE;
     if (t0 >= runs.len(run)) {
       ++run;

@@ -283,12 +283,20 @@ gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *
  *
  * A ring cache holds positions [L_b - C, L_b), so with a window the first token
  * needs C >= window + T - 1 unless the cache never wraps (C >= max_seqlen);
- * otherwise GDATTN_ERR_INVALID_ARG.  The step is one small kernel that writes
- * the T per-token lengths into the workspace, then one decode launch over
- * T x batch query sequences (token-major) in which query sequence t * batch + b
- * reads cache sequence b.  The T tokens of a sequence read the same cache rows
- * from different CTAs at about the same time, so much of the repetition is
- * served from L2 rather than HBM.
+ * otherwise GDATTN_ERR_INVALID_ARG.
+ *
+ * On the pair geometry (two query heads per KV head, head_dim 256, separate V)
+ * with T <= 8 the step is one pass over the cache: a unit's 2T query rows (token,
+ * head) share every K and V tile of the union of their windows, the last
+ * min(L_b, window + T - 1) positions, and each score is masked to its own
+ * token's range; split units are merged by the LSE-combine kernel.  Otherwise
+ * one small kernel writes the T per-token lengths into the workspace, then one
+ * decode launch runs over T x batch query sequences (token-major) in which query
+ * sequence t * batch + b reads cache sequence b; the T tokens of a sequence then
+ * read the same cache rows from different CTAs at about the same time, so much
+ * of the repetition is served from L2 rather than HBM.  A sequence with
+ * L_b < T is a device-side error (GDATTN_ERR_DEVICE_SEQLEN); its tokens below
+ * position 0 get a zero output and LSE -inf.
  */
 size_t gdattn_multi_workspace_size(int32_t batch, int32_t n_tokens, int32_t max_seqlen,
                                    const gdattn_layer_desc *desc);

@@ -11,12 +11,23 @@ from gpu_helpers import Guarded, compare, require_gpu
 
 pytestmark = pytest.mark.gpu
 
-# (T, B, Hq, Hkv, D, C, seqlens, window, softcap, kv_shared, flags)
+# (T, B, Hq, Hkv, D, C, seqlens, window, softcap, kv_shared, flags[, split_ctas])
 CASES = {
-    # tcgen05 pair kernel (sliding): ring of w + T - 1 slots that wraps
+    # single-pass pair kernel (sliding, T <= 8): ring of w + T - 1 slots that wraps
     "pair_ring_t4": (4, 3, 16, 8, 256, 259, [700, 256, 4], 256, 0.0, False, 0),
     "pair_even_t2_cap": (2, 2, 16, 8, 256, 1025, [4000, 4000], 1024, 50.0, False, 1),
     "pair_no_wrap_t7": (7, 2, 16, 8, 256, 300, [300, 9], 128, 0.0, False, 0),
+    # all 16 query rows; ragged lengths, one shorter than a tile, one of exactly T
+    "pair_t8_ragged": (8, 4, 16, 8, 256, 519, [2000, 519, 61, 8], 512, 0.0, False, 0),
+    "pair_t8_even_cap": (8, 3, 32, 16, 256, 1031, [1500, 1500, 1500], 1024, 50.0, False, 1),
+    # one token: the single-pass kernel as a plain decode
+    "pair_t1": (1, 2, 16, 8, 256, 600, [600, 200], 512, 0.0, False, 1),
+    # global pair layer (window 0)
+    "pair_global_t5": (5, 2, 4, 2, 256, 700, [700, 333], 0, 0.0, False, 0),
+    # forced flattened chunks: tokens' windows cut across many parts
+    "pair_split40_t6": (6, 2, 16, 8, 256, 1100, [1100, 800], 1024, 0.0, False, 0, 40),
+    # past 8 tokens the pair geometry runs as T x B sequences
+    "pair_t9_per_token": (9, 2, 16, 8, 256, 300, [300, 50], 128, 0.0, False, 0),
     # tcgen05 16-head kernel (global, K = V)
     "tc16_t3": (3, 2, 16, 1, 512, 400, [400, 77], 0, 0.0, True, 0),
     "tc16_even_t2": (2, 2, 32, 2, 512, 300, [300, 300], 0, 30.0, True, 1),
@@ -29,7 +40,7 @@ CASES = {
 
 
 def case_inputs(name):
-    T, B, Hq, Hkv, D, C, sl, w, cap, shared, flags = CASES[name]
+    T, B, Hq, Hkv, D, C, sl, w, cap, shared, flags = CASES[name][:11]
     idx = sorted(CASES).index(name)
     inp = workloads.random_case(700 + idx, B, Hq, Hkv, D, C, sl, window=w, softcap=cap,
                                 kv_shared=shared)
@@ -41,13 +52,14 @@ def case_inputs(name):
 @pytest.mark.parametrize("name", sorted(CASES))
 def test_multi_matches_oracle(name):
     require_gpu()
-    T, B, Hq, Hkv, D, C, sl, w, cap, shared, flags = CASES[name]
+    T, B, Hq, Hkv, D, C, sl, w, cap, shared, flags = CASES[name][:11]
+    split = CASES[name][11] if len(CASES[name]) > 11 else 0
     q, inp = case_inputs(name)
     s = inp.spec
     o_ref, l_ref = oracle.get().decode_multi(q, inp.k, inp.v, inp.seqlens, s.window, s.softcap,
                                              s.scale)
     dev = "cuda"
-    desc = binding.desc_from_spec(s, capacity=C, flags=flags)
+    desc = binding.desc_from_spec(s, capacity=C, flags=flags, split_ctas=split)
     wsg = Guarded((binding.multi_workspace_size(B, T, max(sl), desc),), torch.uint8, dev)
     ws = wsg.t
     binding.workspace_init(ws)
@@ -68,25 +80,36 @@ def test_multi_matches_oracle(name):
                     what=f"{name} token {t} call {rep}")
 
 
-def test_multi_tokens_before_the_context_are_reported():
+@pytest.mark.parametrize("name,short_len", [("core_g4_t3", 2), ("pair_no_wrap_t7", 5)])
+def test_multi_tokens_before_the_context_are_reported(name, short_len):
     """A sequence shorter than T: its tokens at positions below 0 attend nothing;
-    the device reports it, gives them zero output and LSE -inf, and the other
-    tokens are still right."""
+    the device reports it, gives them zero output and LSE -inf, and its other
+    tokens and the other sequence are still right."""
     require_gpu()
-    q, inp = case_inputs("core_g4_t3")  # T = 3
-    inp.seqlens[1] = 2                  # token 0 of sequence 1 would sit at position -1
+    q, inp = case_inputs(name)
+    inp.seqlens[1] = short_len  # sequence 1's first T - short_len tokens sit below 0
     s = inp.spec
     dev = "cuda"
     desc = binding.desc_from_spec(s, capacity=inp.k.shape[1])
     T = q.shape[0]
-    ws = torch.empty(binding.multi_workspace_size(2, T, 90, desc), dtype=torch.uint8, device=dev)
+    max_len = int(inp.seqlens.max())
+    ws = torch.empty(binding.multi_workspace_size(2, T, max_len, desc), dtype=torch.uint8,
+                     device=dev)
     binding.workspace_init(ws)
-    out, lse = binding.decode_multi(q.to(dev), inp.k.to(dev), inp.v.to(dev), inp.seqlens.to(dev),
-                                    desc, 90, workspace=ws)
+    v = inp.v.to(dev) if inp.v is not None else None
+    out, lse = binding.decode_multi(q.to(dev), inp.k.to(dev), v, inp.seqlens.to(dev), desc,
+                                    max_len, workspace=ws)
     assert binding.check_device_status(ws) == binding.GDATTN_ERR_DEVICE_SEQLEN
-    assert torch.all(out[0, 1] == 0) and torch.all(torch.isneginf(lse[0, 1]))
-    o_ref, l_ref = oracle.get().decode_multi(q[1:, 0:1], inp.k[0:1], inp.v[0:1],
+    missing = T - short_len
+    for t in range(missing):
+        assert torch.all(out[t, 1] == 0) and torch.all(torch.isneginf(lse[t, 1]))
+    o_ref, l_ref = oracle.get().decode_multi(q[missing:, 1:2], inp.k[1:2], inp.v[1:2],
+                                             inp.seqlens[1:2], s.window, s.softcap, s.scale)
+    for t in range(missing, T):
+        compare(out[t, 1:2], lse[t, 1:2], o_ref[t - missing], l_ref[t - missing], ulp_floor=True,
+                what=f"token {t} of the short sequence")
+    o_ref, l_ref = oracle.get().decode_multi(q[:, 0:1], inp.k[0:1], inp.v[0:1],
                                              inp.seqlens[0:1], s.window, s.softcap, s.scale)
-    for t in range(1, T):
-        compare(out[t, 0:1], lse[t, 0:1], o_ref[t - 1], l_ref[t - 1], ulp_floor=True,
+    for t in range(T):
+        compare(out[t, 0:1], lse[t, 0:1], o_ref[t], l_ref[t], ulp_floor=True,
                 what=f"token {t} of the full-length sequence")
