@@ -19,6 +19,7 @@ no collective on the data path); timings are reduced as the max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -738,6 +739,79 @@ def run_ours(args, world, rank, local):
                 raise binding.GdattnError(st, "device status after the multi-query step")
         del g_mq
 
+    # ---- multi-query decode on the sliding layers: verify steps of speculative
+    # decoding, 4 and 8 query tokens per sequence (8: 7 draft tokens and the last
+    # accepted one), one pass over each ring.  Rings of w + 7 slots (the first
+    # token's window must still be in the ring); 8 layers of their own, replayed
+    # in turn (together over 4x the L2 size).
+    multi_sl = {}
+    n_multi_sl = 8
+    if sliding_idx:
+        sp0 = stack.layers[sliding_idx[0]]["spec"]
+        spec_m = dataclasses.replace(sp0, capacity=sp0.window + 7)
+        seqlens_m = w.seqlens()
+        flags_m = binding.GDATTN_FLAG_EVEN_UNITS if w.ragged is None else 0
+        desc_m = binding.desc_from_spec(spec_m, flags=flags_m)
+        caches_m = [workloads.layer_inputs(spec_m, w.batch, seqlens_m,
+                                           w.seed * 1000 + 900 + j + rank_seed_offset(rank),
+                                           device=device)
+                    for j in range(n_multi_sl)]
+        gen_sq = torch.Generator(device="cpu").manual_seed(13 + rank)
+        # one token through gdattn_decode on the same rings: the ratio's base
+        ws1 = [binding.alloc_workspace(w.batch, stack.max_seqlen, desc_m, device)
+               for _ in caches_m]
+        q1 = [torch.randn((w.batch, spec_m.n_q_heads, spec_m.head_dim),
+                          generator=gen_sq).to(torch.bfloat16).to(device) for _ in caches_m]
+
+        def single_sl_step():
+            for inp, qq, wsq in zip(caches_m, q1, ws1):
+                binding.decode(qq, inp.k, inp.v, inp.seqlens, desc_m, stack.max_seqlen,
+                               workspace=wsq, stream=stream)
+
+        g_s1 = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            single_sl_step()
+            stream.synchronize()
+            with torch.cuda.graph(g_s1, stream=stream):
+                single_sl_step()
+        barrier()
+        multi_sl[1] = (max_over_ranks(time_graph(g_s1, stream, replays, 3), world),
+                       n_multi_sl * accounting.layer_multi_kv_bytes(spec_m, seqlens_m.tolist(), 1))
+        del g_s1, ws1, q1
+        for t_m in (4, 8):
+            bufs = []
+            for inp in caches_m:
+                qm = torch.randn((t_m, w.batch, spec_m.n_q_heads, spec_m.head_dim),
+                                 generator=gen_sq).to(torch.bfloat16).to(device)
+                wsm = torch.empty(binding.multi_workspace_size(w.batch, t_m, stack.max_seqlen,
+                                                               desc_m),
+                                  dtype=torch.uint8, device=device)
+                binding.workspace_init(wsm, stream)
+                bufs.append((inp, qm, wsm, torch.empty_like(qm),
+                             torch.empty((t_m, w.batch, spec_m.n_q_heads), device=device)))
+
+            def multi_sl_step():
+                for inp, qm, wsm, om, lm in bufs:
+                    binding.decode_multi(qm, inp.k, inp.v, inp.seqlens, desc_m, stack.max_seqlen,
+                                         out=om, lse=lm, workspace=wsm, stream=stream)
+
+            g_msl = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                multi_sl_step()
+                stream.synchronize()
+                with torch.cuda.graph(g_msl, stream=stream):
+                    multi_sl_step()
+            barrier()
+            ms_m = max_over_ranks(time_graph(g_msl, stream, replays, 3), world)
+            for inp, qm, wsm, om, lm in bufs:
+                st = binding.check_device_status(wsm, stream)
+                if st != binding.GDATTN_OK:
+                    raise binding.GdattnError(st, "device status after the sliding multi-query step")
+            multi_sl[t_m] = (ms_m, n_multi_sl * accounting.layer_multi_kv_bytes(
+                spec_m, seqlens_m.tolist(), t_m))
+            del g_msl, bufs
+        del caches_m
+
     # ---- CPU baseline: the oracle over the whole step (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
@@ -868,6 +942,20 @@ def run_ours(args, world, rank, local):
                    "decode launch over 4 x 8 query sequences that read the 8 caches (the "
                    "tokens of a sequence share its rows through L2); kv_gbs counts each "
                    "token's window; CUDA graph, device time"},
+        "multi_query_sliding": None if not multi_sl else {
+            "stack_sliding_us_per_layer": ms_sl / len(sliding_idx) * 1e3,
+            **{f"t{t_m}": {"tokens": t_m, "us_per_layer": ms_m / n_multi_sl * 1e3,
+                           "vs_single_token": ms_m / multi_sl[1][0],
+                           "kv_gbs": b_m / (ms_m * 1e-3) / 1e9,
+                           "kv_frac": b_m / (ms_m * 1e-3) / 1e9 / peak}
+               for t_m, (ms_m, b_m) in sorted(multi_sl.items())},
+            "how": "8 sliding layers (rings of window + 7 slots, the stack's batch and "
+                   "lengths) through gdattn_decode_multi with 4 and 8 query tokens per "
+                   "sequence (8: 7 draft tokens and the last accepted one): one pass over the "
+                   "union of the tokens' windows (tc_pair_multi_decode_kernel, split units "
+                   "merged in the kernel); t1 is one token through gdattn_decode on the same "
+                   "rings, the base of vs_single_token; kv_gbs counts the union once; CUDA "
+                   "graph, device time, the 8 layers replayed in turn"},
         "gpu_launches": stack.launches_per_step(all_idx) * replays,
         "clocks": clk,
     }

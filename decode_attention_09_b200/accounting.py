@@ -10,6 +10,9 @@ The per-token formula of the "Gemma 4 12B" record (KV GEOMETRY paragraph) counts
 K and V for every layer; ``count_shared_twice=True`` reproduces that figure.
 
 An fp8 cache row is ``head_dim`` one-byte e4m3 codes plus its 4-byte scale.
+
+A multi-token (verify) step of T tokens whose union of windows is read once
+counts the positions of that union: min(L, w + T - 1) for a sliding layer.
 """
 from __future__ import annotations
 
@@ -31,6 +34,20 @@ def layer_kv_bytes(spec, seqlens) -> int:
     """Algorithmic KV bytes for one decode step of one layer over a batch."""
     per = kv_bytes_per_position(spec)
     return sum(attended_positions(spec, int(L)) * per for L in seqlens)
+
+
+def union_positions(spec, seqlen: int, tokens: int) -> int:
+    """Positions the T tokens of a verify step attend together: token t at
+    position L - T + t attends min(w, ...) positions ending at its own, so the
+    union is the last min(L, w + T - 1) positions (all L for a global layer)."""
+    return min(seqlen, spec.window + tokens - 1) if spec.window > 0 else seqlen
+
+
+def layer_multi_kv_bytes(spec, seqlens, tokens: int) -> int:
+    """Algorithmic KV bytes of a T-token step that reads each position of the
+    union of its tokens' windows once."""
+    per = kv_bytes_per_position(spec)
+    return sum(union_positions(spec, int(L), tokens) * per for L in seqlens)
 
 
 FP8_ROW_EXTRA = 4  # the fp32 scale stored with every fp8 cache row

@@ -176,10 +176,24 @@ int query_tc_pair_fp8(const void *fn, int threads, int smem) {
                         const Fp8Scales);
   return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
 }
+using MultiPassFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                             const TcParams, const MultiTokens);
 int query_tc_pair_multi(const void *fn, int threads, int smem) {
-  using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const TcParams,
-                        const MultiTokens);
-  return blocks_per_sm(reinterpret_cast<TcFn>(const_cast<void *>(fn)), threads, smem);
+  return blocks_per_sm(reinterpret_cast<MultiPassFn>(const_cast<void *>(fn)), threads, smem);
+}
+// The single-pass multi-token kernel for T tokens (1..8), else null.
+MultiPassFn multi_pass_kernel(int32_t T) {
+  switch (T) {
+    case 1: return tc_pair_multi_decode_kernel<1>;
+    case 2: return tc_pair_multi_decode_kernel<2>;
+    case 3: return tc_pair_multi_decode_kernel<3>;
+    case 4: return tc_pair_multi_decode_kernel<4>;
+    case 5: return tc_pair_multi_decode_kernel<5>;
+    case 6: return tc_pair_multi_decode_kernel<6>;
+    case 7: return tc_pair_multi_decode_kernel<7>;
+    case 8: return tc_pair_multi_decode_kernel<8>;
+    default: return nullptr;
+  }
 }
 int query_tc_pair_append(const void *fn, int threads, int smem) {
   using TcFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const TcParams,
@@ -276,7 +290,8 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
     pl.units_per_seq = d->n_kv_heads;
     pl.heads_per_unit = d->n_q_heads / d->n_kv_heads;  // 8 or 16 (the kernel pads to 16)
   } else if (tokens > 0) {
-    per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_multi_decode_kernel),
+    if (multi_pass_kernel(tokens) == nullptr) return GDATTN_ERR_UNSUPPORTED;
+    per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(multi_pass_kernel(tokens)),
                                   TcPairMultiConfig::kThreads, TcPairMultiConfig::SMEM,
                                   query_tc_pair_multi);
     min_tokens = 2 * TcPairMultiConfig::TILE;
@@ -337,10 +352,12 @@ gdattn_status make_plan(int32_t batch, int32_t max_seqlen, const gdattn_layer_de
   if (grid > 65535) return GDATTN_ERR_INVALID_ARG;
   pl.grid = static_cast<int32_t>(grid);
   pl.slots = grid + units;
-  // The pair kernels merge split units themselves; the multi-token kernel and
-  // the 16-head kernel leave them to the combine kernel.
-  pl.merge_in_kernel = pl.kind == PathKind::kTcPair && tokens == 0;
-  pl.tagged = pl.merge_in_kernel && pl.split_k > 1;
+  // The pair kernels (single- and multi-token) merge split units themselves;
+  // the 16-head kernel leaves them to the combine kernel.
+  pl.merge_in_kernel = pl.kind == PathKind::kTcPair;
+  // Parts of split units as tagged (value, tag) words: the single-token pair
+  // kernels; the multi-token kernel stores plain partials and counts them.
+  pl.tagged = pl.merge_in_kernel && pl.split_k > 1 && tokens == 0;
   const size_t elem = pl.tagged ? 8 : 4;
   pl.off_cnt = kOffCounters;
   pl.off_epoch = kOffEpochs;
@@ -707,8 +724,8 @@ gdattn_layer_desc union_window_desc(const gdattn_layer_desc *d, int32_t T) {
   return u;
 }
 
-// Enqueues the single-pass multi-token kernel (and the combine when the plan
-// splits units); pl comes from make_plan over union_window_desc(desc, T).
+// Enqueues the single-pass multi-token kernel (it merges split units itself);
+// pl comes from make_plan over union_window_desc(desc, T).
 gdattn_status enqueue_decode_multi_pass(const LayerPlan &pl, const void *q, const void *k_cache,
                                         const void *v_cache, const int32_t *seqlens,
                                         int32_t batch, int32_t T, const gdattn_layer_desc *desc,
@@ -746,21 +763,20 @@ gdattn_status enqueue_decode_multi_pass(const LayerPlan &pl, const void *q, cons
   tp.status = reinterpret_cast<uint32_t *>(ws);
   tp.counters = reinterpret_cast<uint32_t *>(ws + pl.off_cnt);
   tp.epochs = reinterpret_cast<uint32_t *>(ws + pl.off_epoch);
-  tp.merge_in_kernel = 0;
+  tp.merge_in_kernel = pl.merge_in_kernel ? 1 : 0;
   tp.test_withhold = (desc->flags & GDATTN_FLAG_TEST_WITHHOLD_KV) ? 1 : 0;
   tp.split_k = pl.split_k;
   tp.geo = geo;
   tp.n_q_heads = desc->n_q_heads;
   tp.qscale = desc->softcap > 0.f ? desc->scale / desc->softcap : desc->scale * log2e;
   tp.post = desc->softcap > 0.f ? desc->softcap * log2e : 0.f;
-  const MultiTokens mt = {T, desc->window};
+  const MultiTokens mt = {desc->window};
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = launch_config(dim3(pl.grid), TcPairMultiConfig::kThreads,
                                          TcPairMultiConfig::SMEM, stream, attr);
-  if (cudaLaunchKernelEx(&cfg, tc_pair_multi_decode_kernel, kmap, vmap, qmap, tp, mt) !=
-      cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, multi_pass_kernel(T), kmap, vmap, qmap, tp, mt) != cudaSuccess)
     return GDATTN_ERR_CUDA;
-  if (pl.needs_combine())
+  if (pl.needs_combine())  // not with the in-kernel merge; kept for a plan without it
     return launch_combine_internal(pl, geo, tp.ws_lse, tp.ws_o, desc, out, lse, stream, T);
   return GDATTN_OK;
 }

@@ -21,20 +21,27 @@
 // a unit's 2T query rows from q [T][B][Hq][D] into the 16-row operand (rows 2T
 // and up are never read back).
 //
-// Each softmax thread owns one cache token and one head and holds that head's T
-// scores (lanes 0-15: head 0 of their token; lanes 16-31: head 1 of the token of
-// lane - 16).  The reference max is kept per query row and moved lazily as in
-// the single-token kernels.
+// S^T accumulates in one 16-column TMEM accumulator (two buffers), so a thread
+// reads its token's 2T scores in one 16-column load.  Each softmax thread owns
+// one cache token and one head and holds that head's T scores (lanes 0-15: head
+// 0 of their token; lanes 16-31: head 1 of the token of lane - 16).  The
+// reference max is kept per query row and moved lazily as in the single-token
+// kernels.  P is triple buffered: the softmax of tile i needs only the P.V of
+// tile i - 3 done.
 //
-// Split parts are written as partials (normalised O [2T][D] and LSE [2T] per
-// slot) and merged by the LSE-combine kernel; a part that covers its whole
-// unit writes out and lse directly.  out and lse are token-major: [T][B][Hq][D]
-// and [T][B][Hq].
+// A part that covers its whole unit writes out and lse directly (token-major:
+// [T][B][Hq][D] and [T][B][Hq]).  Split units are merged in the kernel by the
+// softmax threads, each for the output elements it computed (2T rows x 2 dims):
+// every part stores its partial (normalised O and LSE per row) and counts
+// itself with one acq_rel atomic, and the part that completes the count folds
+// all parts in slot order (its own from registers).  Nobody waits for another
+// CTA, and the merge costs the last part one atomic and one round of loads of
+// data already written.  No combine kernel runs.
 //
 // Warp roles (256 threads): warp 0 loads K (and Q), warp 7 loads V, warp 1
 // issues QK and owns TMEM, warp 6 issues P.V, warps 2-5 run the softmax.  The
 // stage ring, the dependency rule and the bounded waits are those of the
-// single-token pair kernel.
+// single-token pair kernel.  The kernel is instantiated for each T.
 #pragma once
 
 #include <cstdint>
@@ -47,10 +54,8 @@
 
 namespace gdattn {
 
-// Tokens of a multi-token step and the layer's own window (the geometry holds
-// the union window w + T - 1).
+// The layer's own window (the geometry holds the union window w + T - 1).
 struct MultiTokens {
-  int32_t tokens;  // T, 1..8
   int32_t window;  // w (0: global)
 };
 
@@ -68,14 +73,15 @@ struct TcPairMultiConfig {
   static constexpr int QBOXB = N * 128;               // 16 Q rows x 64 d
   static constexpr int QB = QBOXB * (D / 64);         // 8 KiB per Q buffer
   static constexpr int PB = NP * 128;                 // P: 32 rows x 64 tokens bf16, 4 KiB
+  static constexpr int NPB = 3;                       // P buffers
   static constexpr int OFF_Q = NST * STAGEB;
   static constexpr int OFF_P = OFF_Q + 2 * QB;
-  static constexpr int OFF_BAR = OFF_P + 2 * PB;
+  static constexpr int OFF_BAR = OFF_P + NPB * PB;
   static constexpr int OFF_RED = OFF_BAR + 512;
   static constexpr int SMEM = OFF_RED + 2 * 4 * N * 4 + 1024;
   static constexpr int kThreads = 256;
   static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr uint32_t S_COL = 0;                // 2 buffers x 4 partial sums x 16 columns
+  static constexpr uint32_t S_COL = 0;                // 2 buffers x 16 columns
   static constexpr uint32_t O_COL = 128;              // 2 d-blocks x 32 columns
 };
 static_assert(TcPairMultiConfig::SMEM <= 227 * 1024, "shared memory budget");
@@ -125,13 +131,16 @@ __device__ __forceinline__ void tmem_st32_wait(uint32_t taddr, const float (&v)[
       : "memory");
 }
 
+template <int T>
 __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
     tc_pair_multi_decode_kernel(const __grid_constant__ CUtensorMap kmap,
                                 const __grid_constant__ CUtensorMap vmap,
                                 const __grid_constant__ CUtensorMap qmap, const TcParams p,
                                 const MultiTokens mt) {
   using Cfg = TcPairMultiConfig;
-  constexpr int D = Cfg::D, NST = Cfg::NST, N = Cfg::N, TMAX = Cfg::TMAX;
+  constexpr int D = Cfg::D, NST = Cfg::NST, N = Cfg::N;
+  constexpr int R = 2 * T;  // query rows of a unit
+  static_assert(T >= 1 && T <= Cfg::TMAX, "1 to 8 tokens");
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -146,23 +155,22 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
   uint64_t *qempty = bars + 8;      // [2] QK -> TMA
   uint64_t *sfull = bars + 10;      // [2] QK -> softmax
   uint64_t *sempty = bars + 12;     // [2] softmax -> QK
-  uint64_t *pfull = bars + 14;      // [2] softmax -> P.V
-  uint64_t *ofull = bars + 16;      // [2] P.V -> softmax
-  uint64_t *oempty = bars + 18;     // softmax -> P.V: O of a finished segment read out
-  uint64_t *drain = bars + 19;      // [2] QK warp, P.V warp: all their MMAs done
-  uint64_t *vfull = bars + 21;      // [NST]  V TMA -> P.V (and the softmax, for partial tiles)
-  uint64_t *vempty = bars + 24;     // [NST]  P.V -> V TMA
-  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 27);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 28);
-  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 29);  // 48 bytes
+  uint64_t *pfull = bars + 14;      // [NPB] softmax -> P.V
+  uint64_t *ofull = bars + 17;      // [NPB] P.V -> softmax
+  uint64_t *oempty = bars + 20;     // softmax -> P.V: O of a finished segment read out
+  uint64_t *drain = bars + 21;      // [2] QK warp, P.V warp: all their MMAs done
+  uint64_t *vfull = bars + 23;      // [NST]  V TMA -> P.V (and the softmax, for partial tiles)
+  uint64_t *vempty = bars + 26;     // [NST]  P.V -> V TMA
+  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 29);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 30);
+  ChunkPlan *plan = reinterpret_cast<ChunkPlan *>(bars + 31);  // 48 bytes
+  uint32_t *sh_done = reinterpret_cast<uint32_t *>(bars + 37);  // a counted part's count
   float *redmax = reinterpret_cast<float *>(smem + Cfg::OFF_RED);  // [4 warps][16 rows]
   float *redsum = redmax + 4 * N;                                  // [4 warps][16 rows]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int c = blockIdx.x;
-  const int T = mt.tokens;
-  const int R = 2 * T;  // query rows of a unit
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -176,6 +184,8 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
       mbar_init(&qempty[s], 1);
       mbar_init(&sfull[s], 1);
       mbar_init(&sempty[s], 4);
+    }
+    for (int s = 0; s < Cfg::NPB; ++s) {
       mbar_init(&pfull[s], 4);
       mbar_init(&ofull[s], 1);
     }
@@ -197,9 +207,10 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
   grid_launch_dependents();
   const int32_t split_k = p.split_k > 1 ? p.split_k : 1;
   const bool usplit = split_k > 1;
+  const int32_t crank = c % split_k;
   if (warp == 2) {
     if (usplit)
-      plan_unit_split(p.geo, c / split_k, c % split_k, split_k, Cfg::TILE, plan);
+      plan_unit_split(p.geo, c / split_k, crank, split_k, Cfg::TILE, plan);
     else
       plan_chunk(p.geo, c, plan);
   }
@@ -351,7 +362,7 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = a0 + ((j * Cfg::BOXB + kk * 32) >> 4);
             const uint64_t bd = qdesc + ((qb * Cfg::QB + j * Cfg::QBOXB + kk * 32) >> 4);
-            tc_mma_bf16(tmem + Cfg::S_COL + sb * 64 + kk * 16, ad, bd, idesc_qk, j != 0);
+            tc_mma_bf16(tmem + Cfg::S_COL + sb * 16, ad, bd, idesc_qk, j != 0 || kk != 0);
           }
         }
         tc_commit(&sfull[sb]);
@@ -378,7 +389,7 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
     int32_t row, ntok;
     bool first, last;
     while (ok && it.next(C, row, ntok, first, last)) {
-      bool w = mbar_wait(&pfull[t & 1], (t >> 1) & 1, abort_flag, p.status);
+      bool w = mbar_wait(&pfull[t % Cfg::NPB], (t / Cfg::NPB) & 1, abort_flag, p.status);
       if (w) w = mbar_wait(&vfull[t % NST], (t / NST) & 1, abort_flag, p.status);
       if (w && first && nseg > 0) w = mbar_wait(oempty, (nseg - 1) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, w)) {
@@ -388,7 +399,7 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
       if (first) ++nseg;
       tc_fence_after();
       const uint64_t a0 = vdesc + (((t % NST) * Cfg::STAGEB) >> 4);
-      const uint64_t b0 = pdesc + (((t & 1) * Cfg::PB) >> 4);
+      const uint64_t b0 = pdesc + (((t % Cfg::NPB) * Cfg::PB) >> 4);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
@@ -399,7 +410,7 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
             tc_mma_bf16(tmem + Cfg::O_COL + jb * Cfg::NP, ad, bd, idesc_pv, !(first && kk == 0));
           }
         }
-        tc_commit(&ofull[t & 1]);
+        tc_commit(&ofull[t % Cfg::NPB]);
         tc_commit(&vempty[t % NST]);
       }
       __syncwarp();
@@ -413,28 +424,101 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
     // ---------------------------------------------------------- softmax
     grid_dependency_wait();  // outputs and workspace are written below
     const int qd = warp & 3;
+    const int t128 = threadIdx.x - 64;       // thread within the softmax warps
     const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
     const int tok = 16 * qd + (lane & 15);  // tile token of this lane
     const int hd = lane >> 4;               // head of this lane: rows 2t + hd
+    const int32_t unit_k = c / split_k;  // the unit of a part when units are cut into parts
+    const bool has_part = plan->cs < plan->ce;
+    // This thread's output elements: row r, dims 32 qd + lane and 128 + 32 qd + lane.
+    int ed[2];
+#pragma unroll
+    for (int jb = 0; jb < 2; ++jb) ed[jb] = 128 * jb + 32 * qd + lane;
+    // Output row of query row r of unit (b, x) in the token-major out / lse.
+    auto out_row = [&](int32_t b, int32_t x, int r) -> int64_t {
+      return (static_cast<int64_t>(r >> 1) * p.geo.batch + b) * p.n_q_heads + x * Cfg::G +
+             (r & 1);
+    };
+    // One part of unit (b, x), whose parts sit in slots slot0 .. slot0 + np - 1,
+    // this one in slot `own`: store it (unless a wait failed: has_own false;
+    // an empty part stores LSE -inf), count it, and if it completes the count
+    // fold every part in slot order and write the unit's outputs.  Counted
+    // after a failed wait too, so the counters always return to zero.
+    auto count_and_merge = [&](int32_t unit, int32_t b, int32_t x, int64_t slot0, int32_t np,
+                               int64_t own, bool has_own, bool empty,
+                               const float (&own_v)[2][R], const float (&own_l)[R]) {
+      if (has_own) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+#pragma unroll
+          for (int jb = 0; jb < 2; ++jb) p.ws_o[(own * R + r) * D + ed[jb]] = own_v[jb][r];
+          if (t128 == r) p.ws_lse[own * R + r] = own_l[r];
+        }
+      } else if (empty && t128 < R) {
+        p.ws_lse[own * R + t128] = -INFINITY;
+      }
+      named_bar_sync(1, 128);  // every partial store before the count
+      if (t128 == 0) *sh_done = atomic_add_acq_rel_gpu(p.counters + unit, 1u);
+      named_bar_sync(1, 128);  // the acquire before every thread's reads
+      if (*sh_done == static_cast<uint32_t>(np - 1)) {
+        if (t128 == 0) p.counters[unit] = 0u;
+        PartMerge mg[2][R];
+        for (int32_t q = 0; q < np; ++q) {
+          const int64_t sq = slot0 + q;
+          float l[R], o0[R], o1[R];
+          if (sq == own) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              l[r] = has_own ? own_l[r] : -INFINITY;
+              o0[r] = own_v[0][r];
+              o1[r] = own_v[1][r];
+            }
+          } else {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              l[r] = __ldcg(p.ws_lse + sq * R + r);
+              o0[r] = __ldcg(p.ws_o + (sq * R + r) * D + ed[0]);
+              o1[r] = __ldcg(p.ws_o + (sq * R + r) * D + ed[1]);
+            }
+          }
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            mg[0][r].add(l[r], o0[r]);
+            mg[1][r].add(l[r], o1[r]);
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const int64_t orow = out_row(b, x, r);
+#pragma unroll
+          for (int jb = 0; jb < 2; ++jb) p.out[orow * D + ed[jb]] = f32_to_bf16_rn(mg[jb][r].out());
+          if (t128 == 0 && p.lse != nullptr) p.lse[orow] = mg[0][r].lse();
+        }
+      }
+      named_bar_sync(1, 128);  // sh_done read before the next count
+    };
     // P row r holds query row r's bf16 weights and row N + r their remainders;
     // the rows of r >= R multiply O columns nobody reads: keep them zero.
-    for (int e = threadIdx.x - 64; e < 2 * Cfg::NP * 8; e += 128) {
+    for (int e = t128; e < Cfg::NPB * Cfg::NP * 8; e += 128) {
       const int buf = e / (Cfg::NP * 8), r = (e % (Cfg::NP * 8)) >> 3;
       if ((r & (N - 1)) >= R)
         *reinterpret_cast<uint4 *>(ps + buf * Cfg::PB + r * 128 + (e & 7) * 16) =
             make_uint4(0u, 0u, 0u, 0u);
     }
-    float m_ref[N];     // reference max of every query row (the same in all lanes)
-    float lpart[TMAX];  // this lane's share of the weight sum of row 2t + hd
+    float m_ref[R];  // reference max of every query row (the same in all lanes)
+    float lpart[T];  // this lane's share of the weight sum of row 2t + hd
 #pragma unroll
-    for (int r = 0; r < N; ++r) m_ref[r] = -INFINITY;
+    for (int r = 0; r < R; ++r) m_ref[r] = -INFINITY;
 #pragma unroll
-    for (int t = 0; t < TMAX; ++t) lpart[t] = 0.f;
+    for (int t = 0; t < T; ++t) lpart[t] = 0.f;
     bool ok = true;
-    uint32_t cons0 = 0, cons1 = 0;  // ofull phases consumed on barrier 0 / 1
+    // ofull phases consumed on barriers 0, 1, 2.  Wait until the P.V of tile
+    // tt has completed; phases are consumed in order and never lag by two, so
+    // the parity waits cannot alias.
+    uint32_t cons0 = 0, cons1 = 0, cons2 = 0;
     auto ensure_pv = [&](uint32_t tt) {
-      const uint32_t b = tt & 1, ph = tt >> 1;
-      uint32_t &cons = b ? cons1 : cons0;
+      const uint32_t b = tt % Cfg::NPB, ph = tt / Cfg::NPB;
+      uint32_t &cons = b == 0 ? cons0 : (b == 1 ? cons1 : cons2);
       if (cons <= ph) {
         if (ok && !mbar_wait(&ofull[b], cons & 1, abort_flag, p.status)) ok = false;
         ++cons;
@@ -447,51 +531,53 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
     int32_t row, ntok;
     bool first, last;
     while (it.next(C, row, ntok, first, last)) {
-      const int sb = i & 1, pb = i & 1;
-      if (i >= 2) ensure_pv(i - 2);  // P buffer pb is free again
+      const int sb = i & 1, pb = i % Cfg::NPB;
+      if (i >= Cfg::NPB) ensure_pv(i - Cfg::NPB);  // P buffer pb is free again
       if (first) {
 #pragma unroll
-        for (int r = 0; r < N; ++r) m_ref[r] = -INFINITY;
+        for (int r = 0; r < R; ++r) m_ref[r] = -INFINITY;
 #pragma unroll
-        for (int t = 0; t < TMAX; ++t) lpart[t] = 0.f;
+        for (int t = 0; t < T; ++t) lpart[t] = 0.f;
       }
       const Segment &sg = it.seg;
       const int32_t j = it.off + tok;  // offset of this lane's cache token in the unit's range
-      // --- scores of tile i: each row's column summed over the four accumulators
-      float s[TMAX];
+      // --- scores of tile i
+      float s[T];
       if (ok && !mbar_wait(&sfull[sb], (i >> 1) & 1, abort_flag, p.status)) ok = false;
       ok = __all_sync(0xffffffffu, ok);
       {
-        float acc4[64];
+        // column r of S^T is query row r's score
+        float acc[16];
         if (ok) {
           tc_fence_after();
-          tmem_ld64(tmem + lane_base + Cfg::S_COL + sb * 64, acc4);
+          tmem_ld16(tmem + lane_base + Cfg::S_COL + sb * 16, acc);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sempty[sb]);
         } else {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) acc4[e] = 0.f;
+          for (int r = 0; r < 16; ++r) acc[r] = 0.f;
         }
         // lanes 0-15 keep head 0 (even rows) of their token; lanes 16-31 take
         // head 1 (odd rows) of the token of lane - 16
 #pragma unroll
-        for (int t = 0; t < TMAX; ++t) {
-          const float r0 = (acc4[2 * t] + acc4[16 + 2 * t]) + (acc4[32 + 2 * t] + acc4[48 + 2 * t]);
-          const float r1 =
-              (acc4[2 * t + 1] + acc4[17 + 2 * t]) + (acc4[33 + 2 * t] + acc4[49 + 2 * t]);
-          const float got = __shfl_xor_sync(0xffffffffu, r1, 16);
-          s[t] = (lane < 16) ? r0 : got;
+        for (int t = 0; t < T; ++t) {
+          const float got = __shfl_xor_sync(0xffffffffu, acc[2 * t + 1], 16);
+          s[t] = (lane < 16) ? acc[2 * t] : got;
         }
       }
       // Token t sits at offset n - T + t of the unit's range (positions
-      // [L - n, L) are offsets [0, n)) and attends the offsets of its window.
+      // [L - n, L) are offsets [0, n)) and attends offsets up to its own, from
+      // n - T + t + 1 - w on with a window w: this lane's cache token j is in
+      // the range of the tokens t with j - (n - T) <= t <= j - (n - T + 1 - w)
+      // (no upper bound without a window).
+      const int32_t tmin = j - (sg.n - T);
+      const int32_t tmax = mt.window > 0 ? j - (sg.n - T + 1 - mt.window) : T;
+      const bool tok_ok = ok && tok < ntok;
       bool need = false;
 #pragma unroll
-      for (int t = 0; t < TMAX; ++t) {
-        const int32_t pos = sg.n - T + t;
-        const int32_t lo_t = mt.window > 0 ? pos + 1 - mt.window : 0;
-        const bool valid = ok && t < T && tok < ntok && j >= lo_t && j <= pos;
+      for (int t = 0; t < T; ++t) {
+        const bool valid = tok_ok && t >= tmin && t <= tmax;
         float x = s[t] * p.qscale;
         if (p.post != 0.f) x = p.post * tanhf(x);
         s[t] = valid ? x : -INFINITY;
@@ -501,28 +587,25 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
       // --- move the references only when some score outgrew its own
       if (named_bar_or(1, 128, need)) {
 #pragma unroll
-        for (int t = 0; t < TMAX; ++t) {
+        for (int t = 0; t < T; ++t) {
           float mx = s[t];
 #pragma unroll
           for (int off = 1; off < 16; off <<= 1)
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-          if ((lane & 15) == 0 && t < T) redmax[qd * N + 2 * t + hd] = mx;
+          if ((lane & 15) == 0) redmax[qd * N + 2 * t + hd] = mx;
         }
         named_bar_sync(1, 128);
-        float alpha[N];
+        float alpha[R];
 #pragma unroll
-        for (int r = 0; r < N; ++r) {
-          alpha[r] = 1.f;
-          if (r < R) {
-            const float tm = fmaxf(fmaxf(redmax[r], redmax[N + r]),
-                                   fmaxf(redmax[2 * N + r], redmax[3 * N + r]));
-            const float mn = fmaxf(m_ref[r], tm);
-            alpha[r] = (m_ref[r] == -INFINITY) ? 0.f : exp2f(m_ref[r] - mn);
-            m_ref[r] = mn;
-          }
+        for (int r = 0; r < R; ++r) {
+          const float tm = fmaxf(fmaxf(redmax[r], redmax[N + r]),
+                                 fmaxf(redmax[2 * N + r], redmax[3 * N + r]));
+          const float mn = fmaxf(m_ref[r], tm);
+          alpha[r] = (m_ref[r] == -INFINITY) ? 0.f : exp2f(m_ref[r] - mn);
+          m_ref[r] = mn;
         }
 #pragma unroll
-        for (int t = 0; t < TMAX; ++t) lpart[t] *= hd ? alpha[2 * t + 1] : alpha[2 * t];
+        for (int t = 0; t < T; ++t) lpart[t] *= hd ? alpha[2 * t + 1] : alpha[2 * t];
         if (!first) {
           // O holds tiles < i: wait for the last of them, then rescale it in TMEM.
           ensure_pv(i - 1);
@@ -533,7 +616,7 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
               float o[Cfg::NP];  // columns r (hi) and N + r (lo) of query row r
               tmem_ld32(tmem + lane_base + Cfg::O_COL + jb * Cfg::NP, o);
 #pragma unroll
-              for (int r = 0; r < N; ++r) {
+              for (int r = 0; r < R; ++r) {
                 o[r] *= alpha[r];
                 o[N + r] *= alpha[r];
               }
@@ -546,8 +629,7 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
       {
         uint8_t *pbuf = ps + pb * Cfg::PB;
 #pragma unroll
-        for (int t = 0; t < TMAX; ++t) {
-          if (t >= T) break;
+        for (int t = 0; t < T; ++t) {
           const float mr = hd ? m_ref[2 * t + 1] : m_ref[2 * t];
           const float pe = (s[t] == -INFINITY) ? 0.f : exp2f(s[t] - mr);
           lpart[t] += pe;
@@ -569,7 +651,7 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
         const int per_box = (Cfg::TILE - ntok) * 8;
 #pragma unroll 1
         for (int box = 0; box < D / 64; ++box)
-          for (int e = threadIdx.x - 64; e < per_box; e += 128)
+          for (int e = t128; e < per_box; e += 128)
             *reinterpret_cast<uint4 *>(vt + box * Cfg::BOXB + (ntok + (e >> 3)) * 128 +
                                        (e & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
       }
@@ -581,76 +663,82 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
       if (last) {
         // --- segment end: row sums, then O of the segment's last P.V
 #pragma unroll
-        for (int t = 0; t < TMAX; ++t) {
+        for (int t = 0; t < T; ++t) {
           float ls = lpart[t];
 #pragma unroll
           for (int off = 1; off < 16; off <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
-          if ((lane & 15) == 0 && t < T) redsum[qd * N + 2 * t + hd] = ls;
+          if ((lane & 15) == 0) redsum[qd * N + 2 * t + hd] = ls;
         }
         named_bar_sync(1, 128);
         if (i >= 1) ensure_pv(i - 1);
         ensure_pv(i);
         const bool single = sg.whole() && !usplit;
         const int64_t slot = static_cast<int64_t>(c) + sg.unit;
-        const int h0 = sg.x * Cfg::G;
-        float L[N], inv[N];
+        // Normalised O and LSE of every row of this part.  A row that attends
+        // nothing here (another token's positions only, or a token before the
+        // sequence's start) has LSE -inf and weight 0 in any merge.
+        float val[2][R], lse_v[R];
 #pragma unroll
-        for (int r = 0; r < N; ++r) {
-          L[r] = (redsum[r] + redsum[N + r]) + (redsum[2 * N + r] + redsum[3 * N + r]);
-          // A row that attends nothing here (a token before the sequence's
-          // start) gets a zero output and LSE -inf.
-          inv[r] = L[r] > 0.f ? __fdividef(1.f, L[r]) : 0.f;
+        for (int r = 0; r < R; ++r) {
+          const float L = (redsum[r] + redsum[N + r]) + (redsum[2 * N + r] + redsum[3 * N + r]);
+          const float inv = L > 0.f ? __fdividef(1.f, L) : 0.f;
+          lse_v[r] = L > 0.f ? (m_ref[r] + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+          val[0][r] = inv;  // scaled below
+          val[1][r] = inv;
+        }
+        if (ok) tc_fence_after();
+#pragma unroll
+        for (int jb = 0; jb < 2; ++jb) {
+          float o[Cfg::NP];
+#pragma unroll
+          for (int e = 0; e < Cfg::NP; ++e) o[e] = 0.f;
+          if (ok) tmem_ld32(tmem + lane_base + Cfg::O_COL + jb * Cfg::NP, o);
+#pragma unroll
+          for (int r = 0; r < R; ++r) val[jb][r] *= o[r] + o[N + r];
         }
         if (ok) {
-          tc_fence_after();
-#pragma unroll
-          for (int jb = 0; jb < 2; ++jb) {
-            float o[Cfg::NP];
-            tmem_ld32(tmem + lane_base + Cfg::O_COL + jb * Cfg::NP, o);
-            const int d = 128 * jb + 32 * qd + lane;
-#pragma unroll
-            for (int r = 0; r < N; ++r) {
-              if (r >= R) break;
-              const float val = (o[r] + o[N + r]) * inv[r];
-              const int t = r >> 1, h = r & 1;
-              if (single)
-                p.out[((static_cast<int64_t>(t) * p.geo.batch + sg.b) * p.n_q_heads + h0 + h) *
-                          D +
-                      d] = f32_to_bf16_rn(val);
-              else
-                p.ws_o[(slot * R + r) * D + d] = val;
-            }
-          }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(oempty);
-          if (qd == 0 && lane < R) {  // LSE of query row `lane`
-            float mr = -INFINITY, Lr = 0.f;
+        }
+        if (single) {
+          if (ok) {
 #pragma unroll
-            for (int r = 0; r < N; ++r)
-              if (lane == r) {
-                mr = m_ref[r];
-                Lr = L[r];
-              }
-            const float lse_v =
-                Lr > 0.f ? (mr + log2f(Lr)) * 0.69314718055994530942f : -INFINITY;
-            const int t = lane >> 1, h = lane & 1;
-            if (single) {
-              if (p.lse != nullptr)
-                p.lse[(static_cast<int64_t>(t) * p.geo.batch + sg.b) * p.n_q_heads + h0 + h] =
-                    lse_v;
-            } else {
-              p.ws_lse[slot * R + lane] = lse_v;
+            for (int r = 0; r < R; ++r) {
+              const int64_t orow = out_row(sg.b, sg.x, r);
+#pragma unroll
+              for (int jb = 0; jb < 2; ++jb) p.out[orow * D + ed[jb]] = f32_to_bf16_rn(val[jb][r]);
+              if (t128 == 0 && p.lse != nullptr) p.lse[orow] = lse_v[r];
             }
           }
+        } else {
+          int64_t slot0;
+          int32_t np;
+          if (usplit) {  // part crank of unit c / k sits in slot (c / k) * k + unit + crank
+            slot0 = static_cast<int64_t>(unit_k) * split_k + unit_k;
+            np = split_k;
+          } else {
+            int32_t cf, cl;
+            unit_chunks(sg.unit_start, sg.n, plan->chunk, cf, cl);
+            slot0 = static_cast<int64_t>(cf) + sg.unit;
+            np = cl - cf + 1;
+          }
+          count_and_merge(sg.unit, sg.b, sg.x, slot0, np, slot, ok, false, val, lse_v);
         }
       }
       ++i;
     }
-    if (usplit && i == 0 && qd == 0 && lane < R) {
-      // An empty part (the unit is shorter than split_k tiles): LSE -inf.
-      const int64_t slot = static_cast<int64_t>(c) + c / split_k;
-      p.ws_lse[slot * R + lane] = -INFINITY;
+    if (usplit && !has_part) {
+      // An empty part (the unit is shorter than its parts) still counts.
+      float none_v[2][R], none_l[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        none_v[0][r] = none_v[1][r] = 0.f;
+        none_l[r] = -INFINITY;
+      }
+      const int32_t b = unit_k / p.geo.units_per_seq, x = unit_k - b * p.geo.units_per_seq;
+      const int64_t slot0 = static_cast<int64_t>(unit_k) * split_k + unit_k;
+      count_and_merge(unit_k, b, x, slot0, split_k, slot0 + crank, false, true, none_v, none_l);
     }
   }
 
