@@ -19,6 +19,7 @@
 #include "tc_pair_decode.cuh"
 #include "tc_pair_fp8_decode.cuh"
 #include "tc_pair_multi_decode.cuh"
+#include "tc_pair_prefill.cuh"
 
 using namespace gdattn;
 
@@ -180,6 +181,10 @@ using MultiPassFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtenso
                              const TcParams, const MultiTokens);
 int query_tc_pair_multi(const void *fn, int threads, int smem) {
   return blocks_per_sm(reinterpret_cast<MultiPassFn>(const_cast<void *>(fn)), threads, smem);
+}
+int query_prefill(const void *fn, int threads, int smem) {
+  using Fn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const PrefillParams);
+  return blocks_per_sm(reinterpret_cast<Fn>(const_cast<void *>(fn)), threads, smem);
 }
 // The single-pass multi-token kernel for T tokens (1..8), else null.
 MultiPassFn multi_pass_kernel(int32_t T) {
@@ -437,15 +442,16 @@ bool encode_q_rows_map(EncodeTiledFn enc, CUtensorMap *map, const void *q, int32
 }
 
 // q [T][rows][D] bf16 (rows = B * Hq) as a 3-D tensor map read in
-// {64 d, 2 rows, T tokens} boxes with 128-byte swizzle: the 2T query rows of a
-// pair unit land as 2T consecutive 128-byte rows, token-major.
+// {64 d, 2 rows, box_tokens tokens} boxes with 128-byte swizzle: the query rows
+// of a pair unit (2 heads x box_tokens tokens) land as consecutive 128-byte
+// rows, token-major; tokens past T read as zeros.
 bool encode_q_tokens_map(EncodeTiledFn enc, CUtensorMap *map, const void *q, int32_t D,
-                         int64_t rows, int32_t T) {
+                         int64_t rows, int32_t T, int32_t box_tokens) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(T)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
                                  static_cast<cuuint64_t>(rows) * D * 2};
-  const cuuint32_t box[3] = {64, 2, static_cast<cuuint32_t>(T)};
+  const cuuint32_t box[3] = {64, 2, static_cast<cuuint32_t>(box_tokens)};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -724,6 +730,74 @@ gdattn_layer_desc union_window_desc(const gdattn_layer_desc *d, int32_t T) {
   return u;
 }
 
+// Multi-token steps of more than 8 tokens on the pair geometry (prompt chunks)
+// run as flash prefill (tc_pair_prefill.cuh), up to this many tokens.
+constexpr int32_t kMaxPrefillTokens = 1 << 20;
+bool multi_prefill(const gdattn_layer_desc *d, int32_t T) {
+  return choose_path(d) == PathKind::kTcPair && T > TcPairMultiConfig::TMAX;
+}
+
+// Checks the prefill launch for this geometry (and sets the kernel's shared
+// memory limit); the workspace is the fixed header alone (the status word).
+gdattn_status plan_prefill(int32_t batch, int32_t T, const gdattn_layer_desc *d,
+                           size_t *ws_bytes) {
+  gdattn_status st = check_desc(d);
+  if (st != GDATTN_OK) return st;
+  if (batch <= 0 || T < 1 || T > kMaxPrefillTokens) return GDATTN_ERR_INVALID_ARG;
+  const int64_t nblocks = (T + TcPrefillConfig::QT - 1) / TcPrefillConfig::QT;
+  if (static_cast<int64_t>(batch) * d->n_kv_heads * nblocks > INT32_MAX)
+    return GDATTN_ERR_UNSUPPORTED;
+  if (cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_prefill_kernel),
+                           TcPrefillConfig::kThreads, TcPrefillConfig::SMEM, query_prefill) <= 0)
+    return GDATTN_ERR_CUDA;
+  *ws_bytes = kHeaderBytes;
+  return GDATTN_OK;
+}
+
+gdattn_status enqueue_prefill(const void *q, const void *k_cache, const void *v_cache,
+                              const int32_t *seqlens, int32_t batch, int32_t T,
+                              const gdattn_layer_desc *desc, void *out, float *lse, uint8_t *ws,
+                              cudaStream_t stream) {
+  const int32_t D = desc->head_dim;
+  const int32_t Hkv = desc->n_kv_heads;
+  const int64_t bstride = desc->cache_batch_stride != 0
+                              ? desc->cache_batch_stride
+                              : static_cast<int64_t>(desc->cache_capacity) * Hkv * D;
+  const float log2e = 1.4426950408889634f;
+  EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return GDATTN_ERR_CUDA;
+  CUtensorMap kmap, vmap, qmap;
+  if (!encode_cache_map(enc, &kmap, k_cache, D, Hkv, desc->cache_capacity, batch, bstride,
+                        TcPrefillConfig::TILE) ||
+      !encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, batch, bstride,
+                        TcPrefillConfig::TILE) ||
+      !encode_q_tokens_map(enc, &qmap, q, D, static_cast<int64_t>(batch) * desc->n_q_heads, T,
+                           TcPrefillConfig::QT))
+    return GDATTN_ERR_CUDA;
+  PrefillParams pp;
+  pp.seqlens = seqlens;
+  pp.out = static_cast<uint16_t *>(out);
+  pp.lse = lse;
+  pp.status = reinterpret_cast<uint32_t *>(ws);
+  pp.batch = batch;
+  pp.n_q_heads = desc->n_q_heads;
+  pp.n_kv_heads = Hkv;
+  pp.tokens = T;
+  pp.nblocks = (T + TcPrefillConfig::QT - 1) / TcPrefillConfig::QT;
+  pp.window = desc->window;
+  pp.capacity = desc->cache_capacity;
+  pp.qscale = desc->softcap > 0.f ? desc->scale / desc->softcap : desc->scale * log2e;
+  pp.post = desc->softcap > 0.f ? desc->softcap * log2e : 0.f;
+  pp.test_withhold = (desc->flags & GDATTN_FLAG_TEST_WITHHOLD_KV) ? 1 : 0;
+  const unsigned grid = static_cast<unsigned>(static_cast<int64_t>(batch) * Hkv * pp.nblocks);
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = launch_config(dim3(grid), TcPrefillConfig::kThreads,
+                                         TcPrefillConfig::SMEM, stream, attr);
+  return cudaLaunchKernelEx(&cfg, tc_pair_prefill_kernel, kmap, vmap, qmap, pp) == cudaSuccess
+             ? GDATTN_OK
+             : GDATTN_ERR_CUDA;
+}
+
 // Enqueues the single-pass multi-token kernel (it merges split units itself);
 // pl comes from make_plan over union_window_desc(desc, T).
 gdattn_status enqueue_decode_multi_pass(const LayerPlan &pl, const void *q, const void *k_cache,
@@ -745,7 +819,8 @@ gdattn_status enqueue_decode_multi_pass(const LayerPlan &pl, const void *q, cons
                         TcPairMultiConfig::TILE) ||
       !encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, batch, bstride,
                         TcPairMultiConfig::TILE) ||
-      !encode_q_tokens_map(enc, &qmap, q, D, static_cast<int64_t>(batch) * desc->n_q_heads, T))
+      !encode_q_tokens_map(enc, &qmap, q, D, static_cast<int64_t>(batch) * desc->n_q_heads, T,
+                           T))
     return GDATTN_ERR_CUDA;
   Geometry geo;
   geo.seqlens = seqlens;
@@ -980,7 +1055,12 @@ gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *
 
 size_t gdattn_multi_workspace_size(int32_t batch, int32_t n_tokens, int32_t max_seqlen,
                                    const gdattn_layer_desc *desc) {
-  if (n_tokens < 1 || n_tokens > kMaxMultiTokens || batch <= 0 || desc == nullptr) return 0;
+  if (batch <= 0 || desc == nullptr) return 0;
+  if (multi_prefill(desc, n_tokens)) {
+    size_t bytes = 0;
+    return plan_prefill(batch, n_tokens, desc, &bytes) == GDATTN_OK ? bytes : 0;
+  }
+  if (n_tokens < 1 || n_tokens > kMaxMultiTokens) return 0;
   LayerPlan pl;
   if (multi_single_pass(desc, n_tokens)) {
     const gdattn_layer_desc ud = union_window_desc(desc, n_tokens);
@@ -999,7 +1079,9 @@ gdattn_status gdattn_decode_multi(const void *q, const void *k_cache, const void
   gdattn_status st = check_decode_args(q, k_cache, v_cache, seqlens, batch, max_seqlen, desc,
                                        out, lse);
   if (st != GDATTN_OK) return st;
-  if (n_tokens < 1 || n_tokens > kMaxMultiTokens || n_tokens > max_seqlen)
+  const int32_t max_tokens = choose_path(desc) == PathKind::kTcPair ? kMaxPrefillTokens
+                                                                    : kMaxMultiTokens;
+  if (n_tokens < 1 || n_tokens > max_tokens || n_tokens > max_seqlen)
     return GDATTN_ERR_INVALID_ARG;
   // A ring holds positions [L - C, L): the first token's window must still be in it.
   if (desc->window > 0 && desc->cache_capacity < max_seqlen &&
@@ -1008,6 +1090,14 @@ gdattn_status gdattn_decode_multi(const void *q, const void *k_cache, const void
     return GDATTN_ERR_INVALID_ARG;
   if (workspace == nullptr) return GDATTN_ERR_WORKSPACE;
   if (!aligned16(workspace)) return GDATTN_ERR_MISALIGNED;
+  if (multi_prefill(desc, n_tokens)) {
+    size_t bytes = 0;
+    st = plan_prefill(batch, n_tokens, desc, &bytes);
+    if (st != GDATTN_OK) return st;
+    if (workspace_bytes < bytes) return GDATTN_ERR_WORKSPACE;
+    return enqueue_prefill(q, k_cache, v_cache, seqlens, batch, n_tokens, desc, out, lse,
+                           static_cast<uint8_t *>(workspace), static_cast<cudaStream_t>(stream_));
+  }
   if (multi_single_pass(desc, n_tokens)) {
     const gdattn_layer_desc ud = union_window_desc(desc, n_tokens);
     LayerPlan pl;

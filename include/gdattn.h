@@ -276,7 +276,8 @@ gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *
  *
  *  q         bf16 [T, batch, Hq, D] (token-major), device, read only
  *  out       bf16 [T, batch, Hq, D];  lse: fp32 [T, batch, Hq] or NULL
- *  n_tokens  T, 1 <= T <= 64;  seqlens: L_b >= T, the length with all T tokens
+ *  n_tokens  T: 1 <= T <= 64, or up to 2^20 on the pair geometry (a prompt
+ *            chunk);  seqlens: L_b >= T, the length with all T tokens
  *  workspace at least gdattn_multi_workspace_size bytes (zeroed once by
  *            gdattn_workspace_init)
  *  other arguments, geometries and device-side errors as gdattn_decode.
@@ -289,7 +290,11 @@ gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *
  * with T <= 8 the step is one pass over the cache: a unit's 2T query rows (token,
  * head) share every K and V tile of the union of their windows, the last
  * min(L_b, window + T - 1) positions, and each score is masked to its own
- * token's range; split units are merged by the LSE-combine kernel.  Otherwise
+ * token's range; split units are merged inside the kernel.  With T > 8 on the
+ * same geometry the step is flash prefill ("Gemma support" pull request,
+ * Performance: flash prefill for head_dim 256): one CTA per 64 query tokens of a
+ * (sequence, KV head), 128 query rows per tensor-core tile, streaming that
+ * block's KV range once; its workspace is the fixed header alone.  Otherwise
  * one small kernel writes the T per-token lengths into the workspace, then one
  * decode launch runs over T x batch query sequences (token-major) in which query
  * sequence t * batch + b reads cache sequence b; the T tokens of a sequence then

@@ -26,8 +26,12 @@ CASES = {
     "pair_global_t5": (5, 2, 4, 2, 256, 700, [700, 333], 0, 0.0, False, 0),
     # forced flattened chunks: tokens' windows cut across many parts
     "pair_split40_t6": (6, 2, 16, 8, 256, 1100, [1100, 800], 1024, 0.0, False, 0, 40),
-    # past 8 tokens the pair geometry runs as T x B sequences
-    "pair_t9_per_token": (9, 2, 16, 8, 256, 300, [300, 50], 128, 0.0, False, 0),
+    # past 8 tokens the pair geometry runs as flash prefill: 64-token query blocks
+    "prefill_t9": (9, 3, 16, 8, 256, 600, [600, 9, 300], 512, 0.0, False, 0),
+    "prefill_t64_prompt": (64, 2, 16, 8, 256, 1100, [1100, 64], 1024, 0.0, False, 0),
+    "prefill_t200_ring_cap": (200, 2, 16, 8, 256, 1223, [3000, 1223], 1024, 50.0, False, 0),
+    "prefill_t130_small_w": (130, 2, 16, 8, 256, 300, [300, 131], 100, 0.0, False, 0),
+    "prefill_t513_global": (513, 1, 4, 2, 256, 700, [600], 0, 0.0, False, 0),
     # tcgen05 16-head kernel (global, K = V)
     "tc16_t3": (3, 2, 16, 1, 512, 400, [400, 77], 0, 0.0, True, 0),
     "tc16_even_t2": (2, 2, 32, 2, 512, 300, [300, 300], 0, 30.0, True, 1),
@@ -80,7 +84,8 @@ def test_multi_matches_oracle(name):
                     what=f"{name} token {t} call {rep}")
 
 
-@pytest.mark.parametrize("name,short_len", [("core_g4_t3", 2), ("pair_no_wrap_t7", 5)])
+@pytest.mark.parametrize("name,short_len", [("core_g4_t3", 2), ("pair_no_wrap_t7", 5),
+                                            ("prefill_t130_small_w", 70)])
 def test_multi_tokens_before_the_context_are_reported(name, short_len):
     """A sequence shorter than T: its tokens at positions below 0 attend nothing;
     the device reports it, gives them zero output and LSE -inf, and its other
