@@ -61,6 +61,19 @@ def measured_peak_gbs():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+FALLBACK_BF16_TFLOPS = 1590.0  # an earlier burst measurement on this machine
+
+
+def measured_peak_tflops():
+    """Dense bf16 tensor peak: the measured cuBLAS burst figure, else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
 def kernel_source_hash():
     """Hash of the device code of the profiled kernels: every kernel lives in a
     csrc/*.cuh header (api.cu holds the host-side launches)."""
@@ -812,6 +825,62 @@ def run_ours(args, world, rank, local):
             del g_msl, bufs
         del caches_m
 
+    # ---- flash prefill (gdattn_decode_multi with a prompt chunk) on the sliding
+    # geometry: one 8192-token prompt per layer (a cache of 8192 slots, L = T),
+    # 4 layers of their own replayed in turn (1 GiB of q, K, V and out).
+    prefill = None
+    if sliding_idx:
+        sp0 = stack.layers[sliding_idx[0]]["spec"]
+        t_pf, n_pf = 8192, 4
+        spec_p = dataclasses.replace(sp0, capacity=t_pf)
+        seqlens_p = torch.full((1,), t_pf, dtype=torch.int32)
+        desc_p = binding.desc_from_spec(spec_p)
+        gen_p = torch.Generator(device="cpu").manual_seed(17 + rank)
+        bufs_p = []
+        for j in range(n_pf):
+            inp = workloads.layer_inputs(spec_p, 1, seqlens_p,
+                                         w.seed * 1000 + 950 + j + rank_seed_offset(rank),
+                                         device=device)
+            qp = torch.randn((t_pf, 1, spec_p.n_q_heads, spec_p.head_dim),
+                             generator=gen_p).to(torch.bfloat16).to(device)
+            wsp = torch.empty(binding.multi_workspace_size(1, t_pf, t_pf, desc_p),
+                              dtype=torch.uint8, device=device)
+            binding.workspace_init(wsp, stream)
+            bufs_p.append((inp, qp, wsp, torch.empty_like(qp),
+                           torch.empty((t_pf, 1, spec_p.n_q_heads), device=device)))
+
+        def prefill_step():
+            for inp, qp, wsp, op, lp in bufs_p:
+                binding.decode_multi(qp, inp.k, inp.v, inp.seqlens, desc_p, t_pf, out=op, lse=lp,
+                                     workspace=wsp, stream=stream)
+
+        g_pf = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            prefill_step()
+            stream.synchronize()
+            with torch.cuda.graph(g_pf, stream=stream):
+                prefill_step()
+        barrier()
+        ms_pf = max_over_ranks(time_graph(g_pf, stream, max(3, replays // 20), 3), world)
+        for inp, qp, wsp, op, lp in bufs_p:
+            st = binding.check_device_status(wsp, stream)
+            if st != binding.GDATTN_OK:
+                raise binding.GdattnError(st, "device status after the prefill step")
+        flops = n_pf * accounting.layer_prefill_flops(spec_p, seqlens_p.tolist(), t_pf)
+        tf_peak, tf_kind = measured_peak_tflops()
+        tflops = flops / (ms_pf * 1e-3) / 1e12
+        prefill = {
+            "kernel": "tc_pair_prefill_kernel (tcgen05: S = Q K^T with M = 128 query rows, "
+                      "P.V with bf16 weights plus remainders)",
+            "tokens": t_pf, "us_per_layer": ms_pf / n_pf * 1e3,
+            "tflops": tflops, "peak_tflops": tf_peak, "peak_kind": tf_kind,
+            "frac": tflops / tf_peak, "bound": "tensor",
+            "how": "one 8192-token prompt (window 1024, 16 query / 8 KV heads, head_dim 256) "
+                   "per layer through gdattn_decode_multi, 4 layers replayed in turn in a CUDA "
+                   "graph; useful flops = 4 x head_dim per (query head, token, attended "
+                   "position), so the weight split's second P.V half counts as overhead"}
+        del g_pf, bufs_p
+
     # ---- CPU baseline: the oracle over the whole step (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
@@ -956,6 +1025,7 @@ def run_ours(args, world, rank, local):
                    "merged in the kernel); t1 is one token through gdattn_decode on the same "
                    "rings, the base of vs_single_token; kv_gbs counts the union once; CUDA "
                    "graph, device time, the 8 layers replayed in turn"},
+        "prefill": prefill,
         "gpu_launches": stack.launches_per_step(all_idx) * replays,
         "clocks": clk,
     }

@@ -50,6 +50,27 @@ def layer_multi_kv_bytes(spec, seqlens, tokens: int) -> int:
     return sum(union_positions(spec, int(L), tokens) * per for L in seqlens)
 
 
+def multi_attended_pairs(spec, seqlen: int, tokens: int) -> int:
+    """(query token, attended position) pairs of one query head in a T-token step:
+    token t at p = L - T + t attends min(p + 1, w) positions (p + 1 without a
+    window)."""
+    total = 0
+    for t in range(tokens):
+        p = seqlen - tokens + t
+        if p < 0:
+            continue
+        total += min(p + 1, spec.window) if spec.window > 0 else p + 1
+    return total
+
+
+def layer_prefill_flops(spec, seqlens, tokens: int) -> int:
+    """Useful flops of a T-token step (prefill chunk) of one layer: 2 D for the
+    score and 2 D for the weighted value of every (query head, token, attended
+    position)."""
+    per = 4 * spec.head_dim * spec.n_q_heads
+    return sum(multi_attended_pairs(spec, int(L), tokens) * per for L in seqlens)
+
+
 FP8_ROW_EXTRA = 4  # the fp32 scale stored with every fp8 cache row
 
 

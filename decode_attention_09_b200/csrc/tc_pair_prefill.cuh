@@ -15,9 +15,9 @@
 //
 // Every TMEM lane is a query row, so each softmax thread owns a row: its 64
 // scores, mask, running maximum, row sum and the rescale of its O row need no
-// exchange with other threads.  P is stored as the bf16 weights plus their bf16
-// remainders (two K = 64 halves of the P.V product), the decode kernels' weight
-// split, so the weights keep about 16 significant bits on a bf16 MMA.  The
+// exchange with other threads.  P is stored as bf16 weights plus their bf16
+// remainders (two K = 64 halves of the P.V product), like the decode kernels'
+// weight split, so a weight keeps 2^-14 relative precision on a bf16 MMA.  The
 // reference maximum of a row moves lazily: only when a score exceeds it by
 // more than 2^8, and then the thread rescales its O row in TMEM after the
 // previous P.V completed.
@@ -28,9 +28,14 @@
 // and causal bound, and V rows past a partial tile's end are cleared, since
 // they may hold anything.
 //
-// Shared memory (1 CTA per SM): two K/V stages (32 KiB each of K and V), the
-// block's Q (64 KiB, loaded once), and the two P halves (16 KiB each): 224 KiB.
-// TMEM: S double buffered (2 x 64 columns) and O (256 columns).
+// Shared memory (1 CTA per SM): a ring of three 32 KiB K tiles (a K tile is
+// released as soon as its QK is done, so the K loads run further ahead), a ring
+// of two V tiles, and the block's Q (64 KiB, loaded once): 224 KiB.  TMEM holds the rest: S double
+// buffered (2 x 64 columns), P double buffered (each 32 columns of bf16 pairs
+// for the weights and 32 for their remainders, the A operand of P.V read from
+// tensor memory), and O (256 columns).  With two P buffers the softmax of tile
+// i waits only for the P.V of tile i - 2, so the tensor pipe is not left idle
+// while P is written.
 //
 // Warp roles (256 threads): warp 0 loads Q and K, warp 3 loads V, warp 1 issues
 // QK and owns TMEM, warp 2 issues P.V, warps 4-7 run the softmax (warp 4 + s
@@ -54,20 +59,20 @@ struct TcPrefillConfig {
   static constexpr int QT = 64;                   // query tokens per block
   static constexpr int M = QT * G;                // 128 query rows
   static constexpr int TILE = 64;                 // KV tokens per tile
-  static constexpr int NST = 2;                   // K/V stages
+  static constexpr int NSTK = 3;                  // K ring
+  static constexpr int NSTV = 2;                  // V ring
   static constexpr int BOXB = TILE * 128;         // 64 KV rows x 64 d: 8 KiB
   static constexpr int KB = BOXB * (D / 64);      // 32 KiB
-  static constexpr int STAGEB = 2 * KB;           // K then V
   static constexpr int QBOXB = M * 128;           // 128 rows x 64 d: 16 KiB
   static constexpr int QB = QBOXB * (D / 64);     // 64 KiB
-  static constexpr int PHB = M * 128;             // one P half: 128 rows x 64 KV bf16
-  static constexpr int OFF_Q = NST * STAGEB;
-  static constexpr int OFF_P = OFF_Q + QB;
-  static constexpr int OFF_BAR = OFF_P + 2 * PHB;
+  static constexpr int OFF_V = NSTK * KB;
+  static constexpr int OFF_Q = OFF_V + NSTV * KB;
+  static constexpr int OFF_BAR = OFF_Q + QB;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr int kThreads = 256;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0;            // 2 buffers x 64 columns
+  static constexpr uint32_t P_COL = 128;          // 2 buffers x (32 hi + 32 lo) columns
   static constexpr uint32_t O_COL = 256;          // 256 columns
 };
 static_assert(TcPrefillConfig::SMEM <= 227 * 1024, "shared memory budget");
@@ -113,6 +118,14 @@ struct PrefillTiles {
   }
 };
 
+// 2^x by the hardware's approximate base-2 exponential (relative error about
+// 2^-22, results below 2^-126 flushed to zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Block c -> (sequence b, KV head x, query block qb), heaviest causal blocks first.
 __device__ __forceinline__ void prefill_block(const PrefillParams &p, int32_t c, int32_t &b,
                                               int32_t &x, int32_t &qb) {
@@ -128,27 +141,28 @@ __global__ void __launch_bounds__(TcPrefillConfig::kThreads, 1)
                            const __grid_constant__ CUtensorMap vmap,
                            const __grid_constant__ CUtensorMap qmap, const PrefillParams p) {
   using Cfg = TcPrefillConfig;
-  constexpr int D = Cfg::D, NST = Cfg::NST, TILE = Cfg::TILE;
+  constexpr int D = Cfg::D, NSTK = Cfg::NSTK, NSTV = Cfg::NSTV, TILE = Cfg::TILE;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
-  uint8_t *stages = smem;
+  uint8_t *ks = smem;                // K ring
+  uint8_t *vs = smem + Cfg::OFF_V;   // V ring
   uint8_t *qs = smem + Cfg::OFF_Q;
-  uint8_t *ps = smem + Cfg::OFF_P;  // P_hi, then P_lo
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
-  uint64_t *kfull = bars;          // [NST] K TMA -> QK
-  uint64_t *kempty = bars + 2;     // [NST] QK -> K TMA
-  uint64_t *vfull = bars + 4;      // [NST] V TMA -> P.V (and the softmax, for partial tiles)
-  uint64_t *vempty = bars + 6;     // [NST] P.V -> V TMA
-  uint64_t *sfull = bars + 8;      // [2] QK -> softmax
-  uint64_t *sempty = bars + 10;    // [2] softmax -> QK
-  uint64_t *qfull = bars + 12;     // Q TMA -> QK
-  uint64_t *pfull = bars + 13;     // softmax -> P.V
-  uint64_t *odone = bars + 14;     // P.V -> softmax: a tile's P.V completed (P free, O final)
-  uint64_t *drain = bars + 15;     // [2] QK warp, P.V warp: all their MMAs done
-  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 17);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 18);
+  uint64_t *kfull = bars;          // [NSTK] K TMA -> QK
+  uint64_t *kempty = bars + 3;     // [NSTK] QK -> K TMA
+  uint64_t *vfull = bars + 6;      // [NSTV] V TMA -> P.V (and the softmax, for partial tiles)
+  uint64_t *vempty = bars + 8;     // [NSTV] P.V -> V TMA
+  uint64_t *sfull = bars + 10;     // [2] QK -> softmax
+  uint64_t *sempty = bars + 12;    // [2] softmax -> QK
+  uint64_t *qfull = bars + 14;     // Q TMA -> QK
+  uint64_t *pfull = bars + 15;     // [2] softmax -> P.V, per P buffer
+  uint64_t *odone = bars + 17;     // [2] P.V -> softmax: the P.V of a tile using P buffer
+                                   // i & 1 completed (that buffer free, O up to date)
+  uint64_t *drain = bars + 19;     // [2] QK warp, P.V warp: all their MMAs done
+  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(bars + 21);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 22);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -166,9 +180,11 @@ __global__ void __launch_bounds__(TcPrefillConfig::kThreads, 1)
   const bool bad = L < T || (hi > lo && lo < L - p.capacity);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < NSTK; ++s) {
       mbar_init(&kfull[s], 1);
       mbar_init(&kempty[s], 1);
+    }
+    for (int s = 0; s < NSTV; ++s) {
       mbar_init(&vfull[s], 1);
       mbar_init(&vempty[s], 1);
     }
@@ -177,8 +193,10 @@ __global__ void __launch_bounds__(TcPrefillConfig::kThreads, 1)
       mbar_init(&sempty[s], 4);
     }
     mbar_init(qfull, 1);
-    mbar_init(pfull, 4);
-    mbar_init(odone, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&pfull[s], 4);
+      mbar_init(&odone[s], 1);
+    }
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
     *abort_flag = 0;
@@ -221,13 +239,14 @@ __global__ void __launch_bounds__(TcPrefillConfig::kThreads, 1)
     it.init(lo_t, hi, C);
     int32_t pos0, slot, ntok;
     while (ok && it.next(pos0, slot, ntok)) {
-      const int st = i % NST;
-      if (i >= NST)
-        ok = mbar_wait(is_k ? &kempty[st] : &vempty[st], ((i / NST) - 1) & 1, abort_flag,
+      const int nst = is_k ? NSTK : NSTV;
+      const int st = i % nst;
+      if (i >= static_cast<uint32_t>(nst))
+        ok = mbar_wait(is_k ? &kempty[st] : &vempty[st], ((i / nst) - 1) & 1, abort_flag,
                        p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       if (!(p.test_withhold && is_k && i == 0) && elect_one()) {
-        uint8_t *dst = stages + st * Cfg::STAGEB + (is_k ? 0 : Cfg::KB);
+        uint8_t *dst = (is_k ? ks : vs) + st * Cfg::KB;
         uint64_t *bar = is_k ? &kfull[st] : &vfull[st];
         mbar_arrive_expect_tx(bar, Cfg::KB);
 #pragma unroll
@@ -239,23 +258,24 @@ __global__ void __launch_bounds__(TcPrefillConfig::kThreads, 1)
     }
     // Never leave with copies in flight into shared memory.
     volatile int no_abort = 0;
-    for (uint32_t f = i > NST ? i - NST : 0; f < i; ++f)
+    const uint32_t nst = is_k ? NSTK : NSTV;
+    for (uint32_t f = i > nst ? i - nst : 0; f < i; ++f)
       if (!(p.test_withhold && is_k && f == 0))
-        mbar_wait(is_k ? &kfull[f % NST] : &vfull[f % NST], (f / NST) & 1, &no_abort, p.status);
+        mbar_wait(is_k ? &kfull[f % nst] : &vfull[f % nst], (f / nst) & 1, &no_abort, p.status);
     if (is_k) mbar_wait(qfull, 0, &no_abort, p.status);
   } else if (warp == 1) {
     // --------------------------------------------------------- QK MMA
     const uint32_t idesc = idesc_bf16_f32(128, TILE, false, false);
     const uint64_t qdesc = smem_desc_sw128(smem_u32(qs), 16, 1024);      // Q, K-major
-    const uint64_t kdesc = smem_desc_sw128(smem_u32(stages), 16, 1024);  // K tile, K-major
+    const uint64_t kdesc = smem_desc_sw128(smem_u32(ks), 16, 1024);  // K tile, K-major
     bool ok = mbar_wait(qfull, 0, abort_flag, p.status);
     uint32_t i = 0;
     PrefillTiles it;
     it.init(lo_t, hi, C);
     int32_t pos0, slot, ntok;
     while (__all_sync(0xffffffffu, ok) && it.next(pos0, slot, ntok)) {
-      const int st = i % NST, sb = i & 1;
-      ok = mbar_wait(&kfull[st], (i / NST) & 1, abort_flag, p.status);
+      const int st = i % NSTK, sb = i & 1;
+      ok = mbar_wait(&kfull[st], (i / NSTK) & 1, abort_flag, p.status);
       if (ok && i >= 2) ok = mbar_wait(&sempty[sb], ((i >> 1) - 1) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
@@ -266,7 +286,7 @@ __global__ void __launch_bounds__(TcPrefillConfig::kThreads, 1)
           for (int kk = 0; kk < 4; ++kk)
             tc_mma_bf16(tmem + Cfg::S_COL + sb * TILE,
                         qdesc + ((j * Cfg::QBOXB + kk * 32) >> 4),
-                        kdesc + ((st * Cfg::STAGEB + j * Cfg::BOXB + kk * 32) >> 4), idesc,
+                        kdesc + ((st * Cfg::KB + j * Cfg::BOXB + kk * 32) >> 4), idesc,
                         (j | kk) != 0);
         tc_commit(&sfull[sb]);
         tc_commit(&kempty[st]);
@@ -281,32 +301,33 @@ __global__ void __launch_bounds__(TcPrefillConfig::kThreads, 1)
   } else if (warp == 2) {
     // -------------------------------------------------------- P.V MMA
     const uint32_t idesc = idesc_bf16_f32(128, D, false, true);
-    const uint64_t pdesc = smem_desc_sw128(smem_u32(ps), 16, 1024);  // P, K-major
     // V tile as the MN-major B operand: 64-d chunks Cfg::BOXB apart, 8 KV rows per 1 KiB
-    const uint64_t vdesc = smem_desc_sw128(smem_u32(stages + Cfg::KB), Cfg::BOXB, 1024);
+    const uint64_t vdesc = smem_desc_sw128(smem_u32(vs), Cfg::BOXB, 1024);
     bool ok = true;
     uint32_t i = 0;
     PrefillTiles it;
     it.init(lo_t, hi, C);
     int32_t pos0, slot, ntok;
     while (ok && it.next(pos0, slot, ntok)) {
-      const int st = i % NST;
-      bool w = mbar_wait(pfull, i & 1, abort_flag, p.status);
-      if (w) w = mbar_wait(&vfull[st], (i / NST) & 1, abort_flag, p.status);
+      const int st = i % NSTV;
+      const int pb = i & 1;
+      bool w = mbar_wait(&pfull[pb], (i >> 1) & 1, abort_flag, p.status);
+      if (w) w = mbar_wait(&vfull[st], (i / NSTV) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         break;
       }
       tc_fence_after();
       if (elect_one()) {
+        // A = P from tensor memory: 16 KV tokens are 8 columns of bf16 pairs.
 #pragma unroll
         for (int half = 0; half < 2; ++half)
 #pragma unroll
           for (int kk = 0; kk < TILE / 16; ++kk)
-            tc_mma_bf16(tmem + Cfg::O_COL, pdesc + ((half * Cfg::PHB + kk * 32) >> 4),
-                        vdesc + ((st * Cfg::STAGEB + kk * 2048) >> 4), idesc,
-                        !(i == 0 && half == 0 && kk == 0));
-        tc_commit(odone);
+            tc_mma_bf16_ta(tmem + Cfg::O_COL, tmem + Cfg::P_COL + pb * 64 + half * 32 + kk * 8,
+                           vdesc + ((st * Cfg::KB + kk * 2048) >> 4), idesc,
+                           !(i == 0 && half == 0 && kk == 0));
+        tc_commit(&odone[pb]);
         tc_commit(&vempty[st]);
       }
       __syncwarp();
@@ -326,15 +347,22 @@ __global__ void __launch_bounds__(TcPrefillConfig::kThreads, 1)
     const int tq = r >> 1, h = r & 1;
     const bool row_ok = tq < nq;
     const int32_t prow = P0 + tq;  // the row's position
-    const int32_t rlo = p.window > 0 ? prow + 1 - p.window : INT32_MIN;
     if (bad && t128 == 0) atomicOr(p.status, kStatusSeqlen);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    uint32_t done = 0;  // odone phases consumed
-    auto ensure_pv = [&](uint32_t tt) {  // the P.V of tile tt has completed
-      if (done <= tt) {
-        if (ok && !mbar_wait(odone, done & 1, abort_flag, p.status)) ok = false;
-        ++done;
+    // The P.V of tile tt (and so every earlier one: they complete in order) has
+    // completed.  Each odone barrier's phases are consumed in order, and a
+    // barrier never runs two phases ahead of its waiter (the P.V two tiles on
+    // needs this warp's next P), so the parity waits cannot alias.
+    uint32_t done0 = 0, done1 = 0;  // phases consumed on odone[0], odone[1]
+    auto ensure_pv = [&](uint32_t tt) {
+      const uint32_t ph = tt >> 1;
+      if (tt & 1) {
+        for (; done1 <= ph; ++done1)
+          if (ok && !mbar_wait(&odone[1], done1 & 1, abort_flag, p.status)) ok = false;
+      } else {
+        for (; done0 <= ph; ++done0)
+          if (ok && !mbar_wait(&odone[0], done0 & 1, abort_flag, p.status)) ok = false;
       }
       ok = __all_sync(0xffffffffu, ok);
     };
@@ -342,7 +370,6 @@ __global__ void __launch_bounds__(TcPrefillConfig::kThreads, 1)
     PrefillTiles it;
     it.init(lo_t, hi, C);
     int32_t pos0, slot, ntok;
-    uint8_t *phi = ps + r * 128, *plo = ps + Cfg::PHB + r * 128;
     while (it.next(pos0, slot, ntok)) {
       const int sb = i & 1;
       float s[TILE];
@@ -355,18 +382,31 @@ __global__ void __launch_bounds__(TcPrefillConfig::kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&sempty[sb]);
       }
-      // Column c is position pos0 + c: in the row's range when it is at most
-      // the row's own position and (with a window) at least prow + 1 - w.
-      float mx = -INFINITY;
+      // Scores in log2 units (scale, then the soft-cap if there is one).
+      if (p.post != 0.f) {
 #pragma unroll
-      for (int c = 0; c < TILE; ++c) {
-        const int32_t pos = pos0 + c;
-        const bool valid = ok && row_ok && c < ntok && pos <= prow && pos >= rlo;
-        float v = s[c] * p.qscale;
-        if (p.post != 0.f) v = p.post * tanhf(v);
-        s[c] = valid ? v : -INFINITY;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < TILE; ++c) s[c] = p.post * tanhf(s[c] * p.qscale);
+      } else {
+#pragma unroll
+        for (int c = 0; c < TILE; ++c) s[c] *= p.qscale;
       }
+      // Column c is position pos0 + c: in the row's range when it is at most
+      // the row's own position and (with a window) at least prow + 1 - w, i.e.
+      // c in [c_lo, c_hi).  A tile inside every row's range (all but the
+      // window's first and the diagonal's tiles) needs no mask.
+      const bool inside = ntok == TILE && nq == Cfg::QT && pos0 + TILE - 1 <= P0 &&
+                          (p.window == 0 || pos0 >= P0 + Cfg::QT - p.window);
+      if (!(inside && ok)) {
+        int32_t c_lo = p.window > 0 ? prow + 1 - p.window - pos0 : 0;
+        int32_t c_hi = prow - pos0 + 1 < ntok ? prow - pos0 + 1 : ntok;
+        if (!(ok && row_ok)) c_hi = 0;
+#pragma unroll
+        for (int c = 0; c < TILE; ++c) s[c] = (c >= c_lo && c < c_hi) ? s[c] : -INFINITY;
+      }
+      float mx4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+      for (int c = 4; c < TILE; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       // --- move the reference of a row when a score outgrew it.  The TMEM
       // loads and stores are warp-wide, so a warp with any such row rescales
       // all its rows, by 1 where the reference stays.
@@ -394,30 +434,38 @@ __global__ void __launch_bounds__(TcPrefillConfig::kThreads, 1)
           }
         }
       }
-      // --- weights, as bf16 hi + lo rows of P (K-major, 128-byte swizzle)
-      if (i > 0) ensure_pv(i - 1);  // P is single-buffered: tile i - 1's P.V read it
+      // --- weights: the row's bf16 pairs (column j holds KV tokens 2j, 2j + 1)
+      // and their remainders, into P buffer i & 1 in TMEM.  Both parts are
+      // truncated to bf16 (upper halves of the fp32 bits; the remainder is
+      // exact in fp32 before its own truncation), so the pair keeps a weight to
+      // 2^-14 relative with integer operations only.  A row with no score yet
+      // (reference -inf) has only masked columns here: 2^(-inf) = 0.
+      const float mr = m_ref == -INFINITY ? 0.f : m_ref;
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
+      float wh[TILE / 2], wl[TILE / 2];
 #pragma unroll
-      for (int ch = 0; ch < TILE / 8; ++ch) {
-        uint32_t wh[4], wl[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = s[8 * ch + 2 * e], bb = s[8 * ch + 2 * e + 1];
-          const float pa = (a == -INFINITY) ? 0.f : exp2f(a - m_ref);
-          const float pb = (bb == -INFINITY) ? 0.f : exp2f(bb - m_ref);
-          l += pa + pb;
-          wh[e] = pack_bf16x2(pa, pb);
-          wl[e] = pack_bf16x2(pa - bf16lo(wh[e]), pb - bf16hi(wh[e]));
-        }
-        const uint32_t off = static_cast<uint32_t>((ch ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4 *>(phi + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-        *reinterpret_cast<uint4 *>(plo + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+      for (int j = 0; j < TILE / 2; ++j) {
+        const float pa = ex2_approx(s[2 * j] - mr);
+        const float pb = ex2_approx(s[2 * j + 1] - mr);
+        l4[j & 3] += pa + pb;
+        const uint32_t ua = __float_as_uint(pa), ub = __float_as_uint(pb);
+        const float ra = pa - __uint_as_float(ua & 0xFFFF0000u);
+        const float rb = pb - __uint_as_float(ub & 0xFFFF0000u);
+        wh[j] = __uint_as_float(__byte_perm(ua, ub, 0x7632));  // hi halves: a low, b high
+        wl[j] = __uint_as_float(__byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632));
+      }
+      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      if (i >= 2) ensure_pv(i - 2);  // the P.V of tile i - 2 read this P buffer
+      if (ok) {
+        tmem_st32_wait(tmem + lane_base + Cfg::P_COL + (i & 1) * 64, wh);
+        tmem_st32_wait(tmem + lane_base + Cfg::P_COL + (i & 1) * 64 + 32, wl);
       }
       if (ok && ntok < TILE) {
         // V rows past the tile's end hold other slots (possibly NaN): clear them.
         ok = __all_sync(0xffffffffu,
-                        mbar_wait(&vfull[i % NST], (i / NST) & 1, abort_flag, p.status));
+                        mbar_wait(&vfull[i % NSTV], (i / NSTV) & 1, abort_flag, p.status));
         if (ok) {
-          uint8_t *vt = stages + (i % NST) * Cfg::STAGEB + Cfg::KB;
+          uint8_t *vt = vs + (i % NSTV) * Cfg::KB;
           const int per_box = (TILE - ntok) * 8;
 #pragma unroll 1
           for (int box = 0; box < D / 64; ++box)
@@ -426,10 +474,10 @@ __global__ void __launch_bounds__(TcPrefillConfig::kThreads, 1)
                                          (e & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      fence_proxy_async_smem();
+      fence_proxy_async_smem();  // the cleared V rows, for the tensor core
       tc_fence_before();
       __syncwarp();
-      if (ok && lane == 0) mbar_arrive(pfull);
+      if (ok && lane == 0) mbar_arrive(&pfull[i & 1]);
       ++i;
     }
     // --- the row's output: O / l, and its LSE.  The whole warp loads (the

@@ -111,3 +111,25 @@ def test_peak_falls_back_without_a_measured_record(tmp_path, monkeypatch):
     assert bench.measured_peak_gbs() == (bench.FALLBACK_HBM_GBS, "fallback")
     (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6450.0}))
     assert bench.measured_peak_gbs() == (6450.0, "measured")
+
+
+def test_multi_token_accounting_against_brute_force():
+    """The verify / prefill byte and flop accounting: pairs of (token, attended
+    position) and the union of the tokens' ranges, counted one by one."""
+    import workloads
+    from decode_attention_09_b200 import accounting
+    for spec in (workloads.sliding_spec(4096, 16), workloads.global_spec(4096)):
+        for L, T in ((40, 8), (10, 10), (100, 1), (3, 3), (70, 33)):
+            pairs, union = 0, set()
+            for t in range(T):
+                p = L - T + t
+                lo = max(0, p + 1 - spec.window) if spec.window > 0 else 0
+                rng = range(lo, p + 1)
+                pairs += len(rng)
+                union.update(rng)
+            assert accounting.multi_attended_pairs(spec, L, T) == pairs
+            assert accounting.union_positions(spec, L, T) == len(union)
+            assert accounting.layer_prefill_flops(spec, [L], T) == \
+                pairs * 4 * spec.head_dim * spec.n_q_heads
+            assert accounting.layer_multi_kv_bytes(spec, [L, L], T) == \
+                2 * len(union) * accounting.kv_bytes_per_position(spec)
