@@ -514,7 +514,8 @@ def run_ours(args, world, rank, local):
     step_spread = spread(per_replay, ncopy)
     ms_sl = time_graph(g_sl, stream, replays, 3) if g_sl else None
     ms_gl = time_graph(g_gl, stream, replays, 3) if g_gl else None
-    ceiling = read_ceiling(device, stream) if rank == 0 else None
+    want = lambda name: args.sections == "all" or name in args.sections.split(",")
+    ceiling = read_ceiling(device, stream) if rank == 0 and want("ceiling") else None
     for ly in stack.layers:  # no device-side error latched during any of it
         st = binding.check_device_status(ly["ws"], stream)
         if st != binding.GDATTN_OK:
@@ -640,39 +641,41 @@ def run_ours(args, world, rank, local):
     # ---- the same step with the current token's K/V append fused in
     # (gdattn_decode_append): each layer's new rows are written into their ring
     # slots by the decode kernels.  Last, since it writes into the caches.
-    gen = torch.Generator(device="cpu").manual_seed(7 + rank)
-    new_rows = []
-    for ly in stack.layers:
-        sp = ly["spec"]
-        shape = (w.batch, sp.n_kv_heads, sp.head_dim)
-        kn = torch.randn(shape, generator=gen).to(torch.bfloat16).to(device)
-        vn = None if sp.kv_shared else torch.randn(shape, generator=gen).to(torch.bfloat16).to(device)
-        new_rows.append((kn, vn))
+    ms_app = None
+    if want("append"):
+        gen = torch.Generator(device="cpu").manual_seed(7 + rank)
+        new_rows = []
+        for ly in stack.layers:
+            sp = ly["spec"]
+            shape = (w.batch, sp.n_kv_heads, sp.head_dim)
+            kn = torch.randn(shape, generator=gen).to(torch.bfloat16).to(device)
+            vn = None if sp.kv_shared else torch.randn(shape, generator=gen).to(torch.bfloat16).to(device)
+            new_rows.append((kn, vn))
 
-    def append_step():
-        for ly, (kn, vn) in zip(stack.layers, new_rows):
-            binding.decode_append(ly["inp"].q, kn, vn, ly["inp"].k, ly["inp"].v, ly["inp"].seqlens,
-                                  ly["desc"], stack.max_seqlen, out=ly["out"], lse=ly["lse"],
-                                  workspace=ly["ws"], stream=stream)
+        def append_step():
+            for ly, (kn, vn) in zip(stack.layers, new_rows):
+                binding.decode_append(ly["inp"].q, kn, vn, ly["inp"].k, ly["inp"].v, ly["inp"].seqlens,
+                                      ly["desc"], stack.max_seqlen, out=ly["out"], lse=ly["lse"],
+                                      workspace=ly["ws"], stream=stream)
 
-    g_app = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        append_step()
-        stream.synchronize()
-        with torch.cuda.graph(g_app, stream=stream):
+        g_app = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
             append_step()
-    barrier()
-    ms_app = max_over_ranks(time_graph(g_app, stream, replays, args.warmup) / ncopy, world)
-    for ly in stack.layers:
-        st = binding.check_device_status(ly["ws"], stream)
-        if st != binding.GDATTN_OK:
-            raise binding.GdattnError(st, "device status after the append step")
+            stream.synchronize()
+            with torch.cuda.graph(g_app, stream=stream):
+                append_step()
+        barrier()
+        ms_app = max_over_ranks(time_graph(g_app, stream, replays, args.warmup) / ncopy, world)
+        for ly in stack.layers:
+            st = binding.check_device_status(ly["ws"], stream)
+            if st != binding.GDATTN_OK:
+                raise binding.GdattnError(st, "device status after the append step")
 
     # ---- fp8 KV cache (gdattn_decode_fp8) on the sliding layers: the same
     # geometry and lengths with e4m3 codes and per-row scales; the global layers
     # (no fp8 kernel) stay bf16 in the mixed step.
     fp8_layers = {}
-    for i in sliding_idx:
+    for i in (sliding_idx if want("fp8") else []):
         sp = stack.layers[i]["spec"]
         inp8 = workloads.fp8_layer_inputs(sp, w.batch, w.seqlens(),
                                           w.seed * 1000 + 500 + i + rank_seed_offset(rank),
@@ -715,7 +718,7 @@ def run_ours(args, world, rank, local):
     # ---- multi-query decode (gdattn_decode_multi): a 4-token verify step over the
     # global layers (whole-context caches, so every token's range is resident)
     t_multi, ms_multi = 4, None
-    if global_idx:
+    if global_idx and want("multi"):
         gen_mq = torch.Generator(device="cpu").manual_seed(11 + rank)
         mq = {}
         for i in global_idx:
@@ -759,7 +762,7 @@ def run_ours(args, world, rank, local):
     # in turn (together over 4x the L2 size).
     multi_sl = {}
     n_multi_sl = 8
-    if sliding_idx:
+    if sliding_idx and want("multi"):
         sp0 = stack.layers[sliding_idx[0]]["spec"]
         spec_m = dataclasses.replace(sp0, capacity=sp0.window + 7)
         seqlens_m = w.seqlens()
@@ -829,7 +832,7 @@ def run_ours(args, world, rank, local):
     # geometry: one 8192-token prompt per layer (a cache of 8192 slots, L = T),
     # 4 layers of their own replayed in turn (1 GiB of q, K, V and out).
     prefill = None
-    if sliding_idx:
+    if sliding_idx and want("prefill"):
         sp0 = stack.layers[sliding_idx[0]]["spec"]
         t_pf, n_pf = 8192, 4
         spec_p = dataclasses.replace(sp0, capacity=t_pf)
@@ -995,7 +998,8 @@ def run_ours(args, world, rank, local):
                        "CUDA graph and replayed",
                 "eager_value": job_gbs(kv_step, ms_e2e_eager, world),
                 "eager_ms_per_step": ms_e2e_eager},
-        "append": {"value": job_gbs(kv_step, ms_app, world), "unit": "GB/s",
+        "append": None if ms_app is None else {"value": job_gbs(kv_step, ms_app, world),
+                   "unit": "GB/s",
                    "us_per_step": ms_app * 1e3,
                    "how": "the same 48 layers through gdattn_decode_append: each layer's "
                           "current-token K/V rows written into their ring slots by the decode "
@@ -1042,6 +1046,11 @@ def main():
     ap.add_argument("--workload", default="gemma4_12b_stack_b8_l8192",
                     choices=sorted(workloads.ALL_WORKLOADS))
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--sections", default="all",
+                    help="optional measurements to run beside the timed step, comma "
+                         "separated: ceiling, append, fp8, multi, prefill; 'all' (default) "
+                         "or 'none' (the step, its layer-type split and e2e only, as for "
+                         "profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

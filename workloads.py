@@ -138,8 +138,18 @@ def long_context_b4() -> Workload:
                     seqlen=131072, heavy_row_frac=0.01, heavy_row_scale=8.0)
 
 
+def gemma4_12b_two_layers_b8_l8192() -> Workload:
+    """Layers 0 (sliding) and 5 (global) of the 12B stack at batch 8, context 8192:
+    the headline's per-layer shapes and launch configurations on a few hundred MB
+    of device memory, for profiler captures."""
+    stack = gemma4_12b_stack(1024, 8192)
+    return Workload("gemma4_12b_two_layers_b8_l8192", 8, [stack[0], stack[5]], seed=3,
+                    seqlen=8192)
+
+
 ALL_WORKLOADS = {w().name: w for w in (single_sliding, single_global, gemma4_12b_b8_l8192,
-                                       ragged_b64, long_context_b4)}
+                                       ragged_b64, long_context_b4,
+                                       gemma4_12b_two_layers_b8_l8192)}
 
 
 # --------------------------------------------------------------------------
