@@ -4,8 +4,8 @@ runs out (after about 2 s at the maximum SM clock).  The kernel must drain its
 copies and tensor-core work, free tensor memory and return; the call reports
 GDATTN_ERR_DEVICE_TIMEOUT, the context stays usable, and the same workspace,
 re-initialised, then gives the oracle's result.  Every kernel path is covered:
-the tcgen05 pair kernel (bf16 and fp8 caches), the 16-head kernel, and the
-CUDA-core kernel."""
+the tcgen05 pair kernel (bf16 and fp8 caches), the 16-head kernel, the
+CUDA-core kernel, and the multi-token and prefill kernels."""
 import pytest
 import torch
 
@@ -65,3 +65,43 @@ def test_expired_wait_fp8():
                                            f8.seqlens, s.window, s.softcap, s.scale)
     torch.cuda.synchronize()
     compare(out, lse, o_ref, l_ref, ulp_floor=True, what="fp8 after a timeout")
+
+
+# Multi-token steps on the pair geometry: (T, seqlens, capacity, window, flags):
+# the single-pass kernel with units cut into parts (counted merge) and with
+# flattened chunks, and flash prefill.
+MULTI_CASES = {
+    "verify_t4_even": (4, [600, 600], 600, 512, binding.GDATTN_FLAG_EVEN_UNITS),
+    "verify_t2_chunks": (2, [700, 90], 300, 256, 0),
+    "prefill_t64": (64, [200, 64], 200, 128, 0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MULTI_CASES))
+def test_expired_wait_multi_token(name):
+    require_gpu()
+    T, sl, C, w, flags = MULTI_CASES[name]
+    B = len(sl)
+    inp = workloads.random_case(970 + sorted(MULTI_CASES).index(name), B, 16, 8, 256, C, sl,
+                                window=w)
+    g = torch.Generator().manual_seed(980 + sorted(MULTI_CASES).index(name))
+    q = torch.randn((T, B, 16, 256), generator=g).to(torch.bfloat16)
+    s = inp.spec
+    dev = "cuda"
+    desc = binding.desc_from_spec(s, capacity=C, flags=flags | WITHHOLD)
+    ws = torch.empty(binding.multi_workspace_size(B, T, max(sl), desc), dtype=torch.uint8,
+                     device=dev)
+    binding.workspace_init(ws)
+    args = (q.to(dev), inp.k.to(dev), inp.v.to(dev), inp.seqlens.to(dev))
+    binding.decode_multi(*args, desc, max(sl), workspace=ws)
+    assert binding.check_device_status(ws) == binding.GDATTN_ERR_DEVICE_TIMEOUT
+    binding.workspace_init(ws)
+    out, lse = binding.decode_multi(*args, binding.desc_from_spec(s, capacity=C, flags=flags),
+                                    max(sl), workspace=ws)
+    assert binding.check_device_status(ws) == binding.GDATTN_OK
+    o_ref, l_ref = oracle.get().decode_multi(q, inp.k, inp.v, inp.seqlens, s.window, s.softcap,
+                                             s.scale)
+    torch.cuda.synchronize()
+    for t in range(T):
+        compare(out[t], lse[t], o_ref[t], l_ref[t], ulp_floor=True,
+                what=f"{name} token {t} after a timeout")
