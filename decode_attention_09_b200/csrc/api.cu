@@ -20,6 +20,7 @@
 #include "tc_pair_fp8_decode.cuh"
 #include "tc_pair_multi_decode.cuh"
 #include "tc_pair_prefill.cuh"
+#include "tc_global_prefill.cuh"
 
 using namespace gdattn;
 
@@ -442,16 +443,17 @@ bool encode_q_rows_map(EncodeTiledFn enc, CUtensorMap *map, const void *q, int32
 }
 
 // q [T][rows][D] bf16 (rows = B * Hq) as a 3-D tensor map read in
-// {64 d, 2 rows, box_tokens tokens} boxes with 128-byte swizzle: the query rows
-// of a pair unit (2 heads x box_tokens tokens) land as consecutive 128-byte
-// rows, token-major; tokens past T read as zeros.
+// {64 d, box_heads rows, box_tokens tokens} boxes with 128-byte swizzle: the
+// query rows of a unit (box_heads heads x box_tokens tokens) land as consecutive
+// 128-byte rows, token-major; tokens past T read as zeros.
 bool encode_q_tokens_map(EncodeTiledFn enc, CUtensorMap *map, const void *q, int32_t D,
-                         int64_t rows, int32_t T, int32_t box_tokens) {
+                         int64_t rows, int32_t T, int32_t box_tokens, int32_t box_heads = 2) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(T)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
                                  static_cast<cuuint64_t>(rows) * D * 2};
-  const cuuint32_t box[3] = {64, 2, static_cast<cuuint32_t>(box_tokens)};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_heads),
+                             static_cast<cuuint32_t>(box_tokens)};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -730,11 +732,32 @@ gdattn_layer_desc union_window_desc(const gdattn_layer_desc *d, int32_t T) {
   return u;
 }
 
-// Multi-token steps of more than 8 tokens on the pair geometry (prompt chunks)
-// run as flash prefill (tc_pair_prefill.cuh), up to this many tokens.
+// Multi-token steps of more than 8 tokens (prompt chunks) run as flash prefill
+// on the pair geometry (tc_pair_prefill.cuh) and on the global geometry with
+// K = V (tc_global_prefill.cuh), up to this many tokens.
 constexpr int32_t kMaxPrefillTokens = 1 << 20;
+bool prefill_geometry(const gdattn_layer_desc *d) {
+  const PathKind k = choose_path(d);
+  return k == PathKind::kTcPair || (k == PathKind::kTc && d->kv_shared == 1);
+}
 bool multi_prefill(const gdattn_layer_desc *d, int32_t T) {
-  return choose_path(d) == PathKind::kTcPair && T > TcPairMultiConfig::TMAX;
+  return prefill_geometry(d) && T > TcPairMultiConfig::TMAX;
+}
+
+using GlobalPrefillFn = void (*)(const CUtensorMap, const CUtensorMap, const PrefillParams);
+int query_global_prefill(const void *fn, int threads, int smem) {
+  return blocks_per_sm(reinterpret_cast<GlobalPrefillFn>(const_cast<void *>(fn)), threads, smem);
+}
+
+// Query tokens per prefill block, and CTAs per block (the global kernel splits
+// the head dimension over two).
+int32_t prefill_block_tokens(const gdattn_layer_desc *d) {
+  return choose_path(d) == PathKind::kTcPair
+             ? TcPrefillConfig::QT
+             : TcGlobalPrefillConfig::M / (d->n_q_heads / d->n_kv_heads);
+}
+int32_t prefill_ctas_per_block(const gdattn_layer_desc *d) {
+  return choose_path(d) == PathKind::kTcPair ? 1 : 2;
 }
 
 // Checks the prefill launch for this geometry (and sets the kernel's shared
@@ -744,12 +767,24 @@ gdattn_status plan_prefill(int32_t batch, int32_t T, const gdattn_layer_desc *d,
   gdattn_status st = check_desc(d);
   if (st != GDATTN_OK) return st;
   if (batch <= 0 || T < 1 || T > kMaxPrefillTokens) return GDATTN_ERR_INVALID_ARG;
-  const int64_t nblocks = (T + TcPrefillConfig::QT - 1) / TcPrefillConfig::QT;
-  if (static_cast<int64_t>(batch) * d->n_kv_heads * nblocks > INT32_MAX)
+  if (!prefill_geometry(d)) return GDATTN_ERR_UNSUPPORTED;
+  const int32_t qt = prefill_block_tokens(d);
+  const int64_t nblocks = (T + qt - 1) / qt;
+  if (static_cast<int64_t>(batch) * d->n_kv_heads * nblocks * prefill_ctas_per_block(d) >
+      INT32_MAX)
     return GDATTN_ERR_UNSUPPORTED;
-  if (cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_prefill_kernel),
-                           TcPrefillConfig::kThreads, TcPrefillConfig::SMEM, query_prefill) <= 0)
-    return GDATTN_ERR_CUDA;
+  int per_sm = 0;
+  if (choose_path(d) == PathKind::kTcPair) {
+    per_sm = cached_blocks_per_sm(reinterpret_cast<const void *>(tc_pair_prefill_kernel),
+                                  TcPrefillConfig::kThreads, TcPrefillConfig::SMEM, query_prefill);
+  } else {
+    const void *fn = d->n_q_heads / d->n_kv_heads == 8
+                         ? reinterpret_cast<const void *>(tc_global_prefill_kernel<8>)
+                         : reinterpret_cast<const void *>(tc_global_prefill_kernel<16>);
+    per_sm = cached_blocks_per_sm(fn, TcGlobalPrefillConfig::kThreads, TcGlobalPrefillConfig::SMEM,
+                                  query_global_prefill);
+  }
+  if (per_sm <= 0) return GDATTN_ERR_CUDA;
   *ws_bytes = kHeaderBytes;
   return GDATTN_OK;
 }
@@ -764,15 +799,18 @@ gdattn_status enqueue_prefill(const void *q, const void *k_cache, const void *v_
                               ? desc->cache_batch_stride
                               : static_cast<int64_t>(desc->cache_capacity) * Hkv * D;
   const float log2e = 1.4426950408889634f;
+  const bool pair = choose_path(desc) == PathKind::kTcPair;
+  const int32_t GU = desc->n_q_heads / Hkv;
+  const int32_t qt = prefill_block_tokens(desc);
   EncodeTiledFn enc = encode_tiled();
   if (enc == nullptr) return GDATTN_ERR_CUDA;
   CUtensorMap kmap, vmap, qmap;
   if (!encode_cache_map(enc, &kmap, k_cache, D, Hkv, desc->cache_capacity, batch, bstride,
                         TcPrefillConfig::TILE) ||
-      !encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, batch, bstride,
-                        TcPrefillConfig::TILE) ||
+      (pair && !encode_cache_map(enc, &vmap, v_cache, D, Hkv, desc->cache_capacity, batch,
+                                 bstride, TcPrefillConfig::TILE)) ||
       !encode_q_tokens_map(enc, &qmap, q, D, static_cast<int64_t>(batch) * desc->n_q_heads, T,
-                           TcPrefillConfig::QT))
+                           qt, pair ? 2 : GU))
     return GDATTN_ERR_CUDA;
   PrefillParams pp;
   pp.seqlens = seqlens;
@@ -783,19 +821,27 @@ gdattn_status enqueue_prefill(const void *q, const void *k_cache, const void *v_
   pp.n_q_heads = desc->n_q_heads;
   pp.n_kv_heads = Hkv;
   pp.tokens = T;
-  pp.nblocks = (T + TcPrefillConfig::QT - 1) / TcPrefillConfig::QT;
+  pp.nblocks = (T + qt - 1) / qt;
   pp.window = desc->window;
   pp.capacity = desc->cache_capacity;
   pp.qscale = desc->softcap > 0.f ? desc->scale / desc->softcap : desc->scale * log2e;
   pp.post = desc->softcap > 0.f ? desc->softcap * log2e : 0.f;
   pp.test_withhold = (desc->flags & GDATTN_FLAG_TEST_WITHHOLD_KV) ? 1 : 0;
-  const unsigned grid = static_cast<unsigned>(static_cast<int64_t>(batch) * Hkv * pp.nblocks);
+  const unsigned grid = static_cast<unsigned>(static_cast<int64_t>(batch) * Hkv * pp.nblocks *
+                                              prefill_ctas_per_block(desc));
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = launch_config(dim3(grid), TcPrefillConfig::kThreads,
-                                         TcPrefillConfig::SMEM, stream, attr);
-  return cudaLaunchKernelEx(&cfg, tc_pair_prefill_kernel, kmap, vmap, qmap, pp) == cudaSuccess
-             ? GDATTN_OK
-             : GDATTN_ERR_CUDA;
+  cudaError_t e;
+  if (pair) {
+    cudaLaunchConfig_t cfg = launch_config(dim3(grid), TcPrefillConfig::kThreads,
+                                           TcPrefillConfig::SMEM, stream, attr);
+    e = cudaLaunchKernelEx(&cfg, tc_pair_prefill_kernel, kmap, vmap, qmap, pp);
+  } else {
+    cudaLaunchConfig_t cfg = launch_config(dim3(grid), TcGlobalPrefillConfig::kThreads,
+                                           TcGlobalPrefillConfig::SMEM, stream, attr);
+    e = GU == 8 ? cudaLaunchKernelEx(&cfg, tc_global_prefill_kernel<8>, kmap, qmap, pp)
+                : cudaLaunchKernelEx(&cfg, tc_global_prefill_kernel<16>, kmap, qmap, pp);
+  }
+  return e == cudaSuccess ? GDATTN_OK : GDATTN_ERR_CUDA;
 }
 
 // Enqueues the single-pass multi-token kernel (it merges split units itself);
@@ -1079,8 +1125,7 @@ gdattn_status gdattn_decode_multi(const void *q, const void *k_cache, const void
   gdattn_status st = check_decode_args(q, k_cache, v_cache, seqlens, batch, max_seqlen, desc,
                                        out, lse);
   if (st != GDATTN_OK) return st;
-  const int32_t max_tokens = choose_path(desc) == PathKind::kTcPair ? kMaxPrefillTokens
-                                                                    : kMaxMultiTokens;
+  const int32_t max_tokens = prefill_geometry(desc) ? kMaxPrefillTokens : kMaxMultiTokens;
   if (n_tokens < 1 || n_tokens > max_tokens || n_tokens > max_seqlen)
     return GDATTN_ERR_INVALID_ARG;
   // A ring holds positions [L - C, L): the first token's window must still be in it.

@@ -276,8 +276,9 @@ gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *
  *
  *  q         bf16 [T, batch, Hq, D] (token-major), device, read only
  *  out       bf16 [T, batch, Hq, D];  lse: fp32 [T, batch, Hq] or NULL
- *  n_tokens  T: 1 <= T <= 64, or up to 2^20 on the pair geometry (a prompt
- *            chunk);  seqlens: L_b >= T, the length with all T tokens
+ *  n_tokens  T: 1 <= T <= 64, or up to 2^20 on the pair geometry and on the
+ *            global geometry with K = V (a prompt chunk);  seqlens: L_b >= T,
+ *            the length with all T tokens
  *  workspace at least gdattn_multi_workspace_size bytes (zeroed once by
  *            gdattn_workspace_init)
  *  other arguments, geometries and device-side errors as gdattn_decode.
@@ -294,7 +295,10 @@ gdattn_status gdattn_decode_fp8(const void *q, const void *k_codes, const void *
  * same geometry the step is flash prefill ("Gemma support" pull request,
  * Performance: flash prefill for head_dim 256): one CTA per 64 query tokens of a
  * (sequence, KV head), 128 query rows per tensor-core tile, streaming that
- * block's KV range once; its workspace is the fixed header alone.  Otherwise
+ * block's KV range once; its workspace is the fixed header alone.  The global
+ * geometry with K = V (8 or 16 query heads per KV head, head_dim 512) runs T > 8
+ * as flash prefill too, in blocks of 64 query rows (64 / G tokens), each on two
+ * CTAs that split the output's head dimension.  Otherwise
  * one small kernel writes the T per-token lengths into the workspace, then one
  * decode launch runs over T x batch query sequences (token-major) in which query
  * sequence t * batch + b reads cache sequence b; the T tokens of a sequence then

@@ -32,6 +32,11 @@ CASES = {
     "prefill_t200_ring_cap": (200, 2, 16, 8, 256, 1223, [3000, 1223], 1024, 50.0, False, 0),
     "prefill_t130_small_w": (130, 2, 16, 8, 256, 300, [300, 131], 100, 0.0, False, 0),
     "prefill_t513_global": (513, 1, 4, 2, 256, 700, [600], 0, 0.0, False, 0),
+    # flash prefill on the global geometry (K = V, head_dim 512): 64-row blocks of
+    # 64 / G tokens, each on two CTAs (one per half of the head dimension)
+    "gprefill_t64_g16": (64, 2, 16, 1, 512, 300, [300, 64], 0, 0.0, True, 0),
+    "gprefill_t100_g8_cap": (100, 1, 16, 2, 512, 400, [350], 0, 30.0, True, 0),
+    "gprefill_t40_ring": (40, 2, 16, 1, 512, 200, [900, 150], 128, 0.0, True, 0),
     # tcgen05 16-head kernel (global, K = V)
     "tc16_t3": (3, 2, 16, 1, 512, 400, [400, 77], 0, 0.0, True, 0),
     "tc16_even_t2": (2, 2, 32, 2, 512, 300, [300, 300], 0, 30.0, True, 1),
@@ -85,7 +90,8 @@ def test_multi_matches_oracle(name):
 
 
 @pytest.mark.parametrize("name,short_len", [("core_g4_t3", 2), ("pair_no_wrap_t7", 5),
-                                            ("prefill_t130_small_w", 70)])
+                                            ("prefill_t130_small_w", 70),
+                                            ("gprefill_t64_g16", 20)])
 def test_multi_tokens_before_the_context_are_reported(name, short_len):
     """A sequence shorter than T: its tokens at positions below 0 attend nothing;
     the device reports it, gives them zero output and LSE -inf, and its other
@@ -108,12 +114,13 @@ def test_multi_tokens_before_the_context_are_reported(name, short_len):
     missing = T - short_len
     for t in range(missing):
         assert torch.all(out[t, 1] == 0) and torch.all(torch.isneginf(lse[t, 1]))
-    o_ref, l_ref = oracle.get().decode_multi(q[missing:, 1:2], inp.k[1:2], inp.v[1:2],
+    vs = (lambda i: inp.v[i:i + 1]) if inp.v is not None else (lambda i: None)
+    o_ref, l_ref = oracle.get().decode_multi(q[missing:, 1:2], inp.k[1:2], vs(1),
                                              inp.seqlens[1:2], s.window, s.softcap, s.scale)
     for t in range(missing, T):
         compare(out[t, 1:2], lse[t, 1:2], o_ref[t - missing], l_ref[t - missing], ulp_floor=True,
                 what=f"token {t} of the short sequence")
-    o_ref, l_ref = oracle.get().decode_multi(q[:, 0:1], inp.k[0:1], inp.v[0:1],
+    o_ref, l_ref = oracle.get().decode_multi(q[:, 0:1], inp.k[0:1], vs(0),
                                              inp.seqlens[0:1], s.window, s.softcap, s.scale)
     for t in range(T):
         compare(out[t, 0:1], lse[t, 0:1], o_ref[t], l_ref[t], ulp_floor=True,
