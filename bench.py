@@ -828,21 +828,22 @@ def run_ours(args, world, rank, local):
             del g_msl, bufs
         del caches_m
 
-    # ---- flash prefill (gdattn_decode_multi with a prompt chunk) on the sliding
-    # geometry: one 8192-token prompt per layer (a cache of 8192 slots, L = T),
-    # 4 layers of their own replayed in turn (1 GiB of q, K, V and out).
+    # ---- flash prefill (gdattn_decode_multi with a prompt chunk): one 8192-token
+    # prompt per layer (a cache of 8192 slots, L = T), on the stack's sliding and
+    # global layer shapes, layers of their own replayed in turn (q, K, V and out
+    # over 512 MiB per kind).
     prefill = None
-    if sliding_idx and want("prefill"):
-        sp0 = stack.layers[sliding_idx[0]]["spec"]
-        t_pf, n_pf = 8192, 4
+
+    def time_prefill(sp0, n_pf, seed0, replays_pf):
+        t_pf = 8192
         spec_p = dataclasses.replace(sp0, capacity=t_pf)
         seqlens_p = torch.full((1,), t_pf, dtype=torch.int32)
         desc_p = binding.desc_from_spec(spec_p)
-        gen_p = torch.Generator(device="cpu").manual_seed(17 + rank)
+        gen_p = torch.Generator(device="cpu").manual_seed(seed0 + rank)
         bufs_p = []
         for j in range(n_pf):
             inp = workloads.layer_inputs(spec_p, 1, seqlens_p,
-                                         w.seed * 1000 + 950 + j + rank_seed_offset(rank),
+                                         w.seed * 1000 + seed0 + j + rank_seed_offset(rank),
                                          device=device)
             qp = torch.randn((t_pf, 1, spec_p.n_q_heads, spec_p.head_dim),
                              generator=gen_p).to(torch.bfloat16).to(device)
@@ -864,7 +865,7 @@ def run_ours(args, world, rank, local):
             with torch.cuda.graph(g_pf, stream=stream):
                 prefill_step()
         barrier()
-        ms_pf = max_over_ranks(time_graph(g_pf, stream, max(3, replays // 20), 3), world)
+        ms_pf = max_over_ranks(time_graph(g_pf, stream, replays_pf, 3), world)
         for inp, qp, wsp, op, lp in bufs_p:
             st = binding.check_device_status(wsp, stream)
             if st != binding.GDATTN_OK:
@@ -872,17 +873,32 @@ def run_ours(args, world, rank, local):
         flops = n_pf * accounting.layer_prefill_flops(spec_p, seqlens_p.tolist(), t_pf)
         tf_peak, tf_kind = measured_peak_tflops()
         tflops = flops / (ms_pf * 1e-3) / 1e12
-        prefill = {
-            "kernel": "tc_pair_prefill_kernel (tcgen05: S = Q K^T with M = 128 query rows, "
-                      "P.V with bf16 weights plus remainders)",
-            "tokens": t_pf, "us_per_layer": ms_pf / n_pf * 1e3,
-            "tflops": tflops, "peak_tflops": tf_peak, "peak_kind": tf_kind,
-            "frac": tflops / tf_peak, "bound": "tensor",
-            "how": "one 8192-token prompt (window 1024, 16 query / 8 KV heads, head_dim 256) "
-                   "per layer through gdattn_decode_multi, 4 layers replayed in turn in a CUDA "
-                   "graph; useful flops = 4 x head_dim per (query head, token, attended "
-                   "position), so the weight split's second P.V half counts as overhead"}
         del g_pf, bufs_p
+        return {"tokens": t_pf, "us_per_layer": ms_pf / n_pf * 1e3, "tflops": tflops,
+                "peak_tflops": tf_peak, "peak_kind": tf_kind, "frac": tflops / tf_peak,
+                "bound": "tensor"}
+
+    if want("prefill") and (sliding_idx or global_idx):
+        prefill = {"how": "one 8192-token prompt per layer through gdattn_decode_multi, "
+                          "layers replayed in turn in a CUDA graph; useful flops = 4 x "
+                          "head_dim per (query head, token, attended position), so the weight "
+                          "split's second P.V half (and, on the global layers, the scores "
+                          "computed by both CTAs of a block) count as overhead"}
+        if sliding_idx:
+            prefill["sliding"] = time_prefill(stack.layers[sliding_idx[0]]["spec"], 4, 950,
+                                              max(3, replays // 20))
+            prefill["sliding"]["traffic"] = traffic_for("prefill_sliding")
+            prefill["sliding"]["kernel"] = (
+                "tc_pair_prefill_kernel (window 1024, 16 query / 8 KV heads, head_dim 256; "
+                "M = 128 query rows, P in tensor memory)")
+        if global_idx:
+            prefill["global"] = time_prefill(stack.layers[global_idx[0]]["spec"], 2, 960,
+                                             max(3, replays // 200))
+            prefill["global"]["traffic"] = traffic_for("prefill_global")
+            prefill["global"]["kernel"] = (
+                "tc_global_prefill_kernel<16> (causal over the whole prompt, 16 query heads, "
+                "one K = V head, head_dim 512; M = 64 query rows per CTA pair, each CTA half "
+                "of the output dims)")
 
     # ---- CPU baseline: the oracle over the whole step (rank 0, N = 1 only)
     cpu = None
@@ -1020,7 +1036,8 @@ def run_ours(args, world, rank, local):
             **{f"t{t_m}": {"tokens": t_m, "us_per_layer": ms_m / n_multi_sl * 1e3,
                            "vs_single_token": ms_m / multi_sl[1][0],
                            "kv_gbs": b_m / (ms_m * 1e-3) / 1e9,
-                           "kv_frac": b_m / (ms_m * 1e-3) / 1e9 / peak}
+                           "kv_frac": b_m / (ms_m * 1e-3) / 1e9 / peak,
+                           "traffic": traffic_for("multi_t4_sliding") if t_m == 4 else None}
                for t_m, (ms_m, b_m) in sorted(multi_sl.items())},
             "how": "8 sliding layers (rings of window + 7 slots, the stack's batch and "
                    "lengths) through gdattn_decode_multi with 4 and 8 query tokens per "
