@@ -275,3 +275,27 @@ def test_decode_multi_host_checks(lib):
     assert multi(d, T=2, q=None) == binding.GDATTN_ERR_INVALID_ARG
     assert multi(d, T=2, q=A + 8) == binding.GDATTN_ERR_MISALIGNED
     assert binding.multi_workspace_size(1, 0, 8, good_desc()) == 0
+
+
+def test_prompt_chunks_allowed_where_flash_prefill_runs(lib):
+    """Token limits by geometry: up to 2^20 tokens on the pair geometry and on the
+    global geometry with K = V (flash prefill), 64 elsewhere.  A chunk that passes
+    the host checks reaches the workspace check (here: no workspace)."""
+    def multi(desc, T, ws=None):
+        return binding.decode_multi_raw(A, A, None if desc.kv_shared else A, A, 1, T, 1 << 21,
+                                        desc, A, A, ws, 1 << 24, None)
+    pair = good_desc(window=1024, cache_capacity=1 << 21)  # a cache that never wraps
+    assert multi(pair, 65) == binding.GDATTN_ERR_WORKSPACE
+    assert multi(pair, 1 << 20) == binding.GDATTN_ERR_WORKSPACE
+    assert multi(pair, (1 << 20) + 1) == binding.GDATTN_ERR_INVALID_ARG
+    glob = good_desc(n_q_heads=16, n_kv_heads=1, head_dim=512, window=0, kv_shared=True,
+                     scale=512 ** -0.5, cache_capacity=1 << 21)
+    assert multi(glob, 100) == binding.GDATTN_ERR_WORKSPACE
+    sepv = good_desc(n_q_heads=16, n_kv_heads=1, head_dim=512, window=0, kv_shared=False,
+                     scale=512 ** -0.5, cache_capacity=1 << 21)
+    assert multi(sepv, 64) == binding.GDATTN_ERR_WORKSPACE
+    assert multi(sepv, 65) == binding.GDATTN_ERR_INVALID_ARG
+    core = good_desc(n_q_heads=8, n_kv_heads=2, head_dim=256, window=0,
+                     cache_capacity=1 << 21)
+    assert multi(core, 64) == binding.GDATTN_ERR_WORKSPACE
+    assert multi(core, 65) == binding.GDATTN_ERR_INVALID_ARG
