@@ -503,6 +503,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// 2^x by the hardware's approximate base-2 exponential (relative error about
+// 2^-22, results below 2^-126 flushed to zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // 2^e exactly, for integer e in [-126, 127] (a normal float built from its bits).
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
 

@@ -625,17 +625,21 @@ __global__ void __launch_bounds__(TcPairMultiConfig::kThreads, 1)
           }
         }
       }
-      // --- weights of this lane's (token, head): P rows 2t + hd and N + 2t + hd
+      // --- weights of this lane's (token, head): P rows 2t + hd and N + 2t + hd.
+      // Both bf16 parts are truncations (the upper halves of the fp32 bits; the
+      // remainder is exact in fp32 before its own), 2^-14 relative per weight.
+      // A row with no score yet (reference -inf) has only masked scores: 2^-inf = 0.
       {
         uint8_t *pbuf = ps + pb * Cfg::PB;
 #pragma unroll
         for (int t = 0; t < T; ++t) {
-          const float mr = hd ? m_ref[2 * t + 1] : m_ref[2 * t];
-          const float pe = (s[t] == -INFINITY) ? 0.f : exp2f(s[t] - mr);
+          const float mr0 = hd ? m_ref[2 * t + 1] : m_ref[2 * t];
+          const float pe = ex2_approx(s[t] - (mr0 == -INFINITY ? 0.f : mr0));
           lpart[t] += pe;
-          const uint16_t hi = f32_to_bf16_rn(pe);
+          const uint32_t u = __float_as_uint(pe);
+          const uint16_t hi = static_cast<uint16_t>(u >> 16);
           const uint16_t lo =
-              f32_to_bf16_rn(pe - __uint_as_float(static_cast<uint32_t>(hi) << 16));
+              static_cast<uint16_t>(__float_as_uint(pe - __uint_as_float(u & 0xFFFF0000u)) >> 16);
           *reinterpret_cast<uint16_t *>(pbuf + sw128_offset(2 * t + hd, tok)) = hi;
           *reinterpret_cast<uint16_t *>(pbuf + sw128_offset(N + 2 * t + hd, tok)) = lo;
         }

@@ -118,14 +118,6 @@ struct PrefillTiles {
   }
 };
 
-// 2^x by the hardware's approximate base-2 exponential (relative error about
-// 2^-22, results below 2^-126 flushed to zero; 2^-inf = 0).
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 // Block c -> (sequence b, KV head x, query block qb), heaviest causal blocks first.
 __device__ __forceinline__ void prefill_block(const PrefillParams &p, int32_t c, int32_t &b,
                                               int32_t &x, int32_t &qb) {
