@@ -317,7 +317,7 @@ gdattn_status gdattn_decode_multi(const void *q, const void *k_cache, const void
                                   void *stream);
 
 /*
- * gdattn_decode without a caller workspace.  A library addition: the paper
+ * gdattn_decode without a caller workspace.  A library addition: the pages
  * has no counterpart; it computes exactly what gdattn_decode computes.
  *
  * Same arguments (workspace and workspace_bytes dropped), host checks, kernels

@@ -365,7 +365,7 @@ def test_even_split_workspace_shared_by_two_geometries():
     for rep in range(3):
         for ly, (o_ref, l_ref), name in zip(layers, refs, "ab"):
             out, lse = ly.run()
-            compare(out, lse, o_ref, l_ref, ulp_floor=True, what=f"{name} round {rep}")
+            compare(out, lse, o_ref, l_ref, ulp_floor=True, what=f"{name} call {rep}")
 
 
 def test_workspace_shared_by_plans_with_many_units():

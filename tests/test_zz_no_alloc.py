@@ -1,6 +1,6 @@
 """gdattn_decode_noalloc: gdattn_decode with its split-KV scratch in a fixed
 device array inside the library (a library addition with no counterpart in the
-papers).  Its results must be bit-identical to gdattn_decode's, whatever the
+pages).  Its results must be bit-identical to gdattn_decode's, whatever the
 previous call left in the shared scratch.
 
 This file sorts last so that its GPU tests also run after everything else in
