@@ -317,8 +317,8 @@ gdattn_status gdattn_decode_multi(const void *q, const void *k_cache, const void
                                   void *stream);
 
 /*
- * gdattn_decode without a caller workspace.  A library addition: the pages
- * has no counterpart; it computes exactly what gdattn_decode computes.
+ * gdattn_decode without a caller workspace.  A library addition with no
+ * counterpart in the pages; it computes exactly what gdattn_decode computes.
  *
  * Same arguments (workspace and workspace_bytes dropped), host checks, kernels
  * and results as gdattn_decode: for the same inputs on the same device both
