@@ -15,9 +15,9 @@
 //   O^T[256 d x 32]  += V_tile^T[256 x 64] . P[64 x 32]     (M=128 x2, N=32, K=64)
 //
 // P row r holds query row r's bf16 weights (p_hi) and row 16 + r their
-// remainders (p_lo), the weight split of the single-token pair kernel, so O^T
-// column r plus column 16 + r is row r's output (rows 2T..15 of both halves
-// stay zero).  One 3-D TMA box {64 d, 2 heads, T tokens} per 64-d chunk brings
+// remainders (p_lo), a two-piece weight split like the single-token pair
+// kernel's (here both pieces truncated: 2^-14 relative), so O^T column r plus
+// column 16 + r is row r's output (rows 2T..15 of both halves stay zero).  One 3-D TMA box {64 d, 2 heads, T tokens} per 64-d chunk brings
 // a unit's 2T query rows from q [T][B][Hq][D] into the 16-row operand (rows 2T
 // and up are never read back).
 //
