@@ -386,8 +386,9 @@ def decode_multi(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor],
                  seqlens: torch.Tensor, desc: LayerDesc, max_seqlen: int,
                  out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                  workspace: Optional[torch.Tensor] = None, stream=None):
-    """Multi-query decode through gdattn_decode_multi.  q bf16 [T, B, Hq, D]: token t
-    of sequence b at position L_b - T + t, attending causally.  Returns (out, lse)."""
+    """Multi-token step through gdattn_decode_multi: a verify step, or a prompt chunk
+    (flash prefill).  q bf16 [T, B, Hq, D]: token t of sequence b at position
+    L_b - T + t, attending causally.  Returns (out, lse), token-major."""
     T, B, Hq, D = q.shape
     if out is None:
         out = torch.empty((T, B, Hq, D), dtype=torch.bfloat16, device=q.device)
