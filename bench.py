@@ -23,6 +23,7 @@ import dataclasses
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -74,15 +75,29 @@ def measured_peak_tflops():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def kernel_source_hash():
+_COMMENT_OR_LITERAL = re.compile(r'("(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\')|//[^\n]*|/\*.*?\*/',
+                                 re.S)
+
+
+def code_only(text):
+    """C++ source without its comments and blank lines, each line stripped:
+    what a comment edit or re-indentation leaves unchanged.  String and
+    character literals are kept as written."""
+    text = _COMMENT_OR_LITERAL.sub(lambda m: m.group(1) or "", text)
+    return "\n".join(ln.strip() for ln in text.splitlines() if ln.strip())
+
+
+def kernel_source_hash(csrc=None):
     """Hash of the device code of the profiled kernels: every kernel lives in a
-    csrc/*.cuh header (api.cu holds the host-side launches)."""
+    csrc/*.cuh header (api.cu holds the host-side launches).  Comments are left
+    out, so a record taken on a kernel stays valid across comment edits."""
+    csrc = CSRC if csrc is None else csrc
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
+    for name in sorted(os.listdir(csrc)):
         if name.endswith(".cuh"):
-            with open(os.path.join(CSRC, name), "rb") as f:
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
                 h.update(name.encode())
-                h.update(f.read())
+                h.update(code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -30,12 +30,12 @@
 //
 // Shared memory (1 CTA per SM): a ring of three 32 KiB K tiles (a K tile is
 // released as soon as its QK is done, so the K loads run further ahead), a ring
-// of two V tiles, and the block's Q (64 KiB, loaded once): 224 KiB.  TMEM holds the rest: S double
-// buffered (2 x 64 columns), P double buffered (each 32 columns of bf16 pairs
-// for the weights and 32 for their remainders, the A operand of P.V read from
-// tensor memory), and O (256 columns).  With two P buffers the softmax of tile
-// i waits only for the P.V of tile i - 2, so the tensor pipe is not left idle
-// while P is written.
+// of two V tiles, and the block's Q (64 KiB, loaded once): 224 KiB.  TMEM holds
+// the rest: S double buffered (2 x 64 columns), P double buffered (each 32
+// columns of bf16 pairs for the weights and 32 for their remainders, the A
+// operand of P.V read from tensor memory), and O (256 columns).  With two P
+// buffers the softmax of tile i waits only for the P.V of tile i - 2, so the
+// tensor pipe is not left idle while P is written.
 //
 // Warp roles (256 threads): warp 0 loads Q and K, warp 3 loads V, warp 1 issues
 // QK and owns TMEM, warp 2 issues P.V, warps 4-7 run the softmax (warp 4 + s

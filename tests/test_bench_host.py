@@ -98,6 +98,21 @@ def test_traffic_record_is_used_only_for_the_kernels_it_was_taken_on(tmp_path, m
     assert bench.traffic_for("sliding") is None
 
 
+def test_source_hash_ignores_comments_only(tmp_path):
+    """A comment edit keeps the traffic record valid; a code edit, even one
+    inside a string literal that looks like a comment, does not."""
+    src = tmp_path / "k.cuh"
+    base = 'int a = 1;  // scale\nasm("mov.b32 %0, 1;  // x");\n'
+    src.write_text(base)
+    h0 = bench.kernel_source_hash(str(tmp_path))
+    src.write_text("// header\n" + base.replace("// scale", "/* another\n comment */") + "\n\n")
+    assert bench.kernel_source_hash(str(tmp_path)) == h0
+    src.write_text(base.replace("1;  //", "2;  //"))
+    assert bench.kernel_source_hash(str(tmp_path)) != h0
+    src.write_text(base.replace("// x", "// y"))
+    assert bench.kernel_source_hash(str(tmp_path)) != h0
+
+
 def test_committed_traffic_record_names_every_profiled_kernel():
     with open(bench.TRAFFIC_RECORD) as f:
         rec = json.load(f)
