@@ -80,17 +80,18 @@ _COMMENT_OR_LITERAL = re.compile(r'("(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\')|
 
 
 def code_only(text):
-    """C++ source without its comments and blank lines, each line stripped:
-    what a comment edit or re-indentation leaves unchanged.  String and
-    character literals are kept as written."""
+    """C++ source without its comments and without whitespace, adjacent string
+    literals joined: what a comment edit, re-indentation or re-wrapping leaves
+    unchanged.  Comment markers inside string and character literals are kept."""
     text = _COMMENT_OR_LITERAL.sub(lambda m: m.group(1) or "", text)
-    return "\n".join(ln.strip() for ln in text.splitlines() if ln.strip())
+    return re.sub(r"\s+", "", text).replace('""', "")
 
 
 def kernel_source_hash(csrc=None):
     """Hash of the device code of the profiled kernels: every kernel lives in a
-    csrc/*.cuh header (api.cu holds the host-side launches).  Comments are left
-    out, so a record taken on a kernel stays valid across comment edits."""
+    csrc/*.cuh header (api.cu holds the host-side launches).  Comments and
+    whitespace are left out, so a record taken on a kernel stays valid across
+    comment and layout edits."""
     csrc = CSRC if csrc is None else csrc
     h = hashlib.sha256()
     for name in sorted(os.listdir(csrc)):

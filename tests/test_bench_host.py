@@ -99,13 +99,17 @@ def test_traffic_record_is_used_only_for_the_kernels_it_was_taken_on(tmp_path, m
 
 
 def test_source_hash_ignores_comments_only(tmp_path):
-    """A comment edit keeps the traffic record valid; a code edit, even one
-    inside a string literal that looks like a comment, does not."""
+    """A comment or layout edit keeps the traffic record valid; a code edit,
+    even one inside a string literal that looks like a comment, does not."""
     src = tmp_path / "k.cuh"
     base = 'int a = 1;  // scale\nasm("mov.b32 %0, 1;  // x");\n'
     src.write_text(base)
     h0 = bench.kernel_source_hash(str(tmp_path))
     src.write_text("// header\n" + base.replace("// scale", "/* another\n comment */") + "\n\n")
+    assert bench.kernel_source_hash(str(tmp_path)) == h0
+    src.write_text(base.replace("int a = 1;", "int a =\n    1;"))  # re-wrapped
+    assert bench.kernel_source_hash(str(tmp_path)) == h0
+    src.write_text(base.replace('"mov.b32 %0, 1;', '"mov.b32 "\n    "%0, 1;'))  # literal split
     assert bench.kernel_source_hash(str(tmp_path)) == h0
     src.write_text(base.replace("1;  //", "2;  //"))
     assert bench.kernel_source_hash(str(tmp_path)) != h0
