@@ -329,7 +329,10 @@ int oracle_decode_multi(const uint16_t *q, const uint16_t *k, const uint16_t *v,
 #if ORACLE_MUTATION == 13
       end = L; /* every query sees all T new tokens (not causal) */
 #endif
-      const int32_t start = (window > 0 && end > window) ? end - window : 0;
+      int32_t start = (window > 0 && end > window) ? end - window : 0;
+#if ORACLE_MUTATION == 18
+      if (window > 0 && end > window) start = end - window + 1; /* window one short */
+#endif
       lo[b] = start;
       hi[b] = end;
       if (end < 1 || start < L - C) rc = -1;

@@ -480,12 +480,39 @@ def pin_multi_ring_capacity(orc):
     raise AssertionError("a query reaching an overwritten slot was accepted")
 
 
+def pin_multi_causal_sdpa(orc):
+    """A whole prompt (L_b = T on a linear cache) is textbook causal attention:
+    torch SDPA in float64 with a causal mask, banded for a sliding window, and
+    the LSE from torch.logsumexp over the same masked scores."""
+    for i, (B, Hq, Hkv, D, T, w) in enumerate(((2, 4, 2, 16, 9, 0), (1, 4, 1, 8, 12, 5))):
+        inp = workloads.random_case(4200 + i, B, Hq, Hkv, D, T, [T] * B, window=w)
+        s = inp.spec
+        g = torch.Generator().manual_seed(4300 + i)
+        q = torch.randn((T, B, Hq, D), generator=g).to(torch.bfloat16)
+        o, l = orc.decode_multi(q, inp.k, inp.v, inp.seqlens, s.window, s.softcap, s.scale)
+        tq = torch.arange(T)[:, None]
+        j = torch.arange(T)[None, :]
+        allowed = (j <= tq) & ((j > tq - w) if w > 0 else torch.ones((T, T), dtype=torch.bool))
+        G = Hq // Hkv
+        for b in range(B):
+            Q = q[:, b].to(torch.float64).permute(1, 0, 2)                        # [Hq, T, D]
+            K = inp.k[b, :T].to(torch.float64).permute(1, 0, 2).repeat_interleave(G, dim=0)
+            V = inp.v[b, :T].to(torch.float64).permute(1, 0, 2).repeat_interleave(G, dim=0)
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                Q, K, V, attn_mask=allowed, scale=s.scale)                       # [Hq, T, D]
+            scores = torch.matmul(Q, K.transpose(1, 2)) * s.scale
+            ref_lse = torch.logsumexp(scores.masked_fill(~allowed, -float("inf")), dim=-1)
+            _close(o[:, b], ref.permute(1, 0, 2).numpy(), 1e-12, f"prompt {i} seq {b} out")
+            _close(l[:, b], ref_lse.T.numpy(), 1e-12, f"prompt {i} seq {b} lse")
+
+
 ALL_PINS = [pin_brute_force, pin_sdpa, pin_window_covers_context, pin_cap_to_infinity,
             pin_identical_keys, pin_zero_query, pin_single_position, pin_two_positions,
             pin_softcap_bound, pin_sliding_ignores_old_positions, pin_ring_equals_linear,
             pin_split_recombine, pin_combine_closed_form, pin_separate_v, pin_e4m3_codes,
             pin_fp8_equals_bf16_when_exact, pin_fp8_brute_force, pin_fp8_zero_scale_row,
-            pin_multi_brute_force, pin_multi_reduces_to_decode, pin_multi_ring_capacity]
+            pin_multi_brute_force, pin_multi_reduces_to_decode, pin_multi_ring_capacity,
+            pin_multi_causal_sdpa]
 
 
 def failing_pins(orc):

@@ -26,6 +26,7 @@ MUTATIONS = {
     15: "merge weights relative to the largest part, not normalised",
     16: "soft-cap without its outer factor",
     17: "e4m3 subnormals decoded with a leading one",
+    18: "multi-token window one position short",
 }
 
 
