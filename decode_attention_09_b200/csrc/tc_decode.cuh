@@ -119,49 +119,6 @@ struct TcConfig {
 // weights stay below 256: no overflow in bf16 P, fp32 sums or O.
 constexpr float kTau = 8.f;
 
-// Tiles of one CTA, in order, across its segments.
-template <int TILE>
-struct TileIterT {
-  SegmentIter seg_it;
-  Segment seg;
-  SlotRuns runs;
-  int32_t run, t0;
-  bool have_seg;
-  bool newest;  // the last tile yielded holds the unit's newest position (L - 1)
-  int32_t off;  // offset of the last tile's first token in its unit's attended range
-
-  __device__ __forceinline__ void init(const Geometry &g, const ChunkPlan &p) {
-    seg_it.init(g, p);
-    have_seg = false;
-  }
-  // Yields the next tile: slot row of its first token, valid token count, and
-  // whether it opens / closes its segment.
-  __device__ __forceinline__ bool next(int32_t C, int32_t &row, int32_t &ntok, bool &first,
-                                       bool &last) {
-    first = false;
-    if (!have_seg) {
-      if (!seg_it.next(seg)) return false;
-      runs = segment_runs(seg, C);
-      run = 0;
-      t0 = 0;
-      have_seg = true;
-      first = true;
-    }
-    row = runs.start(run) + t0;
-    ntok = min(TILE, runs.len(run) - t0);
-    off = seg.lo + (run == 1 ? runs.len0 : 0) + t0;
-    newest = off + ntok == seg.n;
-    t0 += TILE;
-    if (t0 >= runs.len(run)) {
-      ++run;
-      t0 = 0;
-    }
-    last = (run >= runs.count);
-    if (last) have_seg = false;
-    return true;
-  }
-};
-
 using TileIter = TileIterT<TcConfig::TILE>;
 
 // Reduce 16 per-lane values over the warp (op = max or sum): after it, lane l

@@ -11,6 +11,8 @@
 //   segments carry the right unit, length and first position, slots c + u are
 //   unique, and unit_chunks names exactly the chunks that touched the unit;
 // - segment_runs: the one or two slot runs are the positions modulo C;
+// - TileIterT: each segment cut into tiles that follow one another, start at
+//   the right slot, never cross the ring's end, and carry the right flags;
 // - plan_unit_split: k parts on tile boundaries that cover a unit once (on up
 //   to 14 units of each batch, evenly spaced, the last one included).
 // Prints "ok <cases>" or the first failure, and exits non-zero on failure.
@@ -155,6 +157,52 @@ char g_err[512];
     }                                                     \
   } while (0)
 
+// Walks chunk c's tiles with TileIterT<TILE> against its segments: each
+// segment's tiles follow one another from lo to hi, start at the slot of
+// their first position, never cross the ring's end, are short only at the end
+// of a slot run, and carry the first / last / newest flags of their place.
+template <int TILE>
+bool check_tiles(const Case &cs, const Geometry &g, const ChunkPlan &p, int32_t c,
+                 const std::vector<Segment> &segs) {
+  TileIterT<TILE> it;
+  it.init(g, p);
+  int32_t row, ntok;
+  bool first, last;
+  size_t si = 0;
+  int32_t next_off = 0;
+  bool in_seg = false;
+  while (it.next(cs.capacity, row, ntok, first, last)) {
+    CHECK(si < segs.size(), "chunk %d: tiles past its %zu segments", c, segs.size());
+    const Segment &s = segs[si];
+    CHECK(first == !in_seg, "chunk %d segment %zu: first flag", c, si);
+    if (first) {
+      next_off = s.lo;
+      in_seg = true;
+    }
+    CHECK(it.seg.unit == s.unit && it.seg.lo == s.lo && it.seg.hi == s.hi,
+          "chunk %d: tile of another segment", c);
+    CHECK(it.off == next_off, "chunk %d unit %d: tile at offset %d, expected %d", c, s.unit,
+          it.off, next_off);
+    CHECK(ntok >= 1 && ntok <= TILE, "chunk %d unit %d: %d tokens", c, s.unit, ntok);
+    CHECK(row == (s.first_pos + it.off) % cs.capacity, "chunk %d unit %d: row %d", c, s.unit,
+          row);
+    CHECK(row + ntok <= cs.capacity, "chunk %d unit %d: tile crosses the ring's end", c, s.unit);
+    CHECK(ntok == TILE || last || row + ntok == cs.capacity,
+          "chunk %d unit %d: short tile inside a run", c, s.unit);
+    CHECK(it.newest == (it.off + ntok == s.n), "chunk %d unit %d: newest flag", c, s.unit);
+    next_off += ntok;
+    CHECK(next_off <= s.hi, "chunk %d unit %d: tiles past the segment", c, s.unit);
+    if (last) {
+      CHECK(next_off == s.hi, "chunk %d unit %d: segment ends at %d, not %d", c, s.unit,
+            next_off, s.hi);
+      ++si;
+      in_seg = false;
+    }
+  }
+  CHECK(si == segs.size() && !in_seg, "chunk %d: %zu of %zu segments tiled", c, si, segs.size());
+  return true;
+}
+
 // Checks one chunk count's whole plan (lane 0 only; plans come from all lanes).
 bool check_chunks(const Case &cs, const Geometry &g, const std::vector<ChunkPlan> &plans) {
   const int32_t B = static_cast<int32_t>(cs.seqlens.size());
@@ -186,7 +234,9 @@ bool check_chunks(const Case &cs, const Geometry &g, const std::vector<ChunkPlan
     it.init(g, p);
     Segment s;
     int64_t pos = p.cs;
+    std::vector<Segment> segs;
     while (it.next(s)) {
+      segs.push_back(s);
       const int32_t b = s.unit / cs.units_per_seq;
       CHECK(b == s.b && s.x == s.unit - b * cs.units_per_seq && s.unit < units,
             "chunk %d: unit %d of (%d, %d)", c, s.unit, s.b, s.x);
@@ -217,6 +267,8 @@ bool check_chunks(const Case &cs, const Geometry &g, const std::vector<ChunkPlan
     }
     CHECK(pos == p.ce || p.cs == p.ce, "chunk %d ends at %lld, not %lld", c, (long long)pos,
           (long long)p.ce);
+    if (!check_tiles<64>(cs, g, p, c, segs) || !check_tiles<128>(cs, g, p, c, segs))
+      return false;
   }
   for (int32_t u = 0; u < units; ++u) {
     for (size_t o = 0; o < cover[u].size(); ++o)

@@ -2,9 +2,10 @@
 
 The header is copied beside an empty ptx.cuh and compiled with g++ together
 with tests/planner_host.cpp, which emulates the warp intrinsics it uses (32
-lanes as fibers) and checks plan_chunk, SegmentIter, unit_chunks, segment_runs
-and plan_unit_split on random ragged batches: every attended position of every
-unit is covered exactly once, slots are unique, chunks and parts are aligned.
+lanes as fibers) and checks plan_chunk, SegmentIter, unit_chunks, segment_runs,
+TileIterT and plan_unit_split on random ragged batches: every attended position
+of every unit is covered exactly once, slots are unique, chunks and parts are
+aligned, and tiles follow their segments without crossing the ring's end.
 A planted mistake in a copy of the header must make the check fail.
 """
 import os
@@ -44,6 +45,7 @@ def test_split_planner_covers_every_position_once(tmp_path):
      "const int64_t ce = imin64(cs + chunk - 1, total);"),
     ("const int32_t first = min(len, C - s0);", "const int32_t first = min(len, C - s0 - 1);"),
     ("if (lane >= o) v += t;", "if (lane > o) v += t;"),
+    ("off = seg.lo + (run == 1 ? runs.len0 : 0) + t0;", "off = seg.lo + t0;"),
 ])
 def test_planted_planner_mistake_is_caught(tmp_path, original, planted):
     with open(PARTITION) as f:
