@@ -2,7 +2,9 @@
 
 bf16 kernels: an MMA's two operands share one type, and V is bf16, so the fp32
 softmax weights go in as two bf16 pieces, p = p_hi + p_lo with p_hi = bf16(p)
-and p_lo = bf16(p - p_hi), in separate MMA columns summed in fp32.
+and p_lo = bf16(p - p_hi), in separate MMA columns summed in fp32.  The
+verify-step and prefill kernels take both pieces by truncation instead (the
+upper halves of the fp32 bits), which keeps 2^-14 relative.
 
 fp8 kernel:
 
@@ -90,3 +92,27 @@ def test_bf16_hi_lo_weight_split():
     assert rel.max().item() <= 2.0 ** -17
     one = (hi.double() - p.double()).abs() / p.double()
     assert 2.0 ** -9 < one.max().item() <= 2.0 ** -8  # what a single piece would keep
+
+
+def truncate_bf16(x: torch.Tensor) -> torch.Tensor:
+    """The upper 16 bits of an fp32 value, as an fp32 value (round toward zero)."""
+    bits = x.float().contiguous().view(torch.int32) & ~0xFFFF
+    return bits.view(torch.float32)
+
+
+def test_bf16_truncation_weight_split():
+    """The verify-step and prefill kernels split a weight by truncation: hi = the
+    upper half of its fp32 bits, lo = the upper half of p - hi (exact in fp32).
+    Two truncated pieces keep a positive weight to 2^-14 relative, never above it."""
+    g = torch.Generator().manual_seed(3)
+    p = torch.exp2(torch.rand(1_000_000, generator=g, dtype=torch.float64) * 40 - 32).float()
+    hi = truncate_bf16(p)
+    r = p - hi
+    assert torch.equal(r.double(), p.double() - hi.double())  # the remainder is exact
+    lo = truncate_bf16(r)
+    assert torch.equal(hi.to(torch.bfloat16).float(), hi)  # both pieces are bf16 numbers
+    assert torch.equal(lo.to(torch.bfloat16).float(), lo)
+    total = hi.double() + lo.double()
+    assert (total <= p.double()).all()
+    rel = (p.double() - total) / p.double()
+    assert 2.0 ** -16 < rel.max().item() < 2.0 ** -14
